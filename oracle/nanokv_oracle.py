@@ -1,0 +1,307 @@
+"""Plain, slow fp64 CPU oracle for NanoKV compressed-history attention.
+
+TEST INFRASTRUCTURE ONLY.  Only the tests, the smoke entry point and the
+benchmark's CPU-baseline leg may import this module.  The CUDA path never
+calls it, and it shares no code with the CUDA path.
+
+Source: "NanoKV: High-Ratio KV Cache Compression for Autoregressive Video
+Generation" (arXiv 2611.06377): abstract; Fig. 2(b,c); Fig. 4(a) joint
+head-channel encoding read through full- or mixed-dimensional attention;
+Fig. 4(b) encoder to INT4 coefficients, decoder adds back centers; Fig. 4(d)
+fixed routing, reduced queries, output restore, LSE merging; Table 5 (rank per
+layer per K/V branch, centers fitted separately for K and V).
+
+The pages print no formulas.  Where they are silent this module takes the
+plain readings below (each also listed in the design notes):
+  * nearest center = smallest squared Euclidean distance in the joint H*d
+    space, ties to the lowest index;
+  * per-token symmetric scale s = stored_dtype(max_i |y_i| / 7), INT4 codes in
+    [-7, 7] (-8 unused), round-half-to-even, s = 0 gives all-zero codes;
+  * softmax scale tau (1/sqrt(d) by default), no mask, natural-log LSE;
+  * head h owns joint columns [h*d, (h+1)*d) of K/V and rows of D;
+  * the current chunk is a third, uncompressed attention branch merged by LSE;
+  * routing: the most recent T_full history tokens are full-dim, the older
+    T - T_full tokens low-dim.
+
+Every stored value (bf16 / fp16 / fp32) converts exactly to fp64, and all
+arithmetic here is fp64 numpy.  Parity of every function is pinned by the
+"not gpu" tests (brute force, closed forms, invariants, the pages' tables).
+"""
+from __future__ import annotations
+
+import numpy as np
+
+QMAX = 7  # symmetric INT4 range [-7, 7]
+
+
+def f64(a) -> np.ndarray:
+    """Exact conversion of a stored array (numpy or torch CPU) to fp64."""
+    if hasattr(a, "detach"):
+        a = a.detach().to("cpu")
+        if a.dtype.is_floating_point:
+            a = a.double()
+        a = a.numpy()
+    return np.asarray(a, dtype=np.float64)
+
+
+def round_to_storage(v: np.ndarray, scale_dtype: str) -> np.ndarray:
+    """Round fp64 values to the scale's storage dtype (RNE), back in fp64."""
+    if scale_dtype == "f16":
+        return np.asarray(v, dtype=np.float64).astype(np.float16).astype(np.float64)
+    if scale_dtype == "f32":
+        return np.asarray(v, dtype=np.float64).astype(np.float32).astype(np.float64)
+    raise ValueError(scale_dtype)
+
+
+# ----------------------------------------------------------------------------
+# Encode (Fig. 4(a,b); abstract: shared content in cluster centers, joint
+# head-channel residuals encoded into low-bit coefficients)
+# ----------------------------------------------------------------------------
+
+def squared_distances(x: np.ndarray, centers: np.ndarray) -> np.ndarray:
+    """dist[t, j] = sum_i (x[t, i] - centers[j, i])^2, one center at a time."""
+    T, C = x.shape[0], centers.shape[0]
+    dist = np.empty((T, C), dtype=np.float64)
+    for j in range(C):
+        diff = x - centers[j][None, :]
+        dist[:, j] = np.einsum("ti,ti->t", diff, diff)
+    return dist
+
+
+def assign(x: np.ndarray, centers: np.ndarray) -> np.ndarray:
+    """Nearest center of each token (lowest index on exact ties)."""
+    return np.argmin(squared_distances(x, centers), axis=1)
+
+
+def project(x: np.ndarray, centers: np.ndarray, ids: np.ndarray, E: np.ndarray) -> np.ndarray:
+    """Residual coefficients y_t = E (x_t - c_{a_t}),  E is [r, J]."""
+    rho = x - centers[ids]
+    return rho @ E.T
+
+
+def scale_of(y: np.ndarray, scale_dtype: str) -> np.ndarray:
+    """Per-token symmetric scale s_t = stored(max_i |y_ti| / 7)."""
+    m = np.max(np.abs(y), axis=1) if y.shape[1] else np.zeros(y.shape[0])
+    return round_to_storage(m / QMAX, scale_dtype)
+
+
+def quantise(y: np.ndarray, s: np.ndarray) -> np.ndarray:
+    """INT4 codes clamp(round_half_even(y / s), -7, 7); s = 0 gives zeros."""
+    codes = np.zeros(y.shape, dtype=np.int64)
+    nz = s > 0
+    codes[nz] = np.clip(np.rint(y[nz] / s[nz, None]), -QMAX, QMAX).astype(np.int64)
+    return codes
+
+
+def encode(x: np.ndarray, centers: np.ndarray, E: np.ndarray, scale_dtype: str) -> dict:
+    """Full encode of tokens x [T, J]: ids, unpacked codes [T, r], scales [T],
+    plus the fp64 intermediates used by the tie accounting."""
+    ids = assign(x, centers)
+    y = project(x, centers, ids, E)
+    s = scale_of(y, scale_dtype)
+    return {"ids": ids, "codes": quantise(y, s), "scales": s, "y": y}
+
+
+def pack_codes(codes: np.ndarray) -> np.ndarray:
+    """[T, r] ints in [-8, 7] -> [T, r/2] bytes; code 2i in the low nibble of
+    byte i, two's complement."""
+    c = (np.asarray(codes, dtype=np.int64) & 0xF).astype(np.uint8)
+    return (c[:, 0::2] | (c[:, 1::2] << 4)).astype(np.uint8)
+
+
+def unpack_codes(packed: np.ndarray) -> np.ndarray:
+    """Inverse of pack_codes: [T, r/2] bytes -> [T, r] int64 in [-8, 7]."""
+    p = np.asarray(packed, dtype=np.uint8).astype(np.int64)
+    lo, hi = p & 0xF, (p >> 4) & 0xF
+    out = np.empty((p.shape[0], 2 * p.shape[1]), dtype=np.int64)
+    out[:, 0::2] = np.where(lo >= 8, lo - 16, lo)
+    out[:, 1::2] = np.where(hi >= 8, hi - 16, hi)
+    return out
+
+
+def decode(ids, codes, scales, centers, D) -> np.ndarray:
+    """x_hat_t = c_{a_t} + s_t * D q_t   (Fig. 4(b): decoder reconstructs the
+    residual and adds back the center).  D is [J, r]."""
+    return centers[ids] + scales[:, None] * (np.asarray(codes, np.float64) @ D.T)
+
+
+# ----------------------------------------------------------------------------
+# Attention branches.  Layout: q [Tq, H, d]; history K/V joint vectors [T, J]
+# with head h in columns [h*d, (h+1)*d); outputs O [Tq, H, d], LSE [H, Tq].
+# ----------------------------------------------------------------------------
+
+def softmax_attention(q: np.ndarray, k: np.ndarray, v: np.ndarray, tau: float):
+    """Textbook softmax attention per head over keys k, v [T, H, d]."""
+    Tq, H, d = q.shape
+    T = k.shape[0]
+    O = np.zeros((Tq, H, d))
+    lse = np.full((H, Tq), -np.inf)
+    if T == 0:
+        return O, lse
+    for h in range(H):
+        z = tau * (q[:, h, :] @ k[:, h, :].T)
+        m = z.max(axis=1, keepdims=True)
+        p = np.exp(z - m)
+        l = p.sum(axis=1, keepdims=True)
+        O[:, h, :] = (p @ v[:, h, :]) / l
+        lse[h] = (m + np.log(l))[:, 0]
+    return O, lse
+
+
+def attend_full(q, ck: dict, cv: dict, hk: dict, hv: dict, tau: float):
+    """Full-dimensional branch (Fig. 4(a), NanoKV): decode K_hat, V_hat to the
+    full joint dimension, then ordinary attention over them."""
+    Tq, H, d = q.shape
+    kh = decode(hk["ids"], hk["codes"], hk["scales"], ck["centers"], ck["D"])
+    vh = decode(hv["ids"], hv["codes"], hv["scales"], cv["centers"], cv["D"])
+    T = kh.shape[0]
+    return softmax_attention(q, kh.reshape(T, H, d), vh.reshape(T, H, d), tau)
+
+
+def attend_low(q, ck: dict, cv: dict, hk: dict, hv: dict, tau: float):
+    """Mixed-dimensional branch (abstract: NanoKV-Fast reuses the stored
+    coefficients; Fig. 4(d): reduce the queries, restore the output dimension).
+
+    Per head h with D_h = rows [h*d, (h+1)*d) of D and c_{j,h} the head's slice
+    of center j:
+        q~   = D_{K,h}^T q                  (reduced query, length r)
+        qc_j = c_{K,j,h} . q                (query against each K center)
+        z_t  = tau * (s_t * q~ . code_t + qc_{a_t})
+        O    = (sum_t p_t c_{V,a_t,h} + D_{V,h} sum_t p_t s_t code^V_t) / sum_t p_t
+    """
+    Tq, H, d = q.shape
+    T = len(hk["ids"])
+    O = np.zeros((Tq, H, d))
+    lse = np.full((H, Tq), -np.inf)
+    if T == 0:
+        return O, lse
+    codes_k = np.asarray(hk["codes"], np.float64)
+    codes_v = np.asarray(hv["codes"], np.float64)
+    sk, sv = hk["scales"], hv["scales"]
+    C_v = cv["centers"].shape[0]
+    onehot_v = np.zeros((T, C_v))
+    onehot_v[np.arange(T), hv["ids"]] = 1.0
+    for h in range(H):
+        cols = slice(h * d, (h + 1) * d)
+        qh = q[:, h, :]
+        q_red = qh @ ck["D"][cols, :]                 # [Tq, r]
+        qc = qh @ ck["centers"][:, cols].T           # [Tq, C]
+        z = tau * (sk[None, :] * (q_red @ codes_k.T) + qc[:, hk["ids"]])
+        m = z.max(axis=1, keepdims=True)
+        p = np.exp(z - m)
+        l = p.sum(axis=1, keepdims=True)
+        o_red = p @ (sv[:, None] * codes_v)          # [Tq, r]
+        p_c = p @ onehot_v                           # [Tq, C]
+        O[:, h, :] = (p_c @ cv["centers"][:, cols] + o_red @ cv["D"][cols, :].T) / l
+        lse[h] = (m + np.log(l))[:, 0]
+    return O, lse
+
+
+def lse_merge(parts):
+    """Combine branch partials (O_i, LSE_i) by log-sum-exp weights (Fig. 4(d)):
+    LSE = log sum_i exp(LSE_i),  O = sum_i exp(LSE_i - LSE) O_i.  Branches with
+    LSE = -inf contribute nothing; if all are empty, O = 0 and LSE = -inf."""
+    lses = np.stack([p[1] for p in parts])           # [n, H, Tq]
+    m = lses.max(axis=0)
+    safe_m = np.where(np.isfinite(m), m, 0.0)
+    w = np.exp(lses - safe_m[None])                  # exp(-inf) = 0
+    tot = w.sum(axis=0)
+    lse = np.where(tot > 0, safe_m + np.log(np.where(tot > 0, tot, 1.0)), -np.inf)
+    O = np.zeros_like(parts[0][0])
+    for (o_i, _), w_i in zip(parts, w):
+        coef = np.where(tot > 0, w_i / np.where(tot > 0, tot, 1.0), 0.0)   # [H, Tq]
+        O += coef.T[:, :, None] * o_i
+    return O, lse
+
+
+def split_history(h: dict, lo: int, hi: int) -> dict:
+    return {"ids": h["ids"][lo:hi], "codes": h["codes"][lo:hi], "scales": h["scales"][lo:hi]}
+
+
+def attend(q, ck, cv, hk, hv, T_full: int, k_cur=None, v_cur=None, tau=None):
+    """Compressed-history attention of a query chunk (Fig. 4(d) with Fig. 4(a)):
+    the oldest T - T_full history tokens go through the low-dim branch, the most
+    recent T_full through full-dim decode-attention, the current chunk's
+    uncompressed K/V through plain attention; the three are LSE-merged."""
+    Tq, H, d = q.shape
+    if tau is None:
+        tau = 1.0 / np.sqrt(d)
+    T = len(hk["ids"])
+    T_low = T - T_full
+    parts = [
+        attend_low(q, ck, cv, split_history(hk, 0, T_low), split_history(hv, 0, T_low), tau),
+        attend_full(q, ck, cv, split_history(hk, T_low, T), split_history(hv, T_low, T), tau),
+    ]
+    if k_cur is not None and len(k_cur):
+        parts.append(softmax_attention(q, k_cur, v_cur, tau))
+    return lse_merge(parts)
+
+
+# ----------------------------------------------------------------------------
+# Tie accounting: an integer decided by floating point (argmin, rounding, the
+# fp16 scale) may legitimately differ between two correct implementations only
+# when the real-valued quantity sits within rounding error of the boundary.
+# ----------------------------------------------------------------------------
+
+TIE_REL = 1e-6
+
+
+def argmin_ties(x: np.ndarray, centers: np.ndarray) -> np.ndarray:
+    """Tokens whose best and second-best center distances are within
+    1e-6 * (|x|^2 + |c_best|^2)."""
+    dist = squared_distances(x, centers)
+    if dist.shape[1] < 2:
+        return np.zeros(dist.shape[0], dtype=bool)
+    srt = np.sort(dist, axis=1)
+    best = np.argmin(dist, axis=1)
+    scale = np.einsum("ti,ti->t", x, x) + np.einsum("ti,ti->t", centers[best], centers[best])
+    return (srt[:, 1] - srt[:, 0]) <= TIE_REL * scale
+
+
+def codes_given_scale(y: np.ndarray, s: np.ndarray) -> np.ndarray:
+    """The oracle's code decision under a given stored scale."""
+    return quantise(y, s)
+
+
+def rounding_ties(x, centers, ids, E, y, s) -> np.ndarray:
+    """Code entries whose y/s lies within 1e-6 * max(1, sum_j |E_ij||rho_j| / s)
+    of a half-integer (the forward-error scale of the dot product)."""
+    rho = x - centers[ids]
+    mag = np.abs(rho) @ np.abs(E).T                  # [T, r]
+    ss = np.where(s > 0, s, 1.0)[:, None]
+    u = y / ss
+    dist = np.abs(u - (np.floor(u) + 0.5))
+    band = TIE_REL * np.maximum(1.0, mag / ss)
+    return (dist <= band) & (s[:, None] > 0)
+
+
+def scale_ties(y: np.ndarray, scale_dtype: str) -> np.ndarray:
+    """Tokens whose max|y|/7 lies within 1e-6 relative of a rounding midpoint of
+    the scale's storage dtype (fp16).  For fp32 scales every value is that close
+    to a midpoint; those are compared with a relative tolerance instead."""
+    v = np.max(np.abs(y), axis=1) / QMAX if y.shape[1] else np.zeros(y.shape[0])
+    if scale_dtype == "f32":
+        return np.ones(v.shape, dtype=bool)
+    f = v.astype(np.float16)
+    up = np.nextafter(f, np.float16(np.inf)).astype(np.float64)
+    dn = np.nextafter(f, np.float16(-np.inf)).astype(np.float64)
+    ff = f.astype(np.float64)
+    mid = np.where(v >= ff, (ff + up) / 2, (ff + dn) / 2)
+    return np.abs(v - mid) <= TIE_REL * np.abs(v)
+
+
+# ----------------------------------------------------------------------------
+# Accounting (Table 5 x Table 9; Table 11)
+# ----------------------------------------------------------------------------
+
+def nominal_coefficient_cr(H: int, d: int, r: int, src_bits: int = 16, code_bits: int = 4) -> float:
+    """Coefficient compression of one token: H*d values of src_bits against r
+    coefficients of code_bits."""
+    return (src_bits * H * d) / (code_bits * r)
+
+
+def overall_saving(historical_share: float, saving_within_history: float) -> float:
+    """Table 11: overall visual-attention MAC saving = historical share x saving
+    within history."""
+    return historical_share * saving_within_history
+

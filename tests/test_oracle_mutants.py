@@ -1,0 +1,107 @@
+"""Plant plausible mistakes in the oracle (on the CPU, one at a time) and check
+that at least one pin catches each of them."""
+import numpy as np
+import pytest
+
+from oracle import nanokv_oracle as orc
+from tests import test_oracle_pins as pins
+
+PINS = [getattr(pins, n) for n in dir(pins) if n.startswith("test_")]
+
+
+def _run_pins():
+    failed = []
+    for fn in PINS:
+        kwargs = {"tau": 1.0} if "tau" in fn.__code__.co_varnames[:fn.__code__.co_argcount] else {}
+        try:
+            fn(**kwargs)
+        except Exception:
+            failed.append(fn.__name__)
+    return failed
+
+
+def _decode_no_center(ids, codes, scales, centers, D):
+    return scales[:, None] * (np.asarray(codes, np.float64) @ D.T)
+
+
+def _decode_no_scale(ids, codes, scales, centers, D):
+    return centers[ids] + (np.asarray(codes, np.float64) @ D.T)
+
+
+def _quantise_floor(y, s):
+    codes = np.zeros(y.shape, dtype=np.int64)
+    nz = s > 0
+    codes[nz] = np.clip(np.floor(y[nz] / s[nz, None] + 0.5), -7, 7).astype(np.int64)
+    return codes
+
+
+def _scale_unrounded(y, scale_dtype):
+    return np.max(np.abs(y), axis=1) / 7
+
+
+def _assign_argmax(x, centers):
+    return np.argmax(orc.squared_distances(x, centers), axis=1)
+
+
+def _project_no_center(x, centers, ids, E):
+    return x @ E.T
+
+
+def _merge_max(parts):
+    lses = np.stack([p[1] for p in parts])
+    idx = np.argmax(lses, axis=0)
+    O = np.zeros_like(parts[0][0])
+    for i, (o, _) in enumerate(parts):
+        O += (idx == i).T[:, :, None] * o
+    return O, lses.max(axis=0)
+
+
+def _pack_swapped(codes):
+    c = (np.asarray(codes, dtype=np.int64) & 0xF).astype(np.uint8)
+    return (c[:, 1::2] | (c[:, 0::2] << 4)).astype(np.uint8)
+
+
+_orig_low = orc.attend_low
+
+
+def _low_wrong_value_scale(q, ck, cv, hk, hv, tau):
+    hv2 = dict(hv, scales=hk["scales"])
+    return _orig_low(q, ck, cv, hk, hv2, tau)
+
+
+def _low_no_key_center(q, ck, cv, hk, hv, tau):
+    ck2 = dict(ck, centers=np.zeros_like(ck["centers"]))
+    return _orig_low(q, ck2, cv, hk, hv, tau)
+
+
+_orig_sm = orc.softmax_attention
+
+
+def _softmax_no_tau(q, k, v, tau):
+    return _orig_sm(q, k, v, 1.0 if tau != 1.0 else 0.5)
+
+
+MUTANTS = {
+    "decode_no_center": ("decode", _decode_no_center),
+    "decode_no_scale": ("decode", _decode_no_scale),
+    "quantise_half_up": ("quantise", _quantise_floor),
+    "scale_unrounded": ("scale_of", _scale_unrounded),
+    "assign_argmax": ("assign", _assign_argmax),
+    "project_no_center": ("project", _project_no_center),
+    "merge_hard_max": ("lse_merge", _merge_max),
+    "pack_nibbles_swapped": ("pack_codes", _pack_swapped),
+    "low_value_uses_key_scale": ("attend_low", _low_wrong_value_scale),
+    "low_drops_key_center": ("attend_low", _low_no_key_center),
+    "softmax_wrong_tau": ("softmax_attention", _softmax_no_tau),
+}
+
+
+def test_pins_pass_unmutated():
+    assert _run_pins() == []
+
+
+@pytest.mark.parametrize("name", sorted(MUTANTS))
+def test_mutant_is_caught(name, monkeypatch):
+    attr, fn = MUTANTS[name]
+    monkeypatch.setattr(orc, attr, fn)
+    assert _run_pins(), f"no pin catches mutant {name}"

@@ -1,0 +1,319 @@
+"""Pins of the fp64 oracle to things other than itself: hand-worked cases, pure
+Python brute force, library routines, closed forms, algebraic invariants and
+the pages' printed tables.  CPU only."""
+import json
+import math
+import os
+
+import numpy as np
+import pytest
+import torch
+
+from oracle import nanokv_oracle as orc
+
+GOLD = os.path.join(os.path.dirname(__file__), "golden")
+
+
+def _load(name):
+    with open(os.path.join(GOLD, name)) as f:
+        return json.load(f)
+
+
+def _rand_codec(rng, H, d, r, C, T):
+    J = H * d
+    ck = {"centers": rng.standard_normal((C, J)), "D": rng.standard_normal((J, r)) / math.sqrt(r)}
+    cv = {"centers": rng.standard_normal((C, J)), "D": rng.standard_normal((J, r)) / math.sqrt(r)}
+
+    def hist():
+        return {"ids": rng.integers(0, C, T), "codes": rng.integers(-7, 8, (T, r)),
+                "scales": rng.uniform(0.05, 0.6, T)}
+    return ck, cv, hist(), hist()
+
+
+# --------------------------------------------------------------------------
+# assignment
+# --------------------------------------------------------------------------
+
+def test_assign_matches_python_loop():
+    rng = np.random.default_rng(11)
+    x = rng.standard_normal((9, 5))
+    cen = rng.standard_normal((4, 5))
+    cen[3] = cen[1]                      # duplicate center: tie -> lowest index
+    x[0] = cen[1] + 1e-3
+    want = []
+    for t in range(9):
+        best, bj = None, None
+        for j in range(4):
+            dd = sum((float(x[t, i]) - float(cen[j, i])) ** 2 for i in range(5))
+            if best is None or dd < best:
+                best, bj = dd, j
+        want.append(bj)
+    assert list(orc.assign(x, cen)) == want
+    assert orc.assign(x, cen)[0] == 1
+
+
+def test_assign_recovers_generator_labels():
+    from synth.gen import WORKLOADS, make_codec, make_tokens, scaled, _gen
+    w = scaled(WORKLOADS["full"], T=300, Tq=8)
+    g = _gen(123, "cpu")
+    codec = make_codec(w, g, "cpu")
+    x, labels = make_tokens(w, codec, 300, g, "cpu")
+    cen = orc.f64(codec["centers"])
+    xx = orc.f64(x)
+    assert np.array_equal(orc.assign(xx, cen), labels.numpy())
+    assert not orc.argmin_ties(xx, cen).any()
+
+
+# --------------------------------------------------------------------------
+# INT4 coefficients
+# --------------------------------------------------------------------------
+
+def test_int4_hand_picked_cases():
+    g = _load("int4_cases.json")
+    for c in g["cases"]:
+        y = np.array([c["y"]], dtype=np.float64)
+        s = orc.scale_of(y, c["scale_dtype"])
+        assert s[0] == c["scale"], c
+        assert list(orc.quantise(y, s)[0]) == c["codes"], c
+    codes = np.array([g["pack"]["codes"]])
+    packed = orc.pack_codes(codes)
+    assert list(packed[0]) == g["pack"]["bytes"]
+    assert np.array_equal(orc.unpack_codes(packed), codes)
+
+
+def test_int4_clamp_and_zero_scale():
+    y = np.array([[10.0, -10.0, 0.2]])
+    assert list(orc.quantise(y, np.array([1.0]))[0]) == [7, -7, 0]
+    assert list(orc.quantise(y, np.array([0.0]))[0]) == [0, 0, 0]
+
+
+def test_pack_roundtrip_all_nibbles():
+    vals = np.arange(-8, 8)
+    codes = np.array(np.meshgrid(vals, vals)).reshape(2, -1).T.reshape(-1, 2)
+    assert np.array_equal(orc.unpack_codes(orc.pack_codes(codes)), codes)
+
+
+# --------------------------------------------------------------------------
+# codec round trip (invariant: unquantised full-rank orthonormal D is exact)
+# --------------------------------------------------------------------------
+
+def test_orthonormal_full_rank_roundtrip():
+    rng = np.random.default_rng(5)
+    J, C, T = 24, 3, 40
+    D = np.linalg.qr(rng.standard_normal((J, J)))[0]
+    E = D.T
+    cen = rng.standard_normal((C, J))
+    x = cen[rng.integers(0, C, T)] + 0.3 * rng.standard_normal((T, J))
+    ids = orc.assign(x, cen)
+    y = orc.project(x, cen, ids, E)
+    xhat = orc.decode(ids, y, np.ones(T), cen, D)
+    assert np.max(np.abs(xhat - x)) < 1e-12
+
+
+def test_decode_adds_center_and_scales_codes():
+    cen = np.array([[1.0, 2.0], [-3.0, 0.5]])
+    D = np.array([[1.0, 0.0, 2.0], [0.0, -1.0, 1.0]])     # J=2, r=3
+    ids = np.array([1, 0])
+    codes = np.array([[1, 2, -1], [0, 7, 3]])
+    s = np.array([0.5, 0.25])
+    want = np.array([[-3.0 + 0.5 * (1 - 2), 0.5 + 0.5 * (-2 - 1)],
+                     [1.0 + 0.25 * (0 + 6), 2.0 + 0.25 * (-7 + 3)]])
+    assert np.allclose(orc.decode(ids, codes, s, cen, D), want, rtol=0, atol=1e-15)
+
+
+# --------------------------------------------------------------------------
+# attention branches
+# --------------------------------------------------------------------------
+
+def _brute_full(q, ck, cv, hk, hv, tau):
+    """Pure-Python loops: decode every key/value element, then softmax."""
+    Tq, H, d = q.shape
+    T = len(hk["ids"])
+    r = ck["D"].shape[1]
+
+    def dec(c, h, t, i):
+        col = h * d + i
+        acc = 0.0
+        for j in range(r):
+            acc += float(c["D"][col, j]) * float(h_["codes"][t][j])
+        return float(c["centers"][h_["ids"][t], col]) + float(h_["scales"][t]) * acc
+
+    O = np.zeros((Tq, H, d))
+    L = np.zeros((H, Tq))
+    for h in range(H):
+        h_ = hk
+        K = [[dec(ck, h, t, i) for i in range(d)] for t in range(T)]
+        h_ = hv
+        V = [[dec(cv, h, t, i) for i in range(d)] for t in range(T)]
+        for a in range(Tq):
+            z = [tau * sum(float(q[a, h, i]) * K[t][i] for i in range(d)) for t in range(T)]
+            m = max(z)
+            p = [math.exp(zz - m) for zz in z]
+            l = sum(p)
+            for i in range(d):
+                O[a, h, i] = sum(p[t] * V[t][i] for t in range(T)) / l
+            L[h, a] = m + math.log(l)
+    return O, L
+
+
+def test_full_branch_matches_python_loops():
+    rng = np.random.default_rng(7)
+    H, d, r, C, T, Tq = 2, 4, 3, 3, 7, 3
+    ck, cv, hk, hv = _rand_codec(rng, H, d, r, C, T)
+    q = rng.standard_normal((Tq, H, d))
+    O, L = orc.attend_full(q, ck, cv, hk, hv, 0.7)
+    Ob, Lb = _brute_full(q, ck, cv, hk, hv, 0.7)
+    assert np.max(np.abs(O - Ob)) < 1e-12
+    assert np.max(np.abs(L - Lb)) < 1e-12
+
+
+def test_textbook_special_case_against_torch_sdpa():
+    """C = 1 zero center, D = I (r = J): K_hat = s * code, so decode-attention
+    is plain softmax attention; torch's SDPA (fp64, CPU) is the reference."""
+    rng = np.random.default_rng(3)
+    H, d, T, Tq = 3, 4, 11, 5
+    J = H * d
+    ck = {"centers": np.zeros((1, J)), "D": np.eye(J)}
+    cv = {"centers": np.zeros((1, J)), "D": np.eye(J)}
+    hk = {"ids": np.zeros(T, int), "codes": rng.integers(-7, 8, (T, J)), "scales": rng.uniform(0.1, 0.5, T)}
+    hv = {"ids": np.zeros(T, int), "codes": rng.integers(-7, 8, (T, J)), "scales": rng.uniform(0.1, 0.5, T)}
+    q = rng.standard_normal((Tq, H, d))
+    tau = 1 / math.sqrt(d)
+    O, L = orc.attend_full(q, ck, cv, hk, hv, tau)
+    K = (hk["scales"][:, None] * hk["codes"]).reshape(T, H, d)
+    V = (hv["scales"][:, None] * hv["codes"]).reshape(T, H, d)
+    qt = torch.tensor(q).permute(1, 0, 2)[None]
+    kt = torch.tensor(K).permute(1, 0, 2)[None]
+    vt = torch.tensor(V).permute(1, 0, 2)[None]
+    ref = torch.nn.functional.scaled_dot_product_attention(qt, kt, vt, scale=tau)[0].permute(1, 0, 2).numpy()
+    assert np.max(np.abs(O - ref)) < 1e-12
+    z = tau * torch.einsum("hqd,hkd->hqk", qt[0], kt[0])
+    assert np.max(np.abs(L - torch.logsumexp(z, dim=-1).numpy())) < 1e-12
+
+
+def test_all_keys_equal_gives_value_mean():
+    rng = np.random.default_rng(4)
+    H, d, r, C, T, Tq = 2, 3, 4, 5, 6, 2
+    ck, cv, hk, hv = _rand_codec(rng, H, d, r, C, T)
+    hk["ids"][:] = 2
+    hk["codes"][:] = hk["codes"][0]
+    hk["scales"][:] = 0.3
+    q = rng.standard_normal((Tq, H, d))
+    O, L = orc.attend_full(q, ck, cv, hk, hv, 1.0)
+    vh = orc.decode(hv["ids"], hv["codes"], hv["scales"], cv["centers"], cv["D"]).reshape(T, H, d)
+    assert np.max(np.abs(O - vh.mean(axis=0)[None])) < 1e-12
+    kh = orc.decode(hk["ids"][:1], hk["codes"][:1], hk["scales"][:1], ck["centers"], ck["D"]).reshape(H, d)
+    z = np.einsum("qhd,hd->hq", q, kh)
+    assert np.max(np.abs(L - (z + math.log(T)))) < 1e-12
+
+
+@pytest.mark.parametrize("tau", [1.0, 0.125])
+def test_low_dim_equals_full_decode(tau):
+    """Invariant: the mixed-dimensional branch is algebraically the
+    full-decode branch on the same compressed data."""
+    rng = np.random.default_rng(8)
+    H, d, r, C, T, Tq = 3, 8, 6, 5, 50, 7
+    ck, cv, hk, hv = _rand_codec(rng, H, d, r, C, T)
+    q = rng.standard_normal((Tq, H, d))
+    Of, Lf = orc.attend_full(q, ck, cv, hk, hv, tau)
+    Ol, Ll = orc.attend_low(q, ck, cv, hk, hv, tau)
+    assert np.max(np.abs(Of - Ol)) < 1e-12 * max(1.0, np.max(np.abs(Of)))
+    assert np.max(np.abs(Lf - Ll)) < 1e-11
+
+
+def test_lse_merge_of_split_history_equals_concatenation():
+    rng = np.random.default_rng(9)
+    H, d, T, Tq = 2, 5, 30, 6
+    q = rng.standard_normal((Tq, H, d))
+    k = rng.standard_normal((T, H, d))
+    v = rng.standard_normal((T, H, d))
+    full = orc.softmax_attention(q, k, v, 0.9)
+    for cuts in ([12], [0, 12], [7, 19, 30]):
+        bounds = [0] + cuts + [T]
+        parts = [orc.softmax_attention(q, k[a:b], v[a:b], 0.9) for a, b in zip(bounds[:-1], bounds[1:])]
+        O, L = orc.lse_merge(parts)
+        assert np.max(np.abs(O - full[0])) < 1e-12
+        assert np.max(np.abs(L - full[1])) < 1e-12
+
+
+def test_lse_merge_closed_forms():
+    rng = np.random.default_rng(10)
+    O1 = rng.standard_normal((4, 2, 3))
+    L1 = rng.standard_normal((2, 4))
+    O, L = orc.lse_merge([(O1, L1)])
+    assert np.array_equal(O, O1) or np.max(np.abs(O - O1)) < 1e-15
+    assert np.max(np.abs(L - L1)) < 1e-15
+    O2 = rng.standard_normal((4, 2, 3))
+    O, L = orc.lse_merge([(O1, L1), (O2, L1.copy())])
+    assert np.max(np.abs(O - (O1 + O2) / 2)) < 1e-15
+    assert np.max(np.abs(L - (L1 + math.log(2)))) < 1e-14
+    empty = (np.zeros_like(O1), np.full_like(L1, -np.inf))
+    O, L = orc.lse_merge([empty, (O1, L1), empty])
+    assert np.max(np.abs(O - O1)) < 1e-15 and np.max(np.abs(L - L1)) < 1e-15
+    O, L = orc.lse_merge([empty, empty])
+    assert np.all(O == 0) and np.all(np.isneginf(L))
+
+
+def test_attend_routing_equals_one_big_attention():
+    """attend() with any split point equals plain attention over the
+    explicitly decoded history concatenated with the current chunk."""
+    rng = np.random.default_rng(12)
+    H, d, r, C, T, Tq = 2, 8, 6, 4, 40, 9
+    ck, cv, hk, hv = _rand_codec(rng, H, d, r, C, T)
+    q = rng.standard_normal((Tq, H, d))
+    kc = rng.standard_normal((Tq, H, d))
+    vc = rng.standard_normal((Tq, H, d))
+    K = orc.decode(hk["ids"], hk["codes"], hk["scales"], ck["centers"], ck["D"]).reshape(T, H, d)
+    V = orc.decode(hv["ids"], hv["codes"], hv["scales"], cv["centers"], cv["D"]).reshape(T, H, d)
+    ref = orc.softmax_attention(q, np.concatenate([K, kc]), np.concatenate([V, vc]), 1 / math.sqrt(d))
+    for T_full in (0, 1, 17, T):
+        O, L = orc.attend(q, ck, cv, hk, hv, T_full, kc, vc)
+        assert np.max(np.abs(O - ref[0])) < 1e-12, T_full
+        assert np.max(np.abs(L - ref[1])) < 1e-12, T_full
+    # no current chunk, empty history -> O = 0, LSE = -inf
+    e = {"ids": hk["ids"][:0], "codes": hk["codes"][:0], "scales": hk["scales"][:0]}
+    O, L = orc.attend(q, ck, cv, e, e, 0)
+    assert np.all(O == 0) and np.all(np.isneginf(L))
+
+
+# --------------------------------------------------------------------------
+# tie accounting
+# --------------------------------------------------------------------------
+
+def test_tie_detectors():
+    # fp16 midpoint: 7 * (1 + 2^-11) lies halfway between 1 and 1 + 2^-10
+    y = np.array([[7 * (1 + 2 ** -11), 1.0], [7.0, 1.0]])
+    assert list(orc.scale_ties(y, "f16")) == [True, False]
+    x = np.array([[1.0, 0.0]])
+    cen = np.array([[0.0, 0.0], [2.0, 0.0], [5.0, 5.0]])
+    assert orc.argmin_ties(x, cen)[0]
+    assert not orc.argmin_ties(np.array([[0.2, 0.0]]), cen)[0]
+    E = np.eye(2)
+    ids = np.array([0])
+    yy = np.array([[2.5, 1.2]])
+    t = orc.rounding_ties(np.array([[2.5, 1.2]]), np.zeros((1, 2)), ids, E, yy, np.array([1.0]))
+    assert list(t[0]) == [True, False]
+
+
+# --------------------------------------------------------------------------
+# the pages' printed numbers: representation and arithmetic accounting
+# --------------------------------------------------------------------------
+
+def test_nominal_cr_matches_table5_table9():
+    g = _load("codec_ranks.json")
+    for row in g["rows"]:
+        cr = orc.nominal_coefficient_cr(row["heads"], row["head_dim"], row["rank"])
+        assert cr == row["budget"], row
+
+
+def test_table11_product_rule():
+    g = _load("fast_macs.json")
+    for row in g["rows"]:
+        prod = orc.overall_saving(row["historical_share"] / 100, row["history_saved"] / 100) * 100
+        assert abs(prod - row["all_saved"]) < 0.006, row
+
+
+def test_table6_head_layer_counts():
+    g = _load("head_dims.json")
+    for row in g["rows"]:
+        assert sum(row["counts"]) == row["layers"] * row["heads"], row
