@@ -1,0 +1,499 @@
+#!/usr/bin/env python
+"""Throughput of the NanoKV compressed-history hot path on B200.
+
+One step = one layer of the path on one batch of seeded synthetic input:
+encode the most recent history chunk (K and V) into the compressed cache,
+then attend the query chunk over the whole compressed history (routed full-
+or low-dim) plus the current chunk, LSE-merged.  Default workload: one layer,
+H=12, d=128 (J=1536), history 3 chunks = 14040 tokens, all full-dim, Tq=4680,
+64 centers, r=192, bf16 I/O, fp16 scales.
+
+    python bench.py [--gpus N] [--steps K] [--warmup W] [--impl ours|reference]
+
+Under torchrun (N > 1) every rank runs its own replica of the workload (no
+data-path collective: the path has no exchange step at one GPU per problem).
+"""
+from __future__ import annotations
+
+import argparse
+import json
+import math
+import os
+import statistics
+import subprocess
+import sys
+import tempfile
+import time
+
+import torch
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+sys.path.insert(0, ROOT)
+
+PEAKS_FALLBACK = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0}
+BAD_REASONS = ("hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown")
+
+
+def load_peaks():
+    p = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    if os.path.exists(p):
+        with open(p) as f:
+            d = json.load(f)
+        return d, "measured"
+    return PEAKS_FALLBACK, "fallback"
+
+
+def args_():
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=10)
+    ap.add_argument("--warmup", type=int, default=3)
+    ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
+    ap.add_argument("--workload", default="full")
+    ap.add_argument("--no-fast", action="store_true", help="skip the mixed-dim (Fast) side measurement")
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--path", type=int, default=0, help="kernel family: 0 auto, 1 CUDA-core, 2 tensor-core")
+    return ap.parse_args()
+
+
+# ---------------------------------------------------------------------------
+# clocks during the timed region
+# ---------------------------------------------------------------------------
+def _same_bus(bus_id, smi_bus: str) -> bool:
+    """torch reports the PCI bus as an int (or a string on some versions);
+    nvidia-smi as 'DDDDDDDD:BB:DD.F'."""
+    try:
+        smi = int(smi_bus.split(":")[1], 16)
+    except Exception:
+        return True
+    if isinstance(bus_id, int):
+        return bus_id == smi
+    try:
+        return int(str(bus_id).split(":")[1], 16) == smi
+    except Exception:
+        return True
+
+
+class ClockSampler:
+    FIELDS = ("index,pci.bus_id,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
+              "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
+              "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+
+    def __init__(self):
+        self.proc = None
+        self.path = None
+
+    def start(self):
+        try:
+            fd, self.path = tempfile.mkstemp(suffix=".csv")
+            os.close(fd)
+            self.proc = subprocess.Popen(
+                ["nvidia-smi", f"--query-gpu={self.FIELDS}", "--format=csv,noheader,nounits", "-lms", "200"],
+                stdout=open(self.path, "w"), stderr=subprocess.DEVNULL)
+        except Exception:
+            self.proc = None
+
+    def stop(self, bus_id: str | None):
+        if self.proc is None:
+            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": ["unsampled"]}
+        self.proc.terminate()
+        try:
+            self.proc.wait(timeout=5)
+        except Exception:
+            self.proc.kill()
+        rows = []
+        for line in open(self.path):
+            parts = [p.strip() for p in line.split(",")]
+            if len(parts) < 10:
+                continue
+            if bus_id is not None and not _same_bus(bus_id, parts[1]):
+                continue
+            rows.append(parts)
+        os.unlink(self.path)
+        if not rows:
+            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": ["unsampled"]}
+        sm = [float(r[2]) for r in rows if r[2].replace(".", "").isdigit()]
+        mx = max(float(r[3]) for r in rows if r[3].replace(".", "").isdigit())
+        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+        reasons = sorted({names[i] for r in rows for i in range(4) if "Active" in r[6 + i]})
+        load = [s for s in sm if s > 0.5 * mx] or sm
+        return {"sm_mhz": statistics.median(load) if load else None, "sm_max_mhz": mx,
+                "reasons": reasons, "samples": len(rows)}
+
+
+# ---------------------------------------------------------------------------
+# our arm
+# ---------------------------------------------------------------------------
+def setup(w, device):
+    import compressed_history_attention_b200 as nk
+    from synth.gen import make_problem
+    prob = make_problem(w, device=device)
+    ck = nk.Codec(w.H, w.d, prob["codec_k"]["centers"], prob["codec_k"]["D"], prob["codec_k"]["E"])
+    cv = nk.Codec(w.H, w.d, prob["codec_v"]["centers"], prob["codec_v"]["D"], prob["codec_v"]["E"])
+    hk, hv = nk.nanokv_encode(ck, cv, prob["hist_k"], prob["hist_v"])
+    n = min(w.chunk, w.T)
+    s = {
+        "prob": prob, "ck": ck, "cv": cv, "hk": hk, "hv": hv,
+        "xk": prob["hist_k"][w.T - n:].contiguous(), "xv": prob["hist_v"][w.T - n:].contiguous(),
+        "tail_k": hk.slice(w.T - n, w.T), "tail_v": hv.slice(w.T - n, w.T), "n_enc": n,
+        "out": torch.empty_like(prob["q"]),
+        "lse": torch.empty(w.H, w.Tq, dtype=torch.float32, device=device),
+    }
+    ws = nk.nanokv_attend_workspace(w.Tq, ck, cv, w.T, w.T_full, w.Tq)
+    s["ws"] = torch.empty(max(ws, 16), dtype=torch.uint8, device=device)
+    # free the raw history: only the compressed cache stays resident
+    prob["hist_k"] = prob["hist_v"] = None
+    return s
+
+
+def step_encode(s):
+    import compressed_history_attention_b200 as nk
+    nk.nanokv_encode(s["ck"], s["cv"], s["xk"], s["xv"], out_k=s["tail_k"], out_v=s["tail_v"])
+
+
+def step_attend(s, w):
+    import compressed_history_attention_b200 as nk
+    p = s["prob"]
+    nk.nanokv_attend(p["q"], s["ck"], s["cv"], s["hk"], s["hv"], w.T_full, p["k_cur"], p["v_cur"],
+                     out=s["out"], lse=s["lse"], workspace=s["ws"])
+
+
+def work_of(w, n_enc):
+    from compressed_history_attention_b200.accounting import attend_flops, encode_bytes, encode_flops
+    af = attend_flops(w.Tq, w.H, w.d, w.r, w.C, w.T_full, w.T_low, w.Tq)
+    ef = 2 * encode_flops(n_enc, w.J, w.r, w.C)
+    eb = 2 * encode_bytes(n_enc, w.J, w.r, 4 if w.fp32 else 2, 4 if w.fp32 else 2)
+    return af, ef, eb
+
+
+def timed_loop(s, w, steps, flush, with_encode=True):
+    """Per-step CUDA events (encode, attend) on the launching stream; the L2
+    flush between steps sits outside the events."""
+    ev = [[torch.cuda.Event(enable_timing=True) for _ in range(3)] for _ in range(steps)]
+    for i in range(steps):
+        flush.zero_()
+        ev[i][0].record()
+        if with_encode:
+            step_encode(s)
+        ev[i][1].record()
+        step_attend(s, w)
+        ev[i][2].record()
+    torch.cuda.synchronize()
+    enc = [e[0].elapsed_time(e[1]) for e in ev]
+    att = [e[1].elapsed_time(e[2]) for e in ev]
+    return enc, att
+
+
+def run_ours(a, rank, world, device):
+    import compressed_history_attention_b200 as nk
+    from synth.gen import WORKLOADS
+    import torch.distributed as dist
+
+    nk.nanokv_set_kernel_path(a.path)
+    peaks, peaks_kind = load_peaks()
+    w = WORKLOADS[a.workload]
+    s = setup(w, device)
+    af, ef, eb = work_of(w, s["n_enc"])
+    flush = torch.empty(256 * 1024 * 1024, dtype=torch.uint8, device=device)
+
+    for _ in range(a.warmup):
+        step_encode(s)
+        step_attend(s, w)
+    torch.cuda.synchronize()
+
+    bus = None
+    try:
+        bus = torch.cuda.get_device_properties(device).pci_bus_id
+    except Exception:
+        pass
+    clocks = None
+    for attempt in range(2):
+        nk.nanokv_timing_read()
+        nk.nanokv_timing_enable(True)
+        sampler = ClockSampler() if rank == 0 else None
+        if sampler:
+            sampler.start()
+        if world > 1:
+            dist.barrier()
+        torch.cuda.synchronize()
+        enc, att = timed_loop(s, w, a.steps, flush)
+        torch.cuda.synchronize()
+        if world > 1:
+            dist.barrier()
+        nk.nanokv_timing_enable(False)
+        kt = nk.nanokv_timing_read()
+        if sampler:
+            clocks = sampler.stop(bus)
+        bad = clocks and any(r in BAD_REASONS for r in clocks.get("reasons", []))
+        if not bad:
+            break
+    nk.nanokv_check()
+
+    step_ms = (sum(enc) + sum(att)) / a.steps
+    enc_ms, att_ms = sum(enc) / a.steps, sum(att) / a.steps
+    if world > 1:
+        t = torch.tensor([step_ms, enc_ms, att_ms], device=device)
+        dist.all_reduce(t, op=dist.ReduceOp.MAX)
+        step_ms, enc_ms, att_ms = t.tolist()
+
+    flops = af["total"] + ef
+    value = world * flops / (step_ms * 1e-3) / 1e12
+    launches = sum(n for _, n in kt.values())
+
+    # dominant kernel: the one with the largest share of the timed region
+    dom = max(kt.items(), key=lambda kv: kv[1][0])
+    dom_name, (dom_ms, dom_n) = dom
+    dom_work = {"attend_full": af["full"], "attend_low": af["low"], "attend_dense": af["current"],
+                "encode": ef / 2, "lse_merge": None}[dom_name]
+    dom_avg_ms = dom_ms / max(dom_n, 1)
+    peak_tf = peaks["bf16_tflops"]
+    if dom_name.startswith("attend"):
+        per_launch = dom_work / (dom_n / a.steps)
+        achieved = per_launch / (dom_avg_ms * 1e-3) / 1e12
+        roof = {"kernel": dom_name, "bound": "tensor", "achieved": round(achieved, 2), "peak": peak_tf,
+                "unit": "TFLOP/s", "frac": round(achieved / peak_tf, 4), "traffic": None,
+                "peak_kind": f"bf16 burst, {peaks_kind}", "avg_launch_ms": round(dom_avg_ms, 4)}
+    else:
+        per_launch = eb / 2 if dom_name == "encode" else None
+        achieved = per_launch / (dom_avg_ms * 1e-3) / 1e9 if per_launch else None
+        roof = {"kernel": dom_name, "bound": "hbm", "achieved": achieved, "peak": peaks["hbm_gbs"],
+                "unit": "GB/s", "frac": (achieved / peaks["hbm_gbs"]) if achieved else None,
+                "traffic": None, "peak_kind": peaks_kind, "avg_launch_ms": round(dom_avg_ms, 4)}
+
+    kernels = {k: {"ms_total": round(v[0], 4), "launches": v[1],
+                   "share": round(v[0] / max(1e-9, sum(x[0] for x in kt.values())), 4)}
+               for k, v in kt.items() if v[1]}
+    attend_tf = af["total"] / (att_ms * 1e-3) / 1e12
+    hist_tf = (af["full"] + af["low"]) / (att_ms * 1e-3) / 1e12
+    enc_gbs = eb / (enc_ms * 1e-3) / 1e9
+
+    e2e = run_e2e(s, w, a, device, flops, world)
+    fast = None if a.no_fast else run_fast(a, device, peaks)
+    cpu = None
+    if rank == 0 and world == 1 and not a.no_cpu_baseline:
+        cpu = cpu_baseline(w, s, budget_s=12.0)
+
+    line = {
+        "metric": "compressed-history attention + encode step throughput (algorithmic TFLOP/s)",
+        "value": round(value, 3), "unit": "TFLOP/s", "n_gpus": world, "steps": a.steps,
+        "warmup": a.warmup, "ms_per_step": round(step_ms, 4), "higher_is_better": True,
+        "scaling": "weak", "vs_baseline": None, "dtype": "bf16" if not w.fp32 else "f32",
+        "data": "synthetic (seeded clustered low-rank generator; random codec params)",
+        "config": {"workload": w.describe(), "H": w.H, "d": w.d, "T": w.T, "T_full": w.T_full,
+                   "T_low": w.T_low, "Tq": w.Tq, "T_cur": w.Tq, "C": w.C, "r": w.r,
+                   "encode_tokens": s["n_enc"], "l2": "flushed between steps (256 MiB write outside the step events)",
+                   "parallelism": f"replicas x{world}"},
+        "attend": {"ms": round(att_ms, 4), "tflops": round(attend_tf, 3),
+                   "history_tflops": round(hist_tf, 3), "frac_bf16_peak": round(attend_tf / peak_tf, 4)},
+        "encode": {"ms": round(enc_ms, 4), "gbs": round(enc_gbs, 2),
+                   "frac_hbm": round(enc_gbs / peaks["hbm_gbs"], 4)},
+        "kernels": kernels,
+        "clocks": clocks, "e2e": e2e, "gpu_launches": launches, "roofline": roof,
+        "cpu_baseline": cpu, "fast": fast,
+    }
+    return line
+
+
+def run_e2e(s, w, a, device, flops, world):
+    """The same step through the public API from pinned host buffers: H2D of
+    the step's inputs and D2H of its output inside the timed region."""
+    import compressed_history_attention_b200 as nk
+    p = s["prob"]
+    host = {k: v.cpu().pin_memory() for k, v in (("q", p["q"]), ("k_cur", p["k_cur"]),
+                                                 ("v_cur", p["v_cur"]), ("xk", s["xk"]), ("xv", s["xv"]))}
+    dev = {k: torch.empty_like(v, device=device) for k, v in host.items()}
+    out_h = torch.empty(s["out"].shape, dtype=s["out"].dtype).pin_memory()
+    lse_h = torch.empty(s["lse"].shape, dtype=torch.float32).pin_memory()
+    bi = sum(t.numel() * t.element_size() for t in host.values())
+    bo = out_h.numel() * out_h.element_size() + lse_h.numel() * 4
+
+    def one():
+        for k in host:
+            dev[k].copy_(host[k], non_blocking=True)
+        nk.nanokv_encode(s["ck"], s["cv"], dev["xk"], dev["xv"], out_k=s["tail_k"], out_v=s["tail_v"])
+        nk.nanokv_attend(dev["q"], s["ck"], s["cv"], s["hk"], s["hv"], w.T_full, dev["k_cur"], dev["v_cur"],
+                         out=s["out"], lse=s["lse"], workspace=s["ws"])
+        out_h.copy_(s["out"], non_blocking=True)
+        lse_h.copy_(s["lse"], non_blocking=True)
+
+    for _ in range(2):
+        one()
+    torch.cuda.synchronize()
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    e0.record()
+    for _ in range(a.steps):
+        one()
+    e1.record()
+    torch.cuda.synchronize()
+    ms = e0.elapsed_time(e1) / a.steps
+    if world > 1:
+        import torch.distributed as dist
+        t = torch.tensor([ms], device=device)
+        dist.all_reduce(t, op=dist.ReduceOp.MAX)
+        ms = t.item()
+    return {"value": round(world * flops / (ms * 1e-3) / 1e12, 3), "unit": "TFLOP/s",
+            "ms_per_step": round(ms, 4), "h2d_bytes_per_step": bi, "d2h_bytes_per_step": bo}
+
+
+def run_fast(a, device, peaks):
+    """Side measurement of the mixed-dimensional (Fast) attend on the mixed
+    workload (same shapes, most recent chunk full-dim, 9360 tokens low-dim)."""
+    from synth.gen import WORKLOADS
+    from compressed_history_attention_b200.accounting import attend_flops
+    w = WORKLOADS["mixed"]
+    s = setup(w, device)
+    for _ in range(2):
+        step_attend(s, w)
+    flush = torch.empty(256 * 1024 * 1024, dtype=torch.uint8, device=device)
+    n = max(3, a.steps // 2)
+    _, att = timed_loop(s, w, n, flush, with_encode=False)
+    ms = sum(att) / n
+    af = attend_flops(w.Tq, w.H, w.d, w.r, w.C, w.T_full, w.T_low, w.Tq)
+    tf = af["total"] / (ms * 1e-3) / 1e12
+    del s
+    torch.cuda.empty_cache()
+    return {"workload": w.describe(), "attend_ms": round(ms, 4), "tflops": round(tf, 3),
+            "frac_bf16_peak": round(tf / peaks["bf16_tflops"], 4), "iters": n}
+
+
+# ---------------------------------------------------------------------------
+# CPU baseline / reference arm: the fp64 oracle as it stands on host cores
+# ---------------------------------------------------------------------------
+def _threads_used():
+    try:
+        from threadpoolctl import threadpool_info
+        info = threadpool_info()
+        if info:
+            return max(i.get("num_threads", 1) for i in info)
+    except Exception:
+        pass
+    return len(os.sched_getaffinity(0))
+
+
+def oracle_data(w, codec_k, codec_v, xk, xv, hk, hv, q, k_cur, v_cur):
+    """fp64 copies of one workload's inputs for the oracle (host memory)."""
+    from oracle import nanokv_oracle as orc
+    return {"ck": {k: orc.f64(codec_k[k]) for k in ("centers", "D", "E")},
+            "cv": {k: orc.f64(codec_v[k]) for k in ("centers", "D", "E")},
+            "xk": orc.f64(xk), "xv": orc.f64(xv), "hk": hk, "hv": hv,
+            "q": orc.f64(q), "kc": orc.f64(k_cur), "vc": orc.f64(v_cur)}
+
+
+def oracle_hist(h):
+    import numpy as np
+    from oracle import nanokv_oracle as orc
+    return {"ids": h.ids.cpu().numpy().astype(np.int64), "codes": orc.unpack_codes(h.codes.cpu().numpy()),
+            "scales": orc.f64(h.scales)}
+
+
+def oracle_sample(w, D, n_rows, n_enc, seed=0):
+    """Runs the oracle on a bounded sample of one step: encode n_enc tokens of
+    K and V and attend n_rows query rows over the whole history plus the
+    current chunk.  Returns (seconds, algorithmic flops of the sample)."""
+    import numpy as np
+    from oracle import nanokv_oracle as orc
+    from compressed_history_attention_b200.accounting import attend_flops, encode_flops
+    sd = "f32" if w.fp32 else "f16"
+    rng = np.random.default_rng(seed)
+    rows = np.sort(rng.choice(w.Tq, min(n_rows, w.Tq), replace=False))
+    n_enc = min(n_enc, D["xk"].shape[0])
+    t0 = time.perf_counter()
+    orc.encode(D["xk"][:n_enc], D["ck"]["centers"], D["ck"]["E"], sd)
+    orc.encode(D["xv"][:n_enc], D["cv"]["centers"], D["cv"]["E"], sd)
+    orc.attend(D["q"][rows], D["ck"], D["cv"], D["hk"], D["hv"], w.T_full, D["kc"], D["vc"])
+    dt = time.perf_counter() - t0
+    fl = (2 * encode_flops(n_enc, w.J, w.r, w.C)
+          + attend_flops(len(rows), w.H, w.d, w.r, w.C, w.T_full, w.T_low, w.Tq)["total"])
+    return dt, fl, len(rows), n_enc
+
+
+def _calibrated(w, D, budget_s, rows0, enc0):
+    dt, _, _, _ = oracle_sample(w, D, rows0, enc0)
+    scale = max(1.0, min(64.0, budget_s / max(dt, 1e-3)))
+    return int(rows0 * scale), int(enc0 * scale)
+
+
+def cpu_baseline(w, s, budget_s=12.0):
+    """The oracle as it stands, timed on this host's cores on a bounded sample
+    of the same workload (the GPU's inputs and compressed history)."""
+    p = s["prob"]
+    D = oracle_data(w, p["codec_k"], p["codec_v"], s["xk"], s["xv"], oracle_hist(s["hk"]),
+                    oracle_hist(s["hv"]), p["q"], p["k_cur"], p["v_cur"])
+    n_rows, n_enc = _calibrated(w, D, budget_s, 16, 64)
+    dt, fl, n_rows, n_enc = oracle_sample(w, D, n_rows, n_enc, seed=1)
+    return {"value": round(fl / dt / 1e12, 6), "unit": "TFLOP/s", "cores": _threads_used(), "kind": "oracle",
+            "sample": f"encode {n_enc} K + {n_enc} V tokens and attend {n_rows} of {w.Tq} query rows "
+                      f"over the full history + current chunk; {dt:.1f} s fp64 numpy"}
+
+
+def run_reference(a, rank, world):
+    """The oracle as it stands on this host's cores, on the same workload (its
+    own encode of the generated history), each step a bounded sample."""
+    if rank != 0:
+        return None
+    import numpy as np
+    from oracle import nanokv_oracle as orc
+    from synth.gen import WORKLOADS, make_problem
+    w = WORKLOADS[a.workload]
+    p = make_problem(w, device="cpu")
+    sd = "f32" if w.fp32 else "f16"
+    hist = []
+    for x, c in ((p["hist_k"], p["codec_k"]), (p["hist_v"], p["codec_v"])):
+        e = orc.encode(orc.f64(x), orc.f64(c["centers"]), orc.f64(c["E"]), sd)
+        hist.append({"ids": e["ids"], "codes": e["codes"], "scales": e["scales"]})
+    n = min(w.chunk, w.T)
+    D = oracle_data(w, p["codec_k"], p["codec_v"], p["hist_k"][w.T - n:], p["hist_v"][w.T - n:],
+                    hist[0], hist[1], p["q"], p["k_cur"], p["v_cur"])
+    budget = 150.0 / max(1, a.steps + a.warmup)
+    n_rows, n_enc = _calibrated(w, D, budget, 8, 32)
+    for _ in range(a.warmup):
+        oracle_sample(w, D, n_rows, n_enc)
+    tot_t, tot_f = 0.0, 0
+    for i in range(a.steps):
+        dt, fl, n_rows, n_enc = oracle_sample(w, D, n_rows, n_enc, seed=i)
+        tot_t += dt
+        tot_f += fl
+    v = tot_f / tot_t / 1e12
+    sample = (f"per step: encode {n_enc} K + {n_enc} V tokens and attend {n_rows} of {w.Tq} query rows "
+              "over the full history + current chunk (fp64 numpy oracle)")
+    return {
+        "impl": "reference",
+        "metric": "compressed-history attention + encode step throughput (algorithmic TFLOP/s)",
+        "value": round(v, 6), "unit": "TFLOP/s", "n_gpus": world, "steps": a.steps, "warmup": a.warmup,
+        "ms_per_step": round(1e3 * tot_t / a.steps, 2), "higher_is_better": True, "scaling": "weak",
+        "vs_baseline": None, "dtype": "f64", "data": "synthetic",
+        "config": {"workload": w.describe(), "H": w.H, "d": w.d, "T": w.T, "T_full": w.T_full,
+                   "T_low": w.T_low, "Tq": w.Tq, "T_cur": w.Tq, "C": w.C, "r": w.r},
+        "cpu_baseline": {"value": round(v, 6), "unit": "TFLOP/s", "cores": _threads_used(), "kind": "oracle",
+                         "sample": sample},
+        "e2e": {"value": round(v, 6), "unit": "TFLOP/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
+    }
+
+
+def main():
+    a = args_()
+    rank = int(os.environ.get("RANK", 0))
+    world = int(os.environ.get("WORLD_SIZE", 1))
+    local = int(os.environ.get("LOCAL_RANK", 0))
+    if a.impl == "reference":
+        line = run_reference(a, rank, world)
+        if line is not None:
+            print(json.dumps(line), flush=True)
+        return
+    import datetime
+    torch.cuda.set_device(local)
+    device = torch.device("cuda", local)
+    if world > 1:
+        import torch.distributed as dist
+        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120), device_id=device)
+    line = run_ours(a, rank, world, device)
+    if rank == 0:
+        print(json.dumps(line), flush=True)
+    if world > 1:
+        import torch.distributed as dist
+        dist.barrier()
+        dist.destroy_process_group()
+
+
+if __name__ == "__main__":
+    main()

@@ -1,0 +1,11 @@
+"""NanoKV compressed-history attention for B200 (sm_100a).
+
+The work runs in libnanokv.so (hand-written CUDA kernels behind a C ABI, see
+include/nanokv.h); this package is its thin Python binding plus the build
+script and the arithmetic accounting used by the benchmark.
+"""
+from ._lib import (  # noqa: F401
+    Codec, Hist, NanoKVError, alloc_hist, lib, nanokv_attend, nanokv_attend_workspace,
+    nanokv_check, nanokv_encode, nanokv_lse_merge, nanokv_set_kernel_path, nanokv_timing_enable,
+    nanokv_timing_read, nanokv_version,
+)

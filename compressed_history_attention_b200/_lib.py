@@ -1,0 +1,271 @@
+"""ctypes binding of libnanokv.so (argument marshalling only).
+
+Every computation runs in the library's CUDA kernels; this module only turns
+torch tensors into device pointers, sizes and the current CUDA stream, and
+allocates outputs with torch.  There is no CPU fallback: if the shared library
+is missing or a call fails, it raises.
+"""
+from __future__ import annotations
+
+import ctypes
+import dataclasses
+import math
+import os
+
+import torch
+
+_PKG = os.path.dirname(os.path.abspath(__file__))
+LIB_PATH = os.path.join(_PKG, "libnanokv.so")
+
+F32, F16, BF16 = 0, 1, 2
+OK, ERR_INVALID, ERR_UNSUPPORTED, ERR_CUDA, ERR_TIMEOUT = 0, -1, -2, -3, -4
+
+SYMBOLS = ("nanokv_encode", "nanokv_attend", "nanokv_attend_workspace", "nanokv_lse_merge",
+           "nanokv_set_kernel_path", "nanokv_check", "nanokv_last_error", "nanokv_version",
+           "nanokv_timing_enable", "nanokv_timing_read")
+
+# kernel identities of the diagnostics (nanokv_kernel_id)
+KERNELS = {0: "encode", 1: "attend_full", 2: "attend_low", 3: "attend_dense", 4: "lse_merge"}
+K_COUNT = 8
+
+
+class NanoKVError(RuntimeError):
+    def __init__(self, status: int, msg: str):
+        super().__init__(f"nanokv status {status}: {msg}")
+        self.status = status
+
+
+class _Codec(ctypes.Structure):
+    _fields_ = [("H", ctypes.c_int32), ("d", ctypes.c_int32), ("r", ctypes.c_int32),
+                ("C", ctypes.c_int32), ("param_dtype", ctypes.c_int32),
+                ("scale_dtype", ctypes.c_int32), ("centers", ctypes.c_void_p),
+                ("D", ctypes.c_void_p), ("E", ctypes.c_void_p)]
+
+
+class _Hist(ctypes.Structure):
+    _fields_ = [("ids", ctypes.c_void_p), ("codes", ctypes.c_void_p), ("scales", ctypes.c_void_p)]
+
+
+_lib = None
+
+
+def lib() -> ctypes.CDLL:
+    """Loads libnanokv.so from the package directory (build it with
+    `python -m compressed_history_attention_b200.build`)."""
+    global _lib
+    if _lib is not None:
+        return _lib
+    if not os.path.exists(LIB_PATH):
+        raise ImportError(f"libnanokv.so not built ({LIB_PATH}); run "
+                          "`python -m compressed_history_attention_b200.build`")
+    L = ctypes.CDLL(LIB_PATH)
+    vp, i32, i64, f32, sz = ctypes.c_void_p, ctypes.c_int32, ctypes.c_int64, ctypes.c_float, ctypes.c_size_t
+    P = ctypes.POINTER
+    L.nanokv_encode.argtypes = [P(_Codec), P(_Codec), vp, vp, i32, i64, vp, vp, vp, vp, vp, vp, vp]
+    L.nanokv_encode.restype = ctypes.c_int
+    L.nanokv_attend.argtypes = [vp, i32, i64, P(_Codec), P(_Codec), P(_Hist), P(_Hist), i64, i64,
+                                vp, vp, i64, f32, vp, vp, vp, sz, vp]
+    L.nanokv_attend.restype = ctypes.c_int
+    L.nanokv_attend_workspace.argtypes = [i64, P(_Codec), P(_Codec), i64, i64, i64]
+    L.nanokv_attend_workspace.restype = sz
+    L.nanokv_lse_merge.argtypes = [i32, P(vp), P(vp), i64, i32, i32, vp, i32, vp, vp]
+    L.nanokv_lse_merge.restype = ctypes.c_int
+    L.nanokv_set_kernel_path.argtypes = [i32]
+    L.nanokv_set_kernel_path.restype = ctypes.c_int
+    L.nanokv_check.argtypes = [vp]
+    L.nanokv_check.restype = ctypes.c_int
+    L.nanokv_last_error.restype = ctypes.c_char_p
+    L.nanokv_version.restype = ctypes.c_char_p
+    L.nanokv_timing_enable.argtypes = [i32]
+    L.nanokv_timing_enable.restype = ctypes.c_int
+    L.nanokv_timing_read.argtypes = [vp, vp]
+    L.nanokv_timing_read.restype = ctypes.c_int
+    _lib = L
+    return L
+
+
+def _raise(status: int):
+    if status != OK:
+        raise NanoKVError(status, lib().nanokv_last_error().decode())
+
+
+def _ptr(t):
+    return None if t is None else ctypes.c_void_p(t.data_ptr())
+
+
+def _stream(device=None):
+    return ctypes.c_void_p(torch.cuda.current_stream(device).cuda_stream)
+
+
+@dataclasses.dataclass
+class Codec:
+    """One K or V codec: centers [C, J], decoder D [J, r], encoder E [r, J]
+    (E may be None for attention-only use).  fp32 tensors select the fp32 mode
+    (fp32 scales), bf16 tensors the bf16 mode (fp16 scales)."""
+    H: int
+    d: int
+    centers: torch.Tensor
+    D: torch.Tensor
+    E: torch.Tensor | None = None
+
+    @property
+    def r(self) -> int:
+        return self.D.shape[1]
+
+    @property
+    def C(self) -> int:
+        return self.centers.shape[0]
+
+    @property
+    def fp32(self) -> bool:
+        return self.centers.dtype == torch.float32
+
+    @property
+    def scale_dtype(self) -> torch.dtype:
+        return torch.float32 if self.fp32 else torch.float16
+
+    def struct(self) -> _Codec:
+        pd = F32 if self.fp32 else BF16
+        sd = F32 if self.fp32 else F16
+        return _Codec(self.H, self.d, self.r, self.C, pd, sd, self.centers.data_ptr(),
+                      self.D.data_ptr(), self.E.data_ptr() if self.E is not None else None)
+
+
+@dataclasses.dataclass
+class Hist:
+    """Compressed history of one branch: ids [T] u8, codes [T, r/2] u8,
+    scales [T] (fp16 or fp32)."""
+    ids: torch.Tensor
+    codes: torch.Tensor
+    scales: torch.Tensor
+
+    def __len__(self):
+        return self.ids.shape[0]
+
+    def struct(self) -> _Hist:
+        return _Hist(self.ids.data_ptr(), self.codes.data_ptr(), self.scales.data_ptr())
+
+    def slice(self, lo: int, hi: int) -> "Hist":
+        return Hist(self.ids[lo:hi], self.codes[lo:hi], self.scales[lo:hi])
+
+
+def _dt(t: torch.Tensor) -> int:
+    return {torch.float32: F32, torch.bfloat16: BF16, torch.float16: F16}[t.dtype]
+
+
+def alloc_hist(codec: Codec, T: int, device) -> Hist:
+    return Hist(torch.empty(T, dtype=torch.uint8, device=device),
+                torch.empty(T, codec.r // 2, dtype=torch.uint8, device=device),
+                torch.empty(T, dtype=codec.scale_dtype, device=device))
+
+
+def nanokv_encode(ck: Codec | None, cv: Codec | None, k: torch.Tensor | None, v: torch.Tensor | None,
+                  out_k: Hist | None = None, out_v: Hist | None = None):
+    """Encode K and V tokens [T, J]; returns (Hist_k, Hist_v) (None for a
+    skipped branch).  Outputs may be preallocated (e.g. views into a cache)."""
+    x0 = k if k is not None else v
+    T = x0.shape[0]
+    dev = x0.device
+    if ck is not None and out_k is None:
+        out_k = alloc_hist(ck, T, dev)
+    if cv is not None and out_v is None:
+        out_v = alloc_hist(cv, T, dev)
+    sk = ck.struct() if ck is not None else None
+    sv = cv.struct() if cv is not None else None
+    st = lib().nanokv_encode(
+        ctypes.byref(sk) if sk is not None else None, ctypes.byref(sv) if sv is not None else None,
+        _ptr(k), _ptr(v), _dt(x0), T,
+        _ptr(out_k.ids if out_k else None), _ptr(out_k.codes if out_k else None),
+        _ptr(out_k.scales if out_k else None),
+        _ptr(out_v.ids if out_v else None), _ptr(out_v.codes if out_v else None),
+        _ptr(out_v.scales if out_v else None), _stream(dev))
+    _raise(st)
+    return out_k, out_v
+
+
+def nanokv_attend_workspace(Tq: int, ck: Codec, cv: Codec, T: int, T_full: int, T_cur: int) -> int:
+    sk, sv = ck.struct(), cv.struct()
+    return int(lib().nanokv_attend_workspace(Tq, ctypes.byref(sk), ctypes.byref(sv), T, T_full, T_cur))
+
+
+def nanokv_attend(q: torch.Tensor, ck: Codec, cv: Codec, hk: Hist | None, hv: Hist | None,
+                  T_full: int, k_cur: torch.Tensor | None = None, v_cur: torch.Tensor | None = None,
+                  softmax_scale: float | None = None, out: torch.Tensor | None = None,
+                  lse: torch.Tensor | bool | None = True, workspace: torch.Tensor | None = None):
+    """Attention of q [Tq, H, d] over compressed history (T_full most recent
+    tokens full-dim, the rest low-dim) plus the current chunk k_cur/v_cur
+    [T_cur, H, d].  Returns (out [Tq, H, d], lse [H, Tq] fp32 or None)."""
+    Tq, H, d = q.shape
+    T = len(hk) if hk is not None else 0
+    T_cur = k_cur.shape[0] if k_cur is not None else 0
+    if softmax_scale is None:
+        softmax_scale = 1.0 / math.sqrt(d)
+    dev = q.device
+    if out is None:
+        out = torch.empty_like(q)
+    if lse is True:
+        lse = torch.empty(H, Tq, dtype=torch.float32, device=dev)
+    elif lse is False:
+        lse = None
+    need = nanokv_attend_workspace(Tq, ck, cv, T, T_full, T_cur)
+    if workspace is None or workspace.numel() * workspace.element_size() < need:
+        workspace = torch.empty(max(need, 16), dtype=torch.uint8, device=dev)
+    sk, sv = ck.struct(), cv.struct()
+    shk = hk.struct() if hk is not None and T else None
+    shv = hv.struct() if hv is not None and T else None
+    st = lib().nanokv_attend(
+        _ptr(q), _dt(q), Tq, ctypes.byref(sk), ctypes.byref(sv),
+        ctypes.byref(shk) if shk else None, ctypes.byref(shv) if shv else None, T, T_full,
+        _ptr(k_cur), _ptr(v_cur), T_cur, ctypes.c_float(softmax_scale), _ptr(out), _ptr(lse),
+        _ptr(workspace), workspace.numel() * workspace.element_size(), _stream(dev))
+    _raise(st)
+    return out, lse
+
+
+def nanokv_lse_merge(o_parts, lse_parts, out_dtype=torch.bfloat16, out=None, lse=True):
+    """LSE-merge fp32 partials O_i [Tq, H, d], LSE_i [H, Tq]."""
+    n = len(o_parts)
+    Tq, H, d = o_parts[0].shape
+    dev = o_parts[0].device
+    if out is None:
+        out = torch.empty(Tq, H, d, dtype=out_dtype, device=dev)
+    if lse is True:
+        lse = torch.empty(H, Tq, dtype=torch.float32, device=dev)
+    elif lse is False:
+        lse = None
+    arr = ctypes.c_void_p * max(n, 1)
+    op = arr(*[p.data_ptr() for p in o_parts])
+    lp = arr(*[p.data_ptr() for p in lse_parts])
+    st = lib().nanokv_lse_merge(n, op, lp, Tq, H, d, _ptr(out), _dt(out), _ptr(lse), _stream(dev))
+    _raise(st)
+    return out, lse
+
+
+def nanokv_set_kernel_path(path: int) -> int:
+    """0 = automatic, 1 = fp32 CUDA-core kernels only, 2 = tensor-core only."""
+    prev = lib().nanokv_set_kernel_path(path)
+    if prev < 0:
+        raise ValueError(path)
+    return prev
+
+
+def nanokv_check(device=None) -> None:
+    _raise(lib().nanokv_check(_stream(device)))
+
+
+def nanokv_version() -> str:
+    return lib().nanokv_version().decode()
+
+
+def nanokv_timing_enable(on: bool) -> bool:
+    """Per-kernel CUDA-event timing of every later launch (diagnostics)."""
+    return bool(lib().nanokv_timing_enable(1 if on else 0))
+
+
+def nanokv_timing_read() -> dict:
+    """{kernel: (total_ms, launches)} since the last read; waits for the
+    recorded events."""
+    ms = (ctypes.c_double * K_COUNT)()
+    n = (ctypes.c_int64 * K_COUNT)()
+    _raise(lib().nanokv_timing_read(ms, n))
+    return {name: (ms[k], n[k]) for k, name in KERNELS.items()}

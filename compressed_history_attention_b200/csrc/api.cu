@@ -1,0 +1,398 @@
+// C ABI of libnanokv: argument validation, workspace layout, kernel selection.
+#include "../../include/nanokv.h"
+#include "common.cuh"
+#include "tc.cuh"
+
+#include <stdarg.h>
+#include <stdio.h>
+#include <string.h>
+
+#include <atomic>
+#include <mutex>
+#include <string>
+#include <vector>
+
+namespace nanokv {
+
+// device error word (bounded waits that expired, bounds violations); read and
+// cleared by nanokv_check
+__device__ unsigned g_error_word = 0;
+
+static thread_local std::string t_last_error;
+static std::atomic<int> g_kernel_path{0};
+
+static int fail(int status, const char *fmt, ...) {
+  char buf[512];
+  va_list ap;
+  va_start(ap, fmt);
+  vsnprintf(buf, sizeof(buf), fmt, ap);
+  va_end(ap);
+  t_last_error = buf;
+  return status;
+}
+
+static int cuda_status(cudaError_t e, const char *what) {
+  if (e == cudaSuccess) return NANOKV_OK;
+  return fail(NANOKV_ERR_CUDA, "%s: %s", what, cudaGetErrorString(e));
+}
+
+// ---------------------------------------------------------------------------
+// diagnostics: launch counts (always) and optional per-kernel event timing
+// ---------------------------------------------------------------------------
+static std::atomic<int> g_timing{0};
+static std::atomic<int64_t> g_launches[NANOKV_K_COUNT];
+struct TimingRec {
+  int kid;
+  cudaEvent_t a, b;
+};
+static std::mutex g_tmu;
+static std::vector<TimingRec> g_recs;
+static std::vector<cudaEvent_t> g_event_pool;
+
+static cudaEvent_t event_get() {
+  std::lock_guard<std::mutex> lk(g_tmu);
+  if (!g_event_pool.empty()) {
+    cudaEvent_t e = g_event_pool.back();
+    g_event_pool.pop_back();
+    return e;
+  }
+  cudaEvent_t e = nullptr;
+  cudaEventCreate(&e);
+  return e;
+}
+
+// runs a launcher that issues `nk` kernels on `st`, counting and (optionally)
+// timing them as kernel `kid`
+template <class F>
+static cudaError_t timed(int kid, int nk, cudaStream_t st, F &&launch) {
+  g_launches[kid] += nk;
+  if (!g_timing.load()) return launch();
+  cudaEvent_t a = event_get(), b = event_get();
+  cudaEventRecord(a, st);
+  cudaError_t e = launch();
+  cudaEventRecord(b, st);
+  std::lock_guard<std::mutex> lk(g_tmu);
+  g_recs.push_back({kid, a, b});
+  return e;
+}
+
+static bool aligned16(const void *p) { return ((uintptr_t)p & 15u) == 0; }
+
+unsigned *error_word_ptr() {
+  // the device address of g_error_word on the current device
+  static thread_local int cached_dev = -1;
+  static thread_local unsigned *cached = nullptr;
+  int dev = 0;
+  cudaGetDevice(&dev);
+  if (dev != cached_dev) {
+    void *p = nullptr;
+    if (cudaGetSymbolAddress(&p, g_error_word) != cudaSuccess) return nullptr;
+    cached = (unsigned *)p;
+    cached_dev = dev;
+  }
+  return cached;
+}
+
+// validates one codec; fills the internal bundle
+static int check_codec(const nanokv_codec *c, const char *name, bool need_E, Codec *out) {
+  if (!c) return fail(NANOKV_ERR_INVALID, "%s: codec is NULL", name);
+  if (c->H < 1 || c->H > 256) return fail(NANOKV_ERR_INVALID, "%s: H=%d out of range [1,256]", name, c->H);
+  if (!(c->d == 16 || c->d == 32 || c->d == 64 || c->d == 128))
+    return fail(NANOKV_ERR_UNSUPPORTED, "%s: d=%d (supported: 16, 32, 64, 128)", name, c->d);
+  if (c->r < 2 || c->r > 512 || (c->r & 1))
+    return fail(NANOKV_ERR_INVALID, "%s: r=%d must be even and in [2,512]", name, c->r);
+  if (c->C < 1 || c->C > 256) return fail(NANOKV_ERR_INVALID, "%s: C=%d out of range [1,256]", name, c->C);
+  int prec;
+  if (c->param_dtype == NANOKV_F32 && c->scale_dtype == NANOKV_F32) prec = PREC_F32;
+  else if (c->param_dtype == NANOKV_BF16 && c->scale_dtype == NANOKV_F16) prec = PREC_BF16;
+  else
+    return fail(NANOKV_ERR_UNSUPPORTED,
+                "%s: param/scale dtype pair (%d,%d) unsupported (F32/F32 or BF16/F16)", name,
+                c->param_dtype, c->scale_dtype);
+  if (!c->centers || !c->D || (need_E && !c->E))
+    return fail(NANOKV_ERR_INVALID, "%s: NULL parameter pointer", name);
+  if (!aligned16(c->centers) || !aligned16(c->D) || (c->E && !aligned16(c->E)))
+    return fail(NANOKV_ERR_INVALID, "%s: parameter pointers must be 16-byte aligned", name);
+  *out = Codec{c->H, c->d, c->r, c->C, prec, c->centers, c->D, c->E};
+  return NANOKV_OK;
+}
+
+static int io_prec(int32_t dt) {
+  if (dt == NANOKV_F32) return PREC_F32;
+  if (dt == NANOKV_BF16) return PREC_BF16;
+  return -1;
+}
+
+// workspace carve-up (every region 256-byte aligned)
+struct WsLayout {
+  size_t off_O[3], off_L[3], off_qred, off_qc, total;
+};
+
+static size_t al256(size_t x) { return (x + 255) & ~(size_t)255; }
+
+static WsLayout ws_layout(int64_t Tq, const Codec &ck, int64_t T_low, int64_t T_full,
+                          int64_t T_cur, bool tc_low) {
+  WsLayout w{};
+  size_t off = 0;
+  const size_t osz = al256((size_t)Tq * ck.H * ck.d * sizeof(float));
+  const size_t lsz = al256((size_t)Tq * ck.H * sizeof(float));
+  const bool on[3] = {T_low > 0, T_full > 0, T_cur > 0};
+  for (int b = 0; b < 3; ++b) {
+    if (!on[b]) continue;
+    w.off_O[b] = off;
+    off += osz;
+    w.off_L[b] = off;
+    off += lsz;
+  }
+  w.off_qred = w.off_qc = off;
+  if (T_low > 0 && !tc_low) {
+    w.off_qred = off;
+    off += al256((size_t)ck.H * Tq * ck.r * sizeof(float));
+    w.off_qc = off;
+    off += al256((size_t)ck.H * Tq * ck.C * sizeof(float));
+  }
+  w.total = off;
+  return w;
+}
+
+}  // namespace nanokv
+
+using namespace nanokv;
+
+extern "C" {
+
+const char *nanokv_last_error(void) { return t_last_error.c_str(); }
+
+const char *nanokv_version(void) { return "nanokv-b200 0.1 (sm_100a)"; }
+
+int nanokv_set_kernel_path(int32_t path) {
+  if (path < 0 || path > 2) return -1;
+  return g_kernel_path.exchange(path);
+}
+
+int nanokv_check(void *stream) {
+  cudaStream_t st = (cudaStream_t)stream;
+  cudaError_t e = cudaStreamSynchronize(st);
+  if (e != cudaSuccess) return cuda_status(e, "stream");
+  unsigned *p = error_word_ptr();
+  if (!p) return fail(NANOKV_ERR_CUDA, "cannot resolve the device error word");
+  unsigned w = 0;
+  e = cudaMemcpy(&w, p, sizeof(w), cudaMemcpyDeviceToHost);
+  if (e != cudaSuccess) return cuda_status(e, "read error word");
+  if (w) {
+    const unsigned zero = 0;
+    cudaMemcpy(p, &zero, sizeof(zero), cudaMemcpyHostToDevice);
+    if (w & ERRW_TIMEOUT) return fail(NANOKV_ERR_TIMEOUT, "a kernel gave up on a bounded wait (word 0x%x)", w);
+    return fail(NANOKV_ERR_CUDA, "device error word 0x%x", w);
+  }
+  return NANOKV_OK;
+}
+
+int nanokv_encode(const nanokv_codec *ck, const nanokv_codec *cv, const void *k, const void *v,
+                  int32_t x_dtype, int64_t T, uint8_t *ids_k, uint8_t *codes_k, void *scales_k,
+                  uint8_t *ids_v, uint8_t *codes_v, void *scales_v, void *stream) {
+  if (T < 0) return fail(NANOKV_ERR_INVALID, "encode: T=%lld < 0", (long long)T);
+  if (!ck && !cv) return fail(NANOKV_ERR_INVALID, "encode: both codecs are NULL");
+  Codec c[2];
+  const nanokv_codec *in[2] = {ck, cv};
+  const void *x[2] = {k, v};
+  uint8_t *ids[2] = {ids_k, ids_v};
+  uint8_t *codes[2] = {codes_k, codes_v};
+  void *scales[2] = {scales_k, scales_v};
+  const int xp = io_prec(x_dtype);
+  for (int b = 0; b < 2; ++b) {
+    if (!in[b]) continue;
+    int s = check_codec(in[b], b ? "encode cv" : "encode ck", true, &c[b]);
+    if (s) return s;
+    if (xp != c[b].prec) return fail(NANOKV_ERR_UNSUPPORTED, "encode: x_dtype must equal param_dtype");
+    if (T > 0 && (!x[b] || !ids[b] || !codes[b] || !scales[b]))
+      return fail(NANOKV_ERR_INVALID, "encode: NULL input/output pointer for branch %d", b);
+    if (T > 0 && (!aligned16(x[b]) || !aligned16(codes[b])))
+      return fail(NANOKV_ERR_INVALID, "encode: pointers must be 16-byte aligned");
+  }
+  if (T == 0) return NANOKV_OK;
+  cudaStream_t st = (cudaStream_t)stream;
+  const int path = g_kernel_path.load();
+  for (int b = 0; b < 2; ++b) {
+    if (!in[b]) continue;
+    const bool tc_ok = tc_encode_supported(c[b]);
+    if (path == 2 && !tc_ok) return fail(NANOKV_ERR_UNSUPPORTED, "encode: no tensor-core kernel for this shape");
+    cudaError_t e = timed(NANOKV_K_ENCODE, 1, st, [&] {
+      return (path != 1 && tc_ok) ? tc_encode(c[b], x[b], T, ids[b], codes[b], scales[b], st)
+                                  : simt_encode(c[b], x[b], T, ids[b], codes[b], scales[b], st);
+    });
+    if (e != cudaSuccess) return cuda_status(e, "encode launch");
+  }
+  return NANOKV_OK;
+}
+
+size_t nanokv_attend_workspace(int64_t Tq, const nanokv_codec *ck, const nanokv_codec *cv,
+                               int64_t T, int64_t T_full, int64_t T_cur) {
+  Codec a, b;
+  if (Tq < 0 || T < 0 || T_full < 0 || T_full > T || T_cur < 0) return 0;
+  if (check_codec(ck, "ck", false, &a) || check_codec(cv, "cv", false, &b)) return 0;
+  const int path = g_kernel_path.load();
+  const bool tc_low = path != 1 && tc_low_supported(a, b);
+  return ws_layout(Tq, a, T - T_full, T_full, T_cur, tc_low).total;
+}
+
+int nanokv_attend(const void *q, int32_t io_dtype, int64_t Tq, const nanokv_codec *ck_,
+                  const nanokv_codec *cv_, const nanokv_hist *hk_, const nanokv_hist *hv_,
+                  int64_t T, int64_t T_full, const void *k_cur, const void *v_cur, int64_t T_cur,
+                  float softmax_scale, void *out, float *lse_out, void *workspace,
+                  size_t workspace_bytes, void *stream) {
+  Codec ck, cv;
+  int s;
+  if ((s = check_codec(ck_, "attend ck", false, &ck))) return s;
+  if ((s = check_codec(cv_, "attend cv", false, &cv))) return s;
+  if (ck.H != cv.H || ck.d != cv.d || ck.prec != cv.prec)
+    return fail(NANOKV_ERR_INVALID, "attend: ck and cv must share H, d and dtypes");
+  const int iop = io_prec(io_dtype);
+  if (iop != ck.prec) return fail(NANOKV_ERR_UNSUPPORTED, "attend: io_dtype must equal param_dtype");
+  if (Tq < 0 || T < 0 || T_cur < 0 || T_full < 0 || T_full > T)
+    return fail(NANOKV_ERR_INVALID, "attend: bad sizes Tq=%lld T=%lld T_full=%lld T_cur=%lld",
+                (long long)Tq, (long long)T, (long long)T_full, (long long)T_cur);
+  if (!(softmax_scale == softmax_scale) || softmax_scale <= 0.f || softmax_scale > 1e4f)
+    return fail(NANOKV_ERR_INVALID, "attend: softmax_scale must be finite and positive");
+  if (Tq == 0) return NANOKV_OK;
+  if (!q || !out) return fail(NANOKV_ERR_INVALID, "attend: NULL q or out");
+  if (!aligned16(q) || !aligned16(out) || (lse_out && !aligned16(lse_out)))
+    return fail(NANOKV_ERR_INVALID, "attend: q/out/lse_out must be 16-byte aligned");
+  if (T > 0) {
+    if (!hk_ || !hv_ || !hk_->ids || !hk_->codes || !hk_->scales || !hv_->ids || !hv_->codes ||
+        !hv_->scales)
+      return fail(NANOKV_ERR_INVALID, "attend: NULL history pointer with T > 0");
+    if (!aligned16(hk_->codes) || !aligned16(hv_->codes))
+      return fail(NANOKV_ERR_INVALID, "attend: code pointers must be 16-byte aligned");
+  }
+  if (T_cur > 0 && (!k_cur || !v_cur || !aligned16(k_cur) || !aligned16(v_cur)))
+    return fail(NANOKV_ERR_INVALID, "attend: k_cur/v_cur NULL or misaligned with T_cur > 0");
+
+  const int path = g_kernel_path.load();
+  const int64_t T_low = T - T_full;
+  const bool tc_full_ok = tc_full_supported(ck, cv);
+  const bool tc_low_ok = tc_low_supported(ck, cv);
+  const bool tc_dense_ok = tc_dense_supported(ck.prec, ck.d);
+  if (path == 2 && ((T_full > 0 && !tc_full_ok) || (T_low > 0 && !tc_low_ok) ||
+                    (T_cur > 0 && !tc_dense_ok)))
+    return fail(NANOKV_ERR_UNSUPPORTED, "attend: no tensor-core kernel for this shape");
+  const bool use_tc_low = path != 1 && tc_low_ok;
+  const WsLayout w = ws_layout(Tq, ck, T_low, T_full, T_cur, use_tc_low);
+  if (w.total > 0 && (!workspace || workspace_bytes < w.total))
+    return fail(NANOKV_ERR_INVALID, "attend: workspace needs %zu bytes, got %zu", w.total,
+                workspace_bytes);
+  if (workspace && !aligned16(workspace))
+    return fail(NANOKV_ERR_INVALID, "attend: workspace must be 16-byte aligned");
+
+  cudaStream_t st = (cudaStream_t)stream;
+  char *ws = (char *)workspace;
+  const Hist hk = T > 0 ? Hist{hk_->ids, hk_->codes, hk_->scales} : Hist{};
+  const Hist hv = T > 0 ? Hist{hv_->ids, hv_->codes, hv_->scales} : Hist{};
+  PartList pl{};
+  cudaError_t e;
+  if (T_low > 0) {
+    Part p{(float *)(ws + w.off_O[0]), (float *)(ws + w.off_L[0])};
+    if (use_tc_low) {
+      e = timed(NANOKV_K_LOW, 1, st, [&] {
+        return tc_attend_low(q, Tq, ck, cv, hk, hv, 0, T_low, softmax_scale, p, st);
+      });
+    } else {
+      float *qred = (float *)(ws + w.off_qred), *qc = (float *)(ws + w.off_qc);
+      e = timed(NANOKV_K_LOW, 2, st, [&] {
+        cudaError_t e2 = simt_low_prep(q, Tq, ck, qred, qc, st);
+        if (e2 == cudaSuccess)
+          e2 = simt_attend_low(qred, qc, Tq, ck, cv, hk, hv, 0, T_low, softmax_scale, p, st);
+        return e2;
+      });
+    }
+    if (e != cudaSuccess) return cuda_status(e, "attend low-dim launch");
+    pl.O[pl.n] = p.O;
+    pl.LSE[pl.n++] = p.LSE;
+  }
+  if (T_full > 0) {
+    Part p{(float *)(ws + w.off_O[1]), (float *)(ws + w.off_L[1])};
+    e = timed(NANOKV_K_FULL, 1, st, [&] {
+      return (path != 1 && tc_full_ok)
+                 ? tc_attend_full(q, Tq, ck, cv, hk, hv, T_low, T_full, softmax_scale, p, st)
+                 : simt_attend_full(q, Tq, ck, cv, hk, hv, T_low, T_full, softmax_scale, p, st);
+    });
+    if (e != cudaSuccess) return cuda_status(e, "attend full-dim launch");
+    pl.O[pl.n] = p.O;
+    pl.LSE[pl.n++] = p.LSE;
+  }
+  if (T_cur > 0) {
+    Part p{(float *)(ws + w.off_O[2]), (float *)(ws + w.off_L[2])};
+    e = timed(NANOKV_K_DENSE, 1, st, [&] {
+      return (path != 1 && tc_dense_ok)
+                 ? tc_attend_dense(q, Tq, ck.H, ck.d, k_cur, v_cur, T_cur, softmax_scale, p, st)
+                 : simt_attend_dense(ck.prec, q, Tq, ck.H, ck.d, k_cur, v_cur, T_cur,
+                                     softmax_scale, p, st);
+    });
+    if (e != cudaSuccess) return cuda_status(e, "attend current-chunk launch");
+    pl.O[pl.n] = p.O;
+    pl.LSE[pl.n++] = p.LSE;
+  }
+  e = timed(NANOKV_K_MERGE, 1, st,
+            [&] { return lse_merge_launch(pl, Tq, ck.H, ck.d, out, ck.prec, lse_out, st); });
+  return cuda_status(e, "attend merge launch");
+}
+
+int nanokv_lse_merge(int32_t n, const float *const *o_parts, const float *const *lse_parts,
+                     int64_t Tq, int32_t H, int32_t d, void *out, int32_t out_dtype,
+                     float *lse_out, void *stream) {
+  if (n < 1 || n > kMaxParts) return fail(NANOKV_ERR_INVALID, "merge: n=%d out of range [1,%d]", n, kMaxParts);
+  if (Tq < 0 || H < 1 || d < 4 || (d & 3)) return fail(NANOKV_ERR_INVALID, "merge: bad sizes (d must be a multiple of 4)");
+  const int op = io_prec(out_dtype);
+  if (op < 0) return fail(NANOKV_ERR_UNSUPPORTED, "merge: out_dtype must be F32 or BF16");
+  if (Tq == 0) return NANOKV_OK;
+  if (!o_parts || !lse_parts || !out) return fail(NANOKV_ERR_INVALID, "merge: NULL pointer");
+  PartList pl{};
+  for (int b = 0; b < n; ++b) {
+    if (!o_parts[b] || !lse_parts[b]) return fail(NANOKV_ERR_INVALID, "merge: NULL part %d", b);
+    if (!aligned16(o_parts[b])) return fail(NANOKV_ERR_INVALID, "merge: part %d misaligned", b);
+    pl.O[b] = o_parts[b];
+    pl.LSE[b] = lse_parts[b];
+  }
+  pl.n = n;
+  if (!aligned16(out)) return fail(NANOKV_ERR_INVALID, "merge: out misaligned");
+  cudaStream_t st = (cudaStream_t)stream;
+  return cuda_status(
+      timed(NANOKV_K_MERGE, 1, st, [&] { return lse_merge_launch(pl, Tq, H, d, out, op, lse_out, st); }),
+      "merge launch");
+}
+
+int nanokv_timing_enable(int32_t on) {
+  return g_timing.exchange(on ? 1 : 0);
+}
+
+int nanokv_timing_read(double *ms_total, int64_t *launches) {
+  std::vector<TimingRec> recs;
+  {
+    std::lock_guard<std::mutex> lk(g_tmu);
+    recs.swap(g_recs);
+  }
+  double tot[NANOKV_K_COUNT] = {0};
+  int status = NANOKV_OK;
+  for (auto &r : recs) {
+    float ms = 0.f;
+    cudaError_t e = cudaEventSynchronize(r.b);
+    if (e == cudaSuccess) e = cudaEventElapsedTime(&ms, r.a, r.b);
+    if (e != cudaSuccess && status == NANOKV_OK) status = cuda_status(e, "timing read");
+    tot[r.kid] += ms;
+  }
+  {
+    std::lock_guard<std::mutex> lk(g_tmu);
+    for (auto &r : recs) {
+      g_event_pool.push_back(r.a);
+      g_event_pool.push_back(r.b);
+    }
+  }
+  for (int k = 0; k < NANOKV_K_COUNT; ++k) {
+    if (ms_total) ms_total[k] = tot[k];
+    const int64_t n = g_launches[k].exchange(0);
+    if (launches) launches[k] = n;
+  }
+  return status;
+}
+
+}  // extern "C"

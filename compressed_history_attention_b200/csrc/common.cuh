@@ -1,0 +1,89 @@
+// Shared device helpers and the internal launcher interface of libnanokv.
+#pragma once
+
+#include <cuda_runtime.h>
+#include <cuda_bf16.h>
+#include <cuda_fp16.h>
+#include <stdint.h>
+#include <stddef.h>
+
+namespace nanokv {
+
+// ---------------------------------------------------------------------------
+// element conversion
+// ---------------------------------------------------------------------------
+template <typename T> __device__ __forceinline__ float to_f(T v);
+template <> __device__ __forceinline__ float to_f<float>(float v) { return v; }
+template <> __device__ __forceinline__ float to_f<__nv_bfloat16>(__nv_bfloat16 v) { return __bfloat162float(v); }
+template <> __device__ __forceinline__ float to_f<__half>(__half v) { return __half2float(v); }
+
+template <typename T> __device__ __forceinline__ T from_f(float v);
+template <> __device__ __forceinline__ float from_f<float>(float v) { return v; }
+template <> __device__ __forceinline__ __nv_bfloat16 from_f<__nv_bfloat16>(float v) { return __float2bfloat16_rn(v); }
+template <> __device__ __forceinline__ __half from_f<__half>(float v) { return __float2half_rn(v); }
+
+__device__ __forceinline__ float warp_sum(float v) {
+#pragma unroll
+  for (int o = 16; o > 0; o >>= 1) v += __shfl_xor_sync(0xffffffffu, v, o);
+  return v;
+}
+__device__ __forceinline__ float warp_max(float v) {
+#pragma unroll
+  for (int o = 16; o > 0; o >>= 1) v = fmaxf(v, __shfl_xor_sync(0xffffffffu, v, o));
+  return v;
+}
+
+// INT4 nibble (two's complement) -> int
+__device__ __forceinline__ int nib_lo(uint8_t b) { return (int)((int8_t)(b << 4) >> 4); }
+__device__ __forceinline__ int nib_hi(uint8_t b) { return (int)((int8_t)b >> 4); }
+
+// error-word bits (device error word, read by nanokv_check)
+enum : unsigned { ERRW_TIMEOUT = 1u, ERRW_BOUNDS = 2u };
+
+// ---------------------------------------------------------------------------
+// internal argument bundles (plain pointers; no torch types anywhere)
+// ---------------------------------------------------------------------------
+struct Codec {
+  int H, d, r, C;
+  int prec;  // 0 = fp32 everywhere, 1 = bf16 params/io + fp16 scales
+  const void *centers, *D, *E;
+};
+struct Hist {
+  const uint8_t *ids, *codes;
+  const void *scales;
+};
+
+enum Prec { PREC_F32 = 0, PREC_BF16 = 1 };
+
+// fp32 partial output of one attention branch: O [Tq, H, d], LSE [H, Tq]
+struct Part {
+  float *O, *LSE;
+};
+
+constexpr int kMaxParts = 8;
+struct PartList {
+  const float *O[kMaxParts];
+  const float *LSE[kMaxParts];
+  int n;
+};
+
+// ---------------------------------------------------------------------------
+// launchers (return cudaError_t of the launch; shapes already validated)
+// ---------------------------------------------------------------------------
+// fp32 CUDA-core kernels
+cudaError_t simt_encode(const Codec &c, const void *x, int64_t T, uint8_t *ids, uint8_t *codes,
+                        void *scales, cudaStream_t st);
+cudaError_t simt_attend_dense(int prec, const void *q, int64_t Tq, int H, int d, const void *k,
+                              const void *v, int64_t T, float tau, Part out, cudaStream_t st);
+cudaError_t simt_attend_full(const void *q, int64_t Tq, const Codec &ck, const Codec &cv,
+                             const Hist &hk, const Hist &hv, int64_t t0, int64_t T, float tau,
+                             Part out, cudaStream_t st);
+cudaError_t simt_low_prep(const void *q, int64_t Tq, const Codec &ck, float *qred, float *qc,
+                          cudaStream_t st);
+cudaError_t simt_attend_low(const float *qred, const float *qc, int64_t Tq, const Codec &ck,
+                            const Codec &cv, const Hist &hk, const Hist &hv, int64_t t0,
+                            int64_t T, float tau, Part out, cudaStream_t st);
+cudaError_t lse_merge_launch(const PartList &parts, int64_t Tq, int H, int d, void *out,
+                             int out_prec, float *lse_out, cudaStream_t st);
+
+}  // namespace nanokv

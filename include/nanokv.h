@@ -1,0 +1,187 @@
+/*
+ * nanokv.h -- C ABI of the NanoKV compressed-history attention library
+ * (libnanokv.so, CUDA, sm_100a).
+ *
+ * Source method: "NanoKV: High-Ratio KV Cache Compression for Autoregressive
+ * Video Generation" (arXiv 2611.06377).  Historical keys and values are stored
+ * per token as a cluster-center id plus INT4 joint head-channel residual
+ * coefficients with a per-token scale, under a linear decoder (abstract;
+ * Fig. 4(a,b)).  Attention of a new chunk's queries reads that history either
+ * fully decoded (NanoKV) or, for history that a fixed policy routes to low
+ * dimension, against the coefficients with reduced queries (NanoKV-Fast,
+ * Fig. 4(d)); branch outputs are combined by log-sum-exp merging.
+ *
+ * Conventions shared by every entry point
+ *  - All tensor pointers are DEVICE pointers owned by the caller; the library
+ *    never allocates, frees or retains them.  Scratch memory is passed in as
+ *    `workspace` where needed.
+ *  - Every call is asynchronous on `stream` (a cudaStream_t; NULL = legacy
+ *    default stream) and never synchronises.
+ *  - Joint dimension J = H * d.  Head h owns joint columns [h*d, (h+1)*d).
+ *  - Row-major layouts, no padding between rows.  Every pointer must be
+ *    16-byte aligned.
+ *  - Codes: r INT4 values per token packed two per byte, code 2i in the low
+ *    nibble of byte i, two's complement; encode emits values in [-7, 7].
+ *  - Return values are nanokv_status.  Argument errors return
+ *    NANOKV_ERR_INVALID (nothing launched); shape/dtype combinations without a
+ *    kernel return NANOKV_ERR_UNSUPPORTED (nothing launched); a launch failure
+ *    returns NANOKV_ERR_CUDA.  nanokv_last_error() describes the last non-OK
+ *    status of the calling thread.
+ *  - Kernels never trap.  A kernel whose internal wait exceeds its iteration
+ *    bound records that in a device error word and returns early;
+ *    nanokv_check() reports it as NANOKV_ERR_TIMEOUT.
+ */
+#ifndef NANOKV_H
+#define NANOKV_H
+
+#include <stddef.h>
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+typedef enum {
+  NANOKV_OK = 0,
+  NANOKV_ERR_INVALID = -1,
+  NANOKV_ERR_UNSUPPORTED = -2,
+  NANOKV_ERR_CUDA = -3,
+  NANOKV_ERR_TIMEOUT = -4
+} nanokv_status;
+
+typedef enum { NANOKV_F32 = 0, NANOKV_F16 = 1, NANOKV_BF16 = 2 } nanokv_dtype;
+
+/*
+ * One codec: per layer and per K or V branch (Table 5: rank per layer per K/V
+ * branch; centers fitted separately for K and V).  All pointers are device
+ * pointers in `param_dtype`.
+ *   centers [C, J]  cluster centers (Fig. 4(a,b): shared content)
+ *   D       [J, r]  linear decoder (Fig. 4(b): reconstructs the residual)
+ *   E       [r, J]  linear encoder (Fig. 4(b): residual -> coefficients);
+ *                   may be NULL for calls that do not encode.
+ * Constraints: 1 <= C <= 256; r even, 2 <= r <= 512; d in {16, 32, 64, 128}.
+ * Precision modes: param_dtype = scale_dtype = F32 (fp32 everywhere), or
+ * param_dtype = BF16 with scale_dtype = F16.
+ */
+typedef struct {
+  int32_t H, d, r, C;
+  int32_t param_dtype; /* nanokv_dtype */
+  int32_t scale_dtype; /* nanokv_dtype */
+  const void *centers;
+  const void *D;
+  const void *E;
+} nanokv_codec;
+
+/* One branch of compressed history, T tokens in time order (oldest first).
+ *   ids    [T]        uint8 center id (values >= C are read as C - 1)
+ *   codes  [T, r/2]   packed INT4 coefficients
+ *   scales [T]        per-token scale in the codec's scale_dtype            */
+typedef struct {
+  const uint8_t *ids;
+  const uint8_t *codes;
+  const void *scales;
+} nanokv_hist;
+
+/*
+ * nanokv_encode -- compress T tokens of K and of V (Fig. 4(b); abstract).
+ * For each token x (J values in x_dtype, which must equal the codec's
+ * param_dtype):
+ *   a = argmin_j |x - c_j|^2            (squared Euclidean, ties -> lowest j)
+ *   y = E (x - c_a)                     (r coefficients)
+ *   s = scale_dtype(max_i |y_i| / 7)    (round to nearest even)
+ *   code_i = clamp(rint(y_i / s), -7, 7), all zero when s == 0
+ * Inputs k, v [T, J]; outputs ids_* [T], codes_* [T, r/2], scales_* [T].
+ * Either branch may be skipped by passing its codec as NULL (then its input
+ * and outputs are ignored).  T = 0 is a no-op.
+ */
+int nanokv_encode(const nanokv_codec *ck, const nanokv_codec *cv,
+                  const void *k, const void *v, int32_t x_dtype, int64_t T,
+                  uint8_t *ids_k, uint8_t *codes_k, void *scales_k,
+                  uint8_t *ids_v, uint8_t *codes_v, void *scales_v,
+                  void *stream);
+
+/*
+ * nanokv_attend -- attention of a query chunk over compressed history plus
+ * the current uncompressed chunk (Fig. 4(a) full-dim decode-attention;
+ * Fig. 4(d) fixed routing to full or low dimension and LSE merging).
+ *   q      [Tq, H, d] in io_dtype (= codec param_dtype)
+ *   hk, hv compressed history of T tokens.  Fixed routing policy: the most
+ *          recent T_full tokens (indices [T - T_full, T)) use full-dim
+ *          decode-attention, K_hat = c_K[a] + s D_K code, decoded on chip and
+ *          never written to memory; the older T - T_full tokens use low-dim
+ *          attention: per head h, scores tau (s (D_{K,h}^T q) . code +
+ *          c_{K,a,h} . q), output (sum p c_{V,a,h} + D_{V,h} sum p s code) / sum p.
+ *   k_cur, v_cur [T_cur, H, d] current chunk in io_dtype (may be NULL if T_cur = 0)
+ *   softmax_scale tau (callers normally pass 1/sqrt(d)); no mask.
+ *   out    [Tq, H, d] in io_dtype.  lse_out [H, Tq] fp32 natural-log LSE, or NULL.
+ *   Rows with no keys at all get out = 0 and lse = -inf.
+ *   workspace: device scratch of at least nanokv_attend_workspace(...) bytes,
+ *   16-byte aligned; contents on entry are ignored.
+ * ck and cv must share H, d, param_dtype and scale_dtype; r and C may differ.
+ */
+int nanokv_attend(const void *q, int32_t io_dtype, int64_t Tq,
+                  const nanokv_codec *ck, const nanokv_codec *cv,
+                  const nanokv_hist *hk, const nanokv_hist *hv,
+                  int64_t T, int64_t T_full,
+                  const void *k_cur, const void *v_cur, int64_t T_cur,
+                  float softmax_scale, void *out, float *lse_out,
+                  void *workspace, size_t workspace_bytes, void *stream);
+
+/* Workspace bytes nanokv_attend needs for these sizes (0 is possible). */
+size_t nanokv_attend_workspace(int64_t Tq, const nanokv_codec *ck, const nanokv_codec *cv,
+                               int64_t T, int64_t T_full, int64_t T_cur);
+
+/*
+ * nanokv_lse_merge -- merge n partial attention results over disjoint key sets
+ * (Fig. 4(d): LSE merging):  LSE = log sum_i exp(LSE_i),
+ * O = sum_i exp(LSE_i - LSE) O_i.  Parts with LSE_i = -inf contribute nothing;
+ * rows where every part is -inf get O = 0, LSE = -inf.
+ *   o_parts[i]   device [Tq, H, d] fp32      lse_parts[i] device [H, Tq] fp32
+ *   o_parts / lse_parts are HOST arrays of n device pointers, 1 <= n <= 8.
+ *   out [Tq, H, d] in out_dtype (F32 or BF16); lse_out [H, Tq] fp32 or NULL.
+ */
+int nanokv_lse_merge(int32_t n, const float *const *o_parts, const float *const *lse_parts,
+                     int64_t Tq, int32_t H, int32_t d, void *out, int32_t out_dtype,
+                     float *lse_out, void *stream);
+
+/* Kernel family selection: 0 = automatic (tensor-core kernels where the shape
+ * has one, fp32 CUDA-core kernels otherwise), 1 = fp32 CUDA-core kernels only,
+ * 2 = tensor-core kernels only (NANOKV_ERR_UNSUPPORTED where none exists).
+ * Process-wide; returns the previous value, or -1 for an invalid argument. */
+int nanokv_set_kernel_path(int32_t path);
+
+/* Reads (and clears) the device error word after synchronising `stream`:
+ * NANOKV_OK, NANOKV_ERR_TIMEOUT if a kernel gave up on a bounded wait, or
+ * NANOKV_ERR_CUDA if the stream reports an error. */
+int nanokv_check(void *stream);
+
+/* Message for the calling thread's last non-OK status ("" if none). */
+const char *nanokv_last_error(void);
+
+/* Kernel identities for the diagnostics below. */
+typedef enum {
+  NANOKV_K_ENCODE = 0,   /* encode (one launch per K or V branch)           */
+  NANOKV_K_FULL = 1,     /* full-dim decode-attention                       */
+  NANOKV_K_LOW = 2,      /* low-dim attention (incl. its query prep)        */
+  NANOKV_K_DENSE = 3,    /* attention over the current uncompressed chunk   */
+  NANOKV_K_MERGE = 4,    /* LSE merge                                       */
+  NANOKV_K_COUNT = 8
+} nanokv_kernel_id;
+
+/* Diagnostics.  nanokv_timing_enable(1) makes every later kernel launch record
+ * a pair of CUDA events on its own stream (the library creates and reuses the
+ * events; no device memory).  nanokv_timing_read() waits for the recorded
+ * events, writes per-kernel total milliseconds and launch counts into the
+ * caller's arrays of NANOKV_K_COUNT entries (either may be NULL), and clears
+ * the record.  Launch counts are kept even when timing is off. */
+int nanokv_timing_enable(int32_t on);
+int nanokv_timing_read(double *ms_total, int64_t *launches);
+
+/* Library version string. */
+const char *nanokv_version(void);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* NANOKV_H */

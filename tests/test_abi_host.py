@@ -1,0 +1,136 @@
+"""Host-side checks of the C ABI that need no GPU: the library loads, exports
+every symbol the header declares, and rejects bad arguments before launching
+anything."""
+import ctypes
+import os
+import re
+
+import pytest
+
+import compressed_history_attention_b200 as nk
+from compressed_history_attention_b200 import _lib
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+
+
+def _header_functions():
+    names = set()
+    for fn in os.listdir(os.path.join(ROOT, "include")):
+        if fn.endswith(".h"):
+            src = open(os.path.join(ROOT, "include", fn)).read()
+            src = re.sub(r"/\*.*?\*/", "", src, flags=re.S)
+            names |= set(re.findall(r"\b(nanokv_\w+)\s*\(", src))
+    return names
+
+
+def test_library_exports_every_declared_symbol():
+    L = nk.lib()
+    declared = _header_functions()
+    assert declared >= set(_lib.SYMBOLS)
+    for name in sorted(declared):
+        assert hasattr(L, name), name
+
+
+def test_version():
+    assert "sm_100a" in nk.nanokv_version()
+
+
+def _codec(**kw):
+    c = dict(H=2, d=16, r=8, C=8, param_dtype=_lib.F32, scale_dtype=_lib.F32,
+             centers=4096, D=8192, E=12288)
+    c.update(kw)
+    return _lib._Codec(**c)
+
+
+BAD_CODECS = [
+    (dict(r=7), _lib.ERR_INVALID),
+    (dict(r=0), _lib.ERR_INVALID),
+    (dict(r=514), _lib.ERR_INVALID),
+    (dict(C=0), _lib.ERR_INVALID),
+    (dict(C=257), _lib.ERR_INVALID),
+    (dict(H=0), _lib.ERR_INVALID),
+    (dict(d=24), _lib.ERR_UNSUPPORTED),
+    (dict(param_dtype=_lib.BF16, scale_dtype=_lib.F32), _lib.ERR_UNSUPPORTED),
+    (dict(centers=0), _lib.ERR_INVALID),
+    (dict(D=4100), _lib.ERR_INVALID),        # misaligned
+]
+
+
+@pytest.mark.parametrize("kw,status", BAD_CODECS)
+def test_encode_rejects_bad_codec(kw, status):
+    L = nk.lib()
+    c = _codec(**kw)
+    p = ctypes.c_void_p(1 << 20)
+    st = L.nanokv_encode(ctypes.byref(c), None, p, None, _lib.F32, 10, p, p, p, None, None, None, None)
+    assert st == status
+    assert L.nanokv_last_error().decode()
+
+
+@pytest.mark.parametrize("kw,status", BAD_CODECS)
+def test_attend_rejects_bad_codec(kw, status):
+    L = nk.lib()
+    c, good = _codec(**kw), _codec()
+    p = ctypes.c_void_p(1 << 20)
+    h = _lib._Hist(1 << 20, 1 << 20, 1 << 20)
+    st = L.nanokv_attend(p, _lib.F32, 4, ctypes.byref(good), ctypes.byref(c), ctypes.byref(h),
+                         ctypes.byref(h), 8, 8, None, None, 0, ctypes.c_float(0.25), p, None, p,
+                         1 << 20, None)
+    assert st == status
+
+
+def test_attend_rejects_bad_sizes_and_pointers():
+    L = nk.lib()
+    c = _codec()
+    p = ctypes.c_void_p(1 << 20)
+    h = _lib._Hist(1 << 20, 1 << 20, 1 << 20)
+    hn = _lib._Hist(0, 1 << 20, 1 << 20)
+    call = lambda **kw: L.nanokv_attend(  # noqa: E731
+        kw.get("q", p), kw.get("dt", _lib.F32), kw.get("Tq", 4), ctypes.byref(c), ctypes.byref(kw.get("cv", c)),
+        ctypes.byref(kw.get("hk", h)), ctypes.byref(h), kw.get("T", 8), kw.get("T_full", 8),
+        kw.get("kc", None), None, kw.get("T_cur", 0), ctypes.c_float(kw.get("tau", 0.25)), kw.get("out", p),
+        None, kw.get("ws", p), kw.get("wsb", 1 << 20), None)
+    assert call(T_full=9) == _lib.ERR_INVALID          # T_full > T
+    assert call(T=-1) == _lib.ERR_INVALID
+    assert call(Tq=-3) == _lib.ERR_INVALID
+    assert call(tau=float("nan")) == _lib.ERR_INVALID
+    assert call(tau=-1.0) == _lib.ERR_INVALID
+    assert call(hk=hn) == _lib.ERR_INVALID              # NULL ids with T > 0
+    assert call(T_cur=4) == _lib.ERR_INVALID            # NULL k_cur with T_cur > 0
+    assert call(q=ctypes.c_void_p((1 << 20) + 2)) == _lib.ERR_INVALID   # misaligned
+    assert call(dt=_lib.BF16) == _lib.ERR_UNSUPPORTED   # io dtype != params
+    assert call(wsb=16) == _lib.ERR_INVALID             # workspace too small
+    assert call(cv=_codec(H=3)) == _lib.ERR_INVALID     # K/V codecs disagree on H
+    assert call(Tq=0) == _lib.OK                         # nothing to do, nothing launched
+
+
+def test_workspace_size_is_deterministic_and_grows():
+    L = nk.lib()
+    c = _codec()
+    f = lambda Tq, T, Tf, Tc: L.nanokv_attend_workspace(Tq, ctypes.byref(c), ctypes.byref(c), T, Tf, Tc)  # noqa: E731
+    assert f(0, 0, 0, 0) == 0
+    assert f(64, 256, 256, 64) > 0
+    assert f(64, 256, 0, 64) > f(64, 256, 256, 64)      # low-dim branch adds prep buffers
+    assert f(64, 256, 300, 64) == 0                      # invalid -> 0
+
+
+def test_merge_rejects_bad_arguments():
+    L = nk.lib()
+    arr = (ctypes.c_void_p * 1)(1 << 20)
+    p = ctypes.c_void_p(1 << 20)
+    assert L.nanokv_lse_merge(0, arr, arr, 4, 2, 16, p, _lib.F32, None, None) == _lib.ERR_INVALID
+    assert L.nanokv_lse_merge(9, arr, arr, 4, 2, 16, p, _lib.F32, None, None) == _lib.ERR_INVALID
+    assert L.nanokv_lse_merge(1, arr, arr, 4, 2, 18, p, _lib.F32, None, None) == _lib.ERR_INVALID
+    assert L.nanokv_lse_merge(1, arr, arr, 4, 2, 16, p, _lib.F16, None, None) == _lib.ERR_UNSUPPORTED
+
+
+def test_kernel_path_switch():
+    prev = nk.nanokv_set_kernel_path(1)
+    assert nk.nanokv_set_kernel_path(prev) == 1
+    assert nk.lib().nanokv_set_kernel_path(7) == -1
+
+
+def test_encode_zero_tokens_is_noop():
+    L = nk.lib()
+    c = _codec()
+    assert L.nanokv_encode(ctypes.byref(c), None, None, None, _lib.F32, 0, None, None, None,
+                           None, None, None, None) == _lib.OK
