@@ -115,7 +115,7 @@ class ClockSampler:
         sm = [float(r[2]) for r in rows if r[2].replace(".", "").isdigit()]
         mx = max(float(r[3]) for r in rows if r[3].replace(".", "").isdigit())
         names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
-        reasons = sorted({names[i] for r in rows for i in range(4) if "Active" in r[6 + i]})
+        reasons = sorted({names[i] for r in rows for i in range(4) if r[6 + i].strip() == "Active"})
         load = [s for s in sm if s > 0.5 * mx] or sm
         return {"sm_mhz": statistics.median(load) if load else None, "sm_max_mhz": mx,
                 "reasons": reasons, "samples": len(rows)}

@@ -1,0 +1,140 @@
+// Host helpers for the tensor-core kernels (tensor maps) and the per-row
+// online-softmax / output stages shared by the attention kernels.
+#pragma once
+
+#include <cudaTypedefs.h>
+
+#include "sm100.cuh"
+#include "tc.cuh"
+
+namespace nanokv {
+
+// ---------------------------------------------------------------------------
+// host: 2-D bf16 tensor map (row-major [rows, cols], row stride in elements),
+// box [64 cols x box_rows], 128-byte swizzle, zero fill out of bounds.
+// ---------------------------------------------------------------------------
+bool make_tmap_bf16_2d(CUtensorMap *map, const void *base, uint64_t rows, uint64_t cols,
+                       uint64_t row_stride_elems, uint32_t box_rows);
+
+namespace tc {
+
+constexpr int BM = 128;  // query rows per CTA (TMEM lanes)
+constexpr int BN = 128;  // keys per tile
+constexpr float kLn2 = 0.6931471805599453f;
+constexpr float kLog2e = 1.4426950408889634f;
+// lazy rescaling: keep the running max until a row's max grows by more than
+// this many powers of two (probabilities then stay below 2^kRescaleLog2)
+constexpr float kRescaleLog2 = 8.0f;
+
+__device__ __forceinline__ float ex2(float x) {
+  float y;
+  asm("ex2.approx.ftz.f32 %0, %1;" : "=f"(y) : "f"(x));
+  return y;
+}
+
+__device__ __forceinline__ uint32_t pack_bf16x2(float lo, float hi) {
+  __nv_bfloat162 v = __floats2bfloat162_rn(lo, hi);
+  return *reinterpret_cast<uint32_t *>(&v);
+}
+
+// TMEM address of (lane base of this warp's quarter, column)
+__device__ __forceinline__ uint32_t tmem_lane_addr(uint32_t base, int warp, uint32_t col) {
+  return base + ((uint32_t)((warp & 3) * 32) << 16) + col;
+}
+
+// Online-softmax state of one query row (one thread), log2 domain.
+struct RowState {
+  float m;  // running max of the scaled scores (log2 units)
+  float l;  // running sum of 2^(z - m)
+};
+
+// One key tile of the online softmax for the calling thread's row.
+// Reads S (fp32, 128 columns at s_col), writes P as packed bf16 into the first
+// 64 of those columns, updates the row state.  `nk` valid keys; `zscale`
+// multiplies raw scores into log2 units.  Returns the factor by which the
+// caller must rescale O (1 if none); *rescale tells whether any row of the
+// warp needs it.
+__device__ __forceinline__ float softmax_tile(uint32_t tbase, int warp, uint32_t s_col, int nk,
+                                              float zscale, RowState &st, bool &warp_rescale) {
+  uint32_t r[32];
+  float mx = -INFINITY;
+#pragma unroll
+  for (int c = 0; c < 4; ++c) {
+    sm100::tmem_ld32(tmem_lane_addr(tbase, warp, s_col + 32 * c), r);
+    sm100::tmem_ld_wait();
+#pragma unroll
+    for (int i = 0; i < 32; ++i) {
+      const float z = (32 * c + i < nk) ? __uint_as_float(r[i]) * zscale : -INFINITY;
+      mx = fmaxf(mx, z);
+    }
+  }
+  float corr = 1.f;
+  const bool need = mx > st.m + kRescaleLog2;  // also true when st.m == -inf
+  if (need) {
+    corr = (st.m == -INFINITY) ? 0.f : ex2(st.m - mx);
+    st.l *= corr;
+    st.m = mx;
+  }
+  warp_rescale = __any_sync(0xffffffffu, need) != 0;
+  const float m = st.m;
+  float lsum = 0.f;
+#pragma unroll
+  for (int c = 0; c < 4; ++c) {
+    sm100::tmem_ld32(tmem_lane_addr(tbase, warp, s_col + 32 * c), r);
+    sm100::tmem_ld_wait();
+    uint32_t pk[16];
+#pragma unroll
+    for (int i = 0; i < 16; ++i) {
+      const int k0 = 32 * c + 2 * i;
+      const float p0 = (k0 < nk) ? ex2(fmaf(__uint_as_float(r[2 * i]), zscale, -m)) : 0.f;
+      const float p1 = (k0 + 1 < nk) ? ex2(fmaf(__uint_as_float(r[2 * i + 1]), zscale, -m)) : 0.f;
+      lsum += p0 + p1;
+      pk[i] = pack_bf16x2(p0, p1);
+    }
+    sm100::tmem_st16(tmem_lane_addr(tbase, warp, s_col + 16 * c), pk);
+  }
+  sm100::tmem_st_wait();
+  st.l += lsum;
+  return corr;
+}
+
+// Multiplies this thread's O row (128 fp32 columns at o_col) by f.
+__device__ __forceinline__ void rescale_o(uint32_t tbase, int warp, uint32_t o_col, float f) {
+  uint32_t r[16];
+#pragma unroll
+  for (int c = 0; c < 8; ++c) {
+    const uint32_t a = tmem_lane_addr(tbase, warp, o_col + 16 * c);
+    sm100::tmem_ld16(a, r);
+    sm100::tmem_ld_wait();
+#pragma unroll
+    for (int i = 0; i < 16; ++i) r[i] = __float_as_uint(__uint_as_float(r[i]) * f);
+    sm100::tmem_st16(a, r);
+  }
+  sm100::tmem_st_wait();
+}
+
+// Writes the normalised O row and its natural-log LSE (fp32 partials).
+__device__ __forceinline__ void write_row(uint32_t tbase, int warp, uint32_t o_col,
+                                          const RowState &st, int64_t row, int64_t Tq, int h, int H,
+                                          float *__restrict__ O, float *__restrict__ L) {
+  const float inv = st.l > 0.f ? 1.f / st.l : 0.f;
+  uint32_t r[32];
+  float *dst = O + (row * H + h) * 128;
+#pragma unroll
+  for (int c = 0; c < 4; ++c) {
+    sm100::tmem_ld32(tmem_lane_addr(tbase, warp, o_col + 32 * c), r);
+    sm100::tmem_ld_wait();
+    if (row < Tq) {
+#pragma unroll
+      for (int i = 0; i < 32; i += 4) {
+        float4 v = make_float4(__uint_as_float(r[i]) * inv, __uint_as_float(r[i + 1]) * inv,
+                               __uint_as_float(r[i + 2]) * inv, __uint_as_float(r[i + 3]) * inv);
+        *reinterpret_cast<float4 *>(dst + 32 * c + i) = v;
+      }
+    }
+  }
+  if (row < Tq) L[(int64_t)h * Tq + row] = st.l > 0.f ? (st.m + log2f(st.l)) * kLn2 : -INFINITY;
+}
+
+}  // namespace tc
+}  // namespace nanokv

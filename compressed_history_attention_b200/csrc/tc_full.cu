@@ -1,0 +1,396 @@
+// Tensor-core full-dimensional decode-attention (NanoKV Fig. 4(a,b)): the
+// history keys and values are decoded on chip,
+//     K_hat_t = c_K[a_t] + s_t D_K code_t,   V_hat_t likewise,
+// and never written to global memory; then S = tau Q K_hat^T, online softmax,
+// O = P V_hat.
+//
+// A cluster of two CTAs serves two 128-row query tiles of one head.  CTA 0
+// decodes K_hat, CTA 1 decodes V_hat, and each writes its decoded bf16 tile
+// into the shared memory of both CTAs, so every decode is shared by 256 query
+// rows and each CTA keeps a single decoder slice D_h resident.
+//
+// Roles (12 warps):
+//   warp 0      TMA: Q tile; packed code chunks [128 keys x 32 B] into staging
+//   warp 1      MMA issuer: X = codes D_h^T (decode), S = Q K_hat^T, O += P V_hat
+//   warps 2,3   unpack INT4 staging -> bf16 operand ring (128 keys x 64 codes)
+//   warps 4..7  decode epilogue: X (TMEM, lane = key) * s + center -> bf16 tile
+//               in both CTAs' shared memory
+//   warps 8..11 softmax, one thread per query row; final O / LSE
+// Codes are unpacked in an order permuted within each group of 8; the
+// decoder slice is stored with the same permutation, so the contraction over
+// the rank index is unchanged.  Every wait is bounded.
+#include "tc_common.cuh"
+
+namespace nanokv {
+
+using namespace sm100;
+using namespace tc;
+
+bool make_tmap_u8_2d(CUtensorMap *map, const void *base, uint64_t rows, uint64_t cols,
+                     uint64_t row_stride_bytes, uint32_t box_cols, uint32_t box_rows);
+
+namespace {
+
+constexpr int DH = 128;
+constexpr uint32_t kTile = 128 * 128 * 2;   // [128 x 128] bf16
+constexpr uint32_t kChunk = 128 * 64 * 2;   // [128 keys x 64 codes] bf16
+constexpr uint32_t kStage = 128 * 32;       // [128 keys x 32 bytes] packed
+constexpr int NRING = 3, NSTAGE = 4;
+constexpr uint32_t IDESC_DEC = idesc_bf16(128, 128, false, false);
+constexpr uint32_t IDESC_S = idesc_bf16(128, 128, false, false);
+constexpr uint32_t IDESC_PV = idesc_bf16(128, 128, false, true);
+constexpr uint32_t TM_O = 0, TM_S = 128, TM_X = 256, TM_COLS = 512;
+
+struct FullArgs {
+  const __nv_bfloat16 *D[2];    // decoders [J, r] (K, V)
+  const __nv_bfloat16 *cen[2];  // centers [C, J]
+  const uint8_t *ids[2];        // [T_total]
+  const __half *scales[2];      // [T_total]
+  int64_t t0, T, Tq;            // branch = history tokens [t0, t0 + T)
+  int H, r, C[2];
+  float zscale;
+  float *O, *L;
+  unsigned *err;
+};
+
+struct FullBars {
+  uint64_t q_full;
+  uint64_t st_full[NSTAGE], st_empty[NSTAGE];
+  uint64_t ring_full[NRING], ring_empty[NRING];
+  uint64_t x_full[2], x_empty[2];
+  uint64_t kh_full, vh_full, kh_empty, vh_empty;
+  uint64_t s_full, p_full, pv_done;
+  uint32_t tmem_base;
+  int abort;
+};
+
+// 8 packed INT4 codes (one 32-bit word, code i in bits [4i, 4i+4)) -> 8 bf16
+// in the order (n0,n4), (n1,n5), (n2,n6), (n3,n7): position p of the group
+// holds code (0,4,1,5,2,6,3,7)[p]
+__device__ __forceinline__ uint4 unpack8(uint32_t w) {
+  const __nv_bfloat162 bias = __floats2bfloat162_rn(136.f, 136.f);
+  uint32_t o[4];
+#pragma unroll
+  for (int i = 0; i < 4; ++i) {
+    // (nibble XOR 8) | 0x4300 encodes 128 + (n + 8) in bf16; subtract 136
+    const uint32_t b = ((w >> (4 * i)) & 0x000F000Fu) ^ 0x43084308u;
+    __nv_bfloat162 v = __hsub2(*reinterpret_cast<const __nv_bfloat162 *>(&b), bias);
+    o[i] = *reinterpret_cast<uint32_t *>(&v);
+  }
+  return make_uint4(o[0], o[1], o[2], o[3]);
+}
+
+__global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(384, 1)
+    tc_full_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUtensorMap tmCk,
+                   const __grid_constant__ CUtensorMap tmCv, const FullArgs A) {
+  extern __shared__ uint8_t smraw[];
+  uint8_t *sm = (uint8_t *)(((uintptr_t)smraw + 1023) & ~(uintptr_t)1023);
+  const int nrb = A.r / 64;  // 64-wide rank blocks
+  uint8_t *sQ = sm;
+  uint8_t *sD = sQ + kTile;
+  uint8_t *sRing = sD + nrb * kChunk;
+  uint8_t *sKh = sRing + NRING * kChunk;
+  uint8_t *sVh = sKh + kTile;
+  uint8_t *sStage = sVh + kTile;
+  __shared__ FullBars B;
+
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const uint32_t rank = cluster_ctarank();  // 0: decodes K, 1: decodes V
+  const uint32_t peer = rank ^ 1u;
+  const int h = blockIdx.y;
+  const int64_t q0 = (int64_t)blockIdx.x * BM;
+  const int ntiles = (int)((A.T + BN - 1) / BN);
+  const int nchunk = ntiles * nrb;
+  const int J = A.H * DH;
+  volatile int *abort = &B.abort;
+  unsigned *err = A.err;
+
+  if (threadIdx.x == 0) {
+    mbar_init(&B.q_full, 1);
+    for (int i = 0; i < NSTAGE; ++i) { mbar_init(&B.st_full[i], 1); mbar_init(&B.st_empty[i], 2); }
+    for (int i = 0; i < NRING; ++i) { mbar_init(&B.ring_full[i], 2); mbar_init(&B.ring_empty[i], 1); }
+    for (int i = 0; i < 2; ++i) { mbar_init(&B.x_full[i], 1); mbar_init(&B.x_empty[i], 4); }
+    mbar_init(&B.kh_full, 4);
+    mbar_init(&B.vh_full, 4);
+    mbar_init(&B.kh_empty, 2);
+    mbar_init(&B.vh_empty, 2);
+    mbar_init(&B.s_full, 1);
+    mbar_init(&B.p_full, 4);
+    mbar_init(&B.pv_done, 1);
+    B.abort = 0;
+    fence_mbar_init();
+  }
+  if (warp == 0) {
+    tmem_alloc(&B.tmem_base, TM_COLS);
+    tmem_relinquish();
+  }
+  // decoder slice of this CTA's branch, rows h*128.. of D [J, r], permuted
+  // within groups of 8 like the unpacked codes; K-major 128B-swizzled
+  if (warp == 0 || warp == 2 || warp == 3) {
+    const int t = (warp == 0 ? 0 : warp - 1) * 32 + lane;  // 0..95
+    const __nv_bfloat16 *Dsrc = A.D[rank] + (size_t)h * DH * A.r;
+    const int groups = DH * A.r / 8;
+    for (int gidx = t; gidx < groups; gidx += 96) {
+      const int row = gidx / (A.r / 8), g = gidx % (A.r / 8);
+      const uint4 v = *reinterpret_cast<const uint4 *>(Dsrc + (size_t)row * A.r + 8 * g);
+      // element order (0,4,1,5,2,6,3,7): 16-bit halves of the source words
+      const uint4 o = make_uint4(__byte_perm(v.x, v.z, 0x5410), __byte_perm(v.x, v.z, 0x7632),
+                                 __byte_perm(v.y, v.w, 0x5410), __byte_perm(v.y, v.w, 0x7632));
+      *reinterpret_cast<uint4 *>(sD + sw128_offset(row, 8 * g, DH)) = o;
+    }
+    fence_proxy_async_smem();
+  }
+  tc_fence_before();
+  __syncthreads();
+  cluster_sync();  // barriers of both CTAs initialised before any remote arrive
+  tc_fence_after();
+  const uint32_t tbase = B.tmem_base;
+
+  if (warp == 0) {
+    // ---------------- TMA producer ----------------
+    if (lane == 0) {
+      const CUtensorMap *tmC = rank == 0 ? &tmCk : &tmCv;
+      prefetch_tmap(&tmQ);
+      prefetch_tmap(tmC);
+      mbar_arrive_expect_tx(&B.q_full, kTile);
+      tma_load_2d(sQ, &tmQ, h * DH, (int)q0, &B.q_full);
+      tma_load_2d(sQ + kTile / 2, &tmQ, h * DH + 64, (int)q0, &B.q_full);
+      int issued = 0;
+      for (int c = 0; c < nchunk; ++c) {
+        const int slot = c % NSTAGE;
+        if (c >= NSTAGE && !mbar_wait(&B.st_empty[slot], ((c / NSTAGE) - 1) & 1, abort, err)) break;
+        const int j = c / nrb, cb = c % nrb;
+        mbar_arrive_expect_tx(&B.st_full[slot], kStage);
+        tma_load_2d(sStage + slot * kStage, tmC, cb * 32, (int)(A.t0 + (int64_t)j * BN), &B.st_full[slot]);
+        issued = c + 1;
+      }
+      mbar_wait(&B.q_full, 0, nullptr, nullptr);
+      for (int c = (issued > NSTAGE ? issued - NSTAGE : 0); c < issued; ++c)
+        mbar_wait(&B.st_full[c % NSTAGE], (c / NSTAGE) & 1, nullptr, nullptr);
+    }
+  } else if (warp == 1) {
+    // ---------------- MMA issuer ----------------
+    if (lane == 0) {
+      const uint32_t aQ = smem_u32(sQ), aD = smem_u32(sD), aR = smem_u32(sRing);
+      const uint32_t aK = smem_u32(sKh), aV = smem_u32(sVh);
+      int cc = 0;  // chunk counter
+      bool ok = mbar_wait(&B.q_full, 0, abort, err);
+      auto decode = [&](int j) -> bool {
+        const int xb = j & 1;
+        if (j >= 2 && !mbar_wait(&B.x_empty[xb], ((j >> 1) - 1) & 1, abort, err)) return false;
+        const uint32_t dX = tbase + TM_X + xb * 128;
+        for (int cb = 0; cb < nrb; ++cb, ++cc) {
+          const int slot = cc % NRING;
+          if (!mbar_wait(&B.ring_full[slot], (cc / NRING) & 1, abort, err)) return false;
+          tc_fence_after();
+          const uint32_t a = aR + slot * kChunk, b = aD + cb * kChunk;
+#pragma unroll
+          for (int k = 0; k < 4; ++k)
+            mma_ss(dX, sdesc_sw128(a + 32 * k, 16, 1024), sdesc_sw128(b + 32 * k, 16, 1024), IDESC_DEC,
+                   (cb > 0 || k > 0));
+          mma_commit(&B.ring_empty[slot]);
+        }
+        mma_commit(&B.x_full[xb]);
+        return true;
+      };
+      auto scores = [&](int j) -> bool {
+        if (!mbar_wait_cluster(&B.kh_full, j & 1, abort, err)) return false;
+        if (j > 0 && !mbar_wait(&B.pv_done, (j - 1) & 1, abort, err)) return false;
+        tc_fence_after();
+#pragma unroll
+        for (int ks = 0; ks < DH / 16; ++ks) {
+          const uint32_t off = (ks >> 2) * (kTile / 2) + (ks & 3) * 32;
+          mma_ss(tbase + TM_S, sdesc_sw128(aQ + off, 16, 1024), sdesc_sw128(aK + off, 16, 1024), IDESC_S,
+                 ks > 0);
+        }
+        mma_commit(&B.s_full);
+        mma_commit_mc(&B.kh_empty, 0x1);  // K_hat consumed here: tell the K decoder (CTA 0)
+        return true;
+      };
+      auto values = [&](int j) -> bool {
+        if (!mbar_wait(&B.p_full, j & 1, abort, err)) return false;
+        if (!mbar_wait_cluster(&B.vh_full, j & 1, abort, err)) return false;
+        tc_fence_after();
+#pragma unroll
+        for (int ks = 0; ks < BN / 16; ++ks)
+          mma_ts(tbase + TM_O, tbase + TM_S + ks * 8, sdesc_sw128(aV + ks * 2048, kTile / 2, 1024),
+                 IDESC_PV, (j > 0 || ks > 0));
+        mma_commit(&B.pv_done);
+        mma_commit_mc(&B.vh_empty, 0x2);  // V_hat consumed: tell the V decoder (CTA 1)
+        return true;
+      };
+      if (ok) ok = decode(0) && scores(0);
+      for (int j = 0; ok && j < ntiles; ++j) {
+        if (j + 1 < ntiles && !decode(j + 1)) break;
+        if (!values(j)) break;
+        if (j + 1 < ntiles && !scores(j + 1)) break;
+      }
+    }
+  } else if (warp == 2 || warp == 3) {
+    // ---------------- unpack: staging (packed) -> ring (bf16, K-major SW128) ----------------
+    const int u = (warp - 2) * 32 + lane;  // keys u and u + 64
+    for (int c = 0; c < nchunk; ++c) {
+      const int slot = c % NSTAGE, rs = c % NRING;
+      if (!mbar_wait(&B.st_full[slot], (c / NSTAGE) & 1, abort, err)) break;
+      const uint4 *src = reinterpret_cast<const uint4 *>(sStage + slot * kStage);
+      const uint4 p0 = src[2 * u], p1 = src[2 * u + 1];
+      const uint4 p2 = src[2 * (u + 64)], p3 = src[2 * (u + 64) + 1];
+      __syncwarp();
+      if (lane == 0) mbar_arrive(&B.st_empty[slot]);
+      if (c >= NRING && !mbar_wait(&B.ring_empty[rs], ((c / NRING) - 1) & 1, abort, err)) break;
+      uint8_t *dst = sRing + rs * kChunk;
+      const uint32_t w0[8] = {p0.x, p0.y, p0.z, p0.w, p1.x, p1.y, p1.z, p1.w};
+      const uint32_t w1[8] = {p2.x, p2.y, p2.z, p2.w, p3.x, p3.y, p3.z, p3.w};
+#pragma unroll
+      for (int g = 0; g < 8; ++g) {
+        *reinterpret_cast<uint4 *>(dst + sw128_offset(u, 8 * g, 128)) = unpack8(w0[g]);
+        *reinterpret_cast<uint4 *>(dst + sw128_offset(u + 64, 8 * g, 128)) = unpack8(w1[g]);
+      }
+      fence_proxy_async_smem();
+      __syncwarp();
+      if (lane == 0) mbar_arrive(&B.ring_full[rs]);
+    }
+  } else if (warp >= 4 && warp < 8) {
+    // ---------------- decode epilogue (thread = key) ----------------
+    const int t = (warp - 4) * 32 + lane;
+    const __nv_bfloat16 *cen = A.cen[rank] + (size_t)h * DH;
+    uint8_t *dstL = rank == 0 ? sKh : sVh;
+    const uint32_t dst_local = smem_u32(dstL);
+    const uint32_t dst_remote = mapa(dst_local, peer);
+    uint64_t *full_bar = rank == 0 ? &B.kh_full : &B.vh_full;
+    uint64_t *empty_bar = rank == 0 ? &B.kh_empty : &B.vh_empty;
+    const uint32_t full_local = mapa(smem_u32(full_bar), rank);
+    const uint32_t full_remote = mapa(smem_u32(full_bar), peer);
+    for (int j = 0; j < ntiles; ++j) {
+      const int64_t tt = A.t0 + (int64_t)j * BN + t;
+      const bool valid = (int64_t)j * BN + t < A.T;
+      int a = valid ? (int)A.ids[rank][tt] : 0;
+      a = a < A.C[rank] ? a : A.C[rank] - 1;
+      const float s = valid ? __half2float(A.scales[rank][tt]) : 0.f;
+      const __nv_bfloat16 *crow = cen + (size_t)a * J;
+      const int xb = j & 1;
+      if (!mbar_wait(&B.x_full[xb], (j >> 1) & 1, abort, err)) break;
+      if (j > 0 && !mbar_wait_cluster(empty_bar, (j - 1) & 1, abort, err)) break;
+      tc_fence_after();
+#pragma unroll 1
+      for (int c = 0; c < 4; ++c) {
+        uint32_t x[32];
+        tmem_ld32(tmem_lane_addr(tbase, warp, TM_X + xb * 128 + 32 * c), x);
+#pragma unroll
+        for (int g = 0; g < 4; ++g) {
+          const uint4 cv = *reinterpret_cast<const uint4 *>(crow + 32 * c + 8 * g);
+          const __nv_bfloat162 *c2 = reinterpret_cast<const __nv_bfloat162 *>(&cv);
+          uint32_t o[4];
+#pragma unroll
+          for (int i = 0; i < 4; ++i) {
+            const float2 cf = __bfloat1622float2(c2[i]);
+            o[i] = pack_bf16x2(fmaf(s, __uint_as_float(x[8 * g + 2 * i]), cf.x),
+                               fmaf(s, __uint_as_float(x[8 * g + 2 * i + 1]), cf.y));
+          }
+          const uint4 v = make_uint4(o[0], o[1], o[2], o[3]);
+          const uint32_t off = sw128_offset(t, 32 * c + 8 * g, 128);
+          st_shared_v4(dst_local + off, v);
+          st_cluster_v4(dst_remote + off, v);
+        }
+      }
+      fence_proxy_async_smem();
+      fence_proxy_async_cluster();
+      tc_fence_before();
+      __syncwarp();
+      if (lane == 0) {
+        mbar_arrive(&B.x_empty[xb]);
+        mbar_arrive_cluster(full_local);
+        mbar_arrive_cluster(full_remote);
+      }
+    }
+  } else if (warp >= 8) {
+    // ---------------- softmax (thread = query row) ----------------
+    const int row = (warp - 8) * 32 + lane;
+    RowState st{-INFINITY, 0.f};
+    bool ok = true;
+    for (int j = 0; j < ntiles; ++j) {
+      if (!mbar_wait(&B.s_full, j & 1, abort, err)) { ok = false; break; }
+      tc_fence_after();
+      const int64_t rem = A.T - (int64_t)j * BN;
+      const int nk = rem < BN ? (int)rem : BN;
+      bool wr;
+      const float corr = softmax_tile(tbase, warp, TM_S, nk, A.zscale, st, wr);
+      if (j > 0 && wr) {
+        if (!mbar_wait(&B.pv_done, (j - 1) & 1, abort, err)) { ok = false; break; }
+        tc_fence_after();
+        rescale_o(tbase, warp, TM_O, corr);
+      }
+      tc_fence_before();
+      __syncwarp();
+      if (lane == 0) mbar_arrive(&B.p_full);
+    }
+    if (ok && mbar_wait(&B.pv_done, (ntiles - 1) & 1, abort, err)) {
+      tc_fence_after();
+      write_row(tbase, warp, TM_O, st, q0 + row, A.Tq, h, A.H, A.O, A.L);
+    }
+  }
+  // the last consumer signals of the peer (multicast commits) must land
+  // before this CTA's shared memory goes away
+  if (threadIdx.x == 0) {
+    if (rank == 0) mbar_wait_cluster(&B.kh_empty, (ntiles - 1) & 1, nullptr, nullptr);
+    else mbar_wait_cluster(&B.vh_empty, (ntiles - 1) & 1, nullptr, nullptr);
+  }
+  tc_fence_before();
+  __syncthreads();
+  cluster_sync();
+  if (warp == 0) {
+    tc_fence_after();
+    tmem_dealloc(tbase, TM_COLS);
+  }
+}
+
+}  // namespace
+
+bool tc_full_supported(const Codec &ck, const Codec &cv) {
+  return ck.prec == PREC_BF16 && ck.d == DH && ck.r == cv.r && ck.r % 64 == 0 && ck.r <= 256;
+}
+
+size_t tc_full_smem(int r) {
+  return (size_t)3 * kTile + (size_t)(r / 64) * kChunk + NRING * kChunk + NSTAGE * kStage + 1024;
+}
+
+cudaError_t tc_attend_full(const void *q, int64_t Tq, const Codec &ck, const Codec &cv,
+                           const Hist &hk, const Hist &hv, int64_t t0, int64_t T, float tau,
+                           Part out, cudaStream_t st) {
+  if (Tq == 0 || T == 0) return cudaSuccess;
+  const int J = ck.H * DH;
+  const int64_t T_total = t0 + T;
+  CUtensorMap mq, mck, mcv;
+  if (!make_tmap_bf16_2d(&mq, q, Tq, J, J, 128) ||
+      !make_tmap_u8_2d(&mck, hk.codes, T_total, ck.r / 2, ck.r / 2, 32, 128) ||
+      !make_tmap_u8_2d(&mcv, hv.codes, T_total, cv.r / 2, cv.r / 2, 32, 128))
+    return cudaErrorInvalidValue;
+  FullArgs a;
+  a.D[0] = (const __nv_bfloat16 *)ck.D;
+  a.D[1] = (const __nv_bfloat16 *)cv.D;
+  a.cen[0] = (const __nv_bfloat16 *)ck.centers;
+  a.cen[1] = (const __nv_bfloat16 *)cv.centers;
+  a.ids[0] = hk.ids;
+  a.ids[1] = hv.ids;
+  a.scales[0] = (const __half *)hk.scales;
+  a.scales[1] = (const __half *)hv.scales;
+  a.t0 = t0;
+  a.T = T;
+  a.Tq = Tq;
+  a.H = ck.H;
+  a.r = ck.r;
+  a.C[0] = ck.C;
+  a.C[1] = cv.C;
+  a.zscale = tau * kLog2e;
+  a.O = out.O;
+  a.L = out.LSE;
+  a.err = error_word_ptr();
+  const size_t smem = tc_full_smem(ck.r);
+  cudaFuncSetAttribute(tc_full_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+  const unsigned qt = (unsigned)((Tq + BM - 1) / BM);
+  dim3 grid((qt + 1) & ~1u, (unsigned)ck.H);
+  tc_full_kernel<<<grid, 384, smem, st>>>(mq, mck, mcv, a);
+  return cudaGetLastError();
+}
+
+}  // namespace nanokv
