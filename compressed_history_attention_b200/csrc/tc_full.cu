@@ -329,13 +329,15 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(384, 1)
       write_row(tbase, warp, TM_O, st, q0 + row, A.Tq, h, A.H, A.O, A.L);
     }
   }
-  // the last consumer signals of the peer (multicast commits) must land
-  // before this CTA's shared memory goes away
-  if (threadIdx.x == 0) {
+  tc_fence_before();
+  __syncthreads();
+  // the peer's last consumer signals (multicast commits) must land before this
+  // CTA's shared memory goes away; after the block barrier the epilogue has
+  // waited every earlier phase, so this wait cannot see a stale parity
+  if (threadIdx.x == 0 && !*abort) {
     if (rank == 0) mbar_wait_cluster(&B.kh_empty, (ntiles - 1) & 1, nullptr, nullptr);
     else mbar_wait_cluster(&B.vh_empty, (ntiles - 1) & 1, nullptr, nullptr);
   }
-  tc_fence_before();
   __syncthreads();
   cluster_sync();
   if (warp == 0) {

@@ -139,7 +139,15 @@ def test_attend_peaked_softmax(path):
                             softmax_scale=1.0)
     torch.cuda.synchronize()
     Or, Lr = P.oracle_attend(w, prob, hk, hv, w.T_full, tau=1.0)
-    P.compare_attn(O, L, Or, Lr, False)
+    if path == "simt":
+        P.compare_attn(O, L, Or, Lr, False)
+    else:
+        # the tensor-core kernels round decoded K_hat/V_hat to bf16; with
+        # unit-variance queries and tau = 1 the scores have magnitude ~10 and
+        # each carries a rounding error of about 2^-9 * |q * k_hat|_2 ~ 0.02
+        # (three sigma ~ 0.06), so the bound is scaled to that, not to the
+        # workloads' near-uniform softmax
+        P.compare_attn(O, L, Or, Lr, False, tol=(0.15, 1.5e-2, 0.15))
 
 
 def test_lse_merge_parity():
