@@ -22,7 +22,8 @@ OK, ERR_INVALID, ERR_UNSUPPORTED, ERR_CUDA, ERR_TIMEOUT = 0, -1, -2, -3, -4
 
 SYMBOLS = ("nanokv_encode", "nanokv_attend", "nanokv_attend_workspace", "nanokv_lse_merge",
            "nanokv_set_kernel_path", "nanokv_check", "nanokv_last_error", "nanokv_version",
-           "nanokv_timing_enable", "nanokv_timing_read")
+           "nanokv_timing_enable", "nanokv_timing_read", "nanokv_codec_aux_bytes",
+           "nanokv_codec_prepare")
 
 # kernel identities of the diagnostics (nanokv_kernel_id)
 KERNELS = {0: "encode", 1: "attend_full", 2: "attend_low", 3: "attend_dense", 4: "lse_merge"}
@@ -39,7 +40,7 @@ class _Codec(ctypes.Structure):
     _fields_ = [("H", ctypes.c_int32), ("d", ctypes.c_int32), ("r", ctypes.c_int32),
                 ("C", ctypes.c_int32), ("param_dtype", ctypes.c_int32),
                 ("scale_dtype", ctypes.c_int32), ("centers", ctypes.c_void_p),
-                ("D", ctypes.c_void_p), ("E", ctypes.c_void_p)]
+                ("D", ctypes.c_void_p), ("E", ctypes.c_void_p), ("aux", ctypes.c_void_p)]
 
 
 class _Hist(ctypes.Structure):
@@ -76,6 +77,10 @@ def lib() -> ctypes.CDLL:
     L.nanokv_check.restype = ctypes.c_int
     L.nanokv_last_error.restype = ctypes.c_char_p
     L.nanokv_version.restype = ctypes.c_char_p
+    L.nanokv_codec_aux_bytes.argtypes = [P(_Codec)]
+    L.nanokv_codec_aux_bytes.restype = sz
+    L.nanokv_codec_prepare.argtypes = [P(_Codec), vp, vp]
+    L.nanokv_codec_prepare.restype = ctypes.c_int
     L.nanokv_timing_enable.argtypes = [i32]
     L.nanokv_timing_enable.restype = ctypes.c_int
     L.nanokv_timing_read.argtypes = [vp, vp]
@@ -107,6 +112,7 @@ class Codec:
     centers: torch.Tensor
     D: torch.Tensor
     E: torch.Tensor | None = None
+    aux: torch.Tensor | None = None
 
     @property
     def r(self) -> int:
@@ -128,7 +134,22 @@ class Codec:
         pd = F32 if self.fp32 else BF16
         sd = F32 if self.fp32 else F16
         return _Codec(self.H, self.d, self.r, self.C, pd, sd, self.centers.data_ptr(),
-                      self.D.data_ptr(), self.E.data_ptr() if self.E is not None else None)
+                      self.D.data_ptr(), self.E.data_ptr() if self.E is not None else None,
+                      self.aux.data_ptr() if self.aux is not None else None)
+
+    def prepare(self) -> "Codec":
+        """Computes the codec's derived encode tables once (nanokv_codec_prepare)
+        into a device buffer kept on this object."""
+        sc = self.struct()
+        sc.aux = None
+        n = int(lib().nanokv_codec_aux_bytes(ctypes.byref(sc)))
+        if n == 0:
+            _raise(ERR_INVALID)
+        aux = torch.empty(n, dtype=torch.uint8, device=self.centers.device)
+        _raise(lib().nanokv_codec_prepare(ctypes.byref(sc), ctypes.c_void_p(aux.data_ptr()),
+                                          _stream(self.centers.device)))
+        self.aux = aux
+        return self
 
 
 @dataclasses.dataclass
@@ -166,6 +187,9 @@ def nanokv_encode(ck: Codec | None, cv: Codec | None, k: torch.Tensor | None, v:
     x0 = k if k is not None else v
     T = x0.shape[0]
     dev = x0.device
+    for c in (ck, cv):
+        if c is not None and c.aux is None and c.E is not None:
+            c.prepare()
     if ck is not None and out_k is None:
         out_k = alloc_hist(ck, T, dev)
     if cv is not None and out_v is None:

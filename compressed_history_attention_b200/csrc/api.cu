@@ -113,7 +113,9 @@ static int check_codec(const nanokv_codec *c, const char *name, bool need_E, Cod
     return fail(NANOKV_ERR_INVALID, "%s: NULL parameter pointer", name);
   if (!aligned16(c->centers) || !aligned16(c->D) || (c->E && !aligned16(c->E)))
     return fail(NANOKV_ERR_INVALID, "%s: parameter pointers must be 16-byte aligned", name);
-  *out = Codec{c->H, c->d, c->r, c->C, prec, c->centers, c->D, c->E};
+  if (c->aux && !aligned16(c->aux))
+    return fail(NANOKV_ERR_INVALID, "%s: aux must be 16-byte aligned", name);
+  *out = Codec{c->H, c->d, c->r, c->C, prec, c->centers, c->D, c->E, c->aux};
   return NANOKV_OK;
 }
 
@@ -213,17 +215,43 @@ int nanokv_encode(const nanokv_codec *ck, const nanokv_codec *cv, const void *k,
   if (T == 0) return NANOKV_OK;
   cudaStream_t st = (cudaStream_t)stream;
   const int path = g_kernel_path.load();
+  bool tc_ok[2] = {false, false};
   for (int b = 0; b < 2; ++b) {
     if (!in[b]) continue;
-    const bool tc_ok = tc_encode_supported(c[b]);
-    if (path == 2 && !tc_ok) return fail(NANOKV_ERR_UNSUPPORTED, "encode: no tensor-core kernel for this shape");
+    tc_ok[b] = tc_encode_supported(c[b]);
+    if (path == 2 && !tc_ok[b])
+      return fail(NANOKV_ERR_UNSUPPORTED, "encode: no tensor-core kernel for this shape (or codec aux missing)");
+  }
+  // both branches in one tensor-core launch when their shapes agree
+  if (path != 1 && in[0] && in[1] && tc_ok[0] && tc_ok[1] && c[0].C == c[1].C && c[0].r == c[1].r) {
     cudaError_t e = timed(NANOKV_K_ENCODE, 1, st, [&] {
-      return (path != 1 && tc_ok) ? tc_encode(c[b], x[b], T, ids[b], codes[b], scales[b], st)
-                                  : simt_encode(c[b], x[b], T, ids[b], codes[b], scales[b], st);
+      return tc_encode_pair(c, x, T, ids, codes, scales, 2, st);
+    });
+    return cuda_status(e, "encode launch");
+  }
+  for (int b = 0; b < 2; ++b) {
+    if (!in[b]) continue;
+    cudaError_t e = timed(NANOKV_K_ENCODE, 1, st, [&] {
+      return (path != 1 && tc_ok[b]) ? tc_encode_pair(&c[b], &x[b], T, &ids[b], &codes[b], &scales[b], 1, st)
+                                     : simt_encode(c[b], x[b], T, ids[b], codes[b], scales[b], st);
     });
     if (e != cudaSuccess) return cuda_status(e, "encode launch");
   }
   return NANOKV_OK;
+}
+
+size_t nanokv_codec_aux_bytes(const nanokv_codec *c_) {
+  Codec c;
+  if (check_codec(c_, "codec", false, &c)) return 0;
+  return codec_aux_bytes(c);
+}
+
+int nanokv_codec_prepare(const nanokv_codec *c_, void *aux, void *stream) {
+  Codec c;
+  int s = check_codec(c_, "prepare", true, &c);
+  if (s) return s;
+  if (!aux || !aligned16(aux)) return fail(NANOKV_ERR_INVALID, "prepare: aux NULL or misaligned");
+  return cuda_status(codec_prepare(c, aux, (cudaStream_t)stream), "prepare launch");
 }
 
 size_t nanokv_attend_workspace(int64_t Tq, const nanokv_codec *ck, const nanokv_codec *cv,

@@ -47,6 +47,7 @@ struct Codec {
   int H, d, r, C;
   int prec;  // 0 = fp32 everywhere, 1 = bf16 params/io + fp16 scales
   const void *centers, *D, *E;
+  const void *aux;  // optional derived encode tables (E c_j, |c_j|^2)
 };
 struct Hist {
   const uint8_t *ids, *codes;

@@ -10,8 +10,11 @@ bool tc_full_supported(const Codec &ck, const Codec &cv);
 bool tc_low_supported(const Codec &ck, const Codec &cv);
 bool tc_dense_supported(int prec, int d);
 
-cudaError_t tc_encode(const Codec &c, const void *x, int64_t T, uint8_t *ids, uint8_t *codes,
-                      void *scales, cudaStream_t st);
+// encodes nbranch (1 or 2) branches with equal C and r in one launch
+cudaError_t tc_encode_pair(const Codec *c, const void *const *x, int64_t T, uint8_t *const *ids,
+                           uint8_t *const *codes, void *const *scales, int nbranch, cudaStream_t st);
+size_t codec_aux_bytes(const Codec &c);
+cudaError_t codec_prepare(const Codec &c, void *aux, cudaStream_t st);
 cudaError_t tc_attend_full(const void *q, int64_t Tq, const Codec &ck, const Codec &cv,
                            const Hist &hk, const Hist &hv, int64_t t0, int64_t T, float tau,
                            Part out, cudaStream_t st);

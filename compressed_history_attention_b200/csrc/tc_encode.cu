@@ -1,0 +1,310 @@
+// Tensor-core encode (NanoKV Fig. 4(b)): for 128 tokens x per CTA,
+//     G = x [C | E]^T           (one GEMM, N = C + r, fp32 in TMEM)
+//     a = argmin_j |c_j|^2 - 2 G[j]          (= argmin |x - c_j|^2)
+//     y = G[C + k] - (E c_a)[k]              (= E (x - c_a))
+//     s = fp16(max|y| / 7),  code = clamp(rint(y / s), -7, 7)
+// The tables E c_j and |c_j|^2 come from nanokv_codec_prepare.  Both
+// branches (K and V) run in one launch (grid.y).
+// The projection part of G is accumulated per 64-wide K block into one of two
+// TMEM buffers and the blocks are summed in fp32 registers by the epilogue,
+// so no fp32 accumulation chain is longer than one block on the tensor core;
+// the codes are decided on values as accurate as a plain fp32 dot product.
+//   warp 0      TMA: token tile and [centers | E] tile per 64-wide K block
+//   warp 1      MMA issuer
+//   warps 2,3   stage the E c table and |c|^2 into shared memory
+//   warps 4..7  epilogue, one thread per token (TMEM lane)
+#include "tc_common.cuh"
+
+namespace nanokv {
+
+using namespace sm100;
+using namespace tc;
+
+namespace {
+
+constexpr int NSTG = 3;
+constexpr uint32_t kA = 128 * 64 * 2;  // token tile [128 x 64] bf16
+
+struct EncArgs {
+  const float *aux[2];  // [C][r] E c_j, then [C] |c_j|^2
+  uint8_t *ids[2];
+  uint8_t *codes[2];
+  __half *scales[2];
+  int64_t T;
+  int J, r, C;
+  unsigned *err;
+};
+
+struct EncBars {
+  uint64_t full[NSTG], empty[NSTG], acc_full, part_full[2], part_empty[2];
+  uint32_t tmem_base;
+  int abort;
+};
+
+template <int R>
+__global__ void __launch_bounds__(256, 1)
+    tc_encode_kernel(const __grid_constant__ CUtensorMap tmX0, const __grid_constant__ CUtensorMap tmC0,
+                     const __grid_constant__ CUtensorMap tmE0, const __grid_constant__ CUtensorMap tmX1,
+                     const __grid_constant__ CUtensorMap tmC1, const __grid_constant__ CUtensorMap tmE1,
+                     const EncArgs A) {
+  extern __shared__ uint8_t smraw[];
+  uint8_t *sm = (uint8_t *)(((uintptr_t)smraw + 1023) & ~(uintptr_t)1023);
+  const int N = A.C + R;
+  const uint32_t kB = (uint32_t)N * 128;  // [N x 64] bf16
+  uint8_t *sA = sm;
+  uint8_t *sB = sA + NSTG * kA;
+  float *sEC = (float *)(sB + NSTG * kB);  // [C][r + 1]
+  float *sCN = sEC + A.C * (R + 1);        // [C]
+  __shared__ EncBars B;
+
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const int br = blockIdx.y;
+  const CUtensorMap *tmX = br ? &tmX1 : &tmX0;
+  const CUtensorMap *tmC = br ? &tmC1 : &tmC0;
+  const CUtensorMap *tmE = br ? &tmE1 : &tmE0;
+  const int64_t t0 = (int64_t)blockIdx.x * 128;
+  const int nkb = A.J / 64;
+  volatile int *abort = &B.abort;
+  unsigned *err = A.err;
+  const uint32_t tmem_cols = 512;  // [0, C) centers | [C, C + R) block buffer 0 | [C + R, C + 2R) buffer 1
+
+  if (threadIdx.x == 0) {
+    for (int i = 0; i < NSTG; ++i) { mbar_init(&B.full[i], 1); mbar_init(&B.empty[i], 1); }
+    mbar_init(&B.acc_full, 1);
+    for (int i = 0; i < 2; ++i) { mbar_init(&B.part_full[i], 1); mbar_init(&B.part_empty[i], 4); }
+    B.abort = 0;
+    fence_mbar_init();
+  }
+  if (warp == 0) {
+    tmem_alloc(&B.tmem_base, tmem_cols);
+    tmem_relinquish();
+  }
+  if (warp == 2 || warp == 3) {
+    const float *aux = A.aux[br];
+    const int n = A.C * R;
+    for (int i = (warp - 2) * 32 + lane; i < n; i += 64) sEC[(i / R) * (R + 1) + i % R] = aux[i];
+    for (int i = (warp - 2) * 32 + lane; i < A.C; i += 64) sCN[i] = aux[n + i];
+  }
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tbase = B.tmem_base;
+
+  if (warp == 0) {
+    if (lane == 0) {
+      prefetch_tmap(tmX);
+      prefetch_tmap(tmC);
+      prefetch_tmap(tmE);
+      int issued = 0;
+      for (int kb = 0; kb < nkb; ++kb) {
+        const int s = kb % NSTG;
+        if (kb >= NSTG && !mbar_wait(&B.empty[s], ((kb / NSTG) - 1) & 1, abort, err)) break;
+        mbar_arrive_expect_tx(&B.full[s], kA + kB);
+        tma_load_2d(sA + s * kA, tmX, kb * 64, (int)t0, &B.full[s]);
+        tma_load_2d(sB + s * kB, tmC, kb * 64, 0, &B.full[s]);
+        tma_load_2d(sB + s * kB + A.C * 128, tmE, kb * 64, 0, &B.full[s]);
+        issued = kb + 1;
+      }
+      for (int kb = (issued > NSTG ? issued - NSTG : 0); kb < issued; ++kb)
+        mbar_wait(&B.full[kb % NSTG], (kb / NSTG) & 1, nullptr, nullptr);
+    }
+  } else if (warp == 1) {
+    if (lane == 0) {
+      const uint32_t idc = idesc_bf16(128, A.C, false, false), ide = idesc_bf16(128, R, false, false);
+      bool ok = true;
+      for (int kb = 0; kb < nkb; ++kb) {
+        const int s = kb % NSTG, pb = kb & 1;
+        if (!mbar_wait(&B.full[s], (kb / NSTG) & 1, abort, err)) { ok = false; break; }
+        if (kb >= 2 && !mbar_wait(&B.part_empty[pb], ((kb >> 1) - 1) & 1, abort, err)) { ok = false; break; }
+        tc_fence_after();
+        const uint32_t a = smem_u32(sA + s * kA), b = smem_u32(sB + s * kB);
+        const uint32_t be = b + A.C * 128;
+#pragma unroll
+        for (int k = 0; k < 4; ++k) {
+          mma_ss(tbase, sdesc_sw128(a + 32 * k, 16, 1024), sdesc_sw128(b + 32 * k, 16, 1024), idc,
+                 (kb > 0 || k > 0));
+          mma_ss(tbase + A.C + pb * R, sdesc_sw128(a + 32 * k, 16, 1024), sdesc_sw128(be + 32 * k, 16, 1024),
+                 ide, k > 0);
+        }
+        mma_commit(&B.empty[s]);
+        mma_commit(&B.part_full[pb]);
+      }
+      if (ok) mma_commit(&B.acc_full);
+    }
+  } else if (warp >= 4) {
+    const int row = (warp - 4) * 32 + lane;
+    const int64_t t = t0 + row;
+    // E x, summed over K blocks in fp32
+    float y[R];
+#pragma unroll
+    for (int k = 0; k < R; ++k) y[k] = 0.f;
+    bool ok = true;
+    for (int kb = 0; kb < nkb; ++kb) {
+      const int pb = kb & 1;
+      if (!mbar_wait(&B.part_full[pb], (kb >> 1) & 1, abort, err)) { ok = false; break; }
+      tc_fence_after();
+      uint32_t g[32];
+#pragma unroll
+      for (int k0 = 0; k0 < R; k0 += 32) {
+        tmem_ld32(tmem_lane_addr(tbase, warp, A.C + pb * R + k0), g);
+#pragma unroll
+        for (int i = 0; i < 32; ++i) y[k0 + i] += __uint_as_float(g[i]);
+      }
+      tc_fence_before();
+      __syncwarp();
+      if (lane == 0) mbar_arrive(&B.part_empty[pb]);
+    }
+    if (ok && mbar_wait(&B.acc_full, 0, abort, err)) {
+      tc_fence_after();
+      uint32_t g[32];
+      // nearest center: argmin |c_j|^2 - 2 x.c_j, strict < keeps the lowest index
+      float best = INFINITY;
+      int a = 0;
+      for (int c0 = 0; c0 < A.C; c0 += 32) {
+        tmem_ld32(tmem_lane_addr(tbase, warp, c0), g);
+#pragma unroll
+        for (int i = 0; i < 32; ++i) {
+          if (c0 + i < A.C) {
+            const float sc = fmaf(-2.f, __uint_as_float(g[i]), sCN[c0 + i]);
+            if (sc < best) { best = sc; a = c0 + i; }
+          }
+        }
+      }
+      // y = E x - E c_a
+      const float *ec = sEC + a * (R + 1);
+      float m = 0.f;
+#pragma unroll
+      for (int k = 0; k < R; ++k) {
+        y[k] -= ec[k];
+        m = fmaxf(m, fabsf(y[k]));
+      }
+      const __half sh = __float2half_rn(m / 7.0f);
+      const float sf = __half2float(sh);
+      // INT4 codes, two per byte (code 2i in the low nibble)
+      uint8_t *crow = A.codes[br] + t * (R / 2);
+#pragma unroll
+      for (int k0 = 0; k0 < R; k0 += 32) {
+        uint32_t w[4];
+#pragma unroll
+        for (int q = 0; q < 4; ++q) {
+          uint32_t acc = 0;
+#pragma unroll
+          for (int i = 0; i < 8; ++i) {
+            int code = 0;
+            if (sf > 0.f) code = (int)fminf(7.f, fmaxf(-7.f, rintf(y[k0 + 8 * q + i] / sf)));
+            acc |= (uint32_t)(code & 0xF) << (4 * i);
+          }
+          w[q] = acc;
+        }
+        if (t < A.T) *reinterpret_cast<uint4 *>(crow + k0 / 2) = make_uint4(w[0], w[1], w[2], w[3]);
+      }
+      if (t < A.T) {
+        A.ids[br][t] = (uint8_t)a;
+        A.scales[br][t] = sh;
+      }
+    }
+  }
+  tc_fence_before();
+  __syncthreads();
+  if (warp == 0) {
+    tc_fence_after();
+    tmem_dealloc(tbase, tmem_cols);
+  }
+}
+
+// EC[j][k] = E[k] . c_j and |c_j|^2 in fp32: one warp per output
+template <typename TP>
+__global__ void codec_prepare_kernel(const TP *__restrict__ cen, const TP *__restrict__ E, int C, int r,
+                                     int J, float *__restrict__ aux) {
+  const int lane = threadIdx.x & 31;
+  const int64_t wid = ((int64_t)blockIdx.x * blockDim.x + threadIdx.x) >> 5;
+  const int64_t n = (int64_t)C * r + C;
+  if (wid >= n) return;
+  float acc = 0.f;
+  if (wid < (int64_t)C * r) {
+    const int j = (int)(wid / r), k = (int)(wid % r);
+    const TP *cr = cen + (size_t)j * J, *er = E + (size_t)k * J;
+    for (int i = lane; i < J; i += 32) acc = fmaf(to_f(er[i]), to_f(cr[i]), acc);
+  } else {
+    const TP *cr = cen + (size_t)(wid - (int64_t)C * r) * J;
+    for (int i = lane; i < J; i += 32) {
+      const float v = to_f(cr[i]);
+      acc = fmaf(v, v, acc);
+    }
+  }
+  acc = warp_sum(acc);
+  if (lane == 0) aux[wid] = acc;
+}
+
+}  // namespace
+
+size_t codec_aux_bytes(const Codec &c) {
+  return (((size_t)c.C * c.r + c.C) * sizeof(float) + 255) & ~(size_t)255;
+}
+
+cudaError_t codec_prepare(const Codec &c, void *aux, cudaStream_t st) {
+  const int64_t n = (int64_t)c.C * c.r + c.C;
+  const int threads = 256;
+  const int64_t blocks = (n * 32 + threads - 1) / threads;
+  if (c.prec == PREC_F32)
+    codec_prepare_kernel<float><<<(unsigned)blocks, threads, 0, st>>>(
+        (const float *)c.centers, (const float *)c.E, c.C, c.r, c.H * c.d, (float *)aux);
+  else
+    codec_prepare_kernel<__nv_bfloat16><<<(unsigned)blocks, threads, 0, st>>>(
+        (const __nv_bfloat16 *)c.centers, (const __nv_bfloat16 *)c.E, c.C, c.r, c.H * c.d, (float *)aux);
+  return cudaGetLastError();
+}
+
+bool tc_encode_supported(const Codec &c) {
+  return c.prec == PREC_BF16 && c.aux && (c.H * c.d) % 64 == 0 && (c.r == 64 || c.r == 128 || c.r == 192) &&
+         c.C % 16 == 0 && c.C <= 64;
+}
+
+static size_t enc_smem(const Codec &c) {
+  const size_t N = c.C + c.r;
+  return NSTG * (kA + N * 128) + ((size_t)c.C * (c.r + 1) + c.C) * sizeof(float) + 1024;
+}
+
+cudaError_t tc_encode_pair(const Codec *c, const void *const *x, int64_t T, uint8_t *const *ids,
+                           uint8_t *const *codes, void *const *scales, int nbranch, cudaStream_t st) {
+  if (T == 0) return cudaSuccess;
+  CUtensorMap m[2][3];
+  EncArgs a{};
+  const int J = c[0].H * c[0].d;
+  for (int b = 0; b < nbranch; ++b) {
+    if (!make_tmap_bf16_2d(&m[b][0], x[b], T, J, J, 128) ||
+        !make_tmap_bf16_2d(&m[b][1], c[b].centers, c[b].C, J, J, c[b].C) ||
+        !make_tmap_bf16_2d(&m[b][2], c[b].E, c[b].r, J, J, c[b].r))
+      return cudaErrorInvalidValue;
+    a.aux[b] = (const float *)c[b].aux;
+    a.ids[b] = ids[b];
+    a.codes[b] = codes[b];
+    a.scales[b] = (__half *)scales[b];
+  }
+  if (nbranch == 1) {
+    for (int i = 0; i < 3; ++i) m[1][i] = m[0][i];
+  }
+  a.T = T;
+  a.J = J;
+  a.r = c[0].r;
+  a.C = c[0].C;
+  a.err = error_word_ptr();
+  const size_t smem = enc_smem(c[0]);
+  dim3 grid((unsigned)((T + 127) / 128), (unsigned)nbranch);
+#define NANOKV_ENC_CASE(RR)                                                                         \
+  case RR:                                                                                          \
+    cudaFuncSetAttribute(tc_encode_kernel<RR>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem); \
+    tc_encode_kernel<RR><<<grid, 256, smem, st>>>(m[0][0], m[0][1], m[0][2], m[1][0], m[1][1], m[1][2], a); \
+    break;
+  switch (c[0].r) {
+    NANOKV_ENC_CASE(64)
+    NANOKV_ENC_CASE(128)
+    NANOKV_ENC_CASE(192)
+    default:
+      return cudaErrorInvalidValue;
+  }
+#undef NANOKV_ENC_CASE
+  return cudaGetLastError();
+}
+
+}  // namespace nanokv

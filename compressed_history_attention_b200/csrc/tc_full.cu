@@ -92,6 +92,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(384, 1)
   uint8_t *sKh = sRing + NRING * kChunk;
   uint8_t *sVh = sKh + kTile;
   uint8_t *sStage = sVh + kTile;
+  uint8_t *sCen = sStage + NSTAGE * kStage;  // this CTA's branch centers, head slice [C][128] bf16
   __shared__ FullBars B;
 
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
@@ -253,7 +254,18 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(384, 1)
   } else if (warp >= 4 && warp < 8) {
     // ---------------- decode epilogue (thread = key) ----------------
     const int t = (warp - 4) * 32 + lane;
-    const __nv_bfloat16 *cen = A.cen[rank] + (size_t)h * DH;
+    const int C = A.C[rank];
+    // head slice of the centers, 16-byte chunk k of row a stored at chunk
+    // (k ^ (a & 15)) so that rows read together spread over the banks
+    {
+      const __nv_bfloat16 *cen = A.cen[rank] + (size_t)h * DH;
+      for (int i = t; i < C * 16; i += 128) {
+        const int a = i >> 4, k = i & 15;
+        *reinterpret_cast<uint4 *>(sCen + a * 256 + ((k ^ (a & 15)) << 4)) =
+            *reinterpret_cast<const uint4 *>(cen + (size_t)a * J + 8 * k);
+      }
+      asm volatile("bar.sync 1, 128;" ::: "memory");
+    }
     uint8_t *dstL = rank == 0 ? sKh : sVh;
     const uint32_t dst_local = smem_u32(dstL);
     const uint32_t dst_remote = mapa(dst_local, peer);
@@ -261,13 +273,22 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(384, 1)
     uint64_t *empty_bar = rank == 0 ? &B.kh_empty : &B.vh_empty;
     const uint32_t full_local = mapa(smem_u32(full_bar), rank);
     const uint32_t full_remote = mapa(smem_u32(full_bar), peer);
-    for (int j = 0; j < ntiles; ++j) {
+    auto key_meta = [&](int j, int &a, float &s) {
       const int64_t tt = A.t0 + (int64_t)j * BN + t;
       const bool valid = (int64_t)j * BN + t < A.T;
-      int a = valid ? (int)A.ids[rank][tt] : 0;
-      a = a < A.C[rank] ? a : A.C[rank] - 1;
-      const float s = valid ? __half2float(A.scales[rank][tt]) : 0.f;
-      const __nv_bfloat16 *crow = cen + (size_t)a * J;
+      a = valid ? (int)A.ids[rank][tt] : 0;
+      a = a < C ? a : C - 1;
+      s = valid ? __half2float(A.scales[rank][tt]) : 0.f;
+    };
+    int a_next;
+    float s_next;
+    key_meta(0, a_next, s_next);
+    for (int j = 0; j < ntiles; ++j) {
+      const int a = a_next;
+      const float s = s_next;
+      if (j + 1 < ntiles) key_meta(j + 1, a_next, s_next);
+      const uint8_t *crow = sCen + a * 256;
+      const int sw = a & 15;
       const int xb = j & 1;
       if (!mbar_wait(&B.x_full[xb], (j >> 1) & 1, abort, err)) break;
       if (j > 0 && !mbar_wait_cluster(empty_bar, (j - 1) & 1, abort, err)) break;
@@ -278,7 +299,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(384, 1)
         tmem_ld32(tmem_lane_addr(tbase, warp, TM_X + xb * 128 + 32 * c), x);
 #pragma unroll
         for (int g = 0; g < 4; ++g) {
-          const uint4 cv = *reinterpret_cast<const uint4 *>(crow + 32 * c + 8 * g);
+          const uint4 cv = *reinterpret_cast<const uint4 *>(crow + (((4 * c + g) ^ sw) << 4));
           const __nv_bfloat162 *c2 = reinterpret_cast<const __nv_bfloat162 *>(&cv);
           uint32_t o[4];
 #pragma unroll
@@ -349,11 +370,14 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(384, 1)
 }  // namespace
 
 bool tc_full_supported(const Codec &ck, const Codec &cv) {
-  return ck.prec == PREC_BF16 && ck.d == DH && ck.r == cv.r && ck.r % 64 == 0 && ck.r <= 256;
+  // shared memory: r <= 192 with up to 64 centers (r = 256 leaves no room for the center slice)
+  return ck.prec == PREC_BF16 && ck.d == DH && ck.r == cv.r && ck.r % 64 == 0 && ck.r <= 192 &&
+         ck.C <= 64 && cv.C <= 64;
 }
 
-size_t tc_full_smem(int r) {
-  return (size_t)3 * kTile + (size_t)(r / 64) * kChunk + NRING * kChunk + NSTAGE * kStage + 1024;
+size_t tc_full_smem(int r, int C) {
+  return (size_t)3 * kTile + (size_t)(r / 64) * kChunk + NRING * kChunk + NSTAGE * kStage + (size_t)C * 256 +
+         1024;
 }
 
 cudaError_t tc_attend_full(const void *q, int64_t Tq, const Codec &ck, const Codec &cv,
@@ -387,7 +411,7 @@ cudaError_t tc_attend_full(const void *q, int64_t Tq, const Codec &ck, const Cod
   a.O = out.O;
   a.L = out.LSE;
   a.err = error_word_ptr();
-  const size_t smem = tc_full_smem(ck.r);
+  const size_t smem = tc_full_smem(ck.r, ck.C > cv.C ? ck.C : cv.C);
   cudaFuncSetAttribute(tc_full_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
   const unsigned qt = (unsigned)((Tq + BM - 1) / BM);
   dim3 grid((qt + 1) & ~1u, (unsigned)ck.H);

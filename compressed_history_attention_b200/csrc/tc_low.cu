@@ -1,0 +1,489 @@
+// Tensor-core mixed-dimensional attention over the history a fixed policy
+// routes to low dimension (NanoKV-Fast; abstract: reuse the stored
+// coefficients; Fig. 4(d): reduce the queries, restore the output dimension).
+// Per head h, with D_h the head's rows of D and c_{j,h} its slice of center j:
+//   prologue   Q~ = Q D_{K,h}  [128 x r],  QC = Q C_{K,h}^T  [128 x C]   (MMA)
+//   per tile   S' = Q~ codes_K^T                                      (MMA)
+//              z  = tau (s_K S' + QC[a_K])          (softmax warps, log2 units)
+//              O~ += (P * s_V) codes_V,   P_C += P onehot(a_V)        (MMA)
+//   epilogue   O  = (O~ D_{V,h}^T + P_C C_{V,h}) / l                  (MMA)
+// P and P * s_V are written back to TMEM as bf16, interleaved per 32 keys.
+// Codes are unpacked in the order (0,4,1,5,2,6,3,7) within each group of 8;
+// Q~ is stored with the same order and O~ is un-permuted before the restore.
+//   warp 0      TMA: Q, D_{K,h}, C_{K,h}; later D_{V,h}, C_{V,h}
+//   warp 1      MMA issuer
+//   warps 4..7  unpack: thread = key; K codes, V codes, one-hot of a_V
+//   warps 8..11 softmax, one thread per query row; prologue/epilogue stores
+#include "tc_common.cuh"
+
+namespace nanokv {
+
+using namespace sm100;
+using namespace tc;
+
+namespace {
+
+constexpr int DH = 128;
+constexpr uint32_t kBlk = 128 * 64 * 2;  // [128 rows x 64] bf16 block
+constexpr uint32_t TM_OT = 0, TM_S0 = 256, TM_COLS = 512;
+
+struct LowArgs {
+  const __nv_bfloat16 *Dk, *Dv;   // decoders [J, r]
+  const __nv_bfloat16 *Ck, *Cv;   // centers [C, J]
+  const uint8_t *idk, *idv;       // [T]
+  const uint8_t *codk, *codv;     // [T, r/2]
+  const __half *sk, *sv;          // [T]
+  int64_t t0, T, Tq;
+  int H, r, C;
+  float zscale;
+  float *O, *L;
+  unsigned *err;
+};
+
+struct KeyInfo {
+  float sK;  // key scale
+  int aK;    // key center id
+  float sV;  // value scale
+};
+
+struct LowBars {
+  uint64_t pro_full, pro_done, qt_ready;
+  uint64_t kc_full, kc_empty, vc_full, v_empty;
+  uint64_t s_full[2], p_full[2], info_full[2], pv_done, last_done;
+  uint64_t fin_a, fin_b, fin_done;
+  uint32_t tmem_base;
+  int abort;
+};
+
+__device__ __forceinline__ uint4 unpack8(uint32_t w) {
+  const __nv_bfloat162 bias = __floats2bfloat162_rn(136.f, 136.f);
+  uint32_t o[4];
+#pragma unroll
+  for (int i = 0; i < 4; ++i) {
+    const uint32_t b = ((w >> (4 * i)) & 0x000F000Fu) ^ 0x43084308u;
+    __nv_bfloat162 v = __hsub2(*reinterpret_cast<const __nv_bfloat162 *>(&b), bias);
+    o[i] = *reinterpret_cast<uint32_t *>(&v);
+  }
+  return make_uint4(o[0], o[1], o[2], o[3]);
+}
+
+// multiplies `ncols` (multiple of 16) fp32 TMEM columns of this thread's row by f
+__device__ __forceinline__ void rescale_cols(uint32_t tbase, int warp, uint32_t col, int ncols, float f) {
+  uint32_t v[16];
+  for (int c = 0; c < ncols; c += 16) {
+    const uint32_t a = tmem_lane_addr(tbase, warp, col + c);
+    tmem_ld16(a, v);
+#pragma unroll
+    for (int i = 0; i < 16; ++i) v[i] = __float_as_uint(__uint_as_float(v[i]) * f);
+    tmem_st16(a, v);
+  }
+  tmem_st_wait();
+}
+
+__global__ void __launch_bounds__(384, 1)
+    tc_low_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUtensorMap tmDk,
+                  const __grid_constant__ CUtensorMap tmCk, const __grid_constant__ CUtensorMap tmDv,
+                  const __grid_constant__ CUtensorMap tmCv, const LowArgs A) {
+  extern __shared__ uint8_t smraw[];
+  uint8_t *sm = (uint8_t *)(((uintptr_t)smraw + 1023) & ~(uintptr_t)1023);
+  const int r = A.r, C = A.C;
+  const int nrb = r / 64;
+  uint8_t *sQt = sm;                           // [128 x r] K-major (persistent)
+  uint8_t *sKc = sQt + nrb * kBlk;             // [128 keys x r] K-major
+  uint8_t *sVc = sKc + nrb * kBlk;             // [128 keys x r] (MN-major use)
+  uint8_t *sOH = sVc + nrb * kBlk;             // [128 keys x C] one-hot
+  float *sQC = (float *)(sOH + kBlk);          // [128][C + 1]
+  KeyInfo *kinfo = (KeyInfo *)(sQC + 128 * (C + 1));  // [2][128]
+  // prologue aliases (inside sKc .. sOH)
+  uint8_t *sQ = sKc;                           // [128 x 128] K-major
+  uint8_t *sDk = sKc + 2 * kBlk;               // D_{K,h} [128 d x r] (MN-major use)
+  uint8_t *sCk = sDk + nrb * kBlk;             // C_{K,h} [C x 128] K-major (2 blocks of C*128 B)
+  // epilogue aliases
+  uint8_t *sAo = sKc;                          // O~ / l  [128 x r] K-major
+  uint8_t *sAp = sOH;                          // P_C / l [128 x C] K-major
+  uint8_t *sDv = sVc;                          // D_{V,h} [128 d x r] K-major
+  uint8_t *sCv = sQt;                          // C_{V,h} [C x 128] (MN-major use)
+  __shared__ LowBars B;
+
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const int h = blockIdx.y;
+  const int64_t q0 = (int64_t)blockIdx.x * BM;
+  const int ntiles = (int)((A.T + BN - 1) / BN);
+  volatile int *abort = &B.abort;
+  unsigned *err = A.err;
+  const uint32_t cblk = (uint32_t)C * 128;  // bytes of one [C rows x 64] block
+
+  if (threadIdx.x == 0) {
+    mbar_init(&B.pro_full, 1);
+    mbar_init(&B.pro_done, 1);
+    mbar_init(&B.qt_ready, 4);
+    mbar_init(&B.kc_full, 4);
+    mbar_init(&B.kc_empty, 1);
+    mbar_init(&B.vc_full, 4);
+    mbar_init(&B.v_empty, 1);
+    mbar_init(&B.s_full[0], 1);
+    mbar_init(&B.s_full[1], 1);
+    mbar_init(&B.p_full[0], 4);
+    mbar_init(&B.p_full[1], 4);
+    mbar_init(&B.info_full[0], 4);
+    mbar_init(&B.info_full[1], 4);
+    mbar_init(&B.pv_done, 1);
+    mbar_init(&B.last_done, 1);
+    mbar_init(&B.fin_a, 4);
+    mbar_init(&B.fin_b, 1);
+    mbar_init(&B.fin_done, 1);
+    B.abort = 0;
+    fence_mbar_init();
+  }
+  if (warp == 0) {
+    tmem_alloc(&B.tmem_base, TM_COLS);
+    tmem_relinquish();
+  }
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tbase = B.tmem_base;
+
+  if (warp == 0) {
+    // ---------------- TMA producer ----------------
+    if (lane == 0) {
+      mbar_arrive_expect_tx(&B.pro_full, 2 * kBlk + nrb * kBlk + 2 * cblk);
+      tma_load_2d(sQ, &tmQ, h * DH, (int)q0, &B.pro_full);
+      tma_load_2d(sQ + kBlk, &tmQ, h * DH + 64, (int)q0, &B.pro_full);
+      for (int b = 0; b < nrb; ++b) tma_load_2d(sDk + b * kBlk, &tmDk, 64 * b, h * DH, &B.pro_full);
+      for (int b = 0; b < 2; ++b) tma_load_2d(sCk + b * cblk, &tmCk, h * DH + 64 * b, 0, &B.pro_full);
+      bool ok = mbar_wait(&B.pro_full, 0, abort, err);
+      // restore operands once every tile's MMAs are done
+      if (ok && mbar_wait(&B.last_done, 0, abort, err)) {
+        mbar_arrive_expect_tx(&B.fin_b, nrb * kBlk + 2 * cblk);
+        for (int b = 0; b < nrb; ++b) tma_load_2d(sDv + b * kBlk, &tmDv, 64 * b, h * DH, &B.fin_b);
+        for (int b = 0; b < 2; ++b) tma_load_2d(sCv + b * cblk, &tmCv, h * DH + 64 * b, 0, &B.fin_b);
+        mbar_wait(&B.fin_b, 0, nullptr, nullptr);
+      }
+    }
+  } else if (warp == 1) {
+    // ---------------- MMA issuer ----------------
+    if (lane == 0) {
+      const uint32_t aQ = smem_u32(sQ), aDk = smem_u32(sDk), aCk = smem_u32(sCk);
+      const uint32_t aQt = smem_u32(sQt), aK = smem_u32(sKc), aV = smem_u32(sVc), aOH = smem_u32(sOH);
+      bool ok = mbar_wait(&B.pro_full, 0, abort, err);
+      if (ok) {
+        tc_fence_after();
+        // Q~ = Q D_{K,h} (B: N = r contiguous -> MN-major); QC = Q C_{K,h}^T (B K-major)
+#pragma unroll
+        for (int ks = 0; ks < DH / 16; ++ks) {
+          const uint32_t offA = (ks >> 2) * kBlk + (ks & 3) * 32;
+          mma_ss(tbase + TM_OT, sdesc_sw128(aQ + offA, 16, 1024), sdesc_sw128(aDk + ks * 2048, kBlk, 1024),
+                 idesc_bf16(128, r, false, true), ks > 0);
+          mma_ss(tbase + TM_OT + r, sdesc_sw128(aQ + offA, 16, 1024),
+                 sdesc_sw128(aCk + (ks >> 2) * cblk + (ks & 3) * 32, 16, 1024), idesc_bf16(128, C, false, false),
+                 ks > 0);
+        }
+        mma_commit(&B.pro_done);
+        ok = mbar_wait(&B.qt_ready, 0, abort, err);
+      }
+      auto scores = [&](int j) -> bool {
+        if (!mbar_wait(&B.kc_full, j & 1, abort, err)) return false;
+        if (j >= 2 && !mbar_wait(&B.pv_done, (j - 2) & 1, abort, err)) return false;
+        tc_fence_after();
+        const uint32_t dS = tbase + TM_S0 + (j & 1) * 128;
+        for (int ks = 0; ks < r / 16; ++ks) {
+          const uint32_t off = (ks >> 2) * kBlk + (ks & 3) * 32;
+          mma_ss(dS, sdesc_sw128(aQt + off, 16, 1024), sdesc_sw128(aK + off, 16, 1024),
+                 idesc_bf16(128, 128, false, false), ks > 0);
+        }
+        mma_commit(&B.s_full[j & 1]);
+        mma_commit(&B.kc_empty);
+        return true;
+      };
+      if (ok) ok = scores(0);
+      if (ok && ntiles > 1) ok = scores(1);
+      for (int j = 0; ok && j < ntiles; ++j) {
+        if (!mbar_wait(&B.p_full[j & 1], (j >> 1) & 1, abort, err)) { ok = false; break; }
+        if (!mbar_wait(&B.vc_full, j & 1, abort, err)) { ok = false; break; }
+        tc_fence_after();
+        const uint32_t sb = tbase + TM_S0 + (j & 1) * 128;
+#pragma unroll
+        for (int ks = 0; ks < BN / 16; ++ks) {
+          const uint32_t pc = sb + 32 * (ks >> 1) + 8 * (ks & 1);
+          const uint32_t acc = (j > 0 || ks > 0);
+          mma_ts(tbase + TM_OT, pc + 16, sdesc_sw128(aV + ks * 2048, kBlk, 1024), idesc_bf16(128, r, false, true),
+                 acc);
+          mma_ts(tbase + TM_OT + r, pc, sdesc_sw128(aOH + ks * 2048, kBlk, 1024), idesc_bf16(128, C, false, true),
+                 acc);
+        }
+        mma_commit(&B.pv_done);
+        mma_commit(&B.v_empty);
+        if (j + 2 < ntiles && !scores(j + 2)) { ok = false; break; }
+      }
+      if (ok) mma_commit(&B.last_done);
+      // restore: O = [O~/l | P_C/l] [D_{V,h} | C_{V,h}^T]^T
+      if (ok && mbar_wait(&B.fin_a, 0, abort, err) && mbar_wait(&B.fin_b, 0, abort, err)) {
+        tc_fence_after();
+        const uint32_t aAo = smem_u32(sAo), aAp = smem_u32(sAp), aDv = smem_u32(sDv), aCv = smem_u32(sCv);
+        for (int ks = 0; ks < r / 16; ++ks) {
+          const uint32_t off = (ks >> 2) * kBlk + (ks & 3) * 32;
+          mma_ss(tbase + TM_S0, sdesc_sw128(aAo + off, 16, 1024), sdesc_sw128(aDv + off, 16, 1024),
+                 idesc_bf16(128, 128, false, false), ks > 0);
+        }
+        for (int ks = 0; ks < C / 16; ++ks) {
+          mma_ss(tbase + TM_S0, sdesc_sw128(aAp + (ks & 3) * 32, 16, 1024),
+                 sdesc_sw128(aCv + ks * 2048, cblk, 1024), idesc_bf16(128, 128, false, true), 1);
+        }
+        mma_commit(&B.fin_done);
+      }
+    }
+  } else if (warp >= 4 && warp < 8) {
+    // ---------------- unpack (thread = key) ----------------
+    const int t = (warp - 4) * 32 + lane;
+    const int cw = r / 32;  // uint4 words of packed codes per key
+    bool ok = mbar_wait(&B.pro_done, 0, abort, err);  // prologue buffers alias the tiles
+    for (int j = 0; ok && j < ntiles; ++j) {
+      const int64_t tt = A.t0 + (int64_t)j * BN + t;
+      const bool valid = (int64_t)j * BN + t < A.T;
+      int ak = valid ? (int)A.idk[tt] : 0, av = valid ? (int)A.idv[tt] : 0;
+      ak = ak < C ? ak : C - 1;
+      av = av < C ? av : C - 1;
+      const float sk = valid ? __half2float(A.sk[tt]) : 0.f;
+      const float sv = valid ? __half2float(A.sv[tt]) : 0.f;
+      const uint4 *pk = reinterpret_cast<const uint4 *>(A.codk + tt * (r / 2));
+      const uint4 *pv = reinterpret_cast<const uint4 *>(A.codv + tt * (r / 2));
+      // ---- K codes
+      // (kinfo[j & 1] was last read by the softmax of tile j - 2, which finished
+      // before PV of tile j - 2, which the V part of tile j - 1 waited for)
+      if (j >= 1 && !mbar_wait(&B.kc_empty, (j - 1) & 1, abort, err)) break;
+      for (int q = 0; q < cw; ++q) {
+        const uint4 v = valid ? pk[q] : make_uint4(0, 0, 0, 0);
+        const uint32_t w[4] = {v.x, v.y, v.z, v.w};
+#pragma unroll
+        for (int i = 0; i < 4; ++i)
+          *reinterpret_cast<uint4 *>(sKc + sw128_offset(t, 32 * q + 8 * i, 128)) = unpack8(w[i]);
+      }
+      kinfo[(j & 1) * 128 + t] = KeyInfo{sk, ak, sv};
+      fence_proxy_async_smem();
+      __syncwarp();
+      if (lane == 0) {
+        mbar_arrive(&B.kc_full);
+        mbar_arrive(&B.info_full[j & 1]);
+      }
+      // ---- V codes and one-hot of the value center
+      if (j >= 1 && !mbar_wait(&B.v_empty, (j - 1) & 1, abort, err)) break;
+      for (int q = 0; q < cw; ++q) {
+        const uint4 v = valid ? pv[q] : make_uint4(0, 0, 0, 0);
+        const uint32_t w[4] = {v.x, v.y, v.z, v.w};
+#pragma unroll
+        for (int i = 0; i < 4; ++i)
+          *reinterpret_cast<uint4 *>(sVc + sw128_offset(t, 32 * q + 8 * i, 128)) = unpack8(w[i]);
+      }
+      for (int g = 0; g < C / 8; ++g) {
+        uint4 z = make_uint4(0, 0, 0, 0);
+        if (valid && (av >> 3) == g) {
+          const uint32_t one = 0x3F80u << (16 * (av & 1));  // bf16 1.0 in the right half
+          const int wsel = (av & 7) >> 1;
+          if (wsel == 0) z.x = one;
+          else if (wsel == 1) z.y = one;
+          else if (wsel == 2) z.z = one;
+          else z.w = one;
+        }
+        *reinterpret_cast<uint4 *>(sOH + sw128_offset(t, 8 * g, 128)) = z;
+      }
+      fence_proxy_async_smem();
+      __syncwarp();
+      if (lane == 0) mbar_arrive(&B.vc_full);
+    }
+  } else if (warp >= 8) {
+    // ---------------- softmax (thread = query row) ----------------
+    const int row = (warp - 8) * 32 + lane;
+    const float zs = A.zscale;
+    bool ok = mbar_wait(&B.pro_done, 0, abort, err);
+    if (ok) {
+      tc_fence_after();
+      uint32_t v[32];
+      // Q~ * tau*log2e -> bf16, stored in the unpack order of the codes
+      for (int c0 = 0; c0 < r; c0 += 32) {
+        tmem_ld32(tmem_lane_addr(tbase, warp, TM_OT + c0), v);
+#pragma unroll
+        for (int g = 0; g < 4; ++g) {
+          const float *f = reinterpret_cast<const float *>(v + 8 * g);
+          const uint4 o = make_uint4(pack_bf16x2(f[0] * zs, f[4] * zs), pack_bf16x2(f[1] * zs, f[5] * zs),
+                                     pack_bf16x2(f[2] * zs, f[6] * zs), pack_bf16x2(f[3] * zs, f[7] * zs));
+          *reinterpret_cast<uint4 *>(sQt + sw128_offset(row, c0 + 8 * g, 128)) = o;
+        }
+      }
+      for (int c0 = 0; c0 < C; c0 += 16) {
+        uint32_t u[16];
+        tmem_ld16(tmem_lane_addr(tbase, warp, TM_OT + r + c0), u);
+#pragma unroll
+        for (int i = 0; i < 16; ++i) sQC[row * (C + 1) + c0 + i] = __uint_as_float(u[i]) * zs;
+      }
+      fence_proxy_async_smem();
+      tc_fence_before();
+      __syncwarp();
+      if (lane == 0) mbar_arrive(&B.qt_ready);
+    }
+    const float *qc = sQC + row * (C + 1);
+    RowState st{-INFINITY, 0.f};
+    for (int j = 0; ok && j < ntiles; ++j) {
+      if (!mbar_wait(&B.s_full[j & 1], (j >> 1) & 1, abort, err)) { ok = false; break; }
+      if (!mbar_wait(&B.info_full[j & 1], (j >> 1) & 1, abort, err)) { ok = false; break; }
+      tc_fence_after();
+      const uint32_t sb = TM_S0 + (j & 1) * 128;
+      const KeyInfo *ki = kinfo + (j & 1) * 128;
+      const int64_t rem = A.T - (int64_t)j * BN;
+      const int nk = rem < BN ? (int)rem : BN;
+      uint32_t v[32];
+      float mx = -INFINITY;
+      for (int c = 0; c < 4; ++c) {
+        tmem_ld32(tmem_lane_addr(tbase, warp, sb + 32 * c), v);
+#pragma unroll
+        for (int i = 0; i < 32; ++i) {
+          const KeyInfo k = ki[32 * c + i];
+          const float z = fmaf(__uint_as_float(v[i]), k.sK, qc[k.aK]);
+          mx = (32 * c + i < nk) ? fmaxf(mx, z) : mx;
+        }
+      }
+      float corr = 1.f;
+      const bool need = mx > st.m + kRescaleLog2;
+      if (need) {
+        corr = (st.m == -INFINITY) ? 0.f : ex2(st.m - mx);
+        st.l *= corr;
+        st.m = mx;
+      }
+      const bool wr = __any_sync(0xffffffffu, need) != 0;
+      const float m = st.m;
+      float lsum = 0.f;
+      for (int c = 0; c < 4; ++c) {
+        tmem_ld32(tmem_lane_addr(tbase, warp, sb + 32 * c), v);
+        uint32_t pp[16], ps[16];
+#pragma unroll
+        for (int i = 0; i < 16; ++i) {
+          const int k0 = 32 * c + 2 * i;
+          const KeyInfo a = ki[k0], b = ki[k0 + 1];
+          const float p0 = (k0 < nk) ? ex2(fmaf(__uint_as_float(v[2 * i]), a.sK, qc[a.aK]) - m) : 0.f;
+          const float p1 = (k0 + 1 < nk) ? ex2(fmaf(__uint_as_float(v[2 * i + 1]), b.sK, qc[b.aK]) - m) : 0.f;
+          lsum += p0 + p1;
+          pp[i] = pack_bf16x2(p0, p1);
+          ps[i] = pack_bf16x2(p0 * a.sV, p1 * b.sV);
+        }
+        tmem_st16(tmem_lane_addr(tbase, warp, sb + 32 * c), pp);
+        tmem_st16(tmem_lane_addr(tbase, warp, sb + 32 * c + 16), ps);
+      }
+      tmem_st_wait();
+      st.l += lsum;
+      if (j > 0 && wr) {
+        if (!mbar_wait(&B.pv_done, (j - 1) & 1, abort, err)) { ok = false; break; }
+        tc_fence_after();
+        rescale_cols(tbase, warp, TM_OT, r + C, corr);
+      }
+      tc_fence_before();
+      __syncwarp();
+      if (lane == 0) mbar_arrive(&B.p_full[j & 1]);
+    }
+    // restore operands: [O~ | P_C] / l in bf16 (O~ un-permuted)
+    if (ok && mbar_wait(&B.last_done, 0, abort, err)) {
+      tc_fence_after();
+      const float inv = st.l > 0.f ? 1.f / st.l : 0.f;
+      uint32_t v[32];
+      for (int c0 = 0; c0 < r; c0 += 32) {
+        tmem_ld32(tmem_lane_addr(tbase, warp, TM_OT + c0), v);
+#pragma unroll
+        for (int g = 0; g < 4; ++g) {
+          // stored position p holds code (0,4,1,5,2,6,3,7)[p]
+          const float *f = reinterpret_cast<const float *>(v + 8 * g);
+          const uint4 o = make_uint4(pack_bf16x2(f[0] * inv, f[2] * inv), pack_bf16x2(f[4] * inv, f[6] * inv),
+                                     pack_bf16x2(f[1] * inv, f[3] * inv), pack_bf16x2(f[5] * inv, f[7] * inv));
+          *reinterpret_cast<uint4 *>(sAo + sw128_offset(row, c0 + 8 * g, 128)) = o;
+        }
+      }
+      for (int c0 = 0; c0 < C; c0 += 16) {
+        uint32_t u[16];
+        tmem_ld16(tmem_lane_addr(tbase, warp, TM_OT + r + c0), u);
+#pragma unroll
+        for (int g = 0; g < 2; ++g) {
+          const float *f = reinterpret_cast<const float *>(u + 8 * g);
+          const uint4 o = make_uint4(pack_bf16x2(f[0] * inv, f[1] * inv), pack_bf16x2(f[2] * inv, f[3] * inv),
+                                     pack_bf16x2(f[4] * inv, f[5] * inv), pack_bf16x2(f[6] * inv, f[7] * inv));
+          *reinterpret_cast<uint4 *>(sAp + sw128_offset(row, c0 + 8 * g, 128)) = o;
+        }
+      }
+      fence_proxy_async_smem();
+      tc_fence_before();
+      __syncwarp();
+      if (lane == 0) mbar_arrive(&B.fin_a);
+      if (mbar_wait(&B.fin_done, 0, abort, err)) {
+        tc_fence_after();
+        const int64_t qrow = q0 + row;
+        float *dst = A.O + (qrow * A.H + h) * DH;
+        for (int c0 = 0; c0 < DH; c0 += 32) {
+          tmem_ld32(tmem_lane_addr(tbase, warp, TM_S0 + c0), v);
+          if (qrow < A.Tq) {
+#pragma unroll
+            for (int i = 0; i < 32; i += 4)
+              *reinterpret_cast<float4 *>(dst + c0 + i) =
+                  make_float4(__uint_as_float(v[i]), __uint_as_float(v[i + 1]), __uint_as_float(v[i + 2]),
+                              __uint_as_float(v[i + 3]));
+          }
+        }
+        if (qrow < A.Tq) A.L[(int64_t)h * A.Tq + qrow] = st.l > 0.f ? (st.m + log2f(st.l)) * kLn2 : -INFINITY;
+      }
+    }
+  }
+  tc_fence_before();
+  __syncthreads();
+  if (warp == 0) {
+    tc_fence_after();
+    tmem_dealloc(tbase, TM_COLS);
+  }
+}
+
+}  // namespace
+
+bool tc_low_supported(const Codec &ck, const Codec &cv) {
+  return ck.prec == PREC_BF16 && ck.d == DH && ck.r == cv.r && ck.C == cv.C && ck.r % 64 == 0 &&
+         ck.r <= 192 && ck.C % 16 == 0 && ck.C <= 64;
+}
+
+static size_t low_smem(int r, int C) {
+  const int nrb = r / 64;
+  return (size_t)(3 * nrb + 1) * kBlk + (size_t)128 * (C + 1) * 4 + 2 * 128 * sizeof(KeyInfo) + 1024;
+}
+
+cudaError_t tc_attend_low(const void *q, int64_t Tq, const Codec &ck, const Codec &cv, const Hist &hk,
+                          const Hist &hv, int64_t t0, int64_t T, float tau, Part out, cudaStream_t st) {
+  if (Tq == 0 || T == 0) return cudaSuccess;
+  const int J = ck.H * DH;
+  CUtensorMap mq, mdk, mck, mdv, mcv;
+  if (!make_tmap_bf16_2d(&mq, q, Tq, J, J, 128) || !make_tmap_bf16_2d(&mdk, ck.D, J, ck.r, ck.r, 128) ||
+      !make_tmap_bf16_2d(&mck, ck.centers, ck.C, J, J, ck.C) ||
+      !make_tmap_bf16_2d(&mdv, cv.D, J, cv.r, cv.r, 128) ||
+      !make_tmap_bf16_2d(&mcv, cv.centers, cv.C, J, J, cv.C))
+    return cudaErrorInvalidValue;
+  LowArgs a;
+  a.Dk = (const __nv_bfloat16 *)ck.D;
+  a.Dv = (const __nv_bfloat16 *)cv.D;
+  a.Ck = (const __nv_bfloat16 *)ck.centers;
+  a.Cv = (const __nv_bfloat16 *)cv.centers;
+  a.idk = hk.ids;
+  a.idv = hv.ids;
+  a.codk = hk.codes;
+  a.codv = hv.codes;
+  a.sk = (const __half *)hk.scales;
+  a.sv = (const __half *)hv.scales;
+  a.t0 = t0;
+  a.T = T;
+  a.Tq = Tq;
+  a.H = ck.H;
+  a.r = ck.r;
+  a.C = ck.C;
+  a.zscale = tau * kLog2e;
+  a.O = out.O;
+  a.L = out.LSE;
+  a.err = error_word_ptr();
+  const size_t smem = low_smem(ck.r, ck.C);
+  cudaFuncSetAttribute(tc_low_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+  dim3 grid((unsigned)((Tq + BM - 1) / BM), (unsigned)ck.H);
+  tc_low_kernel<<<grid, 384, smem, st>>>(mq, mdk, mck, mdv, mcv, a);
+  return cudaGetLastError();
+}
+
+}  // namespace nanokv

@@ -59,6 +59,10 @@ typedef enum { NANOKV_F32 = 0, NANOKV_F16 = 1, NANOKV_BF16 = 2 } nanokv_dtype;
  *   D       [J, r]  linear decoder (Fig. 4(b): reconstructs the residual)
  *   E       [r, J]  linear encoder (Fig. 4(b): residual -> coefficients);
  *                   may be NULL for calls that do not encode.
+ *   aux     optional device buffer of derived encode tables written by
+ *           nanokv_codec_prepare (fp32 E c_j for every center and |c_j|^2);
+ *           NULL is allowed.  nanokv_encode uses its tensor-core kernel only
+ *           when aux is present, and the fp32 CUDA-core kernel otherwise.
  * Constraints: 1 <= C <= 256; r even, 2 <= r <= 512; d in {16, 32, 64, 128}.
  * Precision modes: param_dtype = scale_dtype = F32 (fp32 everywhere), or
  * param_dtype = BF16 with scale_dtype = F16.
@@ -70,7 +74,20 @@ typedef struct {
   const void *centers;
   const void *D;
   const void *E;
+  const void *aux;
 } nanokv_codec;
+
+/* Bytes of the codec's derived encode tables (C*r + C fp32 values, padded). */
+size_t nanokv_codec_aux_bytes(const nanokv_codec *c);
+
+/*
+ * nanokv_codec_prepare -- fill `aux` (device, 16-byte aligned, at least
+ * nanokv_codec_aux_bytes bytes) with the tables the tensor-core encode reads:
+ * EC[j][k] = sum_i E[k][i] c_j[i] (fp32, [C][r]) and |c_j|^2 (fp32, [C]).
+ * They depend on the codec only, so a caller prepares once per codec and
+ * stores the pointer in nanokv_codec.aux.  Needs E.  Asynchronous on stream.
+ */
+int nanokv_codec_prepare(const nanokv_codec *c, void *aux, void *stream);
 
 /* One branch of compressed history, T tokens in time order (oldest first).
  *   ids    [T]        uint8 center id (values >= C are read as C - 1)

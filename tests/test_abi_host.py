@@ -37,7 +37,7 @@ def test_version():
 
 def _codec(**kw):
     c = dict(H=2, d=16, r=8, C=8, param_dtype=_lib.F32, scale_dtype=_lib.F32,
-             centers=4096, D=8192, E=12288)
+             centers=4096, D=8192, E=12288, aux=None)
     c.update(kw)
     return _lib._Codec(**c)
 
@@ -53,6 +53,7 @@ BAD_CODECS = [
     (dict(param_dtype=_lib.BF16, scale_dtype=_lib.F32), _lib.ERR_UNSUPPORTED),
     (dict(centers=0), _lib.ERR_INVALID),
     (dict(D=4100), _lib.ERR_INVALID),        # misaligned
+    (dict(aux=4104), _lib.ERR_INVALID),      # misaligned aux
 ]
 
 
@@ -134,3 +135,13 @@ def test_encode_zero_tokens_is_noop():
     c = _codec()
     assert L.nanokv_encode(ctypes.byref(c), None, None, None, _lib.F32, 0, None, None, None,
                            None, None, None, None) == _lib.OK
+
+
+def test_codec_prepare_validation():
+    L = nk.lib()
+    c = _codec()
+    assert L.nanokv_codec_aux_bytes(ctypes.byref(c)) >= (8 * 8 + 8) * 4
+    assert L.nanokv_codec_aux_bytes(ctypes.byref(_codec(r=7))) == 0
+    assert L.nanokv_codec_prepare(ctypes.byref(c), None, None) == _lib.ERR_INVALID
+    assert L.nanokv_codec_prepare(ctypes.byref(c), ctypes.c_void_p((1 << 20) + 4), None) == _lib.ERR_INVALID
+    assert L.nanokv_codec_prepare(ctypes.byref(_codec(E=0)), ctypes.c_void_p(1 << 20), None) == _lib.ERR_INVALID
