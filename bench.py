@@ -46,7 +46,7 @@ def load_peaks():
 def args_():
     ap = argparse.ArgumentParser()
     ap.add_argument("--gpus", type=int, default=1)
-    ap.add_argument("--steps", type=int, default=10)
+    ap.add_argument("--steps", type=int, default=30)
     ap.add_argument("--warmup", type=int, default=3)
     ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
     ap.add_argument("--workload", default="full")
@@ -75,7 +75,9 @@ def _same_bus(bus_id, smi_bus: str) -> bool:
 
 
 class ClockSampler:
-    FIELDS = ("index,pci.bus_id,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
+    """nvidia-smi sampling (every 50 ms) started before the timed region and
+    stopped after it; samples are matched to the region by timestamp."""
+    FIELDS = ("timestamp,pci.bus_id,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
               "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
               "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
 
@@ -88,19 +90,22 @@ class ClockSampler:
             fd, self.path = tempfile.mkstemp(suffix=".csv")
             os.close(fd)
             self.proc = subprocess.Popen(
-                ["nvidia-smi", f"--query-gpu={self.FIELDS}", "--format=csv,noheader,nounits", "-lms", "200"],
+                ["nvidia-smi", f"--query-gpu={self.FIELDS}", "--format=csv,noheader,nounits", "-lms", "50"],
                 stdout=open(self.path, "w"), stderr=subprocess.DEVNULL)
+            time.sleep(1.0)  # let nvidia-smi start sampling before the region opens
         except Exception:
             self.proc = None
 
-    def stop(self, bus_id: str | None):
+    def stop(self, bus_id, t0: float, t1: float):
         if self.proc is None:
             return {"sm_mhz": None, "sm_max_mhz": None, "reasons": ["unsampled"]}
+        time.sleep(0.2)
         self.proc.terminate()
         try:
             self.proc.wait(timeout=5)
         except Exception:
             self.proc.kill()
+        import datetime
         rows = []
         for line in open(self.path):
             parts = [p.strip() for p in line.split(",")]
@@ -108,17 +113,33 @@ class ClockSampler:
                 continue
             if bus_id is not None and not _same_bus(bus_id, parts[1]):
                 continue
-            rows.append(parts)
+            try:
+                ts = datetime.datetime.strptime(parts[0], "%Y/%m/%d %H:%M:%S.%f").timestamp()
+            except ValueError:
+                continue
+            rows.append((ts, parts))
         os.unlink(self.path)
         if not rows:
             return {"sm_mhz": None, "sm_max_mhz": None, "reasons": ["unsampled"]}
-        sm = [float(r[2]) for r in rows if r[2].replace(".", "").isdigit()]
-        mx = max(float(r[3]) for r in rows if r[3].replace(".", "").isdigit())
+        inside = [r for t, r in rows if t0 - 0.05 <= t <= t1 + 0.05]
+        window = "timed region"
+        if not inside:
+            before = [r for t, r in rows if t < t0][-1:]
+            after = [r for t, r in rows if t > t1][:1]
+            inside = before + after
+            window = "nearest samples (timed region shorter than the sampling period)"
+
+        def num(x):
+            try:
+                return float(x)
+            except ValueError:
+                return None
+        sm = [v for v in (num(r[2]) for r in inside) if v is not None]
+        mx = max((v for v in (num(r[3]) for r in inside) if v is not None), default=None)
         names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
-        reasons = sorted({names[i] for r in rows for i in range(4) if r[6 + i].strip() == "Active"})
-        load = [s for s in sm if s > 0.5 * mx] or sm
-        return {"sm_mhz": statistics.median(load) if load else None, "sm_max_mhz": mx,
-                "reasons": reasons, "samples": len(rows)}
+        reasons = sorted({names[i] for r in inside for i in range(4) if r[6 + i].strip() == "Active"})
+        return {"sm_mhz": statistics.median(sm) if sm else None, "sm_max_mhz": mx, "reasons": reasons,
+                "samples": len(inside), "window": window}
 
 
 # ---------------------------------------------------------------------------
@@ -209,25 +230,31 @@ def run_ours(a, rank, world, device):
     clocks = None
     for attempt in range(2):
         nk.nanokv_timing_read()
-        nk.nanokv_timing_enable(True)
         sampler = ClockSampler() if rank == 0 else None
         if sampler:
             sampler.start()
         if world > 1:
             dist.barrier()
         torch.cuda.synchronize()
+        t_start = time.time()
         enc, att = timed_loop(s, w, a.steps, flush)
         torch.cuda.synchronize()
+        t_end = time.time()
         if world > 1:
             dist.barrier()
-        nk.nanokv_timing_enable(False)
-        kt = nk.nanokv_timing_read()
+        launches = sum(n for _, n in nk.nanokv_timing_read().values())
         if sampler:
-            clocks = sampler.stop(bus)
+            clocks = sampler.stop(bus, t_start, t_end)
         bad = clocks and any(r in BAD_REASONS for r in clocks.get("reasons", []))
         if not bad:
             break
     nk.nanokv_check()
+    # per-kernel durations: a separate loop with the library's per-launch
+    # events (they serialise the kernels, so the step above runs without them)
+    nk.nanokv_timing_enable(True)
+    timed_loop(s, w, a.steps, flush)
+    nk.nanokv_timing_enable(False)
+    kt = nk.nanokv_timing_read()
 
     step_ms = (sum(enc) + sum(att)) / a.steps
     enc_ms, att_ms = sum(enc) / a.steps, sum(att) / a.steps
@@ -238,8 +265,6 @@ def run_ours(a, rank, world, device):
 
     flops = af["total"] + ef
     value = world * flops / (step_ms * 1e-3) / 1e12
-    launches = sum(n for _, n in kt.values())
-
     # dominant kernel: the one with the largest share of the timed region
     dom = max(kt.items(), key=lambda kv: kv[1][0])
     dom_name, (dom_ms, dom_n) = dom

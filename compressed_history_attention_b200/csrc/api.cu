@@ -341,18 +341,23 @@ int nanokv_attend(const void *q, int32_t io_dtype, int64_t Tq, const nanokv_code
     Part p{(float *)(ws + w.off_O[1]), (float *)(ws + w.off_L[1])};
     e = timed(NANOKV_K_FULL, 1, st, [&] {
       return (path != 1 && tc_full_ok)
-                 ? tc_attend_full(q, Tq, ck, cv, hk, hv, T_low, T_full, softmax_scale, p, st)
+                 ? tc_attend_full(q, Tq, ck, cv, hk, hv, T_low, T_full, softmax_scale, p, st,
+                                  T_low > 0 && use_tc_low)
                  : simt_attend_full(q, Tq, ck, cv, hk, hv, T_low, T_full, softmax_scale, p, st);
     });
     if (e != cudaSuccess) return cuda_status(e, "attend full-dim launch");
     pl.O[pl.n] = p.O;
     pl.LSE[pl.n++] = p.LSE;
   }
+  // the current-chunk kernel may overlap the tail of a preceding tensor-core
+  // attention kernel of this call (it reads none of their outputs)
+  const bool prev_tc = (T_full > 0 && path != 1 && tc_full_ok) || (T_full == 0 && T_low > 0 && use_tc_low);
   if (T_cur > 0) {
     Part p{(float *)(ws + w.off_O[2]), (float *)(ws + w.off_L[2])};
     e = timed(NANOKV_K_DENSE, 1, st, [&] {
       return (path != 1 && tc_dense_ok)
-                 ? tc_attend_dense(q, Tq, ck.H, ck.d, k_cur, v_cur, T_cur, softmax_scale, p, st)
+                 ? tc_attend_dense(q, Tq, ck.H, ck.d, k_cur, v_cur, T_cur, softmax_scale, p, st,
+                                   prev_tc)
                  : simt_attend_dense(ck.prec, q, Tq, ck.H, ck.d, k_cur, v_cur, T_cur,
                                      softmax_scale, p, st);
     });

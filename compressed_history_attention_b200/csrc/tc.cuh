@@ -17,12 +17,12 @@ size_t codec_aux_bytes(const Codec &c);
 cudaError_t codec_prepare(const Codec &c, void *aux, cudaStream_t st);
 cudaError_t tc_attend_full(const void *q, int64_t Tq, const Codec &ck, const Codec &cv,
                            const Hist &hk, const Hist &hv, int64_t t0, int64_t T, float tau,
-                           Part out, cudaStream_t st);
+                           Part out, cudaStream_t st, bool pdl);
 cudaError_t tc_attend_low(const void *q, int64_t Tq, const Codec &ck, const Codec &cv,
                           const Hist &hk, const Hist &hv, int64_t t0, int64_t T, float tau,
                           Part out, cudaStream_t st);
 cudaError_t tc_attend_dense(const void *q, int64_t Tq, int H, int d, const void *k, const void *v,
-                            int64_t T, float tau, Part out, cudaStream_t st);
+                            int64_t T, float tau, Part out, cudaStream_t st, bool pdl);
 
 unsigned *error_word_ptr();
 

@@ -15,6 +15,29 @@ namespace nanokv {
 // ---------------------------------------------------------------------------
 bool make_tmap_bf16_2d(CUtensorMap *map, const void *base, uint64_t rows, uint64_t cols,
                        uint64_t row_stride_elems, uint32_t box_rows);
+bool make_tmap_u8_2d(CUtensorMap *map, const void *base, uint64_t rows, uint64_t cols,
+                     uint64_t row_stride_bytes, uint32_t box_cols, uint32_t box_rows);
+
+// Launches `kern` on `st`; with `pdl` the launch may overlap the tail of the
+// previous kernel in the stream (programmatic dependent launch).  Kernels
+// launched this way never read the previous kernel's output and wait for it
+// (griddepcontrol.wait) before they exit, so stream order still holds for
+// whatever comes after them.
+template <typename... KArgs, typename... Args>
+cudaError_t launch_k(void (*kern)(KArgs...), dim3 grid, dim3 block, size_t smem, cudaStream_t st,
+                     bool pdl, Args &&...args) {
+  cudaLaunchConfig_t cfg{};
+  cfg.gridDim = grid;
+  cfg.blockDim = block;
+  cfg.dynamicSmemBytes = smem;
+  cfg.stream = st;
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  attr[0].val.programmaticStreamSerializationAllowed = 1;
+  cfg.attrs = attr;
+  cfg.numAttrs = pdl ? 1 : 0;
+  return cudaLaunchKernelEx(&cfg, kern, std::forward<Args>(args)...);
+}
 
 namespace tc {
 
@@ -56,15 +79,14 @@ struct RowState {
 // warp needs it.
 __device__ __forceinline__ float softmax_tile(uint32_t tbase, int warp, uint32_t s_col, int nk,
                                               float zscale, RowState &st, bool &warp_rescale) {
-  uint32_t r[32];
+  uint32_t r[64];
   float mx = -INFINITY;
 #pragma unroll
-  for (int c = 0; c < 4; ++c) {
-    sm100::tmem_ld32(tmem_lane_addr(tbase, warp, s_col + 32 * c), r);
-    sm100::tmem_ld_wait();
+  for (int c = 0; c < 2; ++c) {
+    sm100::tmem_ld64(tmem_lane_addr(tbase, warp, s_col + 64 * c), r);
 #pragma unroll
-    for (int i = 0; i < 32; ++i) {
-      const float z = (32 * c + i < nk) ? __uint_as_float(r[i]) * zscale : -INFINITY;
+    for (int i = 0; i < 64; ++i) {
+      const float z = (64 * c + i < nk) ? __uint_as_float(r[i]) * zscale : -INFINITY;
       mx = fmaxf(mx, z);
     }
   }
@@ -79,19 +101,23 @@ __device__ __forceinline__ float softmax_tile(uint32_t tbase, int warp, uint32_t
   const float m = st.m;
   float lsum = 0.f;
 #pragma unroll
-  for (int c = 0; c < 4; ++c) {
-    sm100::tmem_ld32(tmem_lane_addr(tbase, warp, s_col + 32 * c), r);
-    sm100::tmem_ld_wait();
-    uint32_t pk[16];
+  for (int c = 0; c < 2; ++c) {
+    sm100::tmem_ld64(tmem_lane_addr(tbase, warp, s_col + 64 * c), r);
+    uint32_t pk[32];
 #pragma unroll
-    for (int i = 0; i < 16; ++i) {
-      const int k0 = 32 * c + 2 * i;
+    for (int i = 0; i < 32; ++i) {
+      const int k0 = 64 * c + 2 * i;
       const float p0 = (k0 < nk) ? ex2(fmaf(__uint_as_float(r[2 * i]), zscale, -m)) : 0.f;
       const float p1 = (k0 + 1 < nk) ? ex2(fmaf(__uint_as_float(r[2 * i + 1]), zscale, -m)) : 0.f;
       lsum += p0 + p1;
       pk[i] = pack_bf16x2(p0, p1);
     }
-    sm100::tmem_st16(tmem_lane_addr(tbase, warp, s_col + 16 * c), pk);
+    // P chunk c covers columns [32c, 32c + 32), all of S chunk c already read
+    uint32_t lo[16], hi[16];
+#pragma unroll
+    for (int i = 0; i < 16; ++i) { lo[i] = pk[i]; hi[i] = pk[16 + i]; }
+    sm100::tmem_st16(tmem_lane_addr(tbase, warp, s_col + 32 * c), lo);
+    sm100::tmem_st16(tmem_lane_addr(tbase, warp, s_col + 32 * c + 16), hi);
   }
   sm100::tmem_st_wait();
   st.l += lsum;

@@ -108,6 +108,7 @@ __global__ void __launch_bounds__(256, 1)
   __syncthreads();
   tc_fence_after();
   const uint32_t tbase = B.tmem_base;
+  pdl_launch_dependents();
 
   if (warp == 0) {
     // ---------------- TMA producer ----------------
@@ -201,6 +202,7 @@ __global__ void __launch_bounds__(256, 1)
     tc_fence_after();
     tmem_dealloc(tbase, TM_COLS);
   }
+  pdl_wait_prior();
 }
 
 }  // namespace
@@ -208,7 +210,7 @@ __global__ void __launch_bounds__(256, 1)
 bool tc_dense_supported(int prec, int d) { return prec == PREC_BF16 && d == DH; }
 
 cudaError_t tc_attend_dense(const void *q, int64_t Tq, int H, int d, const void *k, const void *v,
-                            int64_t T, float tau, Part out, cudaStream_t st) {
+                            int64_t T, float tau, Part out, cudaStream_t st, bool pdl) {
   if (Tq == 0 || T == 0) return cudaSuccess;
   const int J = H * d;
   CUtensorMap mq, mk, mv;
@@ -218,9 +220,8 @@ cudaError_t tc_attend_dense(const void *q, int64_t Tq, int H, int d, const void 
   const size_t smem = 5 * kTileBytes + 1024;
   cudaFuncSetAttribute(tc_dense_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
   dim3 grid((unsigned)((Tq + BM - 1) / BM), (unsigned)H);
-  tc_dense_kernel<<<grid, 256, smem, st>>>(mq, mk, mv, Tq, T, H, tau * kLog2e, out.O, out.LSE,
-                                           error_word_ptr());
-  return cudaGetLastError();
+  return launch_k(tc_dense_kernel, grid, dim3(256), smem, st, pdl, mq, mk, mv, Tq, T, H, tau * kLog2e,
+                  out.O, out.LSE, error_word_ptr());
 }
 
 }  // namespace nanokv

@@ -26,8 +26,19 @@ namespace nanokv {
 using namespace sm100;
 using namespace tc;
 
-bool make_tmap_u8_2d(CUtensorMap *map, const void *base, uint64_t rows, uint64_t cols,
-                     uint64_t row_stride_bytes, uint32_t box_cols, uint32_t box_rows);
+// Optional event trace of the first cluster of head 0 (debug builds with
+// -DNANOKV_TRACE only): clock64 stamps per role and key tile.
+#ifdef NANOKV_TRACE
+__device__ unsigned long long g_full_trace[2][16][128];
+#define FULL_TRACE(ev, j)                                                                    \
+  do {                                                                                       \
+    if (blockIdx.y == 0 && blockIdx.x < 2 && (j) < 128) g_full_trace[rank][ev][j] = clock64(); \
+  } while (0)
+#else
+#define FULL_TRACE(ev, j) \
+  do {                    \
+  } while (0)
+#endif
 
 namespace {
 
@@ -146,6 +157,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(384, 1)
   cluster_sync();  // barriers of both CTAs initialised before any remote arrive
   tc_fence_after();
   const uint32_t tbase = B.tmem_base;
+  pdl_launch_dependents();
 
   if (warp == 0) {
     // ---------------- TMA producer ----------------
@@ -179,6 +191,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(384, 1)
       auto decode = [&](int j) -> bool {
         const int xb = j & 1;
         if (j >= 2 && !mbar_wait(&B.x_empty[xb], ((j >> 1) - 1) & 1, abort, err)) return false;
+        FULL_TRACE(0, j);
         const uint32_t dX = tbase + TM_X + xb * 128;
         for (int cb = 0; cb < nrb; ++cb, ++cc) {
           const int slot = cc % NRING;
@@ -192,11 +205,13 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(384, 1)
           mma_commit(&B.ring_empty[slot]);
         }
         mma_commit(&B.x_full[xb]);
+        FULL_TRACE(1, j);
         return true;
       };
       auto scores = [&](int j) -> bool {
         if (!mbar_wait_cluster(&B.kh_full, j & 1, abort, err)) return false;
         if (j > 0 && !mbar_wait(&B.pv_done, (j - 1) & 1, abort, err)) return false;
+        FULL_TRACE(2, j);
         tc_fence_after();
 #pragma unroll
         for (int ks = 0; ks < DH / 16; ++ks) {
@@ -211,6 +226,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(384, 1)
       auto values = [&](int j) -> bool {
         if (!mbar_wait(&B.p_full, j & 1, abort, err)) return false;
         if (!mbar_wait_cluster(&B.vh_full, j & 1, abort, err)) return false;
+        FULL_TRACE(3, j);
         tc_fence_after();
 #pragma unroll
         for (int ks = 0; ks < BN / 16; ++ks)
@@ -233,12 +249,14 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(384, 1)
     for (int c = 0; c < nchunk; ++c) {
       const int slot = c % NSTAGE, rs = c % NRING;
       if (!mbar_wait(&B.st_full[slot], (c / NSTAGE) & 1, abort, err)) break;
+      if (u == 0 && c % nrb == 0) FULL_TRACE(9, c / nrb);
       const uint4 *src = reinterpret_cast<const uint4 *>(sStage + slot * kStage);
       const uint4 p0 = src[2 * u], p1 = src[2 * u + 1];
       const uint4 p2 = src[2 * (u + 64)], p3 = src[2 * (u + 64) + 1];
       __syncwarp();
       if (lane == 0) mbar_arrive(&B.st_empty[slot]);
       if (c >= NRING && !mbar_wait(&B.ring_empty[rs], ((c / NRING) - 1) & 1, abort, err)) break;
+      if (u == 0 && c % nrb == 0) FULL_TRACE(10, c / nrb);
       uint8_t *dst = sRing + rs * kChunk;
       const uint32_t w0[8] = {p0.x, p0.y, p0.z, p0.w, p1.x, p1.y, p1.z, p1.w};
       const uint32_t w1[8] = {p2.x, p2.y, p2.z, p2.w, p3.x, p3.y, p3.z, p3.w};
@@ -250,6 +268,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(384, 1)
       fence_proxy_async_smem();
       __syncwarp();
       if (lane == 0) mbar_arrive(&B.ring_full[rs]);
+      if (u == 0 && c % nrb == nrb - 1) FULL_TRACE(11, c / nrb);
     }
   } else if (warp >= 4 && warp < 8) {
     // ---------------- decode epilogue (thread = key) ----------------
@@ -291,7 +310,9 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(384, 1)
       const int sw = a & 15;
       const int xb = j & 1;
       if (!mbar_wait(&B.x_full[xb], (j >> 1) & 1, abort, err)) break;
+      if (t == 0) FULL_TRACE(4, j);
       if (j > 0 && !mbar_wait_cluster(empty_bar, (j - 1) & 1, abort, err)) break;
+      if (t == 0) FULL_TRACE(5, j);
       tc_fence_after();
 #pragma unroll 1
       for (int c = 0; c < 4; ++c) {
@@ -323,6 +344,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(384, 1)
         mbar_arrive_cluster(full_local);
         mbar_arrive_cluster(full_remote);
       }
+      if (t == 0) FULL_TRACE(6, j);
     }
   } else if (warp >= 8) {
     // ---------------- softmax (thread = query row) ----------------
@@ -331,6 +353,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(384, 1)
     bool ok = true;
     for (int j = 0; j < ntiles; ++j) {
       if (!mbar_wait(&B.s_full, j & 1, abort, err)) { ok = false; break; }
+      if (row == 0) FULL_TRACE(7, j);
       tc_fence_after();
       const int64_t rem = A.T - (int64_t)j * BN;
       const int nk = rem < BN ? (int)rem : BN;
@@ -344,6 +367,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(384, 1)
       tc_fence_before();
       __syncwarp();
       if (lane == 0) mbar_arrive(&B.p_full);
+      if (row == 0) FULL_TRACE(8, j);
     }
     if (ok && mbar_wait(&B.pv_done, (ntiles - 1) & 1, abort, err)) {
       tc_fence_after();
@@ -365,6 +389,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(384, 1)
     tc_fence_after();
     tmem_dealloc(tbase, TM_COLS);
   }
+  pdl_wait_prior();
 }
 
 }  // namespace
@@ -382,7 +407,7 @@ size_t tc_full_smem(int r, int C) {
 
 cudaError_t tc_attend_full(const void *q, int64_t Tq, const Codec &ck, const Codec &cv,
                            const Hist &hk, const Hist &hv, int64_t t0, int64_t T, float tau,
-                           Part out, cudaStream_t st) {
+                           Part out, cudaStream_t st, bool pdl) {
   if (Tq == 0 || T == 0) return cudaSuccess;
   const int J = ck.H * DH;
   const int64_t T_total = t0 + T;
@@ -415,8 +440,14 @@ cudaError_t tc_attend_full(const void *q, int64_t Tq, const Codec &ck, const Cod
   cudaFuncSetAttribute(tc_full_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
   const unsigned qt = (unsigned)((Tq + BM - 1) / BM);
   dim3 grid((qt + 1) & ~1u, (unsigned)ck.H);
-  tc_full_kernel<<<grid, 384, smem, st>>>(mq, mck, mcv, a);
-  return cudaGetLastError();
+  return launch_k(tc_full_kernel, grid, dim3(384), smem, st, pdl, mq, mck, mcv, a);
 }
+
+#ifdef NANOKV_TRACE
+extern "C" int nanokv_debug_full_trace(void *host, size_t bytes) {
+  if (bytes < sizeof(g_full_trace)) return -1;
+  return cudaMemcpyFromSymbol(host, g_full_trace, sizeof(g_full_trace)) == cudaSuccess ? 0 : -3;
+}
+#endif
 
 }  // namespace nanokv
