@@ -40,12 +40,16 @@ __device__ __forceinline__ void mbar_arrive_expect_tx(uint64_t *bar, uint32_t by
                "r"(bytes)
                : "memory");
 }
+// A waiting thread is suspended until the phase completes or the hint (ns)
+// elapses, so idle roles do not take issue slots from busy warps.
+constexpr uint32_t kSuspendHintNs = 200000;
+
 __device__ __forceinline__ bool mbar_try_wait(uint64_t *bar, uint32_t parity) {
   uint32_t ok;
   asm volatile(
-      "{ .reg .pred p; mbarrier.try_wait.parity.shared::cta.b64 p, [%1], %2; selp.u32 %0, 1, 0, p; }"
+      "{ .reg .pred p; mbarrier.try_wait.parity.shared::cta.b64 p, [%1], %2, %3; selp.u32 %0, 1, 0, p; }"
       : "=r"(ok)
-      : "r"(smem_u32(bar)), "r"(parity)
+      : "r"(smem_u32(bar)), "r"(parity), "r"(kSuspendHintNs)
       : "memory");
   return ok != 0;
 }
@@ -63,7 +67,7 @@ __device__ __forceinline__ bool mbar_wait(uint64_t *bar, uint32_t parity, volati
   uint32_t n = 0;
   while (true) {
     if (mbar_try_wait(bar, parity)) return true;
-    if ((++n & 63u) == 0) {
+    if ((++n & 3u) == 0) {
       if (abort && *abort) return false;
       if (globaltimer() - t0 > kWaitLimitNs) {
         if (abort) *abort = 1;
@@ -241,10 +245,10 @@ __device__ __forceinline__ void mbar_arrive_cluster(uint32_t caddr) {
 __device__ __forceinline__ bool mbar_try_wait_cluster(uint64_t *bar, uint32_t parity) {
   uint32_t ok;
   asm volatile(
-      "{ .reg .pred p; mbarrier.try_wait.parity.acquire.cluster.shared::cta.b64 p, [%1], %2; "
+      "{ .reg .pred p; mbarrier.try_wait.parity.acquire.cluster.shared::cta.b64 p, [%1], %2, %3; "
       "selp.u32 %0, 1, 0, p; }"
       : "=r"(ok)
-      : "r"(smem_u32(bar)), "r"(parity)
+      : "r"(smem_u32(bar)), "r"(parity), "r"(kSuspendHintNs)
       : "memory");
   return ok != 0;
 }
@@ -256,7 +260,7 @@ __device__ __forceinline__ bool mbar_wait_cluster(uint64_t *bar, uint32_t parity
   uint32_t n = 0;
   while (true) {
     if (mbar_try_wait_cluster(bar, parity)) return true;
-    if ((++n & 63u) == 0) {
+    if ((++n & 3u) == 0) {
       if (abort && *abort) return false;
       if (globaltimer() - t0 > kWaitLimitNs) {
         if (abort) *abort = 1;
@@ -265,6 +269,23 @@ __device__ __forceinline__ bool mbar_wait_cluster(uint64_t *bar, uint32_t parity
       }
     }
   }
+}
+// arrive on a (possibly remote) mbarrier and add `bytes` to its expected
+// transaction count, release at cluster scope
+__device__ __forceinline__ void mbar_arrive_expect_tx_cluster(uint32_t caddr, uint32_t bytes) {
+  asm volatile("mbarrier.arrive.expect_tx.release.cluster.shared::cluster.b64 _, [%0], %1;" ::"r"(caddr),
+               "r"(bytes)
+               : "memory");
+}
+// bulk copy of `bytes` from this CTA's shared memory to shared memory of a CTA
+// of the cluster (cluster addresses), completing on that CTA's mbarrier
+__device__ __forceinline__ void bulk_s2cluster(uint32_t dst_caddr, const void *src, uint32_t bytes,
+                                               uint32_t bar_caddr) {
+  asm volatile(
+      "cp.async.bulk.shared::cluster.shared::cta.mbarrier::complete_tx::bytes [%0], [%1], %2, [%3];" ::"r"(
+          dst_caddr),
+      "r"(smem_u32(src)), "r"(bytes), "r"(bar_caddr)
+      : "memory");
 }
 __device__ __forceinline__ void fence_proxy_async_cluster() {
   asm volatile("fence.proxy.async.shared::cluster;" ::: "memory");

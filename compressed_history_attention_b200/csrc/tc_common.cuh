@@ -71,6 +71,19 @@ struct RowState {
   float l;  // running sum of 2^(z - m)
 };
 
+#ifdef NANOKV_TRACE
+// debug builds only: clock64 stamps of the softmax stages of one row
+__device__ unsigned long long g_softmax_trace[4][128];
+#define SOFTMAX_TRACE(i, tj)                                            \
+  do {                                                                  \
+    if ((tj) >= 0 && (tj) < 128) g_softmax_trace[i][tj] = clock64();    \
+  } while (0)
+#else
+#define SOFTMAX_TRACE(i, tj) \
+  do {                       \
+  } while (0)
+#endif
+
 // One key tile of the online softmax for the calling thread's row.
 // Reads S (fp32, 128 columns at s_col), writes P as packed bf16 into the first
 // 64 of those columns, updates the row state.  `nk` valid keys; `zscale`
@@ -78,18 +91,27 @@ struct RowState {
 // caller must rescale O (1 if none); *rescale tells whether any row of the
 // warp needs it.
 __device__ __forceinline__ float softmax_tile(uint32_t tbase, int warp, uint32_t s_col, int nk,
-                                              float zscale, RowState &st, bool &warp_rescale) {
+                                              float zscale, RowState &st, bool &warp_rescale,
+                                              int trace_j = -1) {
   uint32_t r[64];
-  float mx = -INFINITY;
+  const bool full = nk >= 128;
+  // pass 1: row max over the tile, four independent chains
+  float mx4[4] = {-INFINITY, -INFINITY, -INFINITY, -INFINITY};
+  SOFTMAX_TRACE(0, trace_j);
 #pragma unroll
   for (int c = 0; c < 2; ++c) {
     sm100::tmem_ld64(tmem_lane_addr(tbase, warp, s_col + 64 * c), r);
+    if (full) {
 #pragma unroll
-    for (int i = 0; i < 64; ++i) {
-      const float z = (64 * c + i < nk) ? __uint_as_float(r[i]) * zscale : -INFINITY;
-      mx = fmaxf(mx, z);
+      for (int i = 0; i < 64; ++i) mx4[i & 3] = fmaxf(mx4[i & 3], __uint_as_float(r[i]));
+    } else {
+#pragma unroll
+      for (int i = 0; i < 64; ++i)
+        mx4[i & 3] = (64 * c + i < nk) ? fmaxf(mx4[i & 3], __uint_as_float(r[i])) : mx4[i & 3];
     }
   }
+  // scores are scaled after the max (zscale > 0 keeps the order)
+  const float mx = fmaxf(fmaxf(mx4[0], mx4[1]), fmaxf(mx4[2], mx4[3])) * zscale;
   float corr = 1.f;
   const bool need = mx > st.m + kRescaleLog2;  // also true when st.m == -inf
   if (need) {
@@ -98,18 +120,24 @@ __device__ __forceinline__ float softmax_tile(uint32_t tbase, int warp, uint32_t
     st.m = mx;
   }
   warp_rescale = __any_sync(0xffffffffu, need) != 0;
+  SOFTMAX_TRACE(1, trace_j);
   const float m = st.m;
-  float lsum = 0.f;
+  float ls[4] = {0.f, 0.f, 0.f, 0.f};
 #pragma unroll
   for (int c = 0; c < 2; ++c) {
     sm100::tmem_ld64(tmem_lane_addr(tbase, warp, s_col + 64 * c), r);
+    if (c == 0) SOFTMAX_TRACE(2, trace_j);
     uint32_t pk[32];
 #pragma unroll
     for (int i = 0; i < 32; ++i) {
       const int k0 = 64 * c + 2 * i;
-      const float p0 = (k0 < nk) ? ex2(fmaf(__uint_as_float(r[2 * i]), zscale, -m)) : 0.f;
-      const float p1 = (k0 + 1 < nk) ? ex2(fmaf(__uint_as_float(r[2 * i + 1]), zscale, -m)) : 0.f;
-      lsum += p0 + p1;
+      float p0 = ex2(fmaf(__uint_as_float(r[2 * i]), zscale, -m));
+      float p1 = ex2(fmaf(__uint_as_float(r[2 * i + 1]), zscale, -m));
+      if (!full) {
+        p0 = (k0 < nk) ? p0 : 0.f;
+        p1 = (k0 + 1 < nk) ? p1 : 0.f;
+      }
+      ls[i & 3] += p0 + p1;
       pk[i] = pack_bf16x2(p0, p1);
     }
     // P chunk c covers columns [32c, 32c + 32), all of S chunk c already read
@@ -120,7 +148,8 @@ __device__ __forceinline__ float softmax_tile(uint32_t tbase, int warp, uint32_t
     sm100::tmem_st16(tmem_lane_addr(tbase, warp, s_col + 32 * c + 16), hi);
   }
   sm100::tmem_st_wait();
-  st.l += lsum;
+  SOFTMAX_TRACE(3, trace_j);
+  st.l += (ls[0] + ls[1]) + (ls[2] + ls[3]);
   return corr;
 }
 

@@ -61,10 +61,10 @@ constexpr int DH = 128;
 constexpr uint32_t kTileBytes = 128 * 128 * 2;  // one [128 x 128] bf16 operand tile
 constexpr uint32_t IDESC_S = idesc_bf16(128, 128, false, false);
 constexpr uint32_t IDESC_PV = idesc_bf16(128, 128, false, true);
-constexpr uint32_t TM_O = 0, TM_S = 128, TM_COLS = 256;
+constexpr uint32_t TM_O = 0, TM_S = 128, TM_COLS = 512;  // S: two 128-column buffers
 
 struct DenseBars {
-  uint64_t q_full, k_full[2], v_full[2], kv_empty[2], s_full, p_full, pv_done;
+  uint64_t q_full, k_full[2], v_full[2], kv_empty[2], s_full[2], p_full[2], pv_done;
   uint32_t tmem_base;
   int abort;
 };
@@ -94,8 +94,10 @@ __global__ void __launch_bounds__(256, 1)
       mbar_init(&B.v_full[s], 1);
       mbar_init(&B.kv_empty[s], 1);
     }
-    mbar_init(&B.s_full, 1);
-    mbar_init(&B.p_full, 4);
+    for (int s = 0; s < 2; ++s) {
+      mbar_init(&B.s_full[s], 1);
+      mbar_init(&B.p_full[s], 4);
+    }
     mbar_init(&B.pv_done, 1);
     B.abort = 0;
     fence_mbar_init();
@@ -144,30 +146,40 @@ __global__ void __launch_bounds__(256, 1)
     if (lane == 0) {
       bool ok = mbar_wait(&B.q_full, 0, abort, err);
       const uint32_t aQ = smem_u32(sQ);
-      for (int j = 0; ok && j < ntiles; ++j) {
+      auto scores = [&](int j) -> bool {
         const int s = j & 1;
-        if (!mbar_wait(&B.k_full[s], (j >> 1) & 1, abort, err)) break;
-        if (j > 0 && !mbar_wait(&B.pv_done, (j - 1) & 1, abort, err)) break;
+        if (!mbar_wait(&B.k_full[s], (j >> 1) & 1, abort, err)) return false;
+        // the S buffer of tile j last held P of tile j - 2
+        if (j >= 2 && !mbar_wait(&B.pv_done, (j - 2) & 1, abort, err)) return false;
         tc_fence_after();
         const uint32_t aK = smem_u32(sK[s]);
 #pragma unroll
         for (int ks = 0; ks < DH / 16; ++ks) {
           const uint32_t off = (ks >> 2) * (kTileBytes / 2) + (ks & 3) * 32;
-          mma_ss(tbase + TM_S, sdesc_sw128(aQ + off, 16, 1024), sdesc_sw128(aK + off, 16, 1024),
+          mma_ss(tbase + TM_S + s * 128, sdesc_sw128(aQ + off, 16, 1024), sdesc_sw128(aK + off, 16, 1024),
                  IDESC_S, ks > 0);
         }
-        mma_commit(&B.s_full);
-        if (!mbar_wait(&B.p_full, j & 1, abort, err)) break;
-        if (!mbar_wait(&B.v_full[s], (j >> 1) & 1, abort, err)) break;
+        mma_commit(&B.s_full[s]);
+        return true;
+      };
+      auto values = [&](int j) -> bool {
+        const int s = j & 1;
+        if (!mbar_wait(&B.p_full[s], (j >> 1) & 1, abort, err)) return false;
+        if (!mbar_wait(&B.v_full[s], (j >> 1) & 1, abort, err)) return false;
         tc_fence_after();
         const uint32_t aV = smem_u32(sV[s]);
 #pragma unroll
-        for (int ks = 0; ks < BN / 16; ++ks) {
-          mma_ts(tbase + TM_O, tbase + TM_S + ks * 8, sdesc_sw128(aV + ks * 2048, kTileBytes / 2, 1024),
-                 IDESC_PV, (j > 0 || ks > 0));
-        }
+        for (int ks = 0; ks < BN / 16; ++ks)
+          mma_ts(tbase + TM_O, tbase + TM_S + s * 128 + ks * 8,
+                 sdesc_sw128(aV + ks * 2048, kTileBytes / 2, 1024), IDESC_PV, (j > 0 || ks > 0));
         mma_commit(&B.pv_done);
         mma_commit(&B.kv_empty[s]);
+        return true;
+      };
+      if (ok) ok = scores(0);
+      for (int j = 0; ok && j < ntiles; ++j) {
+        if (j + 1 < ntiles && !scores(j + 1)) break;
+        if (!values(j)) break;
       }
     }
   } else if (warp >= 4) {
@@ -176,12 +188,12 @@ __global__ void __launch_bounds__(256, 1)
     RowState st{-INFINITY, 0.f};
     bool ok = true;
     for (int j = 0; j < ntiles; ++j) {
-      if (!mbar_wait(&B.s_full, j & 1, abort, err)) { ok = false; break; }
+      if (!mbar_wait(&B.s_full[j & 1], (j >> 1) & 1, abort, err)) { ok = false; break; }
       tc_fence_after();
       const int64_t rem = T - (int64_t)j * BN;
       const int nk = rem < BN ? (int)rem : BN;
       bool wr;
-      const float corr = softmax_tile(tbase, warp, TM_S, nk, zscale, st, wr);
+      const float corr = softmax_tile(tbase, warp, TM_S + (j & 1) * 128, nk, zscale, st, wr);
       if (j > 0 && wr) {
         if (!mbar_wait(&B.pv_done, (j - 1) & 1, abort, err)) { ok = false; break; }
         tc_fence_after();
@@ -189,8 +201,11 @@ __global__ void __launch_bounds__(256, 1)
       }
       tc_fence_before();
       __syncwarp();
-      if (lane == 0) mbar_arrive(&B.p_full);
+      if (lane == 0) mbar_arrive(&B.p_full[j & 1]);
     }
+    // the value MMAs may trail the softmax by two tiles: wait for the last two
+    // phases in order so that a parity can never be mistaken for an older one
+    if (ok && ntiles >= 2) ok = mbar_wait(&B.pv_done, (ntiles - 2) & 1, abort, err);
     if (ok && mbar_wait(&B.pv_done, (ntiles - 1) & 1, abort, err)) {
       tc_fence_after();
       write_row(tbase, warp, TM_O, st, q0 + row, Tq, h, H, Oout, Lout);

@@ -50,7 +50,7 @@ constexpr int NRING = 3, NSTAGE = 4;
 constexpr uint32_t IDESC_DEC = idesc_bf16(128, 128, false, false);
 constexpr uint32_t IDESC_S = idesc_bf16(128, 128, false, false);
 constexpr uint32_t IDESC_PV = idesc_bf16(128, 128, false, true);
-constexpr uint32_t TM_O = 0, TM_S = 128, TM_X = 256, TM_COLS = 512;
+constexpr uint32_t TM_O = 0, TM_S = 128, TM_X = 384, TM_COLS = 512;  // S: two 128-column buffers
 
 struct FullArgs {
   const __nv_bfloat16 *D[2];    // decoders [J, r] (K, V)
@@ -68,9 +68,9 @@ struct FullBars {
   uint64_t q_full;
   uint64_t st_full[NSTAGE], st_empty[NSTAGE];
   uint64_t ring_full[NRING], ring_empty[NRING];
-  uint64_t x_full[2], x_empty[2];
+  uint64_t x_full, x_empty;
   uint64_t kh_full, vh_full, kh_empty, vh_empty;
-  uint64_t s_full, p_full, pv_done;
+  uint64_t s_full[2], p_full[2], pv_done;
   uint32_t tmem_base;
   int abort;
 };
@@ -121,13 +121,15 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(384, 1)
     mbar_init(&B.q_full, 1);
     for (int i = 0; i < NSTAGE; ++i) { mbar_init(&B.st_full[i], 1); mbar_init(&B.st_empty[i], 2); }
     for (int i = 0; i < NRING; ++i) { mbar_init(&B.ring_full[i], 2); mbar_init(&B.ring_empty[i], 1); }
-    for (int i = 0; i < 2; ++i) { mbar_init(&B.x_full[i], 1); mbar_init(&B.x_empty[i], 4); }
-    mbar_init(&B.kh_full, 4);
-    mbar_init(&B.vh_full, 4);
+    mbar_init(&B.x_full, 1);
+    mbar_init(&B.x_empty, 1);
+    // decoded-tile barriers: one arrive (the decoder's own elected thread,
+    // or its remote expect_tx arrive) plus, for the receiver, the bulk copy bytes
+    mbar_init(&B.kh_full, 1);
+    mbar_init(&B.vh_full, 1);
     mbar_init(&B.kh_empty, 2);
     mbar_init(&B.vh_empty, 2);
-    mbar_init(&B.s_full, 1);
-    mbar_init(&B.p_full, 4);
+    for (int i = 0; i < 2; ++i) { mbar_init(&B.s_full[i], 1); mbar_init(&B.p_full[i], 4); }
     mbar_init(&B.pv_done, 1);
     B.abort = 0;
     fence_mbar_init();
@@ -189,10 +191,9 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(384, 1)
       int cc = 0;  // chunk counter
       bool ok = mbar_wait(&B.q_full, 0, abort, err);
       auto decode = [&](int j) -> bool {
-        const int xb = j & 1;
-        if (j >= 2 && !mbar_wait(&B.x_empty[xb], ((j >> 1) - 1) & 1, abort, err)) return false;
+        if (j >= 1 && !mbar_wait(&B.x_empty, (j - 1) & 1, abort, err)) return false;
         FULL_TRACE(0, j);
-        const uint32_t dX = tbase + TM_X + xb * 128;
+        const uint32_t dX = tbase + TM_X;
         for (int cb = 0; cb < nrb; ++cb, ++cc) {
           const int slot = cc % NRING;
           if (!mbar_wait(&B.ring_full[slot], (cc / NRING) & 1, abort, err)) return false;
@@ -204,43 +205,45 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(384, 1)
                    (cb > 0 || k > 0));
           mma_commit(&B.ring_empty[slot]);
         }
-        mma_commit(&B.x_full[xb]);
+        mma_commit(&B.x_full);
         FULL_TRACE(1, j);
         return true;
       };
       auto scores = [&](int j) -> bool {
         if (!mbar_wait_cluster(&B.kh_full, j & 1, abort, err)) return false;
-        if (j > 0 && !mbar_wait(&B.pv_done, (j - 1) & 1, abort, err)) return false;
+        // the S buffer of tile j last held P of tile j - 2
+        if (j >= 2 && !mbar_wait(&B.pv_done, (j - 2) & 1, abort, err)) return false;
         FULL_TRACE(2, j);
         tc_fence_after();
+        const uint32_t dS = tbase + TM_S + (j & 1) * 128;
 #pragma unroll
         for (int ks = 0; ks < DH / 16; ++ks) {
           const uint32_t off = (ks >> 2) * (kTile / 2) + (ks & 3) * 32;
-          mma_ss(tbase + TM_S, sdesc_sw128(aQ + off, 16, 1024), sdesc_sw128(aK + off, 16, 1024), IDESC_S,
-                 ks > 0);
+          mma_ss(dS, sdesc_sw128(aQ + off, 16, 1024), sdesc_sw128(aK + off, 16, 1024), IDESC_S, ks > 0);
         }
-        mma_commit(&B.s_full);
+        mma_commit(&B.s_full[j & 1]);
         mma_commit_mc(&B.kh_empty, 0x1);  // K_hat consumed here: tell the K decoder (CTA 0)
         return true;
       };
       auto values = [&](int j) -> bool {
-        if (!mbar_wait(&B.p_full, j & 1, abort, err)) return false;
+        if (!mbar_wait(&B.p_full[j & 1], (j >> 1) & 1, abort, err)) return false;
         if (!mbar_wait_cluster(&B.vh_full, j & 1, abort, err)) return false;
         FULL_TRACE(3, j);
         tc_fence_after();
+        const uint32_t sP = tbase + TM_S + (j & 1) * 128;
 #pragma unroll
         for (int ks = 0; ks < BN / 16; ++ks)
-          mma_ts(tbase + TM_O, tbase + TM_S + ks * 8, sdesc_sw128(aV + ks * 2048, kTile / 2, 1024),
-                 IDESC_PV, (j > 0 || ks > 0));
+          mma_ts(tbase + TM_O, sP + ks * 8, sdesc_sw128(aV + ks * 2048, kTile / 2, 1024), IDESC_PV,
+                 (j > 0 || ks > 0));
         mma_commit(&B.pv_done);
         mma_commit_mc(&B.vh_empty, 0x2);  // V_hat consumed: tell the V decoder (CTA 1)
         return true;
       };
+      // issue order keeps the scores of tile j + 1 ahead of the softmax of tile j
       if (ok) ok = decode(0) && scores(0);
       for (int j = 0; ok && j < ntiles; ++j) {
-        if (j + 1 < ntiles && !decode(j + 1)) break;
+        if (j + 1 < ntiles && !(decode(j + 1) && scores(j + 1))) break;
         if (!values(j)) break;
-        if (j + 1 < ntiles && !scores(j + 1)) break;
       }
     }
   } else if (warp == 2 || warp == 3) {
@@ -290,7 +293,6 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(384, 1)
     const uint32_t dst_remote = mapa(dst_local, peer);
     uint64_t *full_bar = rank == 0 ? &B.kh_full : &B.vh_full;
     uint64_t *empty_bar = rank == 0 ? &B.kh_empty : &B.vh_empty;
-    const uint32_t full_local = mapa(smem_u32(full_bar), rank);
     const uint32_t full_remote = mapa(smem_u32(full_bar), peer);
     auto key_meta = [&](int j, int &a, float &s) {
       const int64_t tt = A.t0 + (int64_t)j * BN + t;
@@ -308,43 +310,46 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(384, 1)
       if (j + 1 < ntiles) key_meta(j + 1, a_next, s_next);
       const uint8_t *crow = sCen + a * 256;
       const int sw = a & 15;
-      const int xb = j & 1;
-      if (!mbar_wait(&B.x_full[xb], (j >> 1) & 1, abort, err)) break;
+      if (!mbar_wait(&B.x_full, j & 1, abort, err)) break;
       if (t == 0) FULL_TRACE(4, j);
+      // the previous tile in this buffer was consumed by both CTAs (and the
+      // bulk copy that carried it to the peer had completed before that)
       if (j > 0 && !mbar_wait_cluster(empty_bar, (j - 1) & 1, abort, err)) break;
       if (t == 0) FULL_TRACE(5, j);
       tc_fence_after();
+      // K_hat = c + s x in packed bf16x2: x rounded to bf16, one fused
+      // multiply-add per pair, one rounding of the result
+      const __nv_bfloat162 s2 = __floats2bfloat162_rn(s, s);
 #pragma unroll 1
-      for (int c = 0; c < 4; ++c) {
-        uint32_t x[32];
-        tmem_ld32(tmem_lane_addr(tbase, warp, TM_X + xb * 128 + 32 * c), x);
+      for (int c = 0; c < 2; ++c) {
+        uint32_t x[64];
+        tmem_ld64(tmem_lane_addr(tbase, warp, TM_X + 64 * c), x);
 #pragma unroll
-        for (int g = 0; g < 4; ++g) {
-          const uint4 cv = *reinterpret_cast<const uint4 *>(crow + (((4 * c + g) ^ sw) << 4));
-          const __nv_bfloat162 *c2 = reinterpret_cast<const __nv_bfloat162 *>(&cv);
+        for (int g = 0; g < 8; ++g) {
+          const uint4 cv = *reinterpret_cast<const uint4 *>(crow + (((8 * c + g) ^ sw) << 4));
+          const uint32_t cw[4] = {cv.x, cv.y, cv.z, cv.w};
           uint32_t o[4];
 #pragma unroll
           for (int i = 0; i < 4; ++i) {
-            const float2 cf = __bfloat1622float2(c2[i]);
-            o[i] = pack_bf16x2(fmaf(s, __uint_as_float(x[8 * g + 2 * i]), cf.x),
-                               fmaf(s, __uint_as_float(x[8 * g + 2 * i + 1]), cf.y));
+            const uint32_t xp = pack_bf16x2(__uint_as_float(x[8 * g + 2 * i]), __uint_as_float(x[8 * g + 2 * i + 1]));
+            const __nv_bfloat162 r = __hfma2(s2, *reinterpret_cast<const __nv_bfloat162 *>(&xp),
+                                             *reinterpret_cast<const __nv_bfloat162 *>(&cw[i]));
+            o[i] = *reinterpret_cast<const uint32_t *>(&r);
           }
-          const uint4 v = make_uint4(o[0], o[1], o[2], o[3]);
-          const uint32_t off = sw128_offset(t, 32 * c + 8 * g, 128);
-          st_shared_v4(dst_local + off, v);
-          st_cluster_v4(dst_remote + off, v);
+          st_shared_v4(dst_local + sw128_offset(t, 64 * c + 8 * g, 128), make_uint4(o[0], o[1], o[2], o[3]));
         }
       }
-      fence_proxy_async_smem();
-      fence_proxy_async_cluster();
+      fence_proxy_async_smem();  // the tile is read by this CTA's MMA and by the bulk copy
       tc_fence_before();
-      __syncwarp();
-      if (lane == 0) {
-        mbar_arrive(&B.x_empty[xb]);
-        mbar_arrive_cluster(full_local);
-        mbar_arrive_cluster(full_remote);
+      asm volatile("bar.sync 1, 128;" ::: "memory");
+      if (t == 0) {
+        mbar_arrive(&B.x_empty);
+        mbar_arrive(full_bar);
+        // carry the tile to the peer CTA; completes on the peer's barrier
+        mbar_arrive_expect_tx_cluster(full_remote, kTile);
+        bulk_s2cluster(dst_remote, dstL, kTile, full_remote);
+        FULL_TRACE(6, j);
       }
-      if (t == 0) FULL_TRACE(6, j);
     }
   } else if (warp >= 8) {
     // ---------------- softmax (thread = query row) ----------------
@@ -352,13 +357,18 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(384, 1)
     RowState st{-INFINITY, 0.f};
     bool ok = true;
     for (int j = 0; j < ntiles; ++j) {
-      if (!mbar_wait(&B.s_full, j & 1, abort, err)) { ok = false; break; }
+      if (!mbar_wait(&B.s_full[j & 1], (j >> 1) & 1, abort, err)) { ok = false; break; }
       if (row == 0) FULL_TRACE(7, j);
       tc_fence_after();
       const int64_t rem = A.T - (int64_t)j * BN;
       const int nk = rem < BN ? (int)rem : BN;
       bool wr;
-      const float corr = softmax_tile(tbase, warp, TM_S, nk, A.zscale, st, wr);
+#ifdef NANOKV_TRACE
+      const int tj = (blockIdx.x == 0 && blockIdx.y == 0 && row == 0) ? j : -1;
+#else
+      const int tj = -1;
+#endif
+      const float corr = softmax_tile(tbase, warp, TM_S + (j & 1) * 128, nk, A.zscale, st, wr, tj);
       if (j > 0 && wr) {
         if (!mbar_wait(&B.pv_done, (j - 1) & 1, abort, err)) { ok = false; break; }
         tc_fence_after();
@@ -366,9 +376,12 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(384, 1)
       }
       tc_fence_before();
       __syncwarp();
-      if (lane == 0) mbar_arrive(&B.p_full);
+      if (lane == 0) mbar_arrive(&B.p_full[j & 1]);
       if (row == 0) FULL_TRACE(8, j);
     }
+    // the value MMAs may trail the softmax by two tiles: wait for the last two
+    // phases in order so that a parity can never be mistaken for an older one
+    if (ok && ntiles >= 2) ok = mbar_wait(&B.pv_done, (ntiles - 2) & 1, abort, err);
     if (ok && mbar_wait(&B.pv_done, (ntiles - 1) & 1, abort, err)) {
       tc_fence_after();
       write_row(tbase, warp, TM_O, st, q0 + row, A.Tq, h, A.H, A.O, A.L);
@@ -445,8 +458,12 @@ cudaError_t tc_attend_full(const void *q, int64_t Tq, const Codec &ck, const Cod
 
 #ifdef NANOKV_TRACE
 extern "C" int nanokv_debug_full_trace(void *host, size_t bytes) {
-  if (bytes < sizeof(g_full_trace)) return -1;
-  return cudaMemcpyFromSymbol(host, g_full_trace, sizeof(g_full_trace)) == cudaSuccess ? 0 : -3;
+  if (bytes < sizeof(g_full_trace) + sizeof(g_softmax_trace)) return -1;
+  if (cudaMemcpyFromSymbol(host, g_full_trace, sizeof(g_full_trace)) != cudaSuccess) return -3;
+  return cudaMemcpyFromSymbol((char *)host + sizeof(g_full_trace), g_softmax_trace, sizeof(g_softmax_trace)) ==
+                 cudaSuccess
+             ? 0
+             : -3;
 }
 #endif
 

@@ -333,16 +333,17 @@ __global__ void __launch_bounds__(384, 1)
       const int64_t rem = A.T - (int64_t)j * BN;
       const int nk = rem < BN ? (int)rem : BN;
       uint32_t v[32];
-      float mx = -INFINITY;
+      float mx4[4] = {-INFINITY, -INFINITY, -INFINITY, -INFINITY};
       for (int c = 0; c < 4; ++c) {
         tmem_ld32(tmem_lane_addr(tbase, warp, sb + 32 * c), v);
 #pragma unroll
         for (int i = 0; i < 32; ++i) {
           const KeyInfo k = ki[32 * c + i];
           const float z = fmaf(__uint_as_float(v[i]), k.sK, qc[k.aK]);
-          mx = (32 * c + i < nk) ? fmaxf(mx, z) : mx;
+          mx4[i & 3] = (32 * c + i < nk) ? fmaxf(mx4[i & 3], z) : mx4[i & 3];
         }
       }
+      const float mx = fmaxf(fmaxf(mx4[0], mx4[1]), fmaxf(mx4[2], mx4[3]));
       float corr = 1.f;
       const bool need = mx > st.m + kRescaleLog2;
       if (need) {
@@ -352,7 +353,7 @@ __global__ void __launch_bounds__(384, 1)
       }
       const bool wr = __any_sync(0xffffffffu, need) != 0;
       const float m = st.m;
-      float lsum = 0.f;
+      float ls[4] = {0.f, 0.f, 0.f, 0.f};
       for (int c = 0; c < 4; ++c) {
         tmem_ld32(tmem_lane_addr(tbase, warp, sb + 32 * c), v);
         uint32_t pp[16], ps[16];
@@ -360,15 +361,18 @@ __global__ void __launch_bounds__(384, 1)
         for (int i = 0; i < 16; ++i) {
           const int k0 = 32 * c + 2 * i;
           const KeyInfo a = ki[k0], b = ki[k0 + 1];
-          const float p0 = (k0 < nk) ? ex2(fmaf(__uint_as_float(v[2 * i]), a.sK, qc[a.aK]) - m) : 0.f;
-          const float p1 = (k0 + 1 < nk) ? ex2(fmaf(__uint_as_float(v[2 * i + 1]), b.sK, qc[b.aK]) - m) : 0.f;
-          lsum += p0 + p1;
+          float p0 = ex2(fmaf(__uint_as_float(v[2 * i]), a.sK, qc[a.aK]) - m);
+          float p1 = ex2(fmaf(__uint_as_float(v[2 * i + 1]), b.sK, qc[b.aK]) - m);
+          p0 = (k0 < nk) ? p0 : 0.f;
+          p1 = (k0 + 1 < nk) ? p1 : 0.f;
+          ls[i & 3] += p0 + p1;
           pp[i] = pack_bf16x2(p0, p1);
           ps[i] = pack_bf16x2(p0 * a.sV, p1 * b.sV);
         }
         tmem_st16(tmem_lane_addr(tbase, warp, sb + 32 * c), pp);
         tmem_st16(tmem_lane_addr(tbase, warp, sb + 32 * c + 16), ps);
       }
+      const float lsum = (ls[0] + ls[1]) + (ls[2] + ls[3]);
       tmem_st_wait();
       st.l += lsum;
       if (j > 0 && wr) {
