@@ -6,6 +6,7 @@ script and the arithmetic accounting used by the benchmark.
 """
 from ._lib import (  # noqa: F401
     Codec, Hist, NanoKVError, alloc_hist, lib, nanokv_attend, nanokv_attend_workspace,
-    nanokv_check, nanokv_encode, nanokv_lse_merge, nanokv_set_kernel_path, nanokv_timing_enable,
+    nanokv_attend_static, nanokv_check, nanokv_encode, nanokv_lse_merge, nanokv_set_kernel_path,
+    nanokv_timing_enable,
     nanokv_timing_read, nanokv_version,
 )

@@ -23,7 +23,7 @@ OK, ERR_INVALID, ERR_UNSUPPORTED, ERR_CUDA, ERR_TIMEOUT = 0, -1, -2, -3, -4
 SYMBOLS = ("nanokv_encode", "nanokv_attend", "nanokv_attend_workspace", "nanokv_lse_merge",
            "nanokv_set_kernel_path", "nanokv_check", "nanokv_last_error", "nanokv_version",
            "nanokv_timing_enable", "nanokv_timing_read", "nanokv_codec_aux_bytes",
-           "nanokv_codec_prepare")
+           "nanokv_codec_prepare", "nanokv_attend_static")
 
 # kernel identities of the diagnostics (nanokv_kernel_id)
 KERNELS = {0: "encode", 1: "attend_full", 2: "attend_low", 3: "attend_dense", 4: "lse_merge"}
@@ -67,6 +67,9 @@ def lib() -> ctypes.CDLL:
     L.nanokv_attend.argtypes = [vp, i32, i64, P(_Codec), P(_Codec), P(_Hist), P(_Hist), i64, i64,
                                 vp, vp, i64, f32, vp, vp, vp, sz, vp]
     L.nanokv_attend.restype = ctypes.c_int
+    L.nanokv_attend_static.argtypes = [vp, i32, i64, P(_Codec), P(_Codec), P(_Hist), P(_Hist), i64, i64,
+                                       vp, vp, i64, f32, vp, vp, vp]
+    L.nanokv_attend_static.restype = ctypes.c_int
     L.nanokv_attend_workspace.argtypes = [i64, P(_Codec), P(_Codec), i64, i64, i64]
     L.nanokv_attend_workspace.restype = sz
     L.nanokv_lse_merge.argtypes = [i32, P(vp), P(vp), i64, i32, i32, vp, i32, vp, vp]
@@ -242,6 +245,32 @@ def nanokv_attend(q: torch.Tensor, ck: Codec, cv: Codec, hk: Hist | None, hv: Hi
         ctypes.byref(shk) if shk else None, ctypes.byref(shv) if shv else None, T, T_full,
         _ptr(k_cur), _ptr(v_cur), T_cur, ctypes.c_float(softmax_scale), _ptr(out), _ptr(lse),
         _ptr(workspace), workspace.numel() * workspace.element_size(), _stream(dev))
+    _raise(st)
+    return out, lse
+
+
+def nanokv_attend_static(q: torch.Tensor, ck: Codec, cv: Codec, hk: Hist | None, hv: Hist | None,
+                         T_full: int, k_cur: torch.Tensor | None = None, v_cur: torch.Tensor | None = None,
+                         softmax_scale: float | None = None, out: torch.Tensor | None = None,
+                         lse: torch.Tensor | None = None):
+    """nanokv_attend for callers that cannot allocate device memory: scratch
+    comes from the library's fixed 32 MiB device array; out and lse must be
+    given (no allocation happens here)."""
+    Tq, H, d = q.shape
+    T = len(hk) if hk is not None else 0
+    T_cur = k_cur.shape[0] if k_cur is not None else 0
+    if softmax_scale is None:
+        softmax_scale = 1.0 / math.sqrt(d)
+    if out is None:
+        raise ValueError("nanokv_attend_static needs a preallocated out tensor")
+    sk, sv = ck.struct(), cv.struct()
+    shk = hk.struct() if hk is not None and T else None
+    shv = hv.struct() if hv is not None and T else None
+    st = lib().nanokv_attend_static(
+        _ptr(q), _dt(q), Tq, ctypes.byref(sk), ctypes.byref(sv),
+        ctypes.byref(shk) if shk else None, ctypes.byref(shv) if shv else None, T, T_full,
+        _ptr(k_cur), _ptr(v_cur), T_cur, ctypes.c_float(softmax_scale), _ptr(out), _ptr(lse),
+        _stream(q.device))
     _raise(st)
     return out, lse
 

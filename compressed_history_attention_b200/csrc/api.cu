@@ -31,6 +31,9 @@ static int fail(int status, const char *fmt, ...) {
   return status;
 }
 
+// records `msg` as the calling thread's last error and returns `status`
+int set_error(int status, const char *msg) { return fail(status, "%s", msg); }
+
 static int cuda_status(cudaError_t e, const char *what) {
   if (e == cudaSuccess) return NANOKV_OK;
   return fail(NANOKV_ERR_CUDA, "%s: %s", what, cudaGetErrorString(e));

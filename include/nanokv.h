@@ -144,6 +144,31 @@ int nanokv_attend(const void *q, int32_t io_dtype, int64_t Tq,
                   float softmax_scale, void *out, float *lse_out,
                   void *workspace, size_t workspace_bytes, void *stream);
 
+/*
+ * nanokv_attend_static -- nanokv_attend without a workspace argument, for
+ * callers that cannot allocate device memory: for example code that runs
+ * where the CUDA allocator must not be entered (it can synchronise the device
+ * and take process-wide locks), or a plug-in that is handed only its input and
+ * output buffers by a host that owns the whole memory pool.  (The pages have no
+ * counterpart; this is a property of the library, not of the method.)
+ * Arguments and results are those of nanokv_attend.  The scratch lives in one
+ * fixed device array of 32 MiB inside the library, which every GPU that loads
+ * the library keeps until the process exits; calls whose
+ * nanokv_attend_workspace(...) exceeds it return NANOKV_ERR_INVALID with a
+ * message.  No allocation or free happens in this call.  The first call on a
+ * device looks up the array's device address (cudaGetSymbolAddress) and caches
+ * it, so make that first call before any stream capture.  All calls share the
+ * array: calls that may overlap on the GPU (other streams, other threads) race
+ * on it and must be serialised by the caller.  Nothing in the array needs to be
+ * zero on entry; it keeps the last call's partial results.
+ */
+int nanokv_attend_static(const void *q, int32_t io_dtype, int64_t Tq,
+                         const nanokv_codec *ck, const nanokv_codec *cv,
+                         const nanokv_hist *hk, const nanokv_hist *hv,
+                         int64_t T, int64_t T_full,
+                         const void *k_cur, const void *v_cur, int64_t T_cur,
+                         float softmax_scale, void *out, float *lse_out, void *stream);
+
 /* Workspace bytes nanokv_attend needs for these sizes (0 is possible). */
 size_t nanokv_attend_workspace(int64_t Tq, const nanokv_codec *ck, const nanokv_codec *cv,
                                int64_t T, int64_t T_full, int64_t T_cur);
