@@ -153,6 +153,96 @@ __device__ __forceinline__ float softmax_tile(uint32_t tbase, int warp, uint32_t
   return corr;
 }
 
+// Half-row variant of softmax_tile: two threads share a query row, thread
+// `half` owning S columns [64 half, 64 half + 64).  The two partial maxima meet
+// in `xmax` (shared, [2 halves][128 rows], one buffer per tile parity): every
+// softmax warp arrives on `xbar` (count: all softmax warps) and waits for its
+// phase `parity` with the usual bound.  The scores stay in registers between
+// the passes.  P of this half goes to columns [32 half, 32 half + 32) of the S
+// buffer (columns the other half had read before arriving).  st.l accumulates
+// this half's share of the row sum.  Returns false if the exchange gave up.
+__device__ __forceinline__ bool softmax_tile_half(uint32_t tbase, int warp, uint32_t s_col, int nk, int half,
+                                                  int row, float *xmax, uint64_t *xbar, uint32_t parity,
+                                                  volatile int *abort, unsigned *err, float zscale,
+                                                  RowState &st, bool &warp_rescale, float &corr) {
+  uint32_t r[64];
+  sm100::tmem_ld64(tmem_lane_addr(tbase, warp, s_col + 64 * half), r);
+  const int base = 64 * half;
+  const bool full = nk >= 128;
+  float mx4[4] = {-INFINITY, -INFINITY, -INFINITY, -INFINITY};
+  if (full) {
+#pragma unroll
+    for (int i = 0; i < 64; ++i) mx4[i & 3] = fmaxf(mx4[i & 3], __uint_as_float(r[i]));
+  } else {
+#pragma unroll
+    for (int i = 0; i < 64; ++i) mx4[i & 3] = (base + i < nk) ? fmaxf(mx4[i & 3], __uint_as_float(r[i])) : mx4[i & 3];
+  }
+  xmax[half * 128 + row] = fmaxf(fmaxf(mx4[0], mx4[1]), fmaxf(mx4[2], mx4[3]));
+  __syncwarp();
+  if ((threadIdx.x & 31) == 0) sm100::mbar_arrive(xbar);
+  if (!sm100::mbar_wait(xbar, parity, abort, err)) return false;
+  const float mx = fmaxf(xmax[row], xmax[128 + row]) * zscale;
+  corr = 1.f;
+  const bool need = mx > st.m + kRescaleLog2;  // identical in both halves
+  if (need) {
+    corr = (st.m == -INFINITY) ? 0.f : ex2(st.m - mx);
+    st.l *= corr;
+    st.m = mx;
+  }
+  warp_rescale = __any_sync(0xffffffffu, need) != 0;
+  const float m = st.m;
+  float ls[4] = {0.f, 0.f, 0.f, 0.f};
+  uint32_t pk[32];
+#pragma unroll
+  for (int i = 0; i < 32; ++i) {
+    const int k0 = base + 2 * i;
+    float p0 = ex2(fmaf(__uint_as_float(r[2 * i]), zscale, -m));
+    float p1 = ex2(fmaf(__uint_as_float(r[2 * i + 1]), zscale, -m));
+    if (!full) {
+      p0 = (k0 < nk) ? p0 : 0.f;
+      p1 = (k0 + 1 < nk) ? p1 : 0.f;
+    }
+    ls[i & 3] += p0 + p1;
+    pk[i] = pack_bf16x2(p0, p1);
+  }
+  uint32_t lo[16], hi[16];
+#pragma unroll
+  for (int i = 0; i < 16; ++i) { lo[i] = pk[i]; hi[i] = pk[16 + i]; }
+  sm100::tmem_st16(tmem_lane_addr(tbase, warp, s_col + 32 * half), lo);
+  sm100::tmem_st16(tmem_lane_addr(tbase, warp, s_col + 32 * half + 16), hi);
+  sm100::tmem_st_wait();
+  st.l += (ls[0] + ls[1]) + (ls[2] + ls[3]);
+  return true;
+}
+
+// Multiplies `ncols` (multiple of 16) fp32 columns of this thread's row at col by f.
+__device__ __forceinline__ void rescale_cols(uint32_t tbase, int warp, uint32_t col, int ncols, float f) {
+  uint32_t v[16];
+  for (int c = 0; c < ncols; c += 16) {
+    const uint32_t a = tmem_lane_addr(tbase, warp, col + c);
+    sm100::tmem_ld16(a, v);
+#pragma unroll
+    for (int i = 0; i < 16; ++i) v[i] = __float_as_uint(__uint_as_float(v[i]) * f);
+    sm100::tmem_st16(a, v);
+  }
+  sm100::tmem_st_wait();
+}
+
+// Writes columns [col0, col0 + 64) of the normalised O row (fp32 partials).
+__device__ __forceinline__ void write_row_half(uint32_t tbase, int warp, uint32_t o_col, int col0, float inv,
+                                               int64_t row, int64_t Tq, int h, int H, float *__restrict__ O) {
+  uint32_t r[64];
+  sm100::tmem_ld64(tmem_lane_addr(tbase, warp, o_col + col0), r);
+  if (row < Tq) {
+    float *dst = O + (row * H + h) * 128 + col0;
+#pragma unroll
+    for (int i = 0; i < 64; i += 4)
+      *reinterpret_cast<float4 *>(dst + i) = make_float4(__uint_as_float(r[i]) * inv, __uint_as_float(r[i + 1]) * inv,
+                                                         __uint_as_float(r[i + 2]) * inv,
+                                                         __uint_as_float(r[i + 3]) * inv);
+  }
+}
+
 // Multiplies this thread's O row (128 fp32 columns at o_col) by f.
 __device__ __forceinline__ void rescale_o(uint32_t tbase, int warp, uint32_t o_col, float f) {
   uint32_t r[16];

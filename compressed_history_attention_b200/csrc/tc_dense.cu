@@ -3,7 +3,8 @@
 // (128-row query tile, head):
 //   warp 0      TMA producer: Q once, then K/V tiles (2 stages)
 //   warp 1      MMA issuer:   S = Q K^T (SS), O += P V (P read from TMEM)
-//   warps 4..7  softmax:      one thread per query row (TMEM lane)
+//   warps 4..11 softmax:      two threads per query row (TMEM lane), each
+//                             owning 64 of the tile's 128 keys
 // S and O accumulate in TMEM; P overwrites S as bf16.  Every wait is bounded.
 #include "tc_common.cuh"
 
@@ -67,9 +68,12 @@ struct DenseBars {
   uint64_t q_full, k_full[2], v_full[2], kv_empty[2], s_full[2], p_full[2], pv_done;
   uint32_t tmem_base;
   int abort;
+  uint64_t xbar[2], lbar;  // row-max exchange per tile parity; final row-sum exchange
+  float xmax[2][2][128];   // [tile parity][half][row] partial row maxima
+  float lsum[2][128];      // [half][row] final partial row sums
 };
 
-__global__ void __launch_bounds__(256, 1)
+__global__ void __launch_bounds__(384, 1)
     tc_dense_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUtensorMap tmK,
                     const __grid_constant__ CUtensorMap tmV, int64_t Tq, int64_t T, int H,
                     float zscale, float *__restrict__ Oout, float *__restrict__ Lout,
@@ -96,9 +100,11 @@ __global__ void __launch_bounds__(256, 1)
     }
     for (int s = 0; s < 2; ++s) {
       mbar_init(&B.s_full[s], 1);
-      mbar_init(&B.p_full[s], 4);
+      mbar_init(&B.p_full[s], 8);
+      mbar_init(&B.xbar[s], 8);
     }
     mbar_init(&B.pv_done, 1);
+    mbar_init(&B.lbar, 8);
     B.abort = 0;
     fence_mbar_init();
   }
@@ -183,8 +189,9 @@ __global__ void __launch_bounds__(256, 1)
       }
     }
   } else if (warp >= 4) {
-    // ---------------- softmax (one thread per query row) ----------------
-    const int row = (warp - 4) * 32 + lane;
+    // ---------------- softmax (two threads per query row) ----------------
+    const int half = (warp - 4) >> 2;  // 0: keys 0..63 of a tile, 1: keys 64..127
+    const int row = (warp & 3) * 32 + lane;
     RowState st{-INFINITY, 0.f};
     bool ok = true;
     for (int j = 0; j < ntiles; ++j) {
@@ -193,11 +200,16 @@ __global__ void __launch_bounds__(256, 1)
       const int64_t rem = T - (int64_t)j * BN;
       const int nk = rem < BN ? (int)rem : BN;
       bool wr;
-      const float corr = softmax_tile(tbase, warp, TM_S + (j & 1) * 128, nk, zscale, st, wr);
+      float corr;
+      if (!softmax_tile_half(tbase, warp, TM_S + (j & 1) * 128, nk, half, row, &B.xmax[j & 1][0][0],
+                             &B.xbar[j & 1], (j >> 1) & 1, abort, err, zscale, st, wr, corr)) {
+        ok = false;
+        break;
+      }
       if (j > 0 && wr) {
         if (!mbar_wait(&B.pv_done, (j - 1) & 1, abort, err)) { ok = false; break; }
         tc_fence_after();
-        rescale_o(tbase, warp, TM_O, corr);
+        rescale_cols(tbase, warp, TM_O + 64 * half, 64, corr);
       }
       tc_fence_before();
       __syncwarp();
@@ -206,9 +218,17 @@ __global__ void __launch_bounds__(256, 1)
     // the value MMAs may trail the softmax by two tiles: wait for the last two
     // phases in order so that a parity can never be mistaken for an older one
     if (ok && ntiles >= 2) ok = mbar_wait(&B.pv_done, (ntiles - 2) & 1, abort, err);
-    if (ok && mbar_wait(&B.pv_done, (ntiles - 1) & 1, abort, err)) {
+    if (ok) ok = mbar_wait(&B.pv_done, (ntiles - 1) & 1, abort, err);
+    B.lsum[half][row] = st.l;
+    __syncwarp();
+    if (lane == 0) mbar_arrive(&B.lbar);
+    if (ok) ok = mbar_wait(&B.lbar, 0, abort, err);
+    if (ok) {
       tc_fence_after();
-      write_row(tbase, warp, TM_O, st, q0 + row, Tq, h, H, Oout, Lout);
+      const float l = B.lsum[0][row] + B.lsum[1][row];
+      const int64_t qrow = q0 + row;
+      write_row_half(tbase, warp, TM_O, 64 * half, l > 0.f ? 1.f / l : 0.f, qrow, Tq, h, H, Oout);
+      if (half == 0 && qrow < Tq) Lout[(int64_t)h * Tq + qrow] = l > 0.f ? (st.m + log2f(l)) * kLn2 : -INFINITY;
     }
   }
   tc_fence_before();
@@ -235,7 +255,7 @@ cudaError_t tc_attend_dense(const void *q, int64_t Tq, int H, int d, const void 
   const size_t smem = 5 * kTileBytes + 1024;
   cudaFuncSetAttribute(tc_dense_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
   dim3 grid((unsigned)((Tq + BM - 1) / BM), (unsigned)H);
-  return launch_k(tc_dense_kernel, grid, dim3(256), smem, st, pdl, mq, mk, mv, Tq, T, H, tau * kLog2e,
+  return launch_k(tc_dense_kernel, grid, dim3(384), smem, st, pdl, mq, mk, mv, Tq, T, H, tau * kLog2e,
                   out.O, out.LSE, error_word_ptr());
 }
 

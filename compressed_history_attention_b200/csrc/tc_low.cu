@@ -67,19 +67,6 @@ __device__ __forceinline__ uint4 unpack8(uint32_t w) {
   return make_uint4(o[0], o[1], o[2], o[3]);
 }
 
-// multiplies `ncols` (multiple of 16) fp32 TMEM columns of this thread's row by f
-__device__ __forceinline__ void rescale_cols(uint32_t tbase, int warp, uint32_t col, int ncols, float f) {
-  uint32_t v[16];
-  for (int c = 0; c < ncols; c += 16) {
-    const uint32_t a = tmem_lane_addr(tbase, warp, col + c);
-    tmem_ld16(a, v);
-#pragma unroll
-    for (int i = 0; i < 16; ++i) v[i] = __float_as_uint(__uint_as_float(v[i]) * f);
-    tmem_st16(a, v);
-  }
-  tmem_st_wait();
-}
-
 __global__ void __launch_bounds__(384, 1)
     tc_low_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUtensorMap tmDk,
                   const __grid_constant__ CUtensorMap tmCk, const __grid_constant__ CUtensorMap tmDv,
