@@ -31,6 +31,24 @@ static int fail(int status, const char *fmt, ...) {
   return status;
 }
 
+cudaError_t ensure_smem(const void *kernel, int bytes) {
+  static std::mutex mu;
+  static std::vector<std::pair<std::pair<const void *, int>, int>> done;  // ((kernel, device), bytes)
+  int dev = 0;
+  cudaGetDevice(&dev);
+  std::lock_guard<std::mutex> lk(mu);
+  for (auto &e : done)
+    if (e.first.first == kernel && e.first.second == dev) {
+      if (e.second >= bytes) return cudaSuccess;
+      const cudaError_t r = cudaFuncSetAttribute(kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, bytes);
+      if (r == cudaSuccess) e.second = bytes;
+      return r;
+    }
+  const cudaError_t r = cudaFuncSetAttribute(kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, bytes);
+  if (r == cudaSuccess) done.push_back({{kernel, dev}, bytes});
+  return r;
+}
+
 // records `msg` as the calling thread's last error and returns `status`
 int set_error(int status, const char *msg) { return fail(status, "%s", msg); }
 

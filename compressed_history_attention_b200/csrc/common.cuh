@@ -68,6 +68,11 @@ struct PartList {
   int n;
 };
 
+// Raises a kernel's dynamic shared-memory limit to `bytes` on the current
+// device the first time a launch needs it (the attribute call is not repeated
+// on every launch).
+cudaError_t ensure_smem(const void *kernel, int bytes);
+
 // ---------------------------------------------------------------------------
 // launchers (return cudaError_t of the launch; shapes already validated)
 // ---------------------------------------------------------------------------

@@ -89,13 +89,13 @@ cudaError_t simt_encode(const Codec &c, const void *x, int64_t T, uint8_t *ids, 
   if (blocks > 148 * 16) blocks = 148 * 16;
   if (c.prec == PREC_F32) {
     auto k = encode_simt_kernel<float, float>;
-    cudaFuncSetAttribute(k, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+    ensure_smem((const void *)k, (int)smem);
     k<<<(unsigned)blocks, wpb * 32, smem, st>>>((const float *)x, T, J, c.r, c.C,
                                                 (const float *)c.centers, (const float *)c.E, ids,
                                                 codes, (float *)scales);
   } else {
     auto k = encode_simt_kernel<__nv_bfloat16, __half>;
-    cudaFuncSetAttribute(k, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+    ensure_smem((const void *)k, (int)smem);
     k<<<(unsigned)blocks, wpb * 32, smem, st>>>(
         (const __nv_bfloat16 *)x, T, J, c.r, c.C, (const __nv_bfloat16 *)c.centers,
         (const __nv_bfloat16 *)c.E, ids, codes, (__half *)scales);
@@ -261,7 +261,7 @@ static cudaError_t launch_attn_simt(const void *q, int64_t Tq, int H, const void
   auto kern = attn_simt_kernel<TIO, TS, DH, DECODE>;
   size_t smem = 2 * SA_BK * DH * sizeof(float);
   if (DECODE) smem += (size_t)SA_BK * (ck.r + cv.r);
-  cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+  ensure_smem((const void *)kern, (int)smem);
   dim3 grid((unsigned)((Tq + SA_BQ - 1) / SA_BQ), (unsigned)H);
   kern<<<grid, SA_THREADS, smem, st>>>((const TIO *)q, Tq, H, (const TIO *)k, (const TIO *)v, ck,
                                         cv, hk, hv, t0, T, tau, out.O, out.LSE);
@@ -472,11 +472,11 @@ cudaError_t simt_attend_low(const float *qred, const float *qc, int64_t Tq, cons
   dim3 grid((unsigned)((Tq + SL_BQ - 1) / SL_BQ), (unsigned)ck.H);
   if (ck.prec == PREC_F32) {
     auto k = attn_low_simt_kernel<float, float>;
-    cudaFuncSetAttribute(k, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+    ensure_smem((const void *)k, (int)smem);
     k<<<grid, SL_THREADS, smem, st>>>(qred, qc, Tq, ck, cv, hk, hv, t0, T, tau, out.O, out.LSE);
   } else {
     auto k = attn_low_simt_kernel<__nv_bfloat16, __half>;
-    cudaFuncSetAttribute(k, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+    ensure_smem((const void *)k, (int)smem);
     k<<<grid, SL_THREADS, smem, st>>>(qred, qc, Tq, ck, cv, hk, hv, t0, T, tau, out.O, out.LSE);
   }
   return cudaGetLastError();

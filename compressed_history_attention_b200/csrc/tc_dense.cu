@@ -253,7 +253,7 @@ cudaError_t tc_attend_dense(const void *q, int64_t Tq, int H, int d, const void 
       !make_tmap_bf16_2d(&mv, v, T, J, J, 128))
     return cudaErrorInvalidValue;
   const size_t smem = 5 * kTileBytes + 1024;
-  cudaFuncSetAttribute(tc_dense_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+  ensure_smem((const void *)tc_dense_kernel, (int)smem);
   dim3 grid((unsigned)((Tq + BM - 1) / BM), (unsigned)H);
   return launch_k(tc_dense_kernel, grid, dim3(384), smem, st, pdl, mq, mk, mv, Tq, T, H, tau * kLog2e,
                   out.O, out.LSE, error_word_ptr());

@@ -20,6 +20,18 @@ namespace nanokv {
 using namespace sm100;
 using namespace tc;
 
+#ifdef NANOKV_TRACE
+__device__ unsigned long long g_enc_trace[8][32];
+#define ENC_TRACE(ev, j)                                                                   \
+  do {                                                                                     \
+    if (blockIdx.x == 0 && blockIdx.y == 0 && (j) < 32) g_enc_trace[ev][j] = clock64();   \
+  } while (0)
+#else
+#define ENC_TRACE(ev, j) \
+  do {                   \
+  } while (0)
+#endif
+
 namespace {
 
 constexpr int NSTG = 3;
@@ -79,16 +91,37 @@ __global__ void __launch_bounds__(256, 1)
     tmem_alloc(&B.tmem_base, tmem_cols);
     tmem_relinquish();
   }
-  if (warp == 2 || warp == 3) {
-    const float *aux = A.aux[br];
-    const int n = A.C * R;
-    for (int i = (warp - 2) * 32 + lane; i < n; i += 64) sEC[(i / R) * (R + 1) + i % R] = aux[i];
-    for (int i = (warp - 2) * 32 + lane; i < A.C; i += 64) sCN[i] = aux[n + i];
+  {
+    // stage the E c table (rows padded to R + 1 floats against bank conflicts)
+    // and |c|^2 with all threads, 16-byte loads, several in flight per thread
+    const float4 *aux4 = reinterpret_cast<const float4 *>(A.aux[br]);
+    const int n4 = A.C * R / 4;
+    constexpr int U = 8;
+    for (int i0 = threadIdx.x; i0 < n4; i0 += U * 256) {
+      float4 v[U];
+#pragma unroll
+      for (int u = 0; u < U; ++u)
+        if (i0 + u * 256 < n4) v[u] = aux4[i0 + u * 256];
+#pragma unroll
+      for (int u = 0; u < U; ++u) {
+        const int i = i0 + u * 256;
+        if (i < n4) {
+          const int e = 4 * i, row = e / R, col = e % R;  // R % 4 == 0: a float4 never straddles rows
+          float *d = sEC + row * (R + 1) + col;
+          d[0] = v[u].x;
+          d[1] = v[u].y;
+          d[2] = v[u].z;
+          d[3] = v[u].w;
+        }
+      }
+    }
+    for (int i = threadIdx.x; i < A.C; i += 256) sCN[i] = A.aux[br][A.C * R + i];
   }
   tc_fence_before();
   __syncthreads();
   tc_fence_after();
   const uint32_t tbase = B.tmem_base;
+  if (threadIdx.x == 0) ENC_TRACE(5, 0);
 
   if (warp == 0) {
     if (lane == 0) {
@@ -99,6 +132,7 @@ __global__ void __launch_bounds__(256, 1)
       for (int kb = 0; kb < nkb; ++kb) {
         const int s = kb % NSTG;
         if (kb >= NSTG && !mbar_wait(&B.empty[s], ((kb / NSTG) - 1) & 1, abort, err)) break;
+        ENC_TRACE(4, kb);
         mbar_arrive_expect_tx(&B.full[s], kA + kB);
         tma_load_2d(sA + s * kA, tmX, kb * 64, (int)t0, &B.full[s]);
         tma_load_2d(sB + s * kB, tmC, kb * 64, 0, &B.full[s]);
@@ -116,6 +150,7 @@ __global__ void __launch_bounds__(256, 1)
         const int s = kb % NSTG, pb = kb & 1;
         if (!mbar_wait(&B.full[s], (kb / NSTG) & 1, abort, err)) { ok = false; break; }
         if (kb >= 2 && !mbar_wait(&B.part_empty[pb], ((kb >> 1) - 1) & 1, abort, err)) { ok = false; break; }
+        ENC_TRACE(0, kb);
         tc_fence_after();
         const uint32_t a = smem_u32(sA + s * kA), b = smem_u32(sB + s * kB);
         const uint32_t be = b + A.C * 128;
@@ -142,6 +177,7 @@ __global__ void __launch_bounds__(256, 1)
     for (int kb = 0; kb < nkb; ++kb) {
       const int pb = kb & 1;
       if (!mbar_wait(&B.part_full[pb], (kb >> 1) & 1, abort, err)) { ok = false; break; }
+      if (row == 0) ENC_TRACE(1, kb);
       tc_fence_after();
       uint32_t g[32];
 #pragma unroll
@@ -153,8 +189,10 @@ __global__ void __launch_bounds__(256, 1)
       tc_fence_before();
       __syncwarp();
       if (lane == 0) mbar_arrive(&B.part_empty[pb]);
+      if (row == 0) ENC_TRACE(2, kb);
     }
     if (ok && mbar_wait(&B.acc_full, 0, abort, err)) {
+      if (row == 0) ENC_TRACE(3, 0);
       tc_fence_after();
       uint32_t g[32];
       // nearest center: argmin |c_j|^2 - 2 x.c_j, strict < keeps the lowest index
@@ -178,8 +216,13 @@ __global__ void __launch_bounds__(256, 1)
         y[k] -= ec[k];
         m = fmaxf(m, fabsf(y[k]));
       }
+      if (row == 0) ENC_TRACE(3, 1);
       const __half sh = __float2half_rn(m / 7.0f);
       const float sf = __half2float(sh);
+      // y * (1/s) with a correctly rounded reciprocal: within an ulp or two of
+      // y / s, so a code can differ only for values within ~1e-7 relative of a
+      // rounding boundary (far inside the tie band)
+      const float inv = sf > 0.f ? __frcp_rn(sf) : 0.f;
       // INT4 codes, two per byte (code 2i in the low nibble)
       uint8_t *crow = A.codes[br] + t * (R / 2);
 #pragma unroll
@@ -190,8 +233,7 @@ __global__ void __launch_bounds__(256, 1)
           uint32_t acc = 0;
 #pragma unroll
           for (int i = 0; i < 8; ++i) {
-            int code = 0;
-            if (sf > 0.f) code = (int)fminf(7.f, fmaxf(-7.f, rintf(y[k0 + 8 * q + i] / sf)));
+            const int code = (int)fminf(7.f, fmaxf(-7.f, rintf(y[k0 + 8 * q + i] * inv)));
             acc |= (uint32_t)(code & 0xF) << (4 * i);
           }
           w[q] = acc;
@@ -202,6 +244,7 @@ __global__ void __launch_bounds__(256, 1)
         A.ids[br][t] = (uint8_t)a;
         A.scales[br][t] = sh;
       }
+      if (row == 0) ENC_TRACE(3, 2);
     }
   }
   tc_fence_before();
@@ -293,7 +336,7 @@ cudaError_t tc_encode_pair(const Codec *c, const void *const *x, int64_t T, uint
   dim3 grid((unsigned)((T + 127) / 128), (unsigned)nbranch);
 #define NANOKV_ENC_CASE(RR)                                                                         \
   case RR:                                                                                          \
-    cudaFuncSetAttribute(tc_encode_kernel<RR>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem); \
+    ensure_smem((const void *)tc_encode_kernel<RR>, (int)smem); \
     tc_encode_kernel<RR><<<grid, 256, smem, st>>>(m[0][0], m[0][1], m[0][2], m[1][0], m[1][1], m[1][2], a); \
     break;
   switch (c[0].r) {
@@ -306,5 +349,12 @@ cudaError_t tc_encode_pair(const Codec *c, const void *const *x, int64_t T, uint
 #undef NANOKV_ENC_CASE
   return cudaGetLastError();
 }
+
+#ifdef NANOKV_TRACE
+extern "C" int nanokv_debug_enc_trace(void *host, size_t bytes) {
+  if (bytes < sizeof(g_enc_trace)) return -1;
+  return cudaMemcpyFromSymbol(host, g_enc_trace, sizeof(g_enc_trace)) == cudaSuccess ? 0 : -3;
+}
+#endif
 
 }  // namespace nanokv

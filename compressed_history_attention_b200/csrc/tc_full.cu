@@ -139,18 +139,50 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(384, 1)
     tmem_relinquish();
   }
   // decoder slice of this CTA's branch, rows h*128.. of D [J, r], permuted
-  // within groups of 8 like the unpacked codes; K-major 128B-swizzled
-  if (warp == 0 || warp == 2 || warp == 3) {
-    const int t = (warp == 0 ? 0 : warp - 1) * 32 + lane;  // 0..95
+  // within groups of 8 like the unpacked codes (K-major 128B-swizzled), and
+  // the head slice of its centers, 16-byte chunk k of row a stored at chunk
+  // (k ^ (a & 15)) so that rows read together spread over the banks.  All
+  // threads stage them with several 16-byte loads in flight each.
+  {
     const __nv_bfloat16 *Dsrc = A.D[rank] + (size_t)h * DH * A.r;
-    const int groups = DH * A.r / 8;
-    for (int gidx = t; gidx < groups; gidx += 96) {
-      const int row = gidx / (A.r / 8), g = gidx % (A.r / 8);
-      const uint4 v = *reinterpret_cast<const uint4 *>(Dsrc + (size_t)row * A.r + 8 * g);
-      // element order (0,4,1,5,2,6,3,7): 16-bit halves of the source words
-      const uint4 o = make_uint4(__byte_perm(v.x, v.z, 0x5410), __byte_perm(v.x, v.z, 0x7632),
-                                 __byte_perm(v.y, v.w, 0x5410), __byte_perm(v.y, v.w, 0x7632));
-      *reinterpret_cast<uint4 *>(sD + sw128_offset(row, 8 * g, DH)) = o;
+    const int gpr = A.r / 8;  // 8-element groups per row
+    const int groups = DH * gpr;
+    constexpr int U = 8;
+    for (int g0 = threadIdx.x; g0 < groups; g0 += U * 384) {
+      uint4 v[U];
+#pragma unroll
+      for (int u = 0; u < U; ++u) {
+        const int gidx = g0 + u * 384;
+        if (gidx < groups) v[u] = *reinterpret_cast<const uint4 *>(Dsrc + (size_t)(gidx / gpr) * A.r + 8 * (gidx % gpr));
+      }
+#pragma unroll
+      for (int u = 0; u < U; ++u) {
+        const int gidx = g0 + u * 384;
+        if (gidx < groups) {
+          // element order (0,4,1,5,2,6,3,7): 16-bit halves of the source words
+          const uint4 o = make_uint4(__byte_perm(v[u].x, v[u].z, 0x5410), __byte_perm(v[u].x, v[u].z, 0x7632),
+                                     __byte_perm(v[u].y, v[u].w, 0x5410), __byte_perm(v[u].y, v[u].w, 0x7632));
+          *reinterpret_cast<uint4 *>(sD + sw128_offset(gidx / gpr, 8 * (gidx % gpr), DH)) = o;
+        }
+      }
+    }
+    const int C = A.C[rank];
+    const __nv_bfloat16 *cen = A.cen[rank] + (size_t)h * DH;
+    for (int i0 = threadIdx.x; i0 < C * 16; i0 += 4 * 384) {
+      uint4 v[4];
+#pragma unroll
+      for (int u = 0; u < 4; ++u) {
+        const int i = i0 + u * 384;
+        if (i < C * 16) v[u] = *reinterpret_cast<const uint4 *>(cen + (size_t)(i >> 4) * J + 8 * (i & 15));
+      }
+#pragma unroll
+      for (int u = 0; u < 4; ++u) {
+        const int i = i0 + u * 384;
+        if (i < C * 16) {
+          const int a = i >> 4, k = i & 15;
+          *reinterpret_cast<uint4 *>(sCen + a * 256 + ((k ^ (a & 15)) << 4)) = v[u];
+        }
+      }
     }
     fence_proxy_async_smem();
   }
@@ -277,17 +309,6 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(384, 1)
     // ---------------- decode epilogue (thread = key) ----------------
     const int t = (warp - 4) * 32 + lane;
     const int C = A.C[rank];
-    // head slice of the centers, 16-byte chunk k of row a stored at chunk
-    // (k ^ (a & 15)) so that rows read together spread over the banks
-    {
-      const __nv_bfloat16 *cen = A.cen[rank] + (size_t)h * DH;
-      for (int i = t; i < C * 16; i += 128) {
-        const int a = i >> 4, k = i & 15;
-        *reinterpret_cast<uint4 *>(sCen + a * 256 + ((k ^ (a & 15)) << 4)) =
-            *reinterpret_cast<const uint4 *>(cen + (size_t)a * J + 8 * k);
-      }
-      asm volatile("bar.sync 1, 128;" ::: "memory");
-    }
     uint8_t *dstL = rank == 0 ? sKh : sVh;
     const uint32_t dst_local = smem_u32(dstL);
     const uint32_t dst_remote = mapa(dst_local, peer);
@@ -450,7 +471,7 @@ cudaError_t tc_attend_full(const void *q, int64_t Tq, const Codec &ck, const Cod
   a.L = out.LSE;
   a.err = error_word_ptr();
   const size_t smem = tc_full_smem(ck.r, ck.C > cv.C ? ck.C : cv.C);
-  cudaFuncSetAttribute(tc_full_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+  ensure_smem((const void *)tc_full_kernel, (int)smem);
   const unsigned qt = (unsigned)((Tq + BM - 1) / BM);
   dim3 grid((qt + 1) & ~1u, (unsigned)ck.H);
   return launch_k(tc_full_kernel, grid, dim3(384), smem, st, pdl, mq, mck, mcv, a);

@@ -472,7 +472,7 @@ cudaError_t tc_attend_low(const void *q, int64_t Tq, const Codec &ck, const Code
   a.L = out.LSE;
   a.err = error_word_ptr();
   const size_t smem = low_smem(ck.r, ck.C);
-  cudaFuncSetAttribute(tc_low_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+  ensure_smem((const void *)tc_low_kernel, (int)smem);
   dim3 grid((unsigned)((Tq + BM - 1) / BM), (unsigned)ck.H);
   tc_low_kernel<<<grid, 384, smem, st>>>(mq, mdk, mck, mdv, mcv, a);
   return cudaGetLastError();
