@@ -399,15 +399,30 @@ def run_fast(a, device, peaks):
     for _ in range(2):
         step_attend(s, w)
     flush = torch.empty(256 * 1024 * 1024, dtype=torch.uint8, device=device)
+    import compressed_history_attention_b200 as nk
     n = max(3, a.steps // 2)
-    _, att = timed_loop(s, w, n, flush, with_encode=False)
+    g = capture(lambda: step_attend(s, w))
+    _, att = timed_loop(s, w, n, flush, with_encode=False, graphs=(None, g))
     ms = sum(att) / n
     af = attend_flops(w.Tq, w.H, w.d, w.r, w.C, w.T_full, w.T_low, w.Tq)
     tf = af["total"] / (ms * 1e-3) / 1e12
-    del s
+    # per-kernel durations from the library's per-launch events (separate loop)
+    nk.nanokv_timing_read()
+    nk.nanokv_timing_enable(True)
+    timed_loop(s, w, n, flush, with_encode=False)
+    nk.nanokv_timing_enable(False)
+    kt = nk.nanokv_timing_read()
+    per = {}
+    for name, work in (("attend_low", af["low"]), ("attend_full", af["full"]), ("attend_dense", af["current"])):
+        ms_k, cnt = kt[name]
+        if cnt:
+            avg = ms_k / cnt
+            per[name] = {"ms": round(avg, 4), "tflops": round(work / (avg * 1e-3) / 1e12, 2),
+                         "frac_bf16_peak": round(work / (avg * 1e-3) / 1e12 / peaks["bf16_tflops"], 4)}
+    del s, g
     torch.cuda.empty_cache()
     return {"workload": w.describe(), "attend_ms": round(ms, 4), "tflops": round(tf, 3),
-            "frac_bf16_peak": round(tf / peaks["bf16_tflops"], 4), "iters": n}
+            "frac_bf16_peak": round(tf / peaks["bf16_tflops"], 4), "iters": n, "kernels": per}
 
 
 # ---------------------------------------------------------------------------

@@ -68,9 +68,9 @@ struct FullBars {
   uint64_t q_full;
   uint64_t st_full[NSTAGE], st_empty[NSTAGE];
   uint64_t ring_full[NRING], ring_empty[NRING];
-  uint64_t x_full, x_empty;
+  uint64_t x_full, x_empty, half_done[2];
   uint64_t kh_full, vh_full, kh_empty, vh_empty;
-  uint64_t s_full[2], p_full[2], pv_done;
+  uint64_t s_full[2], p_full[2], pv_done[2];  // pv_done[b]: P*V of the tiles using S buffer b
   uint32_t tmem_base;
   int abort;
 };
@@ -122,15 +122,20 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(384, 1)
     for (int i = 0; i < NSTAGE; ++i) { mbar_init(&B.st_full[i], 1); mbar_init(&B.st_empty[i], 2); }
     for (int i = 0; i < NRING; ++i) { mbar_init(&B.ring_full[i], 2); mbar_init(&B.ring_empty[i], 1); }
     mbar_init(&B.x_full, 1);
-    mbar_init(&B.x_empty, 1);
+    mbar_init(&B.x_empty, 4);  // one arrive per epilogue warp once its last X load is done
+    mbar_init(&B.half_done[0], 4);
+    mbar_init(&B.half_done[1], 4);
     // decoded-tile barriers: one arrive (the decoder's own elected thread,
     // or its remote expect_tx arrive) plus, for the receiver, the bulk copy bytes
     mbar_init(&B.kh_full, 1);
     mbar_init(&B.vh_full, 1);
     mbar_init(&B.kh_empty, 2);
     mbar_init(&B.vh_empty, 2);
-    for (int i = 0; i < 2; ++i) { mbar_init(&B.s_full[i], 1); mbar_init(&B.p_full[i], 4); }
-    mbar_init(&B.pv_done, 1);
+    for (int i = 0; i < 2; ++i) {
+      mbar_init(&B.s_full[i], 1);
+      mbar_init(&B.p_full[i], 4);
+      mbar_init(&B.pv_done[i], 1);
+    }
     B.abort = 0;
     fence_mbar_init();
   }
@@ -220,62 +225,79 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(384, 1)
     if (lane == 0) {
       const uint32_t aQ = smem_u32(sQ), aD = smem_u32(sD), aR = smem_u32(sRing);
       const uint32_t aK = smem_u32(sKh), aV = smem_u32(sVh);
-      int cc = 0;  // chunk counter
       bool ok = mbar_wait(&B.q_full, 0, abort, err);
-      auto decode = [&](int j) -> bool {
-        if (j >= 1 && !mbar_wait(&B.x_empty, (j - 1) & 1, abort, err)) return false;
-        FULL_TRACE(0, j);
-        const uint32_t dX = tbase + TM_X;
-        for (int cb = 0; cb < nrb; ++cb, ++cc) {
+      // Three independent MMA streams, each issued as soon as its inputs are
+      // ready (polled with non-blocking tests), so that none waits behind
+      // another: decode chunks (X = codes D_h^T), scores S_j = Q K_hat_j^T,
+      // values O += P_j V_hat_j.
+      int jd = 0, cb = 0, cc = 0;  // decode: tile, rank block within it, chunk counter
+      int js = 0, jv = 0;          // next scores / values tile
+      uint64_t t_last = globaltimer();
+      while (ok && jv < ntiles) {
+        bool progress = false;
+        // ---- decode stream
+        if (jd < ntiles && (cb > 0 || jd == 0 || mbar_test(&B.x_empty, (jd - 1) & 1))) {
           const int slot = cc % NRING;
-          if (!mbar_wait(&B.ring_full[slot], (cc / NRING) & 1, abort, err)) return false;
+          if (mbar_test(&B.ring_full[slot], (cc / NRING) & 1)) {
+            if (cb == 0) FULL_TRACE(0, jd);
+            tc_fence_after();
+            const uint32_t a = aR + slot * kChunk, b = aD + cb * kChunk;
+#pragma unroll
+            for (int k = 0; k < 4; ++k)
+              mma_ss(tbase + TM_X, sdesc_sw128(a + 32 * k, 16, 1024), sdesc_sw128(b + 32 * k, 16, 1024), IDESC_DEC,
+                     (cb > 0 || k > 0));
+            mma_commit(&B.ring_empty[slot]);
+            ++cc;
+            if (++cb == nrb) {
+              mma_commit(&B.x_full);
+              FULL_TRACE(1, jd);
+              cb = 0;
+              ++jd;
+            }
+            progress = true;
+          }
+        }
+        // ---- scores stream (the S buffer of tile js last held P of js - 2)
+        if (js < ntiles && mbar_test_cluster(&B.kh_full, js & 1) &&
+            (js < 2 || mbar_test(&B.pv_done[js & 1], ((js - 2) >> 1) & 1))) {
+          FULL_TRACE(2, js);
           tc_fence_after();
-          const uint32_t a = aR + slot * kChunk, b = aD + cb * kChunk;
+          const uint32_t dS = tbase + TM_S + (js & 1) * 128;
 #pragma unroll
-          for (int k = 0; k < 4; ++k)
-            mma_ss(dX, sdesc_sw128(a + 32 * k, 16, 1024), sdesc_sw128(b + 32 * k, 16, 1024), IDESC_DEC,
-                   (cb > 0 || k > 0));
-          mma_commit(&B.ring_empty[slot]);
+          for (int ks = 0; ks < DH / 16; ++ks) {
+            const uint32_t off = (ks >> 2) * (kTile / 2) + (ks & 3) * 32;
+            mma_ss(dS, sdesc_sw128(aQ + off, 16, 1024), sdesc_sw128(aK + off, 16, 1024), IDESC_S, ks > 0);
+          }
+          mma_commit(&B.s_full[js & 1]);
+          mma_commit_mc(&B.kh_empty, 0x1);  // K_hat consumed here: tell the K decoder (CTA 0)
+          ++js;
+          progress = true;
         }
-        mma_commit(&B.x_full);
-        FULL_TRACE(1, j);
-        return true;
-      };
-      auto scores = [&](int j) -> bool {
-        if (!mbar_wait_cluster(&B.kh_full, j & 1, abort, err)) return false;
-        // the S buffer of tile j last held P of tile j - 2
-        if (j >= 2 && !mbar_wait(&B.pv_done, (j - 2) & 1, abort, err)) return false;
-        FULL_TRACE(2, j);
-        tc_fence_after();
-        const uint32_t dS = tbase + TM_S + (j & 1) * 128;
+        // ---- values stream
+        if (jv < js && mbar_test(&B.p_full[jv & 1], (jv >> 1) & 1) && mbar_test_cluster(&B.vh_full, jv & 1)) {
+          FULL_TRACE(3, jv);
+          tc_fence_after();
+          const uint32_t sP = tbase + TM_S + (jv & 1) * 128;
 #pragma unroll
-        for (int ks = 0; ks < DH / 16; ++ks) {
-          const uint32_t off = (ks >> 2) * (kTile / 2) + (ks & 3) * 32;
-          mma_ss(dS, sdesc_sw128(aQ + off, 16, 1024), sdesc_sw128(aK + off, 16, 1024), IDESC_S, ks > 0);
+          for (int ks = 0; ks < BN / 16; ++ks)
+            mma_ts(tbase + TM_O, sP + ks * 8, sdesc_sw128(aV + ks * 2048, kTile / 2, 1024), IDESC_PV,
+                   (jv > 0 || ks > 0));
+          mma_commit(&B.pv_done[jv & 1]);
+          mma_commit_mc(&B.vh_empty, 0x2);  // V_hat consumed: tell the V decoder (CTA 1)
+          ++jv;
+          progress = true;
         }
-        mma_commit(&B.s_full[j & 1]);
-        mma_commit_mc(&B.kh_empty, 0x1);  // K_hat consumed here: tell the K decoder (CTA 0)
-        return true;
-      };
-      auto values = [&](int j) -> bool {
-        if (!mbar_wait(&B.p_full[j & 1], (j >> 1) & 1, abort, err)) return false;
-        if (!mbar_wait_cluster(&B.vh_full, j & 1, abort, err)) return false;
-        FULL_TRACE(3, j);
-        tc_fence_after();
-        const uint32_t sP = tbase + TM_S + (j & 1) * 128;
-#pragma unroll
-        for (int ks = 0; ks < BN / 16; ++ks)
-          mma_ts(tbase + TM_O, sP + ks * 8, sdesc_sw128(aV + ks * 2048, kTile / 2, 1024), IDESC_PV,
-                 (j > 0 || ks > 0));
-        mma_commit(&B.pv_done);
-        mma_commit_mc(&B.vh_empty, 0x2);  // V_hat consumed: tell the V decoder (CTA 1)
-        return true;
-      };
-      // issue order keeps the scores of tile j + 1 ahead of the softmax of tile j
-      if (ok) ok = decode(0) && scores(0);
-      for (int j = 0; ok && j < ntiles; ++j) {
-        if (j + 1 < ntiles && !(decode(j + 1) && scores(j + 1))) break;
-        if (!values(j)) break;
+        if (progress) {
+          t_last = globaltimer();
+        } else {
+          if (*abort) break;
+          if (globaltimer() - t_last > kWaitLimitNs) {
+            *abort = 1;
+            atomicOr(err, ERRW_TIMEOUT);
+            break;
+          }
+          __nanosleep(32);
+        }
       }
     }
   } else if (warp == 2 || warp == 3) {
@@ -345,6 +367,12 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(384, 1)
       for (int c = 0; c < 2; ++c) {
         uint32_t x[64];
         tmem_ld64(tmem_lane_addr(tbase, warp, TM_X + 64 * c), x);
+        if (c == 1) {
+          // X is no longer read by this warp: let the next decode start now
+          tc_fence_before();
+          __syncwarp();
+          if (lane == 0) mbar_arrive(&B.x_empty);
+        }
 #pragma unroll
         for (int g = 0; g < 8; ++g) {
           const uint4 cv = *reinterpret_cast<const uint4 *>(crow + (((8 * c + g) ^ sw) << 4));
@@ -359,17 +387,21 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(384, 1)
           }
           st_shared_v4(dst_local + sw128_offset(t, 64 * c + 8 * g, 128), make_uint4(o[0], o[1], o[2], o[3]));
         }
-      }
-      fence_proxy_async_smem();  // the tile is read by this CTA's MMA and by the bulk copy
-      tc_fence_before();
-      asm volatile("bar.sync 1, 128;" ::: "memory");
-      if (t == 0) {
-        mbar_arrive(&B.x_empty);
-        mbar_arrive(full_bar);
-        // carry the tile to the peer CTA; completes on the peer's barrier
-        mbar_arrive_expect_tx_cluster(full_remote, kTile);
-        bulk_s2cluster(dst_remote, dstL, kTile, full_remote);
-        FULL_TRACE(6, j);
+        // columns [64c, 64c + 64) of every key form one 16 KB block of the
+        // tile: hand it to the local MMA / the peer as soon as it is complete
+        fence_proxy_async_smem();  // read by this CTA's MMA and by the bulk copy
+        tc_fence_before();
+        __syncwarp();
+        if (lane == 0) mbar_arrive(&B.half_done[c]);
+        if (t == 0) {
+          if (!mbar_wait(&B.half_done[c], j & 1, abort, err)) break;
+          if (c == 0) mbar_arrive_expect_tx_cluster(full_remote, kTile);
+          bulk_s2cluster(dst_remote + c * (kTile / 2), dstL + c * (kTile / 2), kTile / 2, full_remote);
+          if (c == 1) {
+            mbar_arrive(full_bar);
+            FULL_TRACE(6, j);
+          }
+        }
       }
     }
   } else if (warp >= 8) {
@@ -391,7 +423,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(384, 1)
 #endif
       const float corr = softmax_tile(tbase, warp, TM_S + (j & 1) * 128, nk, A.zscale, st, wr, tj);
       if (j > 0 && wr) {
-        if (!mbar_wait(&B.pv_done, (j - 1) & 1, abort, err)) { ok = false; break; }
+        if (!mbar_wait(&B.pv_done[(j - 1) & 1], ((j - 1) >> 1) & 1, abort, err)) { ok = false; break; }
         tc_fence_after();
         rescale_o(tbase, warp, TM_O, corr);
       }
@@ -402,8 +434,8 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(384, 1)
     }
     // the value MMAs may trail the softmax by two tiles: wait for the last two
     // phases in order so that a parity can never be mistaken for an older one
-    if (ok && ntiles >= 2) ok = mbar_wait(&B.pv_done, (ntiles - 2) & 1, abort, err);
-    if (ok && mbar_wait(&B.pv_done, (ntiles - 1) & 1, abort, err)) {
+    if (ok && ntiles >= 2) ok = mbar_wait(&B.pv_done[(ntiles - 2) & 1], ((ntiles - 2) >> 1) & 1, abort, err);
+    if (ok && mbar_wait(&B.pv_done[(ntiles - 1) & 1], ((ntiles - 1) >> 1) & 1, abort, err)) {
       tc_fence_after();
       write_row(tbase, warp, TM_O, st, q0 + row, A.Tq, h, A.H, A.O, A.L);
     }
