@@ -97,6 +97,50 @@ static cudaError_t timed(int kid, int nk, cudaStream_t st, F &&launch) {
   return e;
 }
 
+// Helper streams on which the independent branch kernels of one attend call
+// (low-dim, full-dim, current chunk) run concurrently.  The full-dim branch
+// gets the highest priority, so its long two-CTA clusters are dispatched
+// first; the current chunk gets the lowest, so its short CTAs fill the SMs
+// the others leave idle (a partial last wave).  Created once per device and
+// kept for the life of the process; callers on several host threads
+// serialise on the mutex while they enqueue.
+struct BranchStreams {
+  cudaStream_t s[3] = {};
+  cudaEvent_t fork = nullptr, join[3] = {};
+  bool ready = false;
+};
+constexpr int kMaxDevices = 64;
+static std::mutex g_bs_mu;
+static BranchStreams g_bs[kMaxDevices];
+
+// with g_bs_mu held
+static cudaError_t branch_streams(BranchStreams **out) {
+  int dev = 0;
+  cudaError_t e = cudaGetDevice(&dev);
+  if (e != cudaSuccess) return e;
+  if (dev < 0 || dev >= kMaxDevices) return cudaErrorInvalidDevice;
+  BranchStreams &b = g_bs[dev];
+  if (!b.ready) {
+    // creating streams and events is not a stream operation; let it proceed
+    // if this thread is capturing a graph
+    cudaStreamCaptureMode mode = cudaStreamCaptureModeRelaxed;
+    cudaThreadExchangeStreamCaptureMode(&mode);
+    int least = 0, greatest = 0;
+    e = cudaDeviceGetStreamPriorityRange(&least, &greatest);
+    // numerically smaller is higher priority
+    const int prio[3] = {greatest < least ? greatest + 1 : least, greatest, least};
+    for (int i = 0; i < 3 && e == cudaSuccess; ++i)
+      e = cudaStreamCreateWithPriority(&b.s[i], cudaStreamNonBlocking, prio[i]);
+    if (e == cudaSuccess) e = cudaEventCreateWithFlags(&b.fork, cudaEventDisableTiming);
+    for (int i = 0; i < 3 && e == cudaSuccess; ++i) e = cudaEventCreateWithFlags(&b.join[i], cudaEventDisableTiming);
+    cudaThreadExchangeStreamCaptureMode(&mode);
+    if (e != cudaSuccess) return e;
+    b.ready = true;
+  }
+  *out = &b;
+  return cudaSuccess;
+}
+
 static bool aligned16(const void *p) { return ((uintptr_t)p & 15u) == 0; }
 
 unsigned *error_word_ptr() {
@@ -338,54 +382,82 @@ int nanokv_attend(const void *q, int32_t io_dtype, int64_t Tq, const nanokv_code
   const Hist hk = T > 0 ? Hist{hk_->ids, hk_->codes, hk_->scales} : Hist{};
   const Hist hv = T > 0 ? Hist{hv_->ids, hv_->codes, hv_->scales} : Hist{};
   PartList pl{};
-  cudaError_t e;
-  if (T_low > 0) {
+  cudaError_t e = cudaSuccess;
+  const bool on[3] = {T_low > 0, T_full > 0, T_cur > 0};
+  const int nbranch = (int)on[0] + (int)on[1] + (int)on[2];
+  // one branch: everything on the caller's stream; several: fork onto the
+  // helper streams after the caller's prior work, join before the merge.
+  // With per-kernel timing on, the branches run one after another on the
+  // caller's stream, so that each kernel's events time it alone.
+  std::unique_lock<std::mutex> lk(g_bs_mu, std::defer_lock);
+  BranchStreams *bs = nullptr;
+  if (nbranch > 1 && !g_timing.load()) {
+    lk.lock();
+    if ((e = branch_streams(&bs)) != cudaSuccess) return cuda_status(e, "attend helper streams");
+    if ((e = cudaEventRecord(bs->fork, st)) != cudaSuccess) return cuda_status(e, "attend fork");
+  }
+  auto bstream = [&](int b) -> cudaStream_t {
+    if (!bs) return st;
+    e = cudaStreamWaitEvent(bs->s[b], bs->fork, 0);
+    return bs->s[b];
+  };
+  auto join = [&](int b) -> cudaError_t {
+    if (!bs) return cudaSuccess;
+    cudaError_t e2 = cudaEventRecord(bs->join[b], bs->s[b]);
+    return e2 == cudaSuccess ? cudaStreamWaitEvent(st, bs->join[b], 0) : e2;
+  };
+  if (on[0]) {
     Part p{(float *)(ws + w.off_O[0]), (float *)(ws + w.off_L[0])};
+    cudaStream_t bst = bstream(0);
+    if (e != cudaSuccess) return cuda_status(e, "attend fork");
     if (use_tc_low) {
-      e = timed(NANOKV_K_LOW, 1, st, [&] {
-        return tc_attend_low(q, Tq, ck, cv, hk, hv, 0, T_low, softmax_scale, p, st);
+      e = timed(NANOKV_K_LOW, 1, bst, [&] {
+        return tc_attend_low(q, Tq, ck, cv, hk, hv, 0, T_low, softmax_scale, p, bst);
       });
     } else {
       float *qred = (float *)(ws + w.off_qred), *qc = (float *)(ws + w.off_qc);
-      e = timed(NANOKV_K_LOW, 2, st, [&] {
-        cudaError_t e2 = simt_low_prep(q, Tq, ck, qred, qc, st);
+      e = timed(NANOKV_K_LOW, 2, bst, [&] {
+        cudaError_t e2 = simt_low_prep(q, Tq, ck, qred, qc, bst);
         if (e2 == cudaSuccess)
-          e2 = simt_attend_low(qred, qc, Tq, ck, cv, hk, hv, 0, T_low, softmax_scale, p, st);
+          e2 = simt_attend_low(qred, qc, Tq, ck, cv, hk, hv, 0, T_low, softmax_scale, p, bst);
         return e2;
       });
     }
+    if (e == cudaSuccess) e = join(0);
     if (e != cudaSuccess) return cuda_status(e, "attend low-dim launch");
     pl.O[pl.n] = p.O;
     pl.LSE[pl.n++] = p.LSE;
   }
-  if (T_full > 0) {
+  if (on[1]) {
     Part p{(float *)(ws + w.off_O[1]), (float *)(ws + w.off_L[1])};
-    e = timed(NANOKV_K_FULL, 1, st, [&] {
+    cudaStream_t bst = bstream(1);
+    if (e != cudaSuccess) return cuda_status(e, "attend fork");
+    e = timed(NANOKV_K_FULL, 1, bst, [&] {
       return (path != 1 && tc_full_ok)
-                 ? tc_attend_full(q, Tq, ck, cv, hk, hv, T_low, T_full, softmax_scale, p, st,
-                                  T_low > 0 && use_tc_low)
-                 : simt_attend_full(q, Tq, ck, cv, hk, hv, T_low, T_full, softmax_scale, p, st);
+                 ? tc_attend_full(q, Tq, ck, cv, hk, hv, T_low, T_full, softmax_scale, p, bst, false)
+                 : simt_attend_full(q, Tq, ck, cv, hk, hv, T_low, T_full, softmax_scale, p, bst);
     });
+    if (e == cudaSuccess) e = join(1);
     if (e != cudaSuccess) return cuda_status(e, "attend full-dim launch");
     pl.O[pl.n] = p.O;
     pl.LSE[pl.n++] = p.LSE;
   }
-  // the current-chunk kernel may overlap the tail of a preceding tensor-core
-  // attention kernel of this call (it reads none of their outputs)
-  const bool prev_tc = (T_full > 0 && path != 1 && tc_full_ok) || (T_full == 0 && T_low > 0 && use_tc_low);
-  if (T_cur > 0) {
+  if (on[2]) {
     Part p{(float *)(ws + w.off_O[2]), (float *)(ws + w.off_L[2])};
-    e = timed(NANOKV_K_DENSE, 1, st, [&] {
+    cudaStream_t bst = bstream(2);
+    if (e != cudaSuccess) return cuda_status(e, "attend fork");
+    e = timed(NANOKV_K_DENSE, 1, bst, [&] {
       return (path != 1 && tc_dense_ok)
-                 ? tc_attend_dense(q, Tq, ck.H, ck.d, k_cur, v_cur, T_cur, softmax_scale, p, st,
-                                   prev_tc)
+                 ? tc_attend_dense(q, Tq, ck.H, ck.d, k_cur, v_cur, T_cur, softmax_scale, p, bst, false)
                  : simt_attend_dense(ck.prec, q, Tq, ck.H, ck.d, k_cur, v_cur, T_cur,
-                                     softmax_scale, p, st);
+                                     softmax_scale, p, bst);
     });
+    if (e == cudaSuccess) e = join(2);
     if (e != cudaSuccess) return cuda_status(e, "attend current-chunk launch");
     pl.O[pl.n] = p.O;
     pl.LSE[pl.n++] = p.LSE;
   }
+  if (lk.owns_lock()) lk.unlock();
   e = timed(NANOKV_K_MERGE, 1, st,
             [&] { return lse_merge_launch(pl, Tq, ck.H, ck.d, out, ck.prec, lse_out, st); });
   return cuda_status(e, "attend merge launch");

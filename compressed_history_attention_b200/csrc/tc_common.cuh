@@ -123,16 +123,18 @@ __device__ __forceinline__ float softmax_tile(uint32_t tbase, int warp, uint32_t
   SOFTMAX_TRACE(1, trace_j);
   const float m = st.m;
   float ls[4] = {0.f, 0.f, 0.f, 0.f};
+  // pass 2 in 32-column chunks (fewer live registers than 64)
 #pragma unroll
-  for (int c = 0; c < 2; ++c) {
-    sm100::tmem_ld64(tmem_lane_addr(tbase, warp, s_col + 64 * c), r);
+  for (int c = 0; c < 4; ++c) {
+    uint32_t r32[32];
+    sm100::tmem_ld32(tmem_lane_addr(tbase, warp, s_col + 32 * c), r32);
     if (c == 0) SOFTMAX_TRACE(2, trace_j);
-    uint32_t pk[32];
+    uint32_t pk[16];
 #pragma unroll
-    for (int i = 0; i < 32; ++i) {
-      const int k0 = 64 * c + 2 * i;
-      float p0 = ex2(fmaf(__uint_as_float(r[2 * i]), zscale, -m));
-      float p1 = ex2(fmaf(__uint_as_float(r[2 * i + 1]), zscale, -m));
+    for (int i = 0; i < 16; ++i) {
+      const int k0 = 32 * c + 2 * i;
+      float p0 = ex2(fmaf(__uint_as_float(r32[2 * i]), zscale, -m));
+      float p1 = ex2(fmaf(__uint_as_float(r32[2 * i + 1]), zscale, -m));
       if (!full) {
         p0 = (k0 < nk) ? p0 : 0.f;
         p1 = (k0 + 1 < nk) ? p1 : 0.f;
@@ -140,12 +142,9 @@ __device__ __forceinline__ float softmax_tile(uint32_t tbase, int warp, uint32_t
       ls[i & 3] += p0 + p1;
       pk[i] = pack_bf16x2(p0, p1);
     }
-    // P chunk c covers columns [32c, 32c + 32), all of S chunk c already read
-    uint32_t lo[16], hi[16];
-#pragma unroll
-    for (int i = 0; i < 16; ++i) { lo[i] = pk[i]; hi[i] = pk[16 + i]; }
-    sm100::tmem_st16(tmem_lane_addr(tbase, warp, s_col + 32 * c), lo);
-    sm100::tmem_st16(tmem_lane_addr(tbase, warp, s_col + 32 * c + 16), hi);
+    // P of S columns [32c, 32c + 32) goes to columns [16c, 16c + 16), all of
+    // which were read by this chunk or an earlier one
+    sm100::tmem_st16(tmem_lane_addr(tbase, warp, s_col + 16 * c), pk);
   }
   sm100::tmem_st_wait();
   SOFTMAX_TRACE(3, trace_j);

@@ -10,9 +10,12 @@
 // rows and each CTA keeps a single decoder slice D_h resident.
 //
 // Roles (12 warps):
-//   warp 0      TMA: Q tile; packed code chunks [128 keys x 32 B] into staging
-//   warp 1      MMA issuer: X = codes D_h^T (decode), S = Q K_hat^T, O += P V_hat
-//   warps 2,3   unpack INT4 staging -> bf16 operand ring (128 keys x 64 codes)
+//   warp 0      TMEM allocation (otherwise idle)
+//   warp 1      TMA (Q tile) and MMA issue: X = codes D_h^T (decode),
+//               S = Q K_hat^T, O += P V_hat
+//   warps 2,3   unpack: packed INT4 codes, read from global memory, -> bf16
+//               operand ring (128 keys x 64 codes per chunk; each warp takes
+//               64 of the keys of every chunk)
 //   warps 4..7  decode epilogue: X (TMEM, lane = key) * s + center -> bf16 tile
 //               in both CTAs' shared memory
 //   warps 8..11 softmax, one thread per query row; final O / LSE
@@ -29,7 +32,7 @@ using namespace tc;
 // Optional event trace of the first cluster of head 0 (debug builds with
 // -DNANOKV_TRACE only): clock64 stamps per role and key tile.
 #ifdef NANOKV_TRACE
-__device__ unsigned long long g_full_trace[2][16][128];
+__device__ unsigned long long g_full_trace[2][24][128];
 #define FULL_TRACE(ev, j)                                                                    \
   do {                                                                                       \
     if (blockIdx.y == 0 && blockIdx.x < 2 && (j) < 128) g_full_trace[rank][ev][j] = clock64(); \
@@ -45,8 +48,7 @@ namespace {
 constexpr int DH = 128;
 constexpr uint32_t kTile = 128 * 128 * 2;   // [128 x 128] bf16
 constexpr uint32_t kChunk = 128 * 64 * 2;   // [128 keys x 64 codes] bf16
-constexpr uint32_t kStage = 128 * 32;       // [128 keys x 32 bytes] packed
-constexpr int NRING = 3, NSTAGE = 4;
+constexpr int NRING = 4;  // unpacked code chunks in flight
 constexpr uint32_t IDESC_DEC = idesc_bf16(128, 128, false, false);
 constexpr uint32_t IDESC_S = idesc_bf16(128, 128, false, false);
 constexpr uint32_t IDESC_PV = idesc_bf16(128, 128, false, true);
@@ -56,6 +58,7 @@ struct FullArgs {
   const __nv_bfloat16 *D[2];    // decoders [J, r] (K, V)
   const __nv_bfloat16 *cen[2];  // centers [C, J]
   const uint8_t *ids[2];        // [T_total]
+  const uint8_t *codes[2];      // [T_total, r / 2] packed INT4
   const __half *scales[2];      // [T_total]
   int64_t t0, T, Tq;            // branch = history tokens [t0, t0 + T)
   int H, r, C[2];
@@ -66,7 +69,6 @@ struct FullArgs {
 
 struct FullBars {
   uint64_t q_full;
-  uint64_t st_full[NSTAGE], st_empty[NSTAGE];
   uint64_t ring_full[NRING], ring_empty[NRING];
   uint64_t x_full, x_empty, half_done[2];
   uint64_t kh_full, vh_full, kh_empty, vh_empty;
@@ -92,8 +94,7 @@ __device__ __forceinline__ uint4 unpack8(uint32_t w) {
 }
 
 __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(384, 1)
-    tc_full_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUtensorMap tmCk,
-                   const __grid_constant__ CUtensorMap tmCv, const FullArgs A) {
+    tc_full_kernel(const __grid_constant__ CUtensorMap tmQ, const FullArgs A) {
   extern __shared__ uint8_t smraw[];
   uint8_t *sm = (uint8_t *)(((uintptr_t)smraw + 1023) & ~(uintptr_t)1023);
   const int nrb = A.r / 64;  // 64-wide rank blocks
@@ -102,8 +103,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(384, 1)
   uint8_t *sRing = sD + nrb * kChunk;
   uint8_t *sKh = sRing + NRING * kChunk;
   uint8_t *sVh = sKh + kTile;
-  uint8_t *sStage = sVh + kTile;
-  uint8_t *sCen = sStage + NSTAGE * kStage;  // this CTA's branch centers, head slice [C][128] bf16
+  uint8_t *sCen = sVh + kTile;  // this CTA's branch centers, head slice [C][128] bf16
   __shared__ FullBars B;
 
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
@@ -119,14 +119,14 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(384, 1)
 
   if (threadIdx.x == 0) {
     mbar_init(&B.q_full, 1);
-    for (int i = 0; i < NSTAGE; ++i) { mbar_init(&B.st_full[i], 1); mbar_init(&B.st_empty[i], 2); }
     for (int i = 0; i < NRING; ++i) { mbar_init(&B.ring_full[i], 2); mbar_init(&B.ring_empty[i], 1); }
     mbar_init(&B.x_full, 1);
     mbar_init(&B.x_empty, 4);  // one arrive per epilogue warp once its last X load is done
     mbar_init(&B.half_done[0], 4);
     mbar_init(&B.half_done[1], 4);
-    // decoded-tile barriers: one arrive (the decoder's own elected thread,
-    // or its remote expect_tx arrive) plus, for the receiver, the bulk copy bytes
+    // decoded-tile barriers: in the decoding CTA one arrive by its epilogue;
+    // in the receiving CTA one expect_tx arrive, by its own MMA thread, that
+    // arms each phase for the bytes of the two bulk copies from the decoder
     mbar_init(&B.kh_full, 1);
     mbar_init(&B.vh_full, 1);
     mbar_init(&B.kh_empty, 2);
@@ -137,6 +137,8 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(384, 1)
       mbar_init(&B.pv_done[i], 1);
     }
     B.abort = 0;
+    // phase 0 of the barrier of the tile this CTA receives
+    mbar_arrive_expect_tx(rank == 1 ? &B.kh_full : &B.vh_full, kTile);
     fence_mbar_init();
   }
   if (warp == 0) {
@@ -198,31 +200,13 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(384, 1)
   const uint32_t tbase = B.tmem_base;
   pdl_launch_dependents();
 
-  if (warp == 0) {
-    // ---------------- TMA producer ----------------
+  if (warp == 1) {
+    // ---------------- Q load and MMA issuer ----------------
     if (lane == 0) {
-      const CUtensorMap *tmC = rank == 0 ? &tmCk : &tmCv;
       prefetch_tmap(&tmQ);
-      prefetch_tmap(tmC);
       mbar_arrive_expect_tx(&B.q_full, kTile);
       tma_load_2d(sQ, &tmQ, h * DH, (int)q0, &B.q_full);
       tma_load_2d(sQ + kTile / 2, &tmQ, h * DH + 64, (int)q0, &B.q_full);
-      int issued = 0;
-      for (int c = 0; c < nchunk; ++c) {
-        const int slot = c % NSTAGE;
-        if (c >= NSTAGE && !mbar_wait(&B.st_empty[slot], ((c / NSTAGE) - 1) & 1, abort, err)) break;
-        const int j = c / nrb, cb = c % nrb;
-        mbar_arrive_expect_tx(&B.st_full[slot], kStage);
-        tma_load_2d(sStage + slot * kStage, tmC, cb * 32, (int)(A.t0 + (int64_t)j * BN), &B.st_full[slot]);
-        issued = c + 1;
-      }
-      mbar_wait(&B.q_full, 0, nullptr, nullptr);
-      for (int c = (issued > NSTAGE ? issued - NSTAGE : 0); c < issued; ++c)
-        mbar_wait(&B.st_full[c % NSTAGE], (c / NSTAGE) & 1, nullptr, nullptr);
-    }
-  } else if (warp == 1) {
-    // ---------------- MMA issuer ----------------
-    if (lane == 0) {
       const uint32_t aQ = smem_u32(sQ), aD = smem_u32(sD), aR = smem_u32(sRing);
       const uint32_t aK = smem_u32(sKh), aV = smem_u32(sVh);
       bool ok = mbar_wait(&B.q_full, 0, abort, err);
@@ -261,6 +245,9 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(384, 1)
         if (js < ntiles && mbar_test_cluster(&B.kh_full, js & 1) &&
             (js < 2 || mbar_test(&B.pv_done[js & 1], ((js - 2) >> 1) & 1))) {
           FULL_TRACE(2, js);
+          // the K_hat receiver arms the next phase (its bytes can only come
+          // after this tile's scores are done in both CTAs)
+          if (rank == 1 && js + 1 < ntiles) mbar_arrive_expect_tx(&B.kh_full, kTile);
           tc_fence_after();
           const uint32_t dS = tbase + TM_S + (js & 1) * 128;
 #pragma unroll
@@ -276,6 +263,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(384, 1)
         // ---- values stream
         if (jv < js && mbar_test(&B.p_full[jv & 1], (jv >> 1) & 1) && mbar_test_cluster(&B.vh_full, jv & 1)) {
           FULL_TRACE(3, jv);
+          if (rank == 0 && jv + 1 < ntiles) mbar_arrive_expect_tx(&B.vh_full, kTile);
           tc_fence_after();
           const uint32_t sP = tbase + TM_S + (jv & 1) * 128;
 #pragma unroll
@@ -301,31 +289,49 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(384, 1)
       }
     }
   } else if (warp == 2 || warp == 3) {
-    // ---------------- unpack: staging (packed) -> ring (bf16, K-major SW128) ----------------
-    const int u = (warp - 2) * 32 + lane;  // keys u and u + 64
-    for (int c = 0; c < nchunk; ++c) {
-      const int slot = c % NSTAGE, rs = c % NRING;
-      if (!mbar_wait(&B.st_full[slot], (c / NSTAGE) & 1, abort, err)) break;
-      if (u == 0 && c % nrb == 0) FULL_TRACE(9, c / nrb);
-      const uint4 *src = reinterpret_cast<const uint4 *>(sStage + slot * kStage);
-      const uint4 p0 = src[2 * u], p1 = src[2 * u + 1];
-      const uint4 p2 = src[2 * (u + 64)], p3 = src[2 * (u + 64) + 1];
-      __syncwarp();
-      if (lane == 0) mbar_arrive(&B.st_empty[slot]);
-      if (c >= NRING && !mbar_wait(&B.ring_empty[rs], ((c / NRING) - 1) & 1, abort, err)) break;
-      if (u == 0 && c % nrb == 0) FULL_TRACE(10, c / nrb);
-      uint8_t *dst = sRing + rs * kChunk;
-      const uint32_t w0[8] = {p0.x, p0.y, p0.z, p0.w, p1.x, p1.y, p1.z, p1.w};
-      const uint32_t w1[8] = {p2.x, p2.y, p2.z, p2.w, p3.x, p3.y, p3.z, p3.w};
+    // ---------------- unpack: packed codes -> ring (bf16, K-major SW128) ----------------
+    // Each thread takes keys kb + lane and kb + 32 + lane of every chunk and
+    // reads their 32 code bytes straight from global memory, one chunk ahead.
+    // (The codes go to registers, not through a shared staging buffer that a
+    // copy engine would refill while these loads might still be in flight.)
+    const uint8_t *codes = A.codes[rank];
+    const int64_t rowb = A.r / 2;        // packed bytes per token
+    const int kb = (warp - 2) * 64;
+    auto load = [&](int c, uint4(&v)[4]) {
+      const int j = c / nrb, cb = c % nrb;
 #pragma unroll
-      for (int g = 0; g < 8; ++g) {
-        *reinterpret_cast<uint4 *>(dst + sw128_offset(u, 8 * g, 128)) = unpack8(w0[g]);
-        *reinterpret_cast<uint4 *>(dst + sw128_offset(u + 64, 8 * g, 128)) = unpack8(w1[g]);
+      for (int i = 0; i < 2; ++i) {
+        int64_t t = (int64_t)j * BN + kb + lane + 32 * i;
+        t = t < A.T ? t : A.T - 1;  // keys past the end: any valid row (masked later)
+        const uint4 *src = reinterpret_cast<const uint4 *>(codes + (A.t0 + t) * rowb + cb * 32);
+        v[2 * i] = __ldg(src);
+        v[2 * i + 1] = __ldg(src + 1);
       }
+    };
+    uint4 cur[4], nxt[4];
+    load(0, cur);
+    for (int c = 0; c < nchunk; ++c) {
+      if (c + 1 < nchunk) load(c + 1, nxt);
+      const int rs = c % NRING, cb = c % nrb;
+      if (warp == 2 && lane == 0 && cb == 0) FULL_TRACE(9, c / nrb);
+      if (c >= NRING && !mbar_wait(&B.ring_empty[rs], ((c / NRING) - 1) & 1, abort, err)) break;
+      if (warp == 2 && lane == 0 && cb == 0) FULL_TRACE(10, c / nrb);
+      const uint32_t dst = smem_u32(sRing + rs * kChunk);
+#pragma unroll
+      for (int i = 0; i < 2; ++i) {
+        const uint32_t w[8] = {cur[2 * i].x,     cur[2 * i].y,     cur[2 * i].z,     cur[2 * i].w,
+                               cur[2 * i + 1].x, cur[2 * i + 1].y, cur[2 * i + 1].z, cur[2 * i + 1].w};
+#pragma unroll
+        for (int g = 0; g < 8; ++g) st_shared_v4(dst + sw128_offset(kb + lane + 32 * i, 8 * g, 128), unpack8(w[g]));
+      }
+      if (warp == 2 && lane == 0 && cb == 1) FULL_TRACE(19, c / nrb);
       fence_proxy_async_smem();
       __syncwarp();
       if (lane == 0) mbar_arrive(&B.ring_full[rs]);
-      if (u == 0 && c % nrb == nrb - 1) FULL_TRACE(11, c / nrb);
+      if (warp == 2 && lane == 0 && cb == nrb - 1) FULL_TRACE(11, c / nrb);
+      if (warp == 2 && lane == 0 && cb == 1) FULL_TRACE(20, c / nrb);
+#pragma unroll
+      for (int k = 0; k < 4; ++k) cur[k] = nxt[k];
     }
   } else if (warp >= 4 && warp < 8) {
     // ---------------- decode epilogue (thread = key) ----------------
@@ -355,47 +361,59 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(384, 1)
       const int sw = a & 15;
       if (!mbar_wait(&B.x_full, j & 1, abort, err)) break;
       if (t == 0) FULL_TRACE(4, j);
-      // the previous tile in this buffer was consumed by both CTAs (and the
-      // bulk copy that carried it to the peer had completed before that)
-      if (j > 0 && !mbar_wait_cluster(empty_bar, (j - 1) & 1, abort, err)) break;
-      if (t == 0) FULL_TRACE(5, j);
       tc_fence_after();
       // K_hat = c + s x in packed bf16x2: x rounded to bf16, one fused
-      // multiply-add per pair, one rounding of the result
+      // multiply-add per pair, one rounding of the result.  The whole row is
+      // computed into registers and X released before the destination
+      // buffer is waited for, so the next decode overlaps the hand-off.
       const __nv_bfloat162 s2 = __floats2bfloat162_rn(s, s);
-#pragma unroll 1
-      for (int c = 0; c < 2; ++c) {
-        uint32_t x[64];
-        tmem_ld64(tmem_lane_addr(tbase, warp, TM_X + 64 * c), x);
-        if (c == 1) {
+      uint32_t o[64];
+#pragma unroll
+      for (int c = 0; c < 4; ++c) {
+        uint32_t x[32];
+        tmem_ld32(tmem_lane_addr(tbase, warp, TM_X + 32 * c), x);
+        if (c == 3) {
           // X is no longer read by this warp: let the next decode start now
           tc_fence_before();
           __syncwarp();
           if (lane == 0) mbar_arrive(&B.x_empty);
         }
 #pragma unroll
-        for (int g = 0; g < 8; ++g) {
-          const uint4 cv = *reinterpret_cast<const uint4 *>(crow + (((8 * c + g) ^ sw) << 4));
+        for (int g = 0; g < 4; ++g) {
+          const uint4 cv = *reinterpret_cast<const uint4 *>(crow + (((4 * c + g) ^ sw) << 4));
           const uint32_t cw[4] = {cv.x, cv.y, cv.z, cv.w};
-          uint32_t o[4];
 #pragma unroll
           for (int i = 0; i < 4; ++i) {
             const uint32_t xp = pack_bf16x2(__uint_as_float(x[8 * g + 2 * i]), __uint_as_float(x[8 * g + 2 * i + 1]));
             const __nv_bfloat162 r = __hfma2(s2, *reinterpret_cast<const __nv_bfloat162 *>(&xp),
                                              *reinterpret_cast<const __nv_bfloat162 *>(&cw[i]));
-            o[i] = *reinterpret_cast<const uint32_t *>(&r);
+            o[16 * c + 4 * g + i] = *reinterpret_cast<const uint32_t *>(&r);
           }
-          st_shared_v4(dst_local + sw128_offset(t, 64 * c + 8 * g, 128), make_uint4(o[0], o[1], o[2], o[3]));
         }
+      }
+      if (t == 0) FULL_TRACE(22, j);
+      // the previous tile in this buffer was consumed by both CTAs (and the
+      // bulk copy that carried it to the peer had completed before that)
+      if (j > 0 && !mbar_wait_cluster(empty_bar, (j - 1) & 1, abort, err)) break;
+      if (t == 0) FULL_TRACE(5, j);
+      bool ok = true;
+#pragma unroll
+      for (int c = 0; c < 2; ++c) {
+#pragma unroll
+        for (int g = 0; g < 8; ++g)
+          st_shared_v4(dst_local + sw128_offset(t, 64 * c + 8 * g, 128),
+                       make_uint4(o[32 * c + 4 * g], o[32 * c + 4 * g + 1], o[32 * c + 4 * g + 2], o[32 * c + 4 * g + 3]));
         // columns [64c, 64c + 64) of every key form one 16 KB block of the
         // tile: hand it to the local MMA / the peer as soon as it is complete
+        if (t == 0 && c == 0) FULL_TRACE(12, j);
         fence_proxy_async_smem();  // read by this CTA's MMA and by the bulk copy
-        tc_fence_before();
+        if (t == 0 && c == 0) FULL_TRACE(13, j);
+        if (t == 96 && c == 0) FULL_TRACE(14, j);
         __syncwarp();
         if (lane == 0) mbar_arrive(&B.half_done[c]);
         if (t == 0) {
-          if (!mbar_wait(&B.half_done[c], j & 1, abort, err)) break;
-          if (c == 0) mbar_arrive_expect_tx_cluster(full_remote, kTile);
+          if (!mbar_wait(&B.half_done[c], j & 1, abort, err)) { ok = false; break; }
+          FULL_TRACE(15 + c, j);
           bulk_s2cluster(dst_remote + c * (kTile / 2), dstL + c * (kTile / 2), kTile / 2, full_remote);
           if (c == 1) {
             mbar_arrive(full_bar);
@@ -403,6 +421,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(384, 1)
           }
         }
       }
+      if (!ok) break;
     }
   } else if (warp >= 8) {
     // ---------------- softmax (thread = query row) ----------------
@@ -467,8 +486,7 @@ bool tc_full_supported(const Codec &ck, const Codec &cv) {
 }
 
 size_t tc_full_smem(int r, int C) {
-  return (size_t)3 * kTile + (size_t)(r / 64) * kChunk + NRING * kChunk + NSTAGE * kStage + (size_t)C * 256 +
-         1024;
+  return (size_t)3 * kTile + (size_t)(r / 64) * kChunk + NRING * kChunk + (size_t)C * 256 + 1024;
 }
 
 cudaError_t tc_attend_full(const void *q, int64_t Tq, const Codec &ck, const Codec &cv,
@@ -476,12 +494,8 @@ cudaError_t tc_attend_full(const void *q, int64_t Tq, const Codec &ck, const Cod
                            Part out, cudaStream_t st, bool pdl) {
   if (Tq == 0 || T == 0) return cudaSuccess;
   const int J = ck.H * DH;
-  const int64_t T_total = t0 + T;
-  CUtensorMap mq, mck, mcv;
-  if (!make_tmap_bf16_2d(&mq, q, Tq, J, J, 128) ||
-      !make_tmap_u8_2d(&mck, hk.codes, T_total, ck.r / 2, ck.r / 2, 32, 128) ||
-      !make_tmap_u8_2d(&mcv, hv.codes, T_total, cv.r / 2, cv.r / 2, 32, 128))
-    return cudaErrorInvalidValue;
+  CUtensorMap mq;
+  if (!make_tmap_bf16_2d(&mq, q, Tq, J, J, 128)) return cudaErrorInvalidValue;
   FullArgs a;
   a.D[0] = (const __nv_bfloat16 *)ck.D;
   a.D[1] = (const __nv_bfloat16 *)cv.D;
@@ -489,6 +503,8 @@ cudaError_t tc_attend_full(const void *q, int64_t Tq, const Codec &ck, const Cod
   a.cen[1] = (const __nv_bfloat16 *)cv.centers;
   a.ids[0] = hk.ids;
   a.ids[1] = hv.ids;
+  a.codes[0] = hk.codes;
+  a.codes[1] = hv.codes;
   a.scales[0] = (const __half *)hk.scales;
   a.scales[1] = (const __half *)hv.scales;
   a.t0 = t0;
@@ -506,7 +522,7 @@ cudaError_t tc_attend_full(const void *q, int64_t Tq, const Codec &ck, const Cod
   ensure_smem((const void *)tc_full_kernel, (int)smem);
   const unsigned qt = (unsigned)((Tq + BM - 1) / BM);
   dim3 grid((qt + 1) & ~1u, (unsigned)ck.H);
-  return launch_k(tc_full_kernel, grid, dim3(384), smem, st, pdl, mq, mck, mcv, a);
+  return launch_k(tc_full_kernel, grid, dim3(384), smem, st, pdl, mq, a);
 }
 
 #ifdef NANOKV_TRACE

@@ -172,3 +172,59 @@ def test_lse_merge_parity():
         fin = np.isfinite(Lr)
         assert np.array_equal(np.isfinite(orc.f64(lse)), fin)
         assert np.abs(orc.f64(lse)[fin] - Lr[fin]).max() <= 1e-5
+
+
+@pytest.mark.parametrize("name", ["mixed_small", "full_small"])
+def test_attend_graph_capture_matches_eager(name):
+    """With several branches the call forks onto helper streams and joins
+    before the merge; captured in a CUDA graph and replayed (after the inputs
+    changed) it must give the eager result for the new inputs, bit for bit."""
+    w = SMALL[name]
+    prob = P.problem(w)
+    ck, cv, hk, hv = P.encode_history(w, prob)
+    q = prob["q"].clone()
+    out = torch.empty_like(q)
+    lse = torch.empty(w.H, w.Tq, dtype=torch.float32, device=q.device)
+    ws = torch.empty(nk.nanokv_attend_workspace(w.Tq, ck, cv, w.T, w.T_full, w.Tq), dtype=torch.uint8,
+                     device=q.device)
+    nk.nanokv_attend(q, ck, cv, hk, hv, w.T_full, prob["k_cur"], prob["v_cur"], out=out, lse=lse, workspace=ws)
+    torch.cuda.synchronize()
+    side = torch.cuda.Stream()
+    side.wait_stream(torch.cuda.current_stream())
+    g = torch.cuda.CUDAGraph()
+    with torch.cuda.stream(side):
+        with torch.cuda.graph(g, stream=side):
+            nk.nanokv_attend(q, ck, cv, hk, hv, w.T_full, prob["k_cur"], prob["v_cur"], out=out, lse=lse,
+                             workspace=ws)
+    torch.cuda.current_stream().wait_stream(side)
+    gen = torch.Generator(device=q.device).manual_seed(11)
+    q.copy_((torch.randn(q.shape, device=q.device, generator=gen) / math.sqrt(w.d)).to(q.dtype))
+    out.zero_()
+    g.replay()
+    torch.cuda.synchronize()
+    Og, Lg = out.clone(), lse.clone()
+    Oe, Le = nk.nanokv_attend(q, ck, cv, hk, hv, w.T_full, prob["k_cur"], prob["v_cur"])
+    torch.cuda.synchronize()
+    assert torch.equal(Og, Oe)
+    assert torch.equal(Lg, Le)
+    del g
+
+
+@pytest.mark.parametrize("name", ["full", "mixed"])
+def test_attend_is_deterministic(name):
+    """Every output is a fixed function of the inputs: repeated calls at the
+    full workload agree bit for bit.  (Rounding-level differences between runs
+    would mean some key was decoded or scored from data a producer had not
+    finished writing, or had already replaced, which a tolerance check on a
+    near-uniform softmax cannot see.)"""
+    w = WORKLOADS[name]
+    prob = P.problem(w)
+    ck, cv, hk, hv = P.encode_history(w, prob)
+    runs = []
+    for _ in range(4):
+        O, L = nk.nanokv_attend(prob["q"], ck, cv, hk, hv, w.T_full, prob["k_cur"], prob["v_cur"])
+        torch.cuda.synchronize()
+        runs.append((O.clone(), L.clone()))
+    for O, L in runs[1:]:
+        assert torch.equal(O, runs[0][0])
+        assert torch.equal(L, runs[0][1])
