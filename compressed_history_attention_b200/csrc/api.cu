@@ -192,24 +192,27 @@ static int io_prec(int32_t dt) {
 
 // workspace carve-up (every region 256-byte aligned)
 struct WsLayout {
-  size_t off_O[3], off_L[3], off_qred, off_qc, total;
+  // branch b (0 low-dim, 1 full-dim, 2 current chunk) has nparts[b]
+  // consecutive partials, osz / lsz bytes apart
+  size_t off_O[3], off_L[3], off_qred, off_qc, total, osz, lsz;
+  int nparts[3];
 };
 
 static size_t al256(size_t x) { return (x + 255) & ~(size_t)255; }
 
 static WsLayout ws_layout(int64_t Tq, const Codec &ck, int64_t T_low, int64_t T_full,
-                          int64_t T_cur, bool tc_low) {
+                          int64_t T_cur, bool tc_low, int full_splits) {
   WsLayout w{};
   size_t off = 0;
-  const size_t osz = al256((size_t)Tq * ck.H * ck.d * sizeof(float));
-  const size_t lsz = al256((size_t)Tq * ck.H * sizeof(float));
+  w.osz = al256((size_t)Tq * ck.H * ck.d * sizeof(float));
+  w.lsz = al256((size_t)Tq * ck.H * sizeof(float));
   const bool on[3] = {T_low > 0, T_full > 0, T_cur > 0};
   for (int b = 0; b < 3; ++b) {
-    if (!on[b]) continue;
+    w.nparts[b] = on[b] ? (b == 1 ? full_splits : 1) : 0;
     w.off_O[b] = off;
-    off += osz;
+    off += w.nparts[b] * w.osz;
     w.off_L[b] = off;
-    off += lsz;
+    off += w.nparts[b] * w.lsz;
   }
   w.off_qred = w.off_qc = off;
   if (T_low > 0 && !tc_low) {
@@ -326,7 +329,9 @@ size_t nanokv_attend_workspace(int64_t Tq, const nanokv_codec *ck, const nanokv_
   if (check_codec(ck, "ck", false, &a) || check_codec(cv, "cv", false, &b)) return 0;
   const int path = g_kernel_path.load();
   const bool tc_low = path != 1 && tc_low_supported(a, b);
-  return ws_layout(Tq, a, T - T_full, T_full, T_cur, tc_low).total;
+  const bool tc_full = path != 1 && tc_full_supported(a, b);
+  const int splits = (tc_full && T_full > 0 && Tq > 0) ? tc_full_splits(Tq, a.H, a.d, T_full) : 1;
+  return ws_layout(Tq, a, T - T_full, T_full, T_cur, tc_low, splits).total;
 }
 
 int nanokv_attend(const void *q, int32_t io_dtype, int64_t Tq, const nanokv_codec *ck_,
@@ -370,7 +375,9 @@ int nanokv_attend(const void *q, int32_t io_dtype, int64_t Tq, const nanokv_code
                     (T_cur > 0 && !tc_dense_ok)))
     return fail(NANOKV_ERR_UNSUPPORTED, "attend: no tensor-core kernel for this shape");
   const bool use_tc_low = path != 1 && tc_low_ok;
-  const WsLayout w = ws_layout(Tq, ck, T_low, T_full, T_cur, use_tc_low);
+  const bool use_tc_full = path != 1 && tc_full_ok;
+  const int full_splits = (use_tc_full && T_full > 0) ? tc_full_splits(Tq, ck.H, ck.d, T_full) : 1;
+  const WsLayout w = ws_layout(Tq, ck, T_low, T_full, T_cur, use_tc_low, full_splits);
   if (w.total > 0 && (!workspace || workspace_bytes < w.total))
     return fail(NANOKV_ERR_INVALID, "attend: workspace needs %zu bytes, got %zu", w.total,
                 workspace_bytes);
@@ -433,14 +440,16 @@ int nanokv_attend(const void *q, int32_t io_dtype, int64_t Tq, const nanokv_code
     cudaStream_t bst = bstream(1);
     if (e != cudaSuccess) return cuda_status(e, "attend fork");
     e = timed(NANOKV_K_FULL, 1, bst, [&] {
-      return (path != 1 && tc_full_ok)
-                 ? tc_attend_full(q, Tq, ck, cv, hk, hv, T_low, T_full, softmax_scale, p, bst, false)
-                 : simt_attend_full(q, Tq, ck, cv, hk, hv, T_low, T_full, softmax_scale, p, bst);
+      return use_tc_full ? tc_attend_full(q, Tq, ck, cv, hk, hv, T_low, T_full, softmax_scale, p, full_splits,
+                                          w.osz / sizeof(float), w.lsz / sizeof(float), bst, false)
+                         : simt_attend_full(q, Tq, ck, cv, hk, hv, T_low, T_full, softmax_scale, p, bst);
     });
     if (e == cudaSuccess) e = join(1);
     if (e != cudaSuccess) return cuda_status(e, "attend full-dim launch");
-    pl.O[pl.n] = p.O;
-    pl.LSE[pl.n++] = p.LSE;
+    for (int z = 0; z < w.nparts[1]; ++z) {
+      pl.O[pl.n] = (const float *)(ws + w.off_O[1] + z * w.osz);
+      pl.LSE[pl.n++] = (const float *)(ws + w.off_L[1] + z * w.lsz);
+    }
   }
   if (on[2]) {
     Part p{(float *)(ws + w.off_O[2]), (float *)(ws + w.off_L[2])};

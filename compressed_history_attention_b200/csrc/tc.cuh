@@ -15,9 +15,15 @@ cudaError_t tc_encode_pair(const Codec *c, const void *const *x, int64_t T, uint
                            uint8_t *const *codes, void *const *scales, int nbranch, cudaStream_t st);
 size_t codec_aux_bytes(const Codec &c);
 cudaError_t codec_prepare(const Codec &c, void *aux, cudaStream_t st);
+// The full-dim kernel may split the history [t0, t0 + T) into nsplit
+// contiguous ranges of whole key tiles (grid z), each writing its own fp32
+// partial: split z at out.O + z * ostride, out.LSE + z * lstride.
+constexpr int kMaxFullSplits = 6;
+int tc_full_splits(int64_t Tq, int H, int d, int64_t T);
 cudaError_t tc_attend_full(const void *q, int64_t Tq, const Codec &ck, const Codec &cv,
                            const Hist &hk, const Hist &hv, int64_t t0, int64_t T, float tau,
-                           Part out, cudaStream_t st, bool pdl);
+                           Part out, int nsplit, size_t ostride, size_t lstride, cudaStream_t st,
+                           bool pdl);
 cudaError_t tc_attend_low(const void *q, int64_t Tq, const Codec &ck, const Codec &cv,
                           const Hist &hk, const Hist &hv, int64_t t0, int64_t T, float tau,
                           Part out, cudaStream_t st);

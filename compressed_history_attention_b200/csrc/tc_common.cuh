@@ -73,7 +73,7 @@ struct RowState {
 
 #ifdef NANOKV_TRACE
 // debug builds only: clock64 stamps of the softmax stages of one row
-__device__ unsigned long long g_softmax_trace[4][128];
+__device__ unsigned long long g_softmax_trace[8][128];
 #define SOFTMAX_TRACE(i, tj)                                            \
   do {                                                                  \
     if ((tj) >= 0 && (tj) < 128) g_softmax_trace[i][tj] = clock64();    \
@@ -145,6 +145,7 @@ __device__ __forceinline__ float softmax_tile(uint32_t tbase, int warp, uint32_t
     // P of S columns [32c, 32c + 32) goes to columns [16c, 16c + 16), all of
     // which were read by this chunk or an earlier one
     sm100::tmem_st16(tmem_lane_addr(tbase, warp, s_col + 16 * c), pk);
+    SOFTMAX_TRACE(4 + c, trace_j);
   }
   sm100::tmem_st_wait();
   SOFTMAX_TRACE(3, trace_j);

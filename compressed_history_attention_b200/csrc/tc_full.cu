@@ -35,7 +35,7 @@ using namespace tc;
 __device__ unsigned long long g_full_trace[2][24][128];
 #define FULL_TRACE(ev, j)                                                                    \
   do {                                                                                       \
-    if (blockIdx.y == 0 && blockIdx.x < 2 && (j) < 128) g_full_trace[rank][ev][j] = clock64(); \
+    if (blockIdx.z == 0 && blockIdx.y == 0 && blockIdx.x < 2 && (j) < 128) g_full_trace[rank][ev][j] = clock64(); \
   } while (0)
 #else
 #define FULL_TRACE(ev, j) \
@@ -61,6 +61,8 @@ struct FullArgs {
   const uint8_t *codes[2];      // [T_total, r / 2] packed INT4
   const __half *scales[2];      // [T_total]
   int64_t t0, T, Tq;            // branch = history tokens [t0, t0 + T)
+  int64_t Tsplit;               // tokens per history split (a multiple of BN); split z = blockIdx.z
+  size_t ostride, lstride;      // floats between the partial outputs of consecutive splits
   int H, r, C[2];
   float zscale;
   float *O, *L;
@@ -111,7 +113,11 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(384, 1)
   const uint32_t peer = rank ^ 1u;
   const int h = blockIdx.y;
   const int64_t q0 = (int64_t)blockIdx.x * BM;
-  const int ntiles = (int)((A.T + BN - 1) / BN);
+  // this CTA's share of the history: split blockIdx.z, tokens [t0, t0 + T)
+  const int64_t tb = (int64_t)blockIdx.z * A.Tsplit;
+  const int64_t t0 = A.t0 + tb;
+  const int64_t T = (A.T - tb) < A.Tsplit ? (A.T - tb) : A.Tsplit;
+  const int ntiles = (int)((T + BN - 1) / BN);
   const int nchunk = ntiles * nrb;
   const int J = A.H * DH;
   volatile int *abort = &B.abort;
@@ -275,6 +281,8 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(384, 1)
           ++jv;
           progress = true;
         }
+        // no sleep between polls: the time to notice a completed barrier is
+        // on every chain through this thread
         if (progress) {
           t_last = globaltimer();
         } else {
@@ -284,7 +292,6 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(384, 1)
             atomicOr(err, ERRW_TIMEOUT);
             break;
           }
-          __nanosleep(32);
         }
       }
     }
@@ -302,8 +309,8 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(384, 1)
 #pragma unroll
       for (int i = 0; i < 2; ++i) {
         int64_t t = (int64_t)j * BN + kb + lane + 32 * i;
-        t = t < A.T ? t : A.T - 1;  // keys past the end: any valid row (masked later)
-        const uint4 *src = reinterpret_cast<const uint4 *>(codes + (A.t0 + t) * rowb + cb * 32);
+        t = t < T ? t : T - 1;  // keys past the end: any valid row (masked later)
+        const uint4 *src = reinterpret_cast<const uint4 *>(codes + (t0 + t) * rowb + cb * 32);
         v[2 * i] = __ldg(src);
         v[2 * i + 1] = __ldg(src + 1);
       }
@@ -344,8 +351,8 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(384, 1)
     uint64_t *empty_bar = rank == 0 ? &B.kh_empty : &B.vh_empty;
     const uint32_t full_remote = mapa(smem_u32(full_bar), peer);
     auto key_meta = [&](int j, int &a, float &s) {
-      const int64_t tt = A.t0 + (int64_t)j * BN + t;
-      const bool valid = (int64_t)j * BN + t < A.T;
+      const int64_t tt = t0 + (int64_t)j * BN + t;
+      const bool valid = (int64_t)j * BN + t < T;
       a = valid ? (int)A.ids[rank][tt] : 0;
       a = a < C ? a : C - 1;
       s = valid ? __half2float(A.scales[rank][tt]) : 0.f;
@@ -432,11 +439,11 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(384, 1)
       if (!mbar_wait(&B.s_full[j & 1], (j >> 1) & 1, abort, err)) { ok = false; break; }
       if (row == 0) FULL_TRACE(7, j);
       tc_fence_after();
-      const int64_t rem = A.T - (int64_t)j * BN;
+      const int64_t rem = T - (int64_t)j * BN;
       const int nk = rem < BN ? (int)rem : BN;
       bool wr;
 #ifdef NANOKV_TRACE
-      const int tj = (blockIdx.x == 0 && blockIdx.y == 0 && row == 0) ? j : -1;
+      const int tj = (blockIdx.x == 0 && blockIdx.y == 0 && blockIdx.z == 0 && row == 0) ? j : -1;
 #else
       const int tj = -1;
 #endif
@@ -456,7 +463,8 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(384, 1)
     if (ok && ntiles >= 2) ok = mbar_wait(&B.pv_done[(ntiles - 2) & 1], ((ntiles - 2) >> 1) & 1, abort, err);
     if (ok && mbar_wait(&B.pv_done[(ntiles - 1) & 1], ((ntiles - 1) >> 1) & 1, abort, err)) {
       tc_fence_after();
-      write_row(tbase, warp, TM_O, st, q0 + row, A.Tq, h, A.H, A.O, A.L);
+      write_row(tbase, warp, TM_O, st, q0 + row, A.Tq, h, A.H, A.O + blockIdx.z * A.ostride,
+                A.L + blockIdx.z * A.lstride);
     }
   }
   tc_fence_before();
@@ -489,10 +497,63 @@ size_t tc_full_smem(int r, int C) {
   return (size_t)3 * kTile + (size_t)(r / 64) * kChunk + NRING * kChunk + (size_t)C * 256 + 1024;
 }
 
+// Largest number of two-CTA clusters of the full-dim kernel that can be
+// resident at once on the current device (cached per device).
+static int full_cluster_capacity() {
+  static int cached[64] = {};
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= 64) return 0;
+  if (cached[dev] > 0) return cached[dev];
+  int sms = 0;
+  cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
+  int cap = sms / 2;
+  const size_t smem = tc_full_smem(192, 64);
+  if (ensure_smem((const void *)tc_full_kernel, (int)smem) == cudaSuccess) {
+    cudaLaunchConfig_t cfg{};
+    cfg.gridDim = dim3(2, 1, 1);
+    cfg.blockDim = dim3(384);
+    cfg.dynamicSmemBytes = smem;
+    int n = 0;
+    if (cudaOccupancyMaxActiveClusters(&n, (const void *)tc_full_kernel, &cfg) == cudaSuccess && n > 0) cap = n;
+  }
+  cudaGetLastError();
+  cached[dev] = cap > 0 ? cap : 1;
+  return cached[dev];
+}
+
+int tc_full_splits(int64_t Tq, int H, int d, int64_t T) {
+  // Cost model in microseconds: the launch runs ceil(units * ns / capacity)
+  // waves of clusters, each cluster ~3.3 us per 128-key tile plus ~3 tiles of
+  // fixed cost (staging, pipeline fill and drain); every extra split adds a
+  // [Tq, H, d] fp32 partial written here and read by the merge (~6 TB/s).
+  if (T <= 0 || Tq <= 0) return 1;
+  const int64_t ntiles = (T + BN - 1) / BN;
+  const int64_t units = (int64_t)H * ((((Tq + BM - 1) / BM) + 1) / 2);
+  const int64_t cap = full_cluster_capacity();
+  if (cap <= 0) return 1;
+  const double part_us = 2.0 * (double)Tq * H * d * 4.0 / 6.0e6;
+  int best = 1;
+  double best_cost = 1e300;
+  for (int ns = 1; ns <= kMaxFullSplits && ns <= ntiles; ++ns) {
+    const int64_t per = (ntiles + ns - 1) / ns;
+    if ((ntiles + per - 1) / per != ns) continue;  // some split would be empty
+    const int64_t waves = (units * ns + cap - 1) / cap;
+    const double cost = (double)waves * ((double)per + 3.0) * 3.3 + (ns - 1) * part_us;
+    if (cost < best_cost * 0.99) {
+      best_cost = cost;
+      best = ns;
+    }
+  }
+  return best;
+}
+
 cudaError_t tc_attend_full(const void *q, int64_t Tq, const Codec &ck, const Codec &cv,
                            const Hist &hk, const Hist &hv, int64_t t0, int64_t T, float tau,
-                           Part out, cudaStream_t st, bool pdl) {
+                           Part out, int nsplit, size_t ostride, size_t lstride, cudaStream_t st,
+                           bool pdl) {
   if (Tq == 0 || T == 0) return cudaSuccess;
+  const int64_t ntiles = (T + BN - 1) / BN;
+  if (nsplit < 1 || nsplit > ntiles) return cudaErrorInvalidValue;
   const int J = ck.H * DH;
   CUtensorMap mq;
   if (!make_tmap_bf16_2d(&mq, q, Tq, J, J, 128)) return cudaErrorInvalidValue;
@@ -509,6 +570,9 @@ cudaError_t tc_attend_full(const void *q, int64_t Tq, const Codec &ck, const Cod
   a.scales[1] = (const __half *)hv.scales;
   a.t0 = t0;
   a.T = T;
+  a.Tsplit = ((ntiles + nsplit - 1) / nsplit) * BN;
+  a.ostride = ostride;
+  a.lstride = lstride;
   a.Tq = Tq;
   a.H = ck.H;
   a.r = ck.r;
@@ -521,7 +585,9 @@ cudaError_t tc_attend_full(const void *q, int64_t Tq, const Codec &ck, const Cod
   const size_t smem = tc_full_smem(ck.r, ck.C > cv.C ? ck.C : cv.C);
   ensure_smem((const void *)tc_full_kernel, (int)smem);
   const unsigned qt = (unsigned)((Tq + BM - 1) / BM);
-  dim3 grid((qt + 1) & ~1u, (unsigned)ck.H);
+  // every split must get at least one key tile (the caller merges nsplit partials)
+  if ((T + a.Tsplit - 1) / a.Tsplit != nsplit) return cudaErrorInvalidValue;
+  dim3 grid((qt + 1) & ~1u, (unsigned)ck.H, (unsigned)nsplit);
   return launch_k(tc_full_kernel, grid, dim3(384), smem, st, pdl, mq, a);
 }
 
