@@ -321,15 +321,20 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(384, 1)
       if (c + 1 < nchunk) load(c + 1, nxt);
       const int rs = c % NRING, cb = c % nrb;
       if (warp == 2 && lane == 0 && cb == 0) FULL_TRACE(9, c / nrb);
+      if (warp == 2 && lane == 0 && cb == 1) FULL_TRACE(17, c / nrb);
       if (c >= NRING && !mbar_wait(&B.ring_empty[rs], ((c / NRING) - 1) & 1, abort, err)) break;
       if (warp == 2 && lane == 0 && cb == 0) FULL_TRACE(10, c / nrb);
+      if (warp == 2 && lane == 0 && cb == 1) FULL_TRACE(18, c / nrb);
       const uint32_t dst = smem_u32(sRing + rs * kChunk);
 #pragma unroll
       for (int i = 0; i < 2; ++i) {
         const uint32_t w[8] = {cur[2 * i].x,     cur[2 * i].y,     cur[2 * i].z,     cur[2 * i].w,
                                cur[2 * i + 1].x, cur[2 * i + 1].y, cur[2 * i + 1].z, cur[2 * i + 1].w};
 #pragma unroll
-        for (int g = 0; g < 8; ++g) st_shared_v4(dst + sw128_offset(kb + lane + 32 * i, 8 * g, 128), unpack8(w[g]));
+        for (int g = 0; g < 8; ++g) {
+          st_shared_v4(dst + sw128_offset(kb + lane + 32 * i, 8 * g, 128), unpack8(w[g]));
+          if (i == 0 && g == 0 && warp == 2 && lane == 0 && cb == 1) FULL_TRACE(21, c / nrb);
+        }
       }
       if (warp == 2 && lane == 0 && cb == 1) FULL_TRACE(19, c / nrb);
       fence_proxy_async_smem();
