@@ -63,6 +63,23 @@ def ncu_traffic(kernel, workload):
     return e[2]
 
 
+def max_over_ranks(vals, world, device):
+    """Element-wise maximum of per-rank timings over all ranks (every rank gets
+    it); the identity on one rank."""
+    if world <= 1:
+        return list(vals)
+    import torch.distributed as dist
+    t = torch.tensor(list(vals), dtype=torch.float64, device=device)
+    dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    return t.tolist()
+
+
+def whole_job_tflops(flops_per_rank, ms, world):
+    """Whole-job throughput: every rank processes its own replica of the
+    workload, so N ranks do N times the work in the slowest rank's time."""
+    return world * flops_per_rank / (ms * 1e-3) / 1e12
+
+
 def load_peaks():
     p = os.path.join(ROOT, "MEASURED_PEAKS.json")
     if os.path.exists(p):
@@ -315,13 +332,10 @@ def run_ours(a, rank, world, device):
 
     step_ms = (sum(enc) + sum(att)) / a.steps
     enc_ms, att_ms = sum(enc) / a.steps, sum(att) / a.steps
-    if world > 1:
-        t = torch.tensor([step_ms, enc_ms, att_ms], device=device)
-        dist.all_reduce(t, op=dist.ReduceOp.MAX)
-        step_ms, enc_ms, att_ms = t.tolist()
+    step_ms, enc_ms, att_ms = max_over_ranks([step_ms, enc_ms, att_ms], world, device)
 
     flops = af["total"] + ef
-    value = world * flops / (step_ms * 1e-3) / 1e12
+    value = whole_job_tflops(flops, step_ms, world)
     # dominant kernel: the one with the largest share of the timed region
     dom = max(kt.items(), key=lambda kv: kv[1][0])
     dom_name, (dom_ms, dom_n) = dom
@@ -410,13 +424,8 @@ def run_e2e(s, w, a, device, flops, world):
         one()
     e1.record()
     torch.cuda.synchronize()
-    ms = e0.elapsed_time(e1) / a.steps
-    if world > 1:
-        import torch.distributed as dist
-        t = torch.tensor([ms], device=device)
-        dist.all_reduce(t, op=dist.ReduceOp.MAX)
-        ms = t.item()
-    return {"value": round(world * flops / (ms * 1e-3) / 1e12, 3), "unit": "TFLOP/s",
+    ms = max_over_ranks([e0.elapsed_time(e1) / a.steps], world, device)[0]
+    return {"value": round(whole_job_tflops(flops, ms, world), 3), "unit": "TFLOP/s",
             "ms_per_step": round(ms, 4), "h2d_bytes_per_step": bi, "d2h_bytes_per_step": bo}
 
 
