@@ -98,6 +98,7 @@ def args_():
     ap.add_argument("--workload", default="full")
     ap.add_argument("--no-fast", action="store_true", help="skip the mixed-dim (Fast) side measurement")
     ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--no-step30", action="store_true", help="skip the 30-layer step (side measurement)")
     ap.add_argument("--path", type=int, default=0, help="kernel family: 0 auto, 1 CUDA-core, 2 tensor-core")
     return ap.parse_args()
 
@@ -192,9 +193,16 @@ class ClockSampler:
 # our arm
 # ---------------------------------------------------------------------------
 def setup(w, device):
+    return setup_layer(w, 0, device, None)
+
+
+def setup_layer(w, layer, device, ws=None):
+    """One layer of a workload: codec, compressed history, the last chunk's raw
+    K/V (re-encoded each step) and the query chunk; `ws` is reused if large
+    enough."""
     import compressed_history_attention_b200 as nk
     from synth.gen import make_problem
-    prob = make_problem(w, device=device)
+    prob = make_problem(w, layer=layer, device=device)
     ck = nk.Codec(w.H, w.d, prob["codec_k"]["centers"], prob["codec_k"]["D"], prob["codec_k"]["E"])
     cv = nk.Codec(w.H, w.d, prob["codec_v"]["centers"], prob["codec_v"]["D"], prob["codec_v"]["E"])
     hk, hv = nk.nanokv_encode(ck, cv, prob["hist_k"], prob["hist_v"])
@@ -206,8 +214,10 @@ def setup(w, device):
         "out": torch.empty_like(prob["q"]),
         "lse": torch.empty(w.H, w.Tq, dtype=torch.float32, device=device),
     }
-    ws = nk.nanokv_attend_workspace(w.Tq, ck, cv, w.T, w.T_full, w.Tq)
-    s["ws"] = torch.empty(max(ws, 16), dtype=torch.uint8, device=device)
+    need = nk.nanokv_attend_workspace(w.Tq, ck, cv, w.T, w.T_full, w.Tq)
+    if ws is None or ws.numel() < need:
+        ws = torch.empty(max(need, 16), dtype=torch.uint8, device=device)
+    s["ws"] = ws
     # free the raw history: only the compressed cache stays resident
     prob["hist_k"] = prob["hist_v"] = None
     return s
@@ -367,6 +377,7 @@ def run_ours(a, rank, world, device):
 
     e2e = run_e2e(s, w, a, device, flops, world)
     fast = None if a.no_fast else run_fast(a, device, peaks)
+    step30 = None if a.no_step30 else run_step30(a, device, peaks)
     cpu = None
     if rank == 0 and world == 1 and not a.no_cpu_baseline:
         cpu = cpu_baseline(w, s, budget_s=12.0)
@@ -388,7 +399,7 @@ def run_ours(a, rank, world, device):
                    "frac_hbm": round(enc_gbs / peaks["hbm_gbs"], 4)},
         "kernels": kernels,
         "clocks": clocks, "e2e": e2e, "gpu_launches": launches, "roofline": roof,
-        "cpu_baseline": cpu, "fast": fast,
+        "cpu_baseline": cpu, "fast": fast, "step30": step30,
     }
     return line
 
@@ -463,6 +474,57 @@ def run_fast(a, device, peaks):
     torch.cuda.empty_cache()
     return {"workload": w.describe(), "attend_ms": round(ms, 4), "tflops": round(tf, 3),
             "frac_bf16_peak": round(tf / peaks["bf16_tflops"], 4), "iters": n, "kernels": per}
+
+
+def run_step30(a, device, peaks):
+    """Side measurement of the 30-layer step: every layer (own seeded codec and
+    10-chunk compressed history) encodes the previous chunk's K and V, then
+    attends the query chunk in mixed mode (most recent chunk full-dim) with the
+    current chunk, and merges.  The 30 layers are captured as one CUDA graph.
+    The layers share one attend workspace (they run one after another)."""
+    from synth.gen import WORKLOADS
+    w = WORKLOADS["step30"]
+    import compressed_history_attention_b200 as nk
+    layers = []
+    ws = None
+    for layer in range(w.layers):
+        s = setup_layer(w, layer, device, ws)
+        ws = s["ws"]
+        layers.append(s)
+    n_enc = layers[0]["n_enc"]
+    af, ef, eb = work_of(w, n_enc)
+    flops = w.layers * (af["total"] + ef)
+
+    def step():
+        for s in layers:
+            step_encode(s)
+            step_attend(s, w)
+
+    step()
+    torch.cuda.synchronize()
+    g = capture(step)
+    flush = torch.empty(256 * 1024 * 1024, dtype=torch.uint8, device=device)
+    for _ in range(2):
+        g.replay()
+    torch.cuda.synchronize()
+    n = max(3, min(a.steps, 10))
+    ts = []
+    for _ in range(n):
+        flush.zero_()
+        e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        e0.record()
+        g.replay()
+        e1.record()
+        torch.cuda.synchronize()
+        ts.append(e0.elapsed_time(e1))
+    nk.nanokv_check()
+    ms = sum(ts) / n
+    tf = flops / (ms * 1e-3) / 1e12
+    del g, layers, ws
+    torch.cuda.empty_cache()
+    return {"workload": w.describe(), "layers": w.layers, "ms": round(ms, 3), "ms_per_layer": round(ms / w.layers, 4),
+            "tflops": round(tf, 3), "frac_bf16_peak": round(tf / peaks["bf16_tflops"], 4), "iters": n,
+            "launch": "one CUDA graph of the 30 layers' encode and attend calls"}
 
 
 # ---------------------------------------------------------------------------
