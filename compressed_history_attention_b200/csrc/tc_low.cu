@@ -26,6 +26,7 @@ namespace {
 constexpr int DH = 128;
 constexpr uint32_t kBlk = 128 * 64 * 2;  // [128 rows x 64] bf16 block
 constexpr uint32_t TM_OT = 0, TM_S0 = 256, TM_COLS = 512;
+constexpr int kMaxCodeWords = 6;  // uint4 words of packed codes per key (r <= 192)
 
 struct LowArgs {
   const __nv_bfloat16 *Dk, *Dv;   // decoders [J, r]
@@ -223,31 +224,48 @@ __global__ void __launch_bounds__(384, 1)
     }
   } else if (warp >= 4 && warp < 8) {
     // ---------------- unpack (thread = key) ----------------
+    // The key's ids, scales and packed K / V codes of tile j + 1 are loaded
+    // into registers while tile j is unpacked, so no global-memory latency
+    // sits between the tiles.
     const int t = (warp - 4) * 32 + lane;
     const int cw = r / 32;  // uint4 words of packed codes per key
-    bool ok = mbar_wait(&B.pro_done, 0, abort, err);  // prologue buffers alias the tiles
-    for (int j = 0; ok && j < ntiles; ++j) {
+    struct KeyData {
+      int ak, av;
+      float sk, sv;
+      uint4 ck[kMaxCodeWords], cv[kMaxCodeWords];
+    };
+    auto load_key = [&](int j, KeyData &d) {
       const int64_t tt = A.t0 + (int64_t)j * BN + t;
       const bool valid = (int64_t)j * BN + t < A.T;
       int ak = valid ? (int)A.idk[tt] : 0, av = valid ? (int)A.idv[tt] : 0;
-      ak = ak < C ? ak : C - 1;
-      av = av < C ? av : C - 1;
-      const float sk = valid ? __half2float(A.sk[tt]) : 0.f;
-      const float sv = valid ? __half2float(A.sv[tt]) : 0.f;
+      d.ak = ak < C ? ak : C - 1;
+      d.av = valid ? (av < C ? av : C - 1) : -1;  // -1: no one-hot entry
+      d.sk = valid ? __half2float(A.sk[tt]) : 0.f;
+      d.sv = valid ? __half2float(A.sv[tt]) : 0.f;
       const uint4 *pk = reinterpret_cast<const uint4 *>(A.codk + tt * (r / 2));
       const uint4 *pv = reinterpret_cast<const uint4 *>(A.codv + tt * (r / 2));
+#pragma unroll
+      for (int q = 0; q < kMaxCodeWords; ++q) {
+        d.ck[q] = (q < cw && valid) ? __ldg(pk + q) : make_uint4(0, 0, 0, 0);
+        d.cv[q] = (q < cw && valid) ? __ldg(pv + q) : make_uint4(0, 0, 0, 0);
+      }
+    };
+    // one tile: unpack `cur` (tile j) after starting the loads of tile j + 1 into `nxt`
+    auto tile = [&](int j, const KeyData &cur, KeyData &nxt) -> bool {
+      if (j + 1 < ntiles) load_key(j + 1, nxt);
       // ---- K codes
       // (kinfo[j & 1] was last read by the softmax of tile j - 2, which finished
       // before PV of tile j - 2, which the V part of tile j - 1 waited for)
-      if (j >= 1 && !mbar_wait(&B.kc_empty, (j - 1) & 1, abort, err)) break;
-      for (int q = 0; q < cw; ++q) {
-        const uint4 v = valid ? pk[q] : make_uint4(0, 0, 0, 0);
-        const uint32_t w[4] = {v.x, v.y, v.z, v.w};
+      if (j >= 1 && !mbar_wait(&B.kc_empty, (j - 1) & 1, abort, err)) return false;
+#pragma unroll
+      for (int q = 0; q < kMaxCodeWords; ++q) {
+        if (q >= cw) break;
+        const uint32_t w[4] = {cur.ck[q].x, cur.ck[q].y, cur.ck[q].z, cur.ck[q].w};
 #pragma unroll
         for (int i = 0; i < 4; ++i)
           *reinterpret_cast<uint4 *>(sKc + sw128_offset(t, 32 * q + 8 * i, 128)) = unpack8(w[i]);
       }
-      kinfo[(j & 1) * 128 + t] = KeyInfo{sk, ak, sv};
+      kinfo[(j & 1) * 128 + t] = KeyInfo{cur.sk, cur.ak, cur.sv};
       fence_proxy_async_smem();
       __syncwarp();
       if (lane == 0) {
@@ -255,17 +273,19 @@ __global__ void __launch_bounds__(384, 1)
         mbar_arrive(&B.info_full[j & 1]);
       }
       // ---- V codes and one-hot of the value center
-      if (j >= 1 && !mbar_wait(&B.v_empty, (j - 1) & 1, abort, err)) break;
-      for (int q = 0; q < cw; ++q) {
-        const uint4 v = valid ? pv[q] : make_uint4(0, 0, 0, 0);
-        const uint32_t w[4] = {v.x, v.y, v.z, v.w};
+      if (j >= 1 && !mbar_wait(&B.v_empty, (j - 1) & 1, abort, err)) return false;
+#pragma unroll
+      for (int q = 0; q < kMaxCodeWords; ++q) {
+        if (q >= cw) break;
+        const uint32_t w[4] = {cur.cv[q].x, cur.cv[q].y, cur.cv[q].z, cur.cv[q].w};
 #pragma unroll
         for (int i = 0; i < 4; ++i)
           *reinterpret_cast<uint4 *>(sVc + sw128_offset(t, 32 * q + 8 * i, 128)) = unpack8(w[i]);
       }
+      const int av = cur.av;
       for (int g = 0; g < C / 8; ++g) {
         uint4 z = make_uint4(0, 0, 0, 0);
-        if (valid && (av >> 3) == g) {
+        if (av >= 0 && (av >> 3) == g) {
           const uint32_t one = 0x3F80u << (16 * (av & 1));  // bf16 1.0 in the right half
           const int wsel = (av & 7) >> 1;
           if (wsel == 0) z.x = one;
@@ -278,6 +298,14 @@ __global__ void __launch_bounds__(384, 1)
       fence_proxy_async_smem();
       __syncwarp();
       if (lane == 0) mbar_arrive(&B.vc_full);
+      return true;
+    };
+    KeyData ka, kb;
+    bool ok = mbar_wait(&B.pro_done, 0, abort, err);  // prologue buffers alias the tiles
+    if (ok && ntiles > 0) load_key(0, ka);
+    for (int j = 0; ok && j < ntiles; j += 2) {
+      ok = tile(j, ka, kb);
+      if (ok && j + 1 < ntiles) ok = tile(j + 1, kb, ka);
     }
   } else if (warp >= 8) {
     // ---------------- softmax (thread = query row) ----------------
