@@ -21,6 +21,20 @@ namespace nanokv {
 using namespace sm100;
 using namespace tc;
 
+// Optional event trace of the first CTA (debug builds with -DNANOKV_TRACE only):
+// clock64 stamps per role and key tile.
+#ifdef NANOKV_TRACE
+__device__ unsigned long long g_low_trace[12][128];
+#define LOW_TRACE(ev, j)                                                                    \
+  do {                                                                                      \
+    if (blockIdx.x == 0 && blockIdx.y == 0 && (j) < 128) g_low_trace[ev][j] = clock64();    \
+  } while (0)
+#else
+#define LOW_TRACE(ev, j) \
+  do {                   \
+  } while (0)
+#endif
+
 namespace {
 
 constexpr int DH = 128;
@@ -41,16 +55,11 @@ struct LowArgs {
   unsigned *err;
 };
 
-struct KeyInfo {
-  float sK;  // key scale
-  int aK;    // key center id
-  float sV;  // value scale
-};
 
 struct LowBars {
   uint64_t pro_full, pro_done, qt_ready;
   uint64_t kc_full, kc_empty, vc_full, v_empty;
-  uint64_t s_full[2], p_full[2], info_full[2], pv_done, last_done;
+  uint64_t s_full[2], p_full[2], info_full[2], pv_done[2], last_done;  // pv_done[b]: P*V of the tiles using S buffer b
   uint64_t fin_a, fin_b, fin_done;
   uint32_t tmem_base;
   int abort;
@@ -81,7 +90,11 @@ __global__ void __launch_bounds__(384, 1)
   uint8_t *sVc = sKc + nrb * kBlk;             // [128 keys x r] (MN-major use)
   uint8_t *sOH = sVc + nrb * kBlk;             // [128 keys x C] one-hot
   float *sQC = (float *)(sOH + kBlk);          // [128][C + 1]
-  KeyInfo *kinfo = (KeyInfo *)(sQC + 128 * (C + 1));  // [2][128]
+  // per-key info of the two tiles in flight, as arrays (16-byte aligned) so
+  // that the softmax reads four keys' values with one broadcast load
+  int *kAK = (int *)(sQC + 128 * (C + 1));  // [2][128] key center id
+  float *kSK = (float *)(kAK + 2 * 128);     // [2][128] key scale
+  float *kSV = kSK + 2 * 128;                // [2][128] value scale
   // prologue aliases (inside sKc .. sOH)
   uint8_t *sQ = sKc;                           // [128 x 128] K-major
   uint8_t *sDk = sKc + 2 * kBlk;               // D_{K,h} [128 d x r] (MN-major use)
@@ -115,7 +128,8 @@ __global__ void __launch_bounds__(384, 1)
     mbar_init(&B.p_full[1], 4);
     mbar_init(&B.info_full[0], 4);
     mbar_init(&B.info_full[1], 4);
-    mbar_init(&B.pv_done, 1);
+    mbar_init(&B.pv_done[0], 1);
+    mbar_init(&B.pv_done[1], 1);
     mbar_init(&B.last_done, 1);
     mbar_init(&B.fin_a, 4);
     mbar_init(&B.fin_b, 1);
@@ -171,39 +185,60 @@ __global__ void __launch_bounds__(384, 1)
         mma_commit(&B.pro_done);
         ok = mbar_wait(&B.qt_ready, 0, abort, err);
       }
-      auto scores = [&](int j) -> bool {
-        if (!mbar_wait(&B.kc_full, j & 1, abort, err)) return false;
-        if (j >= 2 && !mbar_wait(&B.pv_done, (j - 2) & 1, abort, err)) return false;
-        tc_fence_after();
-        const uint32_t dS = tbase + TM_S0 + (j & 1) * 128;
-        for (int ks = 0; ks < r / 16; ++ks) {
-          const uint32_t off = (ks >> 2) * kBlk + (ks & 3) * 32;
-          mma_ss(dS, sdesc_sw128(aQt + off, 16, 1024), sdesc_sw128(aK + off, 16, 1024),
-                 idesc_bf16(128, 128, false, false), ks > 0);
-        }
-        mma_commit(&B.s_full[j & 1]);
-        mma_commit(&B.kc_empty);
-        return true;
-      };
-      if (ok) ok = scores(0);
-      if (ok && ntiles > 1) ok = scores(1);
-      for (int j = 0; ok && j < ntiles; ++j) {
-        if (!mbar_wait(&B.p_full[j & 1], (j >> 1) & 1, abort, err)) { ok = false; break; }
-        if (!mbar_wait(&B.vc_full, j & 1, abort, err)) { ok = false; break; }
-        tc_fence_after();
-        const uint32_t sb = tbase + TM_S0 + (j & 1) * 128;
+      // Two MMA streams polled with non-blocking tests and issued as soon as
+      // their inputs are ready, so that neither waits behind the other:
+      // scores S'_j = Q~ codes_K^T (S buffer j & 1, which last held P of
+      // tile j - 2) and values O~ += (P s_V) codes_V, P_C += P onehot.
+      int js = 0, jv = 0;
+      uint64_t t_last = globaltimer();
+      while (ok && jv < ntiles) {
+        bool progress = false;
+        // ---- values stream (frees the V code buffer for the unpackers)
+        if (jv < js && mbar_test(&B.p_full[jv & 1], (jv >> 1) & 1) && mbar_test(&B.vc_full, jv & 1)) {
+          LOW_TRACE(1, jv);
+          tc_fence_after();
+          const uint32_t sb = tbase + TM_S0 + (jv & 1) * 128;
 #pragma unroll
-        for (int ks = 0; ks < BN / 16; ++ks) {
-          const uint32_t pc = sb + 32 * (ks >> 1) + 8 * (ks & 1);
-          const uint32_t acc = (j > 0 || ks > 0);
-          mma_ts(tbase + TM_OT, pc + 16, sdesc_sw128(aV + ks * 2048, kBlk, 1024), idesc_bf16(128, r, false, true),
-                 acc);
-          mma_ts(tbase + TM_OT + r, pc, sdesc_sw128(aOH + ks * 2048, kBlk, 1024), idesc_bf16(128, C, false, true),
-                 acc);
+          for (int ks = 0; ks < BN / 16; ++ks) {
+            const uint32_t pc = sb + 32 * (ks >> 1) + 8 * (ks & 1);
+            const uint32_t acc = (jv > 0 || ks > 0);
+            mma_ts(tbase + TM_OT, pc + 16, sdesc_sw128(aV + ks * 2048, kBlk, 1024), idesc_bf16(128, r, false, true),
+                   acc);
+            mma_ts(tbase + TM_OT + r, pc, sdesc_sw128(aOH + ks * 2048, kBlk, 1024), idesc_bf16(128, C, false, true),
+                   acc);
+          }
+          mma_commit(&B.pv_done[jv & 1]);
+          mma_commit(&B.v_empty);
+          ++jv;
+          progress = true;
         }
-        mma_commit(&B.pv_done);
-        mma_commit(&B.v_empty);
-        if (j + 2 < ntiles && !scores(j + 2)) { ok = false; break; }
+        // ---- scores stream
+        if (js < ntiles && mbar_test(&B.kc_full, js & 1) &&
+            (js < 2 || mbar_test(&B.pv_done[js & 1], ((js - 2) >> 1) & 1))) {
+          LOW_TRACE(0, js);
+          tc_fence_after();
+          const uint32_t dS = tbase + TM_S0 + (js & 1) * 128;
+          for (int ks = 0; ks < r / 16; ++ks) {
+            const uint32_t off = (ks >> 2) * kBlk + (ks & 3) * 32;
+            mma_ss(dS, sdesc_sw128(aQt + off, 16, 1024), sdesc_sw128(aK + off, 16, 1024),
+                   idesc_bf16(128, 128, false, false), ks > 0);
+          }
+          mma_commit(&B.s_full[js & 1]);
+          mma_commit(&B.kc_empty);
+          ++js;
+          progress = true;
+        }
+        if (progress) {
+          t_last = globaltimer();
+        } else {
+          if (*abort) { ok = false; break; }
+          if (globaltimer() - t_last > kWaitLimitNs) {
+            *abort = 1;
+            atomicOr(err, ERRW_TIMEOUT);
+            ok = false;
+            break;
+          }
+        }
       }
       if (ok) mma_commit(&B.last_done);
       // restore: O = [O~/l | P_C/l] [D_{V,h} | C_{V,h}^T]^T
@@ -254,9 +289,10 @@ __global__ void __launch_bounds__(384, 1)
     auto tile = [&](int j, const KeyData &cur, KeyData &nxt) -> bool {
       if (j + 1 < ntiles) load_key(j + 1, nxt);
       // ---- K codes
-      // (kinfo[j & 1] was last read by the softmax of tile j - 2, which finished
+      // (key info [j & 1] was last read by the softmax of tile j - 2, which finished
       // before PV of tile j - 2, which the V part of tile j - 1 waited for)
       if (j >= 1 && !mbar_wait(&B.kc_empty, (j - 1) & 1, abort, err)) return false;
+      if (t == 0) LOW_TRACE(4, j);
 #pragma unroll
       for (int q = 0; q < kMaxCodeWords; ++q) {
         if (q >= cw) break;
@@ -265,15 +301,19 @@ __global__ void __launch_bounds__(384, 1)
         for (int i = 0; i < 4; ++i)
           *reinterpret_cast<uint4 *>(sKc + sw128_offset(t, 32 * q + 8 * i, 128)) = unpack8(w[i]);
       }
-      kinfo[(j & 1) * 128 + t] = KeyInfo{cur.sk, cur.ak, cur.sv};
+      kAK[(j & 1) * 128 + t] = cur.ak;
+      kSK[(j & 1) * 128 + t] = cur.sk;
+      kSV[(j & 1) * 128 + t] = cur.sv;
       fence_proxy_async_smem();
       __syncwarp();
       if (lane == 0) {
         mbar_arrive(&B.kc_full);
         mbar_arrive(&B.info_full[j & 1]);
       }
+      if (t == 0) LOW_TRACE(5, j);
       // ---- V codes and one-hot of the value center
       if (j >= 1 && !mbar_wait(&B.v_empty, (j - 1) & 1, abort, err)) return false;
+      if (t == 0) LOW_TRACE(6, j);
 #pragma unroll
       for (int q = 0; q < kMaxCodeWords; ++q) {
         if (q >= cw) break;
@@ -298,6 +338,7 @@ __global__ void __launch_bounds__(384, 1)
       fence_proxy_async_smem();
       __syncwarp();
       if (lane == 0) mbar_arrive(&B.vc_full);
+      if (t == 0) LOW_TRACE(7, j);
       return true;
     };
     KeyData ka, kb;
@@ -342,22 +383,44 @@ __global__ void __launch_bounds__(384, 1)
     for (int j = 0; ok && j < ntiles; ++j) {
       if (!mbar_wait(&B.s_full[j & 1], (j >> 1) & 1, abort, err)) { ok = false; break; }
       if (!mbar_wait(&B.info_full[j & 1], (j >> 1) & 1, abort, err)) { ok = false; break; }
+      if (row == 0) LOW_TRACE(2, j);
       tc_fence_after();
       const uint32_t sb = TM_S0 + (j & 1) * 128;
-      const KeyInfo *ki = kinfo + (j & 1) * 128;
+      const int *aKj = kAK + (j & 1) * 128;
+      const float *sKj = kSK + (j & 1) * 128, *sVj = kSV + (j & 1) * 128;
       const int64_t rem = A.T - (int64_t)j * BN;
       const int nk = rem < BN ? (int)rem : BN;
+      const bool full = nk >= BN;
       uint32_t v[32];
+      // pass 1: z = s_K S' + QC[a_K] per key (one gather per key), row max;
+      // z replaces S' in TMEM for pass 2
       float mx4[4] = {-INFINITY, -INFINITY, -INFINITY, -INFINITY};
+#pragma unroll 1
       for (int c = 0; c < 4; ++c) {
-        tmem_ld32(tmem_lane_addr(tbase, warp, sb + 32 * c), v);
+        const uint32_t taddr = tmem_lane_addr(tbase, warp, sb + 32 * c);
+        tmem_ld32(taddr, v);
 #pragma unroll
-        for (int i = 0; i < 32; ++i) {
-          const KeyInfo k = ki[32 * c + i];
-          const float z = fmaf(__uint_as_float(v[i]), k.sK, qc[k.aK]);
-          mx4[i & 3] = (32 * c + i < nk) ? fmaxf(mx4[i & 3], z) : mx4[i & 3];
+        for (int q = 0; q < 8; ++q) {
+          const int4 a4 = *reinterpret_cast<const int4 *>(aKj + 32 * c + 4 * q);
+          const float4 s4 = *reinterpret_cast<const float4 *>(sKj + 32 * c + 4 * q);
+          const int aa[4] = {a4.x, a4.y, a4.z, a4.w};
+          const float ss[4] = {s4.x, s4.y, s4.z, s4.w};
+#pragma unroll
+          for (int u = 0; u < 4; ++u) {
+            const int i = 4 * q + u;
+            const float z = fmaf(__uint_as_float(v[i]), ss[u], qc[aa[u]]);
+            v[i] = __float_as_uint(z);
+            if (full) mx4[u] = fmaxf(mx4[u], z);
+            else mx4[u] = (32 * c + i < nk) ? fmaxf(mx4[u], z) : mx4[u];
+          }
         }
+        uint32_t lo[16], hi[16];
+#pragma unroll
+        for (int i = 0; i < 16; ++i) { lo[i] = v[i]; hi[i] = v[16 + i]; }
+        tmem_st16(taddr, lo);
+        tmem_st16(taddr + 16, hi);
       }
+      tmem_st_wait();
       const float mx = fmaxf(fmaxf(mx4[0], mx4[1]), fmaxf(mx4[2], mx4[3]));
       float corr = 1.f;
       const bool need = mx > st.m + kRescaleLog2;
@@ -367,22 +430,31 @@ __global__ void __launch_bounds__(384, 1)
         st.m = mx;
       }
       const bool wr = __any_sync(0xffffffffu, need) != 0;
+      if (row == 0) LOW_TRACE(8, j);
       const float m = st.m;
       float ls[4] = {0.f, 0.f, 0.f, 0.f};
+      // pass 2: P and P * s_V, interleaved per 32 keys over the z columns
       for (int c = 0; c < 4; ++c) {
         tmem_ld32(tmem_lane_addr(tbase, warp, sb + 32 * c), v);
         uint32_t pp[16], ps[16];
 #pragma unroll
-        for (int i = 0; i < 16; ++i) {
-          const int k0 = 32 * c + 2 * i;
-          const KeyInfo a = ki[k0], b = ki[k0 + 1];
-          float p0 = ex2(fmaf(__uint_as_float(v[2 * i]), a.sK, qc[a.aK]) - m);
-          float p1 = ex2(fmaf(__uint_as_float(v[2 * i + 1]), b.sK, qc[b.aK]) - m);
-          p0 = (k0 < nk) ? p0 : 0.f;
-          p1 = (k0 + 1 < nk) ? p1 : 0.f;
-          ls[i & 3] += p0 + p1;
-          pp[i] = pack_bf16x2(p0, p1);
-          ps[i] = pack_bf16x2(p0 * a.sV, p1 * b.sV);
+        for (int q = 0; q < 8; ++q) {
+          const float4 sv4 = *reinterpret_cast<const float4 *>(sVj + 32 * c + 4 * q);
+          const float svv[4] = {sv4.x, sv4.y, sv4.z, sv4.w};
+#pragma unroll
+          for (int h2 = 0; h2 < 2; ++h2) {
+            const int i = 2 * q + h2;  // pair index within the chunk
+            const int k0 = 32 * c + 2 * i;
+            float p0 = ex2(__uint_as_float(v[2 * i]) - m);
+            float p1 = ex2(__uint_as_float(v[2 * i + 1]) - m);
+            if (!full) {
+              p0 = (k0 < nk) ? p0 : 0.f;
+              p1 = (k0 + 1 < nk) ? p1 : 0.f;
+            }
+            ls[i & 3] += p0 + p1;
+            pp[i] = pack_bf16x2(p0, p1);
+            ps[i] = pack_bf16x2(p0 * svv[2 * h2], p1 * svv[2 * h2 + 1]);
+          }
         }
         tmem_st16(tmem_lane_addr(tbase, warp, sb + 32 * c), pp);
         tmem_st16(tmem_lane_addr(tbase, warp, sb + 32 * c + 16), ps);
@@ -391,13 +463,14 @@ __global__ void __launch_bounds__(384, 1)
       tmem_st_wait();
       st.l += lsum;
       if (j > 0 && wr) {
-        if (!mbar_wait(&B.pv_done, (j - 1) & 1, abort, err)) { ok = false; break; }
+        if (!mbar_wait(&B.pv_done[(j - 1) & 1], ((j - 1) >> 1) & 1, abort, err)) { ok = false; break; }
         tc_fence_after();
         rescale_cols(tbase, warp, TM_OT, r + C, corr);
       }
       tc_fence_before();
       __syncwarp();
       if (lane == 0) mbar_arrive(&B.p_full[j & 1]);
+      if (row == 0) LOW_TRACE(3, j);
     }
     // restore operands: [O~ | P_C] / l in bf16 (O~ un-permuted)
     if (ok && mbar_wait(&B.last_done, 0, abort, err)) {
@@ -458,6 +531,13 @@ __global__ void __launch_bounds__(384, 1)
 
 }  // namespace
 
+#ifdef NANOKV_TRACE
+extern "C" int nanokv_debug_low_trace(void *host, size_t bytes) {
+  if (bytes < sizeof(g_low_trace)) return -1;
+  return cudaMemcpyFromSymbol(host, g_low_trace, sizeof(g_low_trace)) == cudaSuccess ? 0 : -3;
+}
+#endif
+
 bool tc_low_supported(const Codec &ck, const Codec &cv) {
   return ck.prec == PREC_BF16 && ck.d == DH && ck.r == cv.r && ck.C == cv.C && ck.r % 64 == 0 &&
          ck.r <= 192 && ck.C % 16 == 0 && ck.C <= 64;
@@ -465,7 +545,7 @@ bool tc_low_supported(const Codec &ck, const Codec &cv) {
 
 static size_t low_smem(int r, int C) {
   const int nrb = r / 64;
-  return (size_t)(3 * nrb + 1) * kBlk + (size_t)128 * (C + 1) * 4 + 2 * 128 * sizeof(KeyInfo) + 1024;
+  return (size_t)(3 * nrb + 1) * kBlk + (size_t)128 * (C + 1) * 4 + 3 * 2 * 128 * 4 + 1024;
 }
 
 cudaError_t tc_attend_low(const void *q, int64_t Tq, const Codec &ck, const Codec &cv, const Hist &hk,
