@@ -39,7 +39,7 @@ BAD_REASONS = ("hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown")
 # of the sources they were taken on: a kernel whose source has changed since
 # reports null traffic.
 NCU_TRAFFIC = {
-    ("attend_full", "full"): ("tc_full", "993e3a782c099ca0", 18821888 + 8109568),
+    ("attend_full", "full"): ("tc_full", "08ac9cd11bfcb180", 18886400 + 5319424),
     ("attend_low", "mixed"): ("tc_low", "0e8341580862d853", 17918464 + 15104),
     ("attend_dense", "full"): ("tc_dense", "c7fd737aad612d75", 43223040 + 1623296),
     ("encode", "full"): ("tc_encode", "cc83ab4e475cecac", 30489088 + 3072),

@@ -528,22 +528,25 @@ static int full_cluster_capacity() {
 
 int tc_full_splits(int64_t Tq, int H, int d, int64_t T) {
   // Cost model in microseconds: the launch runs ceil(units * ns / capacity)
-  // waves of clusters, each cluster ~3.3 us per 128-key tile plus ~3 tiles of
+  // waves of clusters, each cluster ~3.3 us per 128-key tile plus ~6 tiles of
   // fixed cost (staging, pipeline fill and drain); every extra split adds a
-  // [Tq, H, d] fp32 partial written here and read by the merge (~6 TB/s).
+  // [Tq, H, d] fp32 partial written here and read by the merge, counted
+  // twice over because the other branches' kernels, which run alongside,
+  // fill part of a ragged last wave anyway.  (Measured on the full-size
+  // workloads: 2 splits best at 110 key tiles, 1 at 37.)
   if (T <= 0 || Tq <= 0) return 1;
   const int64_t ntiles = (T + BN - 1) / BN;
   const int64_t units = (int64_t)H * ((((Tq + BM - 1) / BM) + 1) / 2);
   const int64_t cap = full_cluster_capacity();
   if (cap <= 0) return 1;
-  const double part_us = 2.0 * (double)Tq * H * d * 4.0 / 6.0e6;
+  const double part_us = 4.0 * (double)Tq * H * d * 4.0 / 6.0e6;
   int best = 1;
   double best_cost = 1e300;
   for (int ns = 1; ns <= kMaxFullSplits && ns <= ntiles; ++ns) {
     const int64_t per = (ntiles + ns - 1) / ns;
     if ((ntiles + per - 1) / per != ns) continue;  // some split would be empty
     const int64_t waves = (units * ns + cap - 1) / cap;
-    const double cost = (double)waves * ((double)per + 3.0) * 3.3 + (ns - 1) * part_us;
+    const double cost = (double)waves * ((double)per + 6.0) * 3.3 + (ns - 1) * part_us;
     if (cost < best_cost * 0.99) {
       best_cost = cost;
       best = ns;
