@@ -23,7 +23,7 @@ OK, ERR_INVALID, ERR_UNSUPPORTED, ERR_CUDA, ERR_TIMEOUT = 0, -1, -2, -3, -4
 SYMBOLS = ("nanokv_encode", "nanokv_attend", "nanokv_attend_workspace", "nanokv_lse_merge",
            "nanokv_set_kernel_path", "nanokv_check", "nanokv_last_error", "nanokv_version",
            "nanokv_timing_enable", "nanokv_timing_read", "nanokv_codec_aux_bytes",
-           "nanokv_codec_prepare", "nanokv_attend_static")
+           "nanokv_codec_prepare", "nanokv_attend_static", "nanokv_selftest_wait")
 
 # kernel identities of the diagnostics (nanokv_kernel_id)
 KERNELS = {0: "encode", 1: "attend_full", 2: "attend_low", 3: "attend_dense", 4: "lse_merge"}
@@ -88,6 +88,8 @@ def lib() -> ctypes.CDLL:
     L.nanokv_timing_enable.restype = ctypes.c_int
     L.nanokv_timing_read.argtypes = [vp, vp]
     L.nanokv_timing_read.restype = ctypes.c_int
+    L.nanokv_selftest_wait.argtypes = [ctypes.c_uint64, vp]
+    L.nanokv_selftest_wait.restype = ctypes.c_int
     _lib = L
     return L
 
@@ -304,6 +306,12 @@ def nanokv_set_kernel_path(path: int) -> int:
 
 def nanokv_check(device=None) -> None:
     _raise(lib().nanokv_check(_stream(device)))
+
+
+def nanokv_selftest_wait(limit_ms: float = 50.0, device=None) -> None:
+    """Failure-detection self-test: a kernel gives up on a wait nothing
+    satisfies after ~limit_ms; the next nanokv_check() reports the timeout."""
+    _raise(lib().nanokv_selftest_wait(ctypes.c_uint64(int(limit_ms * 1e6)), _stream(device)))
 
 
 def nanokv_version() -> str:

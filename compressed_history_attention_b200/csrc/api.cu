@@ -1,6 +1,7 @@
 // C ABI of libnanokv: argument validation, workspace layout, kernel selection.
 #include "../../include/nanokv.h"
 #include "common.cuh"
+#include "sm100.cuh"
 #include "tc.cuh"
 
 #include <stdarg.h>
@@ -95,6 +96,24 @@ static cudaError_t timed(int kid, int nk, cudaStream_t st, F &&launch) {
   std::lock_guard<std::mutex> lk(g_tmu);
   g_recs.push_back({kid, a, b});
   return e;
+}
+
+// A wait that is never satisfied, bounded like every pipeline wait: thread 0
+// initialises an mbarrier that nothing arrives on, polls it until `limit_ns`
+// of wall time has passed, then records the timeout in the error word.
+__global__ void selftest_wait_kernel(uint64_t limit_ns, unsigned *err) {
+  __shared__ uint64_t bar;
+  if (threadIdx.x == 0) {
+    sm100::mbar_init(&bar, 1);
+    sm100::fence_mbar_init();
+    const uint64_t t0 = sm100::globaltimer();
+    bool done = false;
+    while (!done) {
+      done = sm100::mbar_test(&bar, 0);
+      if (!done && sm100::globaltimer() - t0 > limit_ns) break;
+    }
+    if (!done) atomicOr(err, ERRW_TIMEOUT);
+  }
 }
 
 // Helper streams on which the independent branch kernels of one attend call
@@ -256,6 +275,14 @@ int nanokv_check(void *stream) {
     return fail(NANOKV_ERR_CUDA, "device error word 0x%x", w);
   }
   return NANOKV_OK;
+}
+
+int nanokv_selftest_wait(uint64_t limit_ns, void *stream) {
+  const uint64_t lim = limit_ns < 1000000ull ? 1000000ull : (limit_ns > 2000000000ull ? 2000000000ull : limit_ns);
+  unsigned *errw = error_word_ptr();
+  if (!errw) return fail(NANOKV_ERR_CUDA, "cannot resolve the device error word");
+  selftest_wait_kernel<<<1, 32, 0, (cudaStream_t)stream>>>(lim, errw);
+  return cuda_status(cudaGetLastError(), "selftest launch");
 }
 
 int nanokv_encode(const nanokv_codec *ck, const nanokv_codec *cv, const void *k, const void *v,

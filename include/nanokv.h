@@ -197,6 +197,16 @@ int nanokv_set_kernel_path(int32_t path);
  * NANOKV_ERR_CUDA if the stream reports an error. */
 int nanokv_check(void *stream);
 
+/* Failure-detection self-test (diagnostic; the method has no counterpart).
+ * Launches one small kernel on `stream` that waits on an mbarrier nothing
+ * arrives on, gives up after about `limit_ns` nanoseconds (clamped to
+ * [1e6, 2e9]) exactly as every pipeline wait of the attention and encode
+ * kernels does on expiry, records the timeout in the device error word and
+ * returns.  The next nanokv_check() on that stream then reports
+ * NANOKV_ERR_TIMEOUT and clears the word; the CUDA context stays usable.
+ * Returns NANOKV_OK once launched, NANOKV_ERR_CUDA on a launch error. */
+int nanokv_selftest_wait(uint64_t limit_ns, void *stream);
+
 /* Message for the calling thread's last non-OK status ("" if none). */
 const char *nanokv_last_error(void);
 
