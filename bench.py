@@ -235,12 +235,27 @@ def step_attend(s, w):
                      out=s["out"], lse=s["lse"], workspace=s["ws"])
 
 
-def work_of(w, n_enc):
+def full_tokens(w, s):
+    """History tokens the library attends on the full-dim path: T_full, or T
+    when the codec shape has no low-dim tensor-core kernel (the low-dim tokens
+    then run through the full-dim kernel, which gives the same result)."""
+    import compressed_history_attention_b200 as nk
+    return nk.nanokv_attend_full_tokens(s["ck"], s["cv"], w.T, w.T_full)
+
+
+def work_of(w, n_enc, s):
+    """Algorithmic work of one step.  `af` splits the history as the workload
+    does (T_full full-dim, T_low low-dim): the method's work, the same that
+    the oracle arm counts, and the numerator of every throughput figure for
+    the step.  `ak` splits it as the kernels run (full_tokens), for each
+    kernel's own roofline."""
     from compressed_history_attention_b200.accounting import attend_flops, encode_bytes, encode_flops
     af = attend_flops(w.Tq, w.H, w.d, w.r, w.C, w.T_full, w.T_low, w.Tq)
+    tf = full_tokens(w, s)
+    ak = attend_flops(w.Tq, w.H, w.d, w.r, w.C, tf, w.T - tf, w.Tq)
     ef = 2 * encode_flops(n_enc, w.J, w.r, w.C)
     eb = 2 * encode_bytes(n_enc, w.J, w.r, 4 if w.fp32 else 2, 4 if w.fp32 else 2)
-    return af, ef, eb
+    return af, ak, ef, eb
 
 
 def capture(fn):
@@ -287,7 +302,7 @@ def run_ours(a, rank, world, device):
     peaks, peaks_kind = load_peaks()
     w = WORKLOADS[a.workload]
     s = setup(w, device)
-    af, ef, eb = work_of(w, s["n_enc"])
+    af, ak, ef, eb = work_of(w, s["n_enc"], s)
     flush = torch.empty(256 * 1024 * 1024, dtype=torch.uint8, device=device)
 
     for _ in range(a.warmup):
@@ -349,7 +364,7 @@ def run_ours(a, rank, world, device):
     # dominant kernel: the one with the largest share of the timed region
     dom = max(kt.items(), key=lambda kv: kv[1][0])
     dom_name, (dom_ms, dom_n) = dom
-    dom_work = {"attend_full": af["full"], "attend_low": af["low"], "attend_dense": af["current"],
+    dom_work = {"attend_full": ak["full"], "attend_low": ak["low"], "attend_dense": ak["current"],
                 "encode": ef / 2, "lse_merge": None}[dom_name]
     dom_avg_ms = dom_ms / max(dom_n, 1)
     peak_tf = peaks["bf16_tflops"]
@@ -390,6 +405,7 @@ def run_ours(a, rank, world, device):
         "data": "synthetic (seeded clustered low-rank generator; random codec params)",
         "config": {"workload": w.describe(), "H": w.H, "d": w.d, "T": w.T, "T_full": w.T_full,
                    "T_low": w.T_low, "Tq": w.Tq, "T_cur": w.Tq, "C": w.C, "r": w.r,
+                   "T_full_attended": full_tokens(w, s),
                    "encode_tokens": s["n_enc"], "l2": "flushed between steps (256 MiB write outside the step events)",
                    "launch": "CUDA graph replay of the encode and attend calls",
                    "parallelism": f"replicas x{world}"},
@@ -444,7 +460,6 @@ def run_fast(a, device, peaks):
     """Side measurement of the mixed-dimensional (Fast) attend on the mixed
     workload (same shapes, most recent chunk full-dim, 9360 tokens low-dim)."""
     from synth.gen import WORKLOADS
-    from compressed_history_attention_b200.accounting import attend_flops
     w = WORKLOADS["mixed"]
     s = setup(w, device)
     for _ in range(2):
@@ -455,7 +470,7 @@ def run_fast(a, device, peaks):
     g = capture(lambda: step_attend(s, w))
     _, att = timed_loop(s, w, n, flush, with_encode=False, graphs=(None, g))
     ms = sum(att) / n
-    af = attend_flops(w.Tq, w.H, w.d, w.r, w.C, w.T_full, w.T_low, w.Tq)
+    af, ak, _, _ = work_of(w, s["n_enc"], s)
     tf = af["total"] / (ms * 1e-3) / 1e12
     # per-kernel durations from the library's per-launch events (separate loop)
     nk.nanokv_timing_read()
@@ -464,7 +479,7 @@ def run_fast(a, device, peaks):
     nk.nanokv_timing_enable(False)
     kt = nk.nanokv_timing_read()
     per = {}
-    for name, work in (("attend_low", af["low"]), ("attend_full", af["full"]), ("attend_dense", af["current"])):
+    for name, work in (("attend_low", ak["low"]), ("attend_full", ak["full"]), ("attend_dense", ak["current"])):
         ms_k, cnt = kt[name]
         if cnt:
             avg = ms_k / cnt
@@ -492,7 +507,7 @@ def run_step30(a, device, peaks):
         ws = s["ws"]
         layers.append(s)
     n_enc = layers[0]["n_enc"]
-    af, ef, eb = work_of(w, n_enc)
+    af, _, ef, eb = work_of(w, n_enc, layers[0])
     flops = w.layers * (af["total"] + ef)
 
     def step():

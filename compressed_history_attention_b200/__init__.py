@@ -8,5 +8,5 @@ from ._lib import (  # noqa: F401
     Codec, Hist, NanoKVError, alloc_hist, lib, nanokv_attend, nanokv_attend_workspace,
     nanokv_attend_static, nanokv_check, nanokv_encode, nanokv_lse_merge, nanokv_set_kernel_path,
     nanokv_timing_enable,
-    nanokv_timing_read, nanokv_version, nanokv_selftest_wait,
+    nanokv_timing_read, nanokv_version, nanokv_selftest_wait, nanokv_attend_full_tokens,
 )

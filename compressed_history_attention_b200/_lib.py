@@ -23,7 +23,8 @@ OK, ERR_INVALID, ERR_UNSUPPORTED, ERR_CUDA, ERR_TIMEOUT = 0, -1, -2, -3, -4
 SYMBOLS = ("nanokv_encode", "nanokv_attend", "nanokv_attend_workspace", "nanokv_lse_merge",
            "nanokv_set_kernel_path", "nanokv_check", "nanokv_last_error", "nanokv_version",
            "nanokv_timing_enable", "nanokv_timing_read", "nanokv_codec_aux_bytes",
-           "nanokv_codec_prepare", "nanokv_attend_static", "nanokv_selftest_wait")
+           "nanokv_codec_prepare", "nanokv_attend_static", "nanokv_selftest_wait",
+           "nanokv_attend_full_tokens")
 
 # kernel identities of the diagnostics (nanokv_kernel_id)
 KERNELS = {0: "encode", 1: "attend_full", 2: "attend_low", 3: "attend_dense", 4: "lse_merge"}
@@ -90,6 +91,8 @@ def lib() -> ctypes.CDLL:
     L.nanokv_timing_read.restype = ctypes.c_int
     L.nanokv_selftest_wait.argtypes = [ctypes.c_uint64, vp]
     L.nanokv_selftest_wait.restype = ctypes.c_int
+    L.nanokv_attend_full_tokens.argtypes = [P(_Codec), P(_Codec), i64, i64]
+    L.nanokv_attend_full_tokens.restype = i64
     _lib = L
     return L
 
@@ -306,6 +309,16 @@ def nanokv_set_kernel_path(path: int) -> int:
 
 def nanokv_check(device=None) -> None:
     _raise(lib().nanokv_check(_stream(device)))
+
+
+def nanokv_attend_full_tokens(ck: Codec, cv: Codec, T: int, T_full: int) -> int:
+    """History tokens nanokv_attend takes on the full-dim path (T_full, or T
+    when the codec shape has no low-dim tensor-core kernel)."""
+    sk, sv = ck.struct(), cv.struct()
+    n = int(lib().nanokv_attend_full_tokens(ctypes.byref(sk), ctypes.byref(sv), T, T_full))
+    if n < 0:
+        raise NanoKVError(ERR_INVALID, "nanokv_attend_full_tokens: invalid arguments")
+    return n
 
 
 def nanokv_selftest_wait(limit_ms: float = 50.0, device=None) -> None:

@@ -209,6 +209,16 @@ static int io_prec(int32_t dt) {
   return -1;
 }
 
+// Tokens attended on the full-dim path.  The low-dim and full-dim paths give
+// the same attention over the same compressed tokens (the low-dim form only
+// reorders the contraction), so when the tensor-core kernels have no low-dim
+// kernel for a codec shape but do have the full-dim one, the low-dim tokens
+// are attended there too (paths 0 and 2); path 1 keeps the routing as given.
+static int64_t effective_T_full(int path, bool tc_low_ok, bool tc_full_ok, int64_t T, int64_t T_full) {
+  if (path != 1 && T > T_full && !tc_low_ok && tc_full_ok) return T;
+  return T_full;
+}
+
 // workspace carve-up (every region 256-byte aligned)
 struct WsLayout {
   // branch b (0 low-dim, 1 full-dim, 2 current chunk) has nparts[b]
@@ -275,6 +285,13 @@ int nanokv_check(void *stream) {
     return fail(NANOKV_ERR_CUDA, "device error word 0x%x", w);
   }
   return NANOKV_OK;
+}
+
+int64_t nanokv_attend_full_tokens(const nanokv_codec *ck, const nanokv_codec *cv, int64_t T, int64_t T_full) {
+  Codec a, b;
+  if (T < 0 || T_full < 0 || T_full > T) return -1;
+  if (check_codec(ck, "ck", false, &a) || check_codec(cv, "cv", false, &b)) return -1;
+  return effective_T_full(g_kernel_path.load(), tc_low_supported(a, b), tc_full_supported(a, b), T, T_full);
 }
 
 int nanokv_selftest_wait(uint64_t limit_ns, void *stream) {
@@ -357,6 +374,7 @@ size_t nanokv_attend_workspace(int64_t Tq, const nanokv_codec *ck, const nanokv_
   const int path = g_kernel_path.load();
   const bool tc_low = path != 1 && tc_low_supported(a, b);
   const bool tc_full = path != 1 && tc_full_supported(a, b);
+  T_full = effective_T_full(path, tc_low_supported(a, b), tc_full_supported(a, b), T, T_full);
   const int splits = (tc_full && T_full > 0 && Tq > 0) ? tc_full_splits(Tq, a.H, a.d, T_full) : 1;
   return ws_layout(Tq, a, T - T_full, T_full, T_cur, tc_low, splits).total;
 }
@@ -394,9 +412,10 @@ int nanokv_attend(const void *q, int32_t io_dtype, int64_t Tq, const nanokv_code
     return fail(NANOKV_ERR_INVALID, "attend: k_cur/v_cur NULL or misaligned with T_cur > 0");
 
   const int path = g_kernel_path.load();
-  const int64_t T_low = T - T_full;
   const bool tc_full_ok = tc_full_supported(ck, cv);
   const bool tc_low_ok = tc_low_supported(ck, cv);
+  T_full = effective_T_full(path, tc_low_ok, tc_full_ok, T, T_full);
+  const int64_t T_low = T - T_full;
   const bool tc_dense_ok = tc_dense_supported(ck.prec, ck.d);
   if (path == 2 && ((T_full > 0 && !tc_full_ok) || (T_low > 0 && !tc_low_ok) ||
                     (T_cur > 0 && !tc_dense_ok)))

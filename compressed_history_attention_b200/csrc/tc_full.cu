@@ -48,7 +48,7 @@ namespace {
 constexpr int DH = 128;
 constexpr uint32_t kTile = 128 * 128 * 2;   // [128 x 128] bf16
 constexpr uint32_t kChunk = 128 * 64 * 2;   // [128 keys x 64 codes] bf16
-constexpr int NRING = 4;  // unpacked code chunks in flight
+constexpr int NRING = 4;  // unpacked code chunks in flight (2 for r > 192: shared memory)
 constexpr uint32_t IDESC_DEC = idesc_bf16(128, 128, false, false);
 constexpr uint32_t IDESC_S = idesc_bf16(128, 128, false, false);
 constexpr uint32_t IDESC_PV = idesc_bf16(128, 128, false, true);
@@ -95,6 +95,11 @@ __device__ __forceinline__ uint4 unpack8(uint32_t w) {
   return make_uint4(o[0], o[1], o[2], o[3]);
 }
 
+// kLarge (codecs with r > 192 or C > 64): the branch's centers are read from
+// global memory (L2) by the epilogue instead of being staged in shared
+// memory, and the code ring has 2 slots, so that a resident decoder slice of
+// up to r = 384 fits.
+template <bool kLarge>
 __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(384, 1)
     tc_full_kernel(const __grid_constant__ CUtensorMap tmQ, const FullArgs A) {
   extern __shared__ uint8_t smraw[];
@@ -103,7 +108,9 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(384, 1)
   uint8_t *sQ = sm;
   uint8_t *sD = sQ + kTile;
   uint8_t *sRing = sD + nrb * kChunk;
-  uint8_t *sKh = sRing + NRING * kChunk;
+  constexpr bool kCenGlobal = kLarge;
+  constexpr int nring = kLarge ? 2 : NRING;
+  uint8_t *sKh = sRing + nring * kChunk;
   uint8_t *sVh = sKh + kTile;
   uint8_t *sCen = sVh + kTile;  // this CTA's branch centers, head slice [C][128] bf16
   __shared__ FullBars B;
@@ -125,7 +132,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(384, 1)
 
   if (threadIdx.x == 0) {
     mbar_init(&B.q_full, 1);
-    for (int i = 0; i < NRING; ++i) { mbar_init(&B.ring_full[i], 2); mbar_init(&B.ring_empty[i], 1); }
+    for (int i = 0; i < nring; ++i) { mbar_init(&B.ring_full[i], 2); mbar_init(&B.ring_empty[i], 1); }
     mbar_init(&B.x_full, 1);
     mbar_init(&B.x_empty, 4);  // one arrive per epilogue warp once its last X load is done
     mbar_init(&B.half_done[0], 4);
@@ -179,7 +186,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(384, 1)
         }
       }
     }
-    const int C = A.C[rank];
+    const int C = kCenGlobal ? 0 : A.C[rank];  // nothing to stage when centers are read from L2
     const __nv_bfloat16 *cen = A.cen[rank] + (size_t)h * DH;
     for (int i0 = threadIdx.x; i0 < C * 16; i0 += 4 * 384) {
       uint4 v[4];
@@ -227,8 +234,8 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(384, 1)
         bool progress = false;
         // ---- decode stream
         if (jd < ntiles && (cb > 0 || jd == 0 || mbar_test(&B.x_empty, (jd - 1) & 1))) {
-          const int slot = cc % NRING;
-          if (mbar_test(&B.ring_full[slot], (cc / NRING) & 1)) {
+          const int slot = cc % nring;
+          if (mbar_test(&B.ring_full[slot], (cc / nring) & 1)) {
             if (cb == 0) FULL_TRACE(0, jd);
             tc_fence_after();
             const uint32_t a = aR + slot * kChunk, b = aD + cb * kChunk;
@@ -319,10 +326,10 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(384, 1)
     load(0, cur);
     for (int c = 0; c < nchunk; ++c) {
       if (c + 1 < nchunk) load(c + 1, nxt);
-      const int rs = c % NRING, cb = c % nrb;
+      const int rs = c % nring, cb = c % nrb;
       if (warp == 2 && lane == 0 && cb == 0) FULL_TRACE(9, c / nrb);
       if (warp == 2 && lane == 0 && cb == 1) FULL_TRACE(17, c / nrb);
-      if (c >= NRING && !mbar_wait(&B.ring_empty[rs], ((c / NRING) - 1) & 1, abort, err)) break;
+      if (c >= nring && !mbar_wait(&B.ring_empty[rs], ((c / nring) - 1) & 1, abort, err)) break;
       if (warp == 2 && lane == 0 && cb == 0) FULL_TRACE(10, c / nrb);
       if (warp == 2 && lane == 0 && cb == 1) FULL_TRACE(18, c / nrb);
       const uint32_t dst = smem_u32(sRing + rs * kChunk);
@@ -371,6 +378,20 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(384, 1)
       if (j + 1 < ntiles) key_meta(j + 1, a_next, s_next);
       const uint8_t *crow = sCen + a * 256;
       const int sw = a & 15;
+      uint32_t o[64];
+      if constexpr (kCenGlobal) {
+        // the key's center row (known a tile ahead) from L2, into the output
+        // registers, before X is ready: o = c + s x is then formed in place
+        const uint4 *src = reinterpret_cast<const uint4 *>(A.cen[rank] + (size_t)a * J + (size_t)h * DH);
+#pragma unroll
+        for (int g = 0; g < 16; ++g) {
+          const uint4 cv = __ldg(src + g);
+          o[4 * g] = cv.x;
+          o[4 * g + 1] = cv.y;
+          o[4 * g + 2] = cv.z;
+          o[4 * g + 3] = cv.w;
+        }
+      }
       if (!mbar_wait(&B.x_full, j & 1, abort, err)) break;
       if (t == 0) FULL_TRACE(4, j);
       tc_fence_after();
@@ -379,7 +400,6 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(384, 1)
       // computed into registers and X released before the destination
       // buffer is waited for, so the next decode overlaps the hand-off.
       const __nv_bfloat162 s2 = __floats2bfloat162_rn(s, s);
-      uint32_t o[64];
 #pragma unroll
       for (int c = 0; c < 4; ++c) {
         uint32_t x[32];
@@ -392,8 +412,17 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(384, 1)
         }
 #pragma unroll
         for (int g = 0; g < 4; ++g) {
-          const uint4 cv = *reinterpret_cast<const uint4 *>(crow + (((4 * c + g) ^ sw) << 4));
-          const uint32_t cw[4] = {cv.x, cv.y, cv.z, cv.w};
+          uint32_t cw[4];
+          if constexpr (kCenGlobal) {
+#pragma unroll
+            for (int i = 0; i < 4; ++i) cw[i] = o[16 * c + 4 * g + i];
+          } else {
+            const uint4 cv = *reinterpret_cast<const uint4 *>(crow + (((4 * c + g) ^ sw) << 4));
+            cw[0] = cv.x;
+            cw[1] = cv.y;
+            cw[2] = cv.z;
+            cw[3] = cv.w;
+          }
 #pragma unroll
           for (int i = 0; i < 4; ++i) {
             const uint32_t xp = pack_bf16x2(__uint_as_float(x[8 * g + 2 * i]), __uint_as_float(x[8 * g + 2 * i + 1]));
@@ -492,14 +521,20 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(384, 1)
 
 }  // namespace
 
-bool tc_full_supported(const Codec &ck, const Codec &cv) {
-  // shared memory: r <= 192 with up to 64 centers (r = 256 leaves no room for the center slice)
-  return ck.prec == PREC_BF16 && ck.d == DH && ck.r == cv.r && ck.r % 64 == 0 && ck.r <= 192 &&
-         ck.C <= 64 && cv.C <= 64;
-}
+static bool full_large(int r, int C) { return r > 192 || C > 64; }
 
 size_t tc_full_smem(int r, int C) {
-  return (size_t)3 * kTile + (size_t)(r / 64) * kChunk + NRING * kChunk + (size_t)C * 256 + 1024;
+  const bool large = full_large(r, C);
+  return (size_t)3 * kTile + (size_t)(r / 64) * kChunk + (size_t)(large ? 2 : NRING) * kChunk +
+         (large ? 0 : (size_t)C * 256) + 1024;
+}
+
+bool tc_full_supported(const Codec &ck, const Codec &cv) {
+  // shared memory: Q, the resident decoder slice (r / 64 blocks), the code
+  // ring, two decoded tiles and, for at most 64 centers, the center slice
+  const int C = ck.C > cv.C ? ck.C : cv.C;
+  return ck.prec == PREC_BF16 && ck.d == DH && ck.r == cv.r && ck.r % 64 == 0 && ck.r <= 384 &&
+         C <= 256 && tc_full_smem(ck.r, C) <= 232448;
 }
 
 // Largest number of two-CTA clusters of the full-dim kernel that can be
@@ -513,13 +548,14 @@ static int full_cluster_capacity() {
   cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
   int cap = sms / 2;
   const size_t smem = tc_full_smem(192, 64);
-  if (ensure_smem((const void *)tc_full_kernel, (int)smem) == cudaSuccess) {
+  if (ensure_smem((const void *)tc_full_kernel<false>, (int)smem) == cudaSuccess) {
     cudaLaunchConfig_t cfg{};
     cfg.gridDim = dim3(2, 1, 1);
     cfg.blockDim = dim3(384);
     cfg.dynamicSmemBytes = smem;
     int n = 0;
-    if (cudaOccupancyMaxActiveClusters(&n, (const void *)tc_full_kernel, &cfg) == cudaSuccess && n > 0) cap = n;
+    if (cudaOccupancyMaxActiveClusters(&n, (const void *)tc_full_kernel<false>, &cfg) == cudaSuccess && n > 0)
+      cap = n;
   }
   cudaGetLastError();
   cached[dev] = cap > 0 ? cap : 1;
@@ -590,13 +626,16 @@ cudaError_t tc_attend_full(const void *q, int64_t Tq, const Codec &ck, const Cod
   a.O = out.O;
   a.L = out.LSE;
   a.err = error_word_ptr();
-  const size_t smem = tc_full_smem(ck.r, ck.C > cv.C ? ck.C : cv.C);
-  ensure_smem((const void *)tc_full_kernel, (int)smem);
+  const int Cmax = ck.C > cv.C ? ck.C : cv.C;
+  const bool large = full_large(ck.r, Cmax);
+  const size_t smem = tc_full_smem(ck.r, Cmax);
+  ensure_smem(large ? (const void *)tc_full_kernel<true> : (const void *)tc_full_kernel<false>, (int)smem);
   const unsigned qt = (unsigned)((Tq + BM - 1) / BM);
   // every split must get at least one key tile (the caller merges nsplit partials)
   if ((T + a.Tsplit - 1) / a.Tsplit != nsplit) return cudaErrorInvalidValue;
   dim3 grid((qt + 1) & ~1u, (unsigned)ck.H, (unsigned)nsplit);
-  return launch_k(tc_full_kernel, grid, dim3(384), smem, st, pdl, mq, a);
+  return large ? launch_k(tc_full_kernel<true>, grid, dim3(384), smem, st, pdl, mq, a)
+               : launch_k(tc_full_kernel<false>, grid, dim3(384), smem, st, pdl, mq, a);
 }
 
 #ifdef NANOKV_TRACE

@@ -128,6 +128,11 @@ int nanokv_encode(const nanokv_codec *ck, const nanokv_codec *cv,
  *          never written to memory; the older T - T_full tokens use low-dim
  *          attention: per head h, scores tau (s (D_{K,h}^T q) . code +
  *          c_{K,a,h} . q), output (sum p c_{V,a,h} + D_{V,h} sum p s code) / sum p.
+ *          The two forms compute the same attention (the low-dim one only
+ *          reorders the contraction).  When the tensor-core kernels have no
+ *          low-dim kernel for the codec shape (r > 192 or C > 64) but have the
+ *          full-dim one, the low-dim tokens are attended with the full-dim
+ *          kernel as well (kernel paths 0 and 2; path 1 keeps the routing).
  *   k_cur, v_cur [T_cur, H, d] current chunk in io_dtype (may be NULL if T_cur = 0)
  *   softmax_scale tau (callers normally pass 1/sqrt(d)); no mask.
  *   out    [Tq, H, d] in io_dtype.  lse_out [H, Tq] fp32 natural-log LSE, or NULL.
@@ -196,6 +201,13 @@ int nanokv_set_kernel_path(int32_t path);
  * NANOKV_OK, NANOKV_ERR_TIMEOUT if a kernel gave up on a bounded wait, or
  * NANOKV_ERR_CUDA if the stream reports an error. */
 int nanokv_check(void *stream);
+
+/* Number of history tokens nanokv_attend attends on the full-dim path for
+ * these codecs under the current kernel path (T_full as given, or T when the
+ * low-dim tokens are attended with the full-dim kernel; see nanokv_attend).
+ * For work accounting and planning; -1 for invalid arguments. */
+int64_t nanokv_attend_full_tokens(const nanokv_codec *ck, const nanokv_codec *cv, int64_t T,
+                                  int64_t T_full);
 
 /* Failure-detection self-test (diagnostic; the method has no counterpart).
  * Launches one small kernel on `stream` that waits on an mbarrier nothing
