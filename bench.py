@@ -244,11 +244,13 @@ def full_tokens(w, s):
 
 
 def work_of(w, n_enc, s):
-    """Algorithmic work of one step.  `af` splits the history as the workload
-    does (T_full full-dim, T_low low-dim): the method's work, the same that
-    the oracle arm counts, and the numerator of every throughput figure for
-    the step.  `ak` splits it as the kernels run (full_tokens), for each
-    kernel's own roofline."""
+    """Algorithmic work of one step.  `ak` splits the history as the kernels
+    run it (full_tokens) and is the numerator of every throughput figure.
+    `af` splits it as the workload names it (T_full full-dim, T_low
+    low-dim).  The two differ only when low-dim tokens run full-dim; with
+    r > d that route does less arithmetic than the low-dim form (scores of
+    width d instead of r per head), so counting `af` there would credit
+    work that never ran.  `af` is reported beside it."""
     from compressed_history_attention_b200.accounting import attend_flops, encode_bytes, encode_flops
     af = attend_flops(w.Tq, w.H, w.d, w.r, w.C, w.T_full, w.T_low, w.Tq)
     tf = full_tokens(w, s)
@@ -359,7 +361,7 @@ def run_ours(a, rank, world, device):
     enc_ms, att_ms = sum(enc) / a.steps, sum(att) / a.steps
     step_ms, enc_ms, att_ms = max_over_ranks([step_ms, enc_ms, att_ms], world, device)
 
-    flops = af["total"] + ef
+    flops = ak["total"] + ef
     value = whole_job_tflops(flops, step_ms, world)
     # dominant kernel: the one with the largest share of the timed region
     dom = max(kt.items(), key=lambda kv: kv[1][0])
@@ -386,8 +388,8 @@ def run_ours(a, rank, world, device):
     kernels = {k: {"ms_total": round(v[0], 4), "launches": v[1],
                    "share": round(v[0] / max(1e-9, sum(x[0] for x in kt.values())), 4)}
                for k, v in kt.items() if v[1]}
-    attend_tf = af["total"] / (att_ms * 1e-3) / 1e12
-    hist_tf = (af["full"] + af["low"]) / (att_ms * 1e-3) / 1e12
+    attend_tf = ak["total"] / (att_ms * 1e-3) / 1e12
+    hist_tf = (ak["full"] + ak["low"]) / (att_ms * 1e-3) / 1e12
     enc_gbs = eb / (enc_ms * 1e-3) / 1e9
 
     e2e = run_e2e(s, w, a, device, flops, world)
@@ -406,6 +408,8 @@ def run_ours(a, rank, world, device):
         "config": {"workload": w.describe(), "H": w.H, "d": w.d, "T": w.T, "T_full": w.T_full,
                    "T_low": w.T_low, "Tq": w.Tq, "T_cur": w.Tq, "C": w.C, "r": w.r,
                    "T_full_attended": full_tokens(w, s),
+                   "step_gflop": round((ak["total"] + ef) / 1e9, 3),
+                   "step_gflop_as_named": round((af["total"] + ef) / 1e9, 3),
                    "encode_tokens": s["n_enc"], "l2": "flushed between steps (256 MiB write outside the step events)",
                    "launch": "CUDA graph replay of the encode and attend calls",
                    "parallelism": f"replicas x{world}"},
@@ -471,7 +475,7 @@ def run_fast(a, device, peaks):
     _, att = timed_loop(s, w, n, flush, with_encode=False, graphs=(None, g))
     ms = sum(att) / n
     af, ak, _, _ = work_of(w, s["n_enc"], s)
-    tf = af["total"] / (ms * 1e-3) / 1e12
+    tf = ak["total"] / (ms * 1e-3) / 1e12
     # per-kernel durations from the library's per-launch events (separate loop)
     nk.nanokv_timing_read()
     nk.nanokv_timing_enable(True)
@@ -507,8 +511,8 @@ def run_step30(a, device, peaks):
         ws = s["ws"]
         layers.append(s)
     n_enc = layers[0]["n_enc"]
-    af, _, ef, eb = work_of(w, n_enc, layers[0])
-    flops = w.layers * (af["total"] + ef)
+    _, ak, ef, eb = work_of(w, n_enc, layers[0])
+    flops = w.layers * (ak["total"] + ef)
 
     def step():
         for s in layers:
