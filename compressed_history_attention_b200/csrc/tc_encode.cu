@@ -255,6 +255,278 @@ __global__ void __launch_bounds__(256, 1)
   }
 }
 
+// Large codecs (C up to 256, r up to 384): G = x [C | E]^T no longer fits in
+// 512 TMEM columns next to the per-block projection buffers, and E x no longer
+// fits in one thread's registers.  The K loop therefore runs once per pass:
+//   pass 0        x C^T, N = C, accumulated in TMEM columns [0, C)
+//   pass 1 + p    x E_p^T for the p-th 128-row slice of E, per 64-wide K block
+//                 into one of two TMEM buffers (columns [256, 384), [384, 512)),
+//                 summed in fp32 registers as in the small-codec kernel
+// The token tile is re-read once per pass (from L2: a 128-token tile of a
+// 3072-wide x is 768 KB).  The epilogue is two warpgroups, each owning half of
+// every slice's columns; a finished slice (y - E c_a) is parked in TMEM
+// columns [128 p, 128 p + 128), where pass 0's center scores were, until the
+// row maximum, and so the scale, is known.
+//   warp 0       TMA: token tile and [centers] or [E slice] tile per K block
+//   warp 1       MMA issuer
+//   warps 4..11  epilogue: thread (row, half) with row = lane quarter of TMEM
+constexpr int LSTG = 4;
+constexpr int kRS = 128;  // E rows (projection columns) per pass
+
+struct EncLBars {
+  uint64_t full[LSTG], empty[LSTG], acc_full, part_full[2], part_empty[2], cen_read, max_full;
+  uint32_t tmem_base;
+  int abort;
+};
+
+__global__ void __launch_bounds__(384, 1)
+    tc_encode_large_kernel(const __grid_constant__ CUtensorMap tmX0, const __grid_constant__ CUtensorMap tmC0,
+                           const __grid_constant__ CUtensorMap tmE0, const __grid_constant__ CUtensorMap tmX1,
+                           const __grid_constant__ CUtensorMap tmC1, const __grid_constant__ CUtensorMap tmE1,
+                           const EncArgs A) {
+  extern __shared__ uint8_t smraw[];
+  uint8_t *sm = (uint8_t *)(((uintptr_t)smraw + 1023) & ~(uintptr_t)1023);
+  const int C = A.C, R = A.r;
+  const uint32_t kBmax = (uint32_t)(C > kRS ? C : kRS) * 128;
+  uint8_t *sA = sm;
+  uint8_t *sB = sA + LSTG * kA;
+  float *sCN = (float *)(sB + LSTG * kBmax);  // [C] |c_j|^2
+  float *sMax = sCN + C;                      // [2][128] per-half row maxima
+  __shared__ EncLBars B;
+
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const int br = blockIdx.y;
+  const CUtensorMap *tmX = br ? &tmX1 : &tmX0;
+  const CUtensorMap *tmC = br ? &tmC1 : &tmC0;
+  const CUtensorMap *tmE = br ? &tmE1 : &tmE0;
+  const int64_t t0 = (int64_t)blockIdx.x * 128;
+  const int nkb = A.J / 64;
+  const int ns = (R + kRS - 1) / kRS;  // projection passes
+  volatile int *abort = &B.abort;
+  unsigned *err = A.err;
+  constexpr uint32_t tmem_cols = 512;
+  constexpr uint32_t kPartCol = 256;
+
+  if (threadIdx.x == 0) {
+    for (int i = 0; i < LSTG; ++i) { mbar_init(&B.full[i], 1); mbar_init(&B.empty[i], 1); }
+    mbar_init(&B.acc_full, 1);
+    for (int i = 0; i < 2; ++i) { mbar_init(&B.part_full[i], 1); mbar_init(&B.part_empty[i], 8); }
+    mbar_init(&B.cen_read, 8);
+    mbar_init(&B.max_full, 8);
+    B.abort = 0;
+    fence_mbar_init();
+  }
+  if (warp == 0) {
+    tmem_alloc(&B.tmem_base, tmem_cols);
+    tmem_relinquish();
+  }
+  for (int i = threadIdx.x; i < C; i += blockDim.x) sCN[i] = A.aux[br][(size_t)C * R + i];
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tbase = B.tmem_base;
+
+  if (warp == 0) {
+    if (lane == 0) {
+      prefetch_tmap(tmX);
+      prefetch_tmap(tmC);
+      prefetch_tmap(tmE);
+      int q = 0;
+      bool ok = true;
+      for (int p = 0; p <= ns && ok; ++p) {
+        const uint32_t bbytes = p == 0 ? (uint32_t)C * 128 : (uint32_t)kRS * 128;
+        for (int kb = 0; kb < nkb; ++kb, ++q) {
+          const int s = q % LSTG;
+          if (q >= LSTG && !mbar_wait(&B.empty[s], ((q / LSTG) - 1) & 1, abort, err)) { ok = false; break; }
+          mbar_arrive_expect_tx(&B.full[s], kA + bbytes);
+          tma_load_2d(sA + s * kA, tmX, kb * 64, (int)t0, &B.full[s]);
+          if (p == 0)
+            tma_load_2d(sB + s * kBmax, tmC, kb * 64, 0, &B.full[s]);
+          else
+            tma_load_2d(sB + s * kBmax, tmE, kb * 64, (p - 1) * kRS, &B.full[s]);
+        }
+      }
+      // every issued copy lands before the CTA can exit
+      for (int i = (q > LSTG ? q - LSTG : 0); i < q; ++i) mbar_wait(&B.full[i % LSTG], (i / LSTG) & 1, nullptr, nullptr);
+    }
+  } else if (warp == 1) {
+    if (lane == 0) {
+      bool ok = true;
+      int q = 0;
+      const uint32_t idc = idesc_bf16(128, C, false, false);
+      for (int kb = 0; kb < nkb; ++kb, ++q) {
+        const int s = q % LSTG;
+        if (!mbar_wait(&B.full[s], (q / LSTG) & 1, abort, err)) { ok = false; break; }
+        tc_fence_after();
+        const uint32_t a = smem_u32(sA + s * kA), b = smem_u32(sB + s * kBmax);
+#pragma unroll
+        for (int k = 0; k < 4; ++k)
+          mma_ss(tbase, sdesc_sw128(a + 32 * k, 16, 1024), sdesc_sw128(b + 32 * k, 16, 1024), idc,
+                 (kb > 0 || k > 0));
+        mma_commit(&B.empty[s]);
+      }
+      if (ok) mma_commit(&B.acc_full);
+      int g = 0;  // projection block counter across passes
+      for (int p = 0; p < ns && ok; ++p) {
+        const int width = R - p * kRS < kRS ? R - p * kRS : kRS;
+        const uint32_t ide = idesc_bf16(128, width, false, false);
+        for (int kb = 0; kb < nkb; ++kb, ++q, ++g) {
+          const int s = q % LSTG, pb = g & 1;
+          if (!mbar_wait(&B.full[s], (q / LSTG) & 1, abort, err)) { ok = false; break; }
+          if (g >= 2 && !mbar_wait(&B.part_empty[pb], ((g >> 1) - 1) & 1, abort, err)) { ok = false; break; }
+          tc_fence_after();
+          const uint32_t a = smem_u32(sA + s * kA), b = smem_u32(sB + s * kBmax);
+#pragma unroll
+          for (int k = 0; k < 4; ++k)
+            mma_ss(tbase + kPartCol + pb * kRS, sdesc_sw128(a + 32 * k, 16, 1024),
+                   sdesc_sw128(b + 32 * k, 16, 1024), ide, k > 0);
+          mma_commit(&B.empty[s]);
+          mma_commit(&B.part_full[pb]);
+        }
+      }
+    }
+  } else if (warp >= 4) {
+    const int row = (warp & 3) * 32 + lane;
+    const int half = (warp - 4) >> 2;  // columns [64 half, 64 half + 64) of every slice
+    const int64_t t = t0 + row;
+    bool ok = mbar_wait(&B.acc_full, 0, abort, err);
+    int a = 0;
+    float m = 0.f;
+    if (ok) {
+      tc_fence_after();
+      uint32_t g[32];
+      // nearest center: argmin |c_j|^2 - 2 x.c_j, strict < keeps the lowest index
+      float best = INFINITY;
+      for (int c0 = 0; c0 < C; c0 += 32) {
+        tmem_ld32(tmem_lane_addr(tbase, warp, c0), g);
+#pragma unroll
+        for (int i = 0; i < 32; ++i) {
+          if (c0 + i < C) {
+            const float sc = fmaf(-2.f, __uint_as_float(g[i]), sCN[c0 + i]);
+            if (sc < best) { best = sc; a = c0 + i; }
+          }
+        }
+      }
+    }
+    // both halves read the center scores of a row before either parks a
+    // slice over them
+    tc_fence_before();
+    __syncwarp();
+    if (lane == 0) mbar_arrive(&B.cen_read);
+    bool cen_free = false;
+    const float *ec = A.aux[br] + (size_t)a * R;
+    float y[64];
+    int g = 0;
+    int last_w = 0;  // this thread's column count in the last slice
+    for (int p = 0; p < ns && ok; ++p) {
+      const int width = R - p * kRS < kRS ? R - p * kRS : kRS;
+      const int col0 = half * 64;
+      const bool mine = col0 < width;  // a 64-wide last slice belongs to half 0
+#pragma unroll
+      for (int k = 0; k < 64; ++k) y[k] = 0.f;
+      for (int kb = 0; kb < nkb; ++kb, ++g) {
+        const int pb = g & 1;
+        if (!mbar_wait(&B.part_full[pb], (g >> 1) & 1, abort, err)) { ok = false; break; }
+        tc_fence_after();
+        if (mine) {
+          uint32_t v[32];
+#pragma unroll
+          for (int k0 = 0; k0 < 64; k0 += 32) {
+            tmem_ld32(tmem_lane_addr(tbase, warp, kPartCol + pb * kRS + col0 + k0), v);
+#pragma unroll
+            for (int i = 0; i < 32; ++i) y[k0 + i] += __uint_as_float(v[i]);
+          }
+        }
+        tc_fence_before();
+        __syncwarp();
+        if (lane == 0) mbar_arrive(&B.part_empty[pb]);
+      }
+      if (!ok || !mine) continue;
+      // y = E x - E c_a for this slice
+      const float4 *e4 = reinterpret_cast<const float4 *>(ec + p * kRS + col0);
+#pragma unroll
+      for (int k4 = 0; k4 < 16; ++k4) {
+        const float4 e = __ldg(e4 + k4);
+        y[4 * k4 + 0] -= e.x;
+        y[4 * k4 + 1] -= e.y;
+        y[4 * k4 + 2] -= e.z;
+        y[4 * k4 + 3] -= e.w;
+      }
+#pragma unroll
+      for (int k = 0; k < 64; ++k) m = fmaxf(m, fabsf(y[k]));
+      if (p + 1 < ns) {
+        // park the slice where pass 0's center scores were
+        if (!cen_free) {
+          if (!(cen_free = mbar_wait(&B.cen_read, 0, abort, err))) { ok = false; continue; }
+          tc_fence_after();
+        }
+#pragma unroll
+        for (int k0 = 0; k0 < 64; k0 += 16) {
+          uint32_t v[16];
+#pragma unroll
+          for (int i = 0; i < 16; ++i) v[i] = __float_as_uint(y[k0 + i]);
+          tmem_st16(tmem_lane_addr(tbase, warp, p * kRS + col0 + k0), v);
+        }
+        tmem_st_wait();
+      } else {
+        last_w = 64;
+      }
+    }
+    // row maximum over both halves
+    sMax[half * 128 + row] = m;
+    __syncwarp();
+    if (lane == 0) mbar_arrive(&B.max_full);
+    if (ok) ok = mbar_wait(&B.max_full, 0, abort, err);
+    if (ok) {
+      m = fmaxf(sMax[row], sMax[128 + row]);
+      const __half sh = __float2half_rn(m / 7.0f);
+      const float sf = __half2float(sh);
+      // y * (1/s) with a correctly rounded reciprocal, as in the small-codec kernel
+      const float inv = sf > 0.f ? __frcp_rn(sf) : 0.f;
+      uint8_t *crow = A.codes[br] + t * (R / 2);
+      auto pack8 = [&](const float *v) {
+        uint32_t acc = 0;
+#pragma unroll
+        for (int i = 0; i < 8; ++i) {
+          const int code = (int)fminf(7.f, fmaxf(-7.f, rintf(v[i] * inv)));
+          acc |= (uint32_t)(code & 0xF) << (4 * i);
+        }
+        return acc;
+      };
+      for (int p = 0; p + 1 < ns; ++p) {
+#pragma unroll
+        for (int k0 = 0; k0 < 64; k0 += 32) {
+          uint32_t v[32];
+          tmem_ld32(tmem_lane_addr(tbase, warp, p * kRS + half * 64 + k0), v);
+          float f[32];
+#pragma unroll
+          for (int i = 0; i < 32; ++i) f[i] = __uint_as_float(v[i]);
+          const uint4 w = make_uint4(pack8(f), pack8(f + 8), pack8(f + 16), pack8(f + 24));
+          if (t < A.T) *reinterpret_cast<uint4 *>(crow + (p * kRS + half * 64 + k0) / 2) = w;
+        }
+      }
+      if (last_w) {
+        const int p = ns - 1;
+#pragma unroll
+        for (int k0 = 0; k0 < 64; k0 += 32) {
+          const uint4 w = make_uint4(pack8(y + k0), pack8(y + k0 + 8), pack8(y + k0 + 16), pack8(y + k0 + 24));
+          if (t < A.T) *reinterpret_cast<uint4 *>(crow + (p * kRS + half * 64 + k0) / 2) = w;
+        }
+      }
+      if (half == 0 && t < A.T) {
+        A.ids[br][t] = (uint8_t)a;
+        A.scales[br][t] = sh;
+      }
+    }
+  }
+  tc_fence_before();
+  __syncthreads();
+  if (warp == 0) {
+    tc_fence_after();
+    tmem_dealloc(tbase, tmem_cols);
+  }
+}
+
 // EC[j][k] = E[k] . c_j and |c_j|^2 in fp32: one warp per output
 template <typename TP>
 __global__ void codec_prepare_kernel(const TP *__restrict__ cen, const TP *__restrict__ E, int C, int r,
@@ -298,12 +570,19 @@ cudaError_t codec_prepare(const Codec &c, void *aux, cudaStream_t st) {
   return cudaGetLastError();
 }
 
+// the single-pass kernel holds E x in registers and [C | E] in one TMEM tile
+static bool enc_small(const Codec &c) { return (c.r == 64 || c.r == 128 || c.r == 192) && c.C <= 64; }
+
 bool tc_encode_supported(const Codec &c) {
-  return c.prec == PREC_BF16 && c.aux && (c.H * c.d) % 64 == 0 && (c.r == 64 || c.r == 128 || c.r == 192) &&
-         c.C % 16 == 0 && c.C <= 64;
+  if (!(c.prec == PREC_BF16 && c.aux && (c.H * c.d) % 64 == 0 && c.C % 16 == 0 && c.C >= 16)) return false;
+  return enc_small(c) || (c.r % 64 == 0 && c.r >= 64 && c.r <= 384 && c.C <= 256);
 }
 
 static size_t enc_smem(const Codec &c) {
+  if (!enc_small(c)) {
+    const size_t kb = (size_t)(c.C > kRS ? c.C : kRS) * 128;
+    return LSTG * (kA + kb) + ((size_t)c.C + 256) * sizeof(float) + 1024;
+  }
   const size_t N = c.C + c.r;
   return NSTG * (kA + N * 128) + ((size_t)c.C * (c.r + 1) + c.C) * sizeof(float) + 1024;
 }
@@ -314,10 +593,11 @@ cudaError_t tc_encode_pair(const Codec *c, const void *const *x, int64_t T, uint
   CUtensorMap m[2][3];
   EncArgs a{};
   const int J = c[0].H * c[0].d;
+  const bool small = enc_small(c[0]);
   for (int b = 0; b < nbranch; ++b) {
     if (!make_tmap_bf16_2d(&m[b][0], x[b], T, J, J, 128) ||
         !make_tmap_bf16_2d(&m[b][1], c[b].centers, c[b].C, J, J, c[b].C) ||
-        !make_tmap_bf16_2d(&m[b][2], c[b].E, c[b].r, J, J, c[b].r))
+        !make_tmap_bf16_2d(&m[b][2], c[b].E, c[b].r, J, J, small ? c[b].r : kRS))
       return cudaErrorInvalidValue;
     a.aux[b] = (const float *)c[b].aux;
     a.ids[b] = ids[b];
@@ -334,6 +614,11 @@ cudaError_t tc_encode_pair(const Codec *c, const void *const *x, int64_t T, uint
   a.err = error_word_ptr();
   const size_t smem = enc_smem(c[0]);
   dim3 grid((unsigned)((T + 127) / 128), (unsigned)nbranch);
+  if (!small) {
+    ensure_smem((const void *)tc_encode_large_kernel, (int)smem);
+    tc_encode_large_kernel<<<grid, 384, smem, st>>>(m[0][0], m[0][1], m[0][2], m[1][0], m[1][1], m[1][2], a);
+    return cudaGetLastError();
+  }
 #define NANOKV_ENC_CASE(RR)                                                                         \
   case RR:                                                                                          \
     ensure_smem((const void *)tc_encode_kernel<RR>, (int)smem); \
