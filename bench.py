@@ -39,10 +39,10 @@ BAD_REASONS = ("hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown")
 # of the sources they were taken on: a kernel whose source has changed since
 # reports null traffic.
 NCU_TRAFFIC = {
-    ("attend_full", "full"): ("tc_full", "08ac9cd11bfcb180", 18886400 + 5319424),
-    ("attend_low", "mixed"): ("tc_low", "0e8341580862d853", 17918464 + 15104),
-    ("attend_dense", "full"): ("tc_dense", "c7fd737aad612d75", 43223040 + 1623296),
-    ("encode", "full"): ("tc_encode", "cc83ab4e475cecac", 30489088 + 3072),
+    ("attend_full", "full"): ("tc_full", "4deaa1093a4d50d4", 18819072 + 5870336),
+    ("attend_low", "mixed"): ("tc_low", "4fcc55f69a077271", 17918464 + 15104),
+    ("attend_dense", "full"): ("tc_dense", "0b2aa648c02231cb", 43223040 + 1623296),
+    ("encode", "full"): ("tc_encode", "c8fa4e3280375134", 30489600 + 19712),
 }
 
 

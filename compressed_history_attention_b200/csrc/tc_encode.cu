@@ -1,18 +1,14 @@
-// Tensor-core encode (NanoKV Fig. 4(b)): for 128 tokens x per CTA,
-//     G = x [C | E]^T           (one GEMM, N = C + r, fp32 in TMEM)
+// Tensor-core encode (NanoKV Fig. 4(b)): for each token x,
+//     G = x [C | E]^T           (a GEMM, N = C + r, fp32)
 //     a = argmin_j |c_j|^2 - 2 G[j]          (= argmin |x - c_j|^2)
 //     y = G[C + k] - (E c_a)[k]              (= E (x - c_a))
 //     s = fp16(max|y| / 7),  code = clamp(rint(y / s), -7, 7)
 // The tables E c_j and |c_j|^2 come from nanokv_codec_prepare.  Both
 // branches (K and V) run in one launch (grid.y).
-// The projection part of G is accumulated per 64-wide K block into one of two
-// TMEM buffers and the blocks are summed in fp32 registers by the epilogue,
-// so no fp32 accumulation chain is longer than one block on the tensor core;
-// the codes are decided on values as accurate as a plain fp32 dot product.
-//   warp 0      TMA: token tile and [centers | E] tile per 64-wide K block
-//   warp 1      MMA issuer
-//   warps 2,3   stage the E c table and |c|^2 into shared memory
-//   warps 4..7  epilogue, one thread per token (TMEM lane)
+// G is accumulated per 64-wide K block into one of two TMEM buffers and the
+// blocks are summed in fp32 registers by the epilogue, so no fp32
+// accumulation chain is longer than one block on the tensor core; codes and
+// ids are decided on values as accurate as a plain fp32 dot product.
 #include "tc_common.cuh"
 
 namespace nanokv {
@@ -21,10 +17,11 @@ using namespace sm100;
 using namespace tc;
 
 #ifdef NANOKV_TRACE
-__device__ unsigned long long g_enc_trace[8][32];
-#define ENC_TRACE(ev, j)                                                                   \
-  do {                                                                                     \
-    if (blockIdx.x == 0 && blockIdx.y == 0 && (j) < 32) g_enc_trace[ev][j] = clock64();   \
+// clock64 events of both CTAs of the first cluster of the 2-CTA kernel
+__device__ unsigned long long g_enc_trace[2][8][32];
+#define ENC_TRACE(ev, j)                                                                             \
+  do {                                                                                               \
+    if (blockIdx.x < 2 && blockIdx.y == 0 && (j) < 32) g_enc_trace[blockIdx.x][ev][j] = clock64();  \
   } while (0)
 #else
 #define ENC_TRACE(ev, j) \
@@ -34,7 +31,6 @@ __device__ unsigned long long g_enc_trace[8][32];
 
 namespace {
 
-constexpr int NSTG = 3;
 constexpr uint32_t kA = 128 * 64 * 2;  // token tile [128 x 64] bf16
 
 struct EncArgs {
@@ -47,43 +43,81 @@ struct EncArgs {
   unsigned *err;
 };
 
-struct EncBars {
-  uint64_t full[NSTG], empty[NSTG], acc_full, part_full[2], part_empty[2];
+// Small codecs (C <= 64, r in {64, 128, 192}), the columns of G = x [C | E]^T
+// split over a 2-CTA cluster per 128-token tile so that a chunk of 4680 tokens
+// per branch fills all SMs and every CTA issues one MMA per K step:
+//   CTA 0   centers (padded to 64 rows; rows >= C read as zero) and E rows [0, P0)
+//   CTA 1   E rows [P0, r)
+// with P0 chosen so both sides have about the same N.  Each side accumulates
+// its columns per 64-wide K block into one of two TMEM buffers and sums the
+// blocks in fp32 registers.  CTA 0 finds the nearest center and hands the id
+// to CTA 1 through distributed shared memory; the two exchange their row
+// maxima the same way, so both derive the same scale and each packs its own
+// codes.  One MMA per K step reads the token tile once, and each CTA moves
+// the token tile plus half the [C | E] tile per K block (32 KB).  The K loop
+// runs at the rate TMA delivers those bytes to the SM; the tail after it
+// (argmin, hand-off, E c_a, scale, packing) is kept short by staging this
+// CTA's columns of the E c table in shared memory while the loop runs.
+//   warp 0      TMA: token tile and this CTA's [C | E] rows per K block
+//   warp 1      MMA issuer
+//   warps 2,3   stage |c|^2 and this CTA's columns of E c into shared memory
+//   warps 4..7  epilogue, thread = token (TMEM lane)
+constexpr int SSTG = 5;
+
+template <int R>
+struct SplitCols {
+  static constexpr int P0 = ((R - 64) / 2) / 32 * 32;  // E rows on CTA 0: 0, 32, 64 for r = 64, 128, 192
+  static constexpr int N0 = 64 + P0;                   // CTA 0: padded centers + E rows [0, P0)
+  static constexpr int N1 = R - P0;                    // CTA 1: E rows [P0, r)
+  static constexpr int ECS = N1 + 4;                   // row stride of the staged E c slice (floats)
+  static_assert(N0 % 32 == 0 && N1 % 32 == 0 && N0 <= 128 && N1 <= 128, "column split");
+};
+
+struct EncSBars {
+  uint64_t full[SSTG], empty[SSTG], part_full[2], part_empty[2], ec_full, ids_full, max_full;
   uint32_t tmem_base;
   int abort;
+  uint32_t ids[128];     // CTA 1: center id of each row, written by CTA 0
+  float peer_max[128];   // the other CTA's row maxima
 };
 
 template <int R>
-__global__ void __launch_bounds__(256, 1)
-    tc_encode_kernel(const __grid_constant__ CUtensorMap tmX0, const __grid_constant__ CUtensorMap tmC0,
-                     const __grid_constant__ CUtensorMap tmE0, const __grid_constant__ CUtensorMap tmX1,
-                     const __grid_constant__ CUtensorMap tmC1, const __grid_constant__ CUtensorMap tmE1,
-                     const EncArgs A) {
+__global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(256, 1)
+    tc_encode_split_kernel(const __grid_constant__ CUtensorMap tmX0, const __grid_constant__ CUtensorMap tmC0,
+                           const __grid_constant__ CUtensorMap tmEa0, const __grid_constant__ CUtensorMap tmEb0,
+                           const __grid_constant__ CUtensorMap tmX1, const __grid_constant__ CUtensorMap tmC1,
+                           const __grid_constant__ CUtensorMap tmEa1, const __grid_constant__ CUtensorMap tmEb1,
+                           const EncArgs A) {
+  using S = SplitCols<R>;
   extern __shared__ uint8_t smraw[];
   uint8_t *sm = (uint8_t *)(((uintptr_t)smraw + 1023) & ~(uintptr_t)1023);
-  const int N = A.C + R;
-  const uint32_t kB = (uint32_t)N * 128;  // [N x 64] bf16
+  constexpr uint32_t kBs = 128 * 128;  // up to 128 rows x 64 bf16
   uint8_t *sA = sm;
-  uint8_t *sB = sA + NSTG * kA;
-  float *sEC = (float *)(sB + NSTG * kB);  // [C][r + 1]
-  float *sCN = sEC + A.C * (R + 1);        // [C]
-  __shared__ EncBars B;
+  uint8_t *sB = sA + SSTG * kA;
+  float *sEC = (float *)(sB + SSTG * kBs);  // [C][ECS] this CTA's columns of E c_j
+  float *sCN = sEC + A.C * S::ECS;          // [C] |c_j|^2 (CTA 0)
+  __shared__ EncSBars B;
 
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const uint32_t rank = cluster_ctarank();
+  const uint32_t peer = rank ^ 1u;
   const int br = blockIdx.y;
   const CUtensorMap *tmX = br ? &tmX1 : &tmX0;
-  const CUtensorMap *tmC = br ? &tmC1 : &tmC0;
-  const CUtensorMap *tmE = br ? &tmE1 : &tmE0;
-  const int64_t t0 = (int64_t)blockIdx.x * 128;
+  const int64_t t0 = (int64_t)(blockIdx.x >> 1) * 128;
   const int nkb = A.J / 64;
+  const int C = A.C;
+  const int ncols = rank ? S::N1 : S::N0;
   volatile int *abort = &B.abort;
   unsigned *err = A.err;
-  const uint32_t tmem_cols = 512;  // [0, C) centers | [C, C + R) block buffer 0 | [C + R, C + 2R) buffer 1
+  constexpr uint32_t tmem_cols = 256;  // two per-block buffers of up to 128 columns
+  if (threadIdx.x == 0) ENC_TRACE(5, 0);
 
   if (threadIdx.x == 0) {
-    for (int i = 0; i < NSTG; ++i) { mbar_init(&B.full[i], 1); mbar_init(&B.empty[i], 1); }
-    mbar_init(&B.acc_full, 1);
+    for (int i = 0; i < SSTG; ++i) { mbar_init(&B.full[i], 1); mbar_init(&B.empty[i], 1); }
     for (int i = 0; i < 2; ++i) { mbar_init(&B.part_full[i], 1); mbar_init(&B.part_empty[i], 4); }
+    mbar_init(&B.ec_full, 64);
+    mbar_init(&B.ids_full, 128);
+    mbar_init(&B.max_full, 128);
     B.abort = 0;
     fence_mbar_init();
   }
@@ -91,88 +125,79 @@ __global__ void __launch_bounds__(256, 1)
     tmem_alloc(&B.tmem_base, tmem_cols);
     tmem_relinquish();
   }
-  {
-    // stage the E c table (rows padded to R + 1 floats against bank conflicts)
-    // and |c|^2 with all threads, 16-byte loads, several in flight per thread
-    const float4 *aux4 = reinterpret_cast<const float4 *>(A.aux[br]);
-    const int n4 = A.C * R / 4;
-    constexpr int U = 8;
-    for (int i0 = threadIdx.x; i0 < n4; i0 += U * 256) {
-      float4 v[U];
-#pragma unroll
-      for (int u = 0; u < U; ++u)
-        if (i0 + u * 256 < n4) v[u] = aux4[i0 + u * 256];
-#pragma unroll
-      for (int u = 0; u < U; ++u) {
-        const int i = i0 + u * 256;
-        if (i < n4) {
-          const int e = 4 * i, row = e / R, col = e % R;  // R % 4 == 0: a float4 never straddles rows
-          float *d = sEC + row * (R + 1) + col;
-          d[0] = v[u].x;
-          d[1] = v[u].y;
-          d[2] = v[u].z;
-          d[3] = v[u].w;
-        }
-      }
-    }
-    for (int i = threadIdx.x; i < A.C; i += 256) sCN[i] = A.aux[br][A.C * R + i];
-  }
   tc_fence_before();
   __syncthreads();
+  // both CTAs' barriers are initialised before any remote access: every
+  // thread arrives here and waits before its first remote access (epilogue)
+  // or at the end (the other warps)
+  cluster_arrive();
   tc_fence_after();
   const uint32_t tbase = B.tmem_base;
-  if (threadIdx.x == 0) ENC_TRACE(5, 0);
+  if (threadIdx.x == 0) ENC_TRACE(5, 1);
 
   if (warp == 0) {
     if (lane == 0) {
+      const CUtensorMap *tmB0 = rank ? (br ? &tmEb1 : &tmEb0) : (br ? &tmC1 : &tmC0);
+      const CUtensorMap *tmB1 = br ? &tmEa1 : &tmEa0;  // CTA 0's E rows [0, P0)
       prefetch_tmap(tmX);
-      prefetch_tmap(tmC);
-      prefetch_tmap(tmE);
+      prefetch_tmap(tmB0);
+      if (rank == 0 && S::P0 > 0) prefetch_tmap(tmB1);
+      const uint32_t bytes = kA + (uint32_t)ncols * 128;
       int issued = 0;
       for (int kb = 0; kb < nkb; ++kb) {
-        const int s = kb % NSTG;
-        if (kb >= NSTG && !mbar_wait(&B.empty[s], ((kb / NSTG) - 1) & 1, abort, err)) break;
+        const int s = kb % SSTG;
+        if (kb >= SSTG && !mbar_wait(&B.empty[s], ((kb / SSTG) - 1) & 1, abort, err)) break;
         ENC_TRACE(4, kb);
-        mbar_arrive_expect_tx(&B.full[s], kA + kB);
+        mbar_arrive_expect_tx(&B.full[s], bytes);
         tma_load_2d(sA + s * kA, tmX, kb * 64, (int)t0, &B.full[s]);
-        tma_load_2d(sB + s * kB, tmC, kb * 64, 0, &B.full[s]);
-        tma_load_2d(sB + s * kB + A.C * 128, tmE, kb * 64, 0, &B.full[s]);
+        if (rank == 0) {
+          tma_load_2d(sB + s * kBs, tmB0, kb * 64, 0, &B.full[s]);
+          if (S::P0 > 0) tma_load_2d(sB + s * kBs + 64 * 128, tmB1, kb * 64, 0, &B.full[s]);
+        } else {
+          tma_load_2d(sB + s * kBs, tmB0, kb * 64, S::P0, &B.full[s]);
+        }
         issued = kb + 1;
       }
-      for (int kb = (issued > NSTG ? issued - NSTG : 0); kb < issued; ++kb)
-        mbar_wait(&B.full[kb % NSTG], (kb / NSTG) & 1, nullptr, nullptr);
+      for (int kb = (issued > SSTG ? issued - SSTG : 0); kb < issued; ++kb)
+        mbar_wait(&B.full[kb % SSTG], (kb / SSTG) & 1, nullptr, nullptr);
     }
   } else if (warp == 1) {
     if (lane == 0) {
-      const uint32_t idc = idesc_bf16(128, A.C, false, false), ide = idesc_bf16(128, R, false, false);
-      bool ok = true;
+      const uint32_t idesc = idesc_bf16(128, ncols, false, false);
       for (int kb = 0; kb < nkb; ++kb) {
-        const int s = kb % NSTG, pb = kb & 1;
-        if (!mbar_wait(&B.full[s], (kb / NSTG) & 1, abort, err)) { ok = false; break; }
-        if (kb >= 2 && !mbar_wait(&B.part_empty[pb], ((kb >> 1) - 1) & 1, abort, err)) { ok = false; break; }
+        const int s = kb % SSTG, pb = kb & 1;
+        if (!mbar_wait(&B.full[s], (kb / SSTG) & 1, abort, err)) break;
+        if (kb >= 2 && !mbar_wait(&B.part_empty[pb], ((kb >> 1) - 1) & 1, abort, err)) break;
         ENC_TRACE(0, kb);
         tc_fence_after();
-        const uint32_t a = smem_u32(sA + s * kA), b = smem_u32(sB + s * kB);
-        const uint32_t be = b + A.C * 128;
+        const uint32_t a = smem_u32(sA + s * kA), b = smem_u32(sB + s * kBs);
 #pragma unroll
-        for (int k = 0; k < 4; ++k) {
-          mma_ss(tbase, sdesc_sw128(a + 32 * k, 16, 1024), sdesc_sw128(b + 32 * k, 16, 1024), idc,
-                 (kb > 0 || k > 0));
-          mma_ss(tbase + A.C + pb * R, sdesc_sw128(a + 32 * k, 16, 1024), sdesc_sw128(be + 32 * k, 16, 1024),
-                 ide, k > 0);
-        }
+        for (int k = 0; k < 4; ++k)
+          mma_ss(tbase + pb * 128, sdesc_sw128(a + 32 * k, 16, 1024), sdesc_sw128(b + 32 * k, 16, 1024), idesc,
+                 k > 0);
         mma_commit(&B.empty[s]);
         mma_commit(&B.part_full[pb]);
       }
-      if (ok) mma_commit(&B.acc_full);
     }
-  } else if (warp >= 4) {
+  } else if (warp < 4) {
+    // E c slice for this CTA's projection columns, rows padded to ECS floats
+    const int ecol = rank ? S::P0 : 0, ncol = rank ? S::N1 : S::P0;
+    const int i0 = threadIdx.x - 64, n4 = ncol / 4;
+    for (int i = i0; i < C * n4; i += 64) {
+      const int j = i / n4, k4 = i - j * n4;
+      const float4 v = __ldg(reinterpret_cast<const float4 *>(A.aux[br] + (size_t)j * R + ecol) + k4);
+      *reinterpret_cast<float4 *>(sEC + j * S::ECS + 4 * k4) = v;
+    }
+    if (rank == 0)
+      for (int i = i0; i < C; i += 64) sCN[i] = A.aux[br][(size_t)C * R + i];
+    mbar_arrive(&B.ec_full);
+  } else {
     const int row = (warp - 4) * 32 + lane;
     const int64_t t = t0 + row;
-    // E x, summed over K blocks in fp32
-    float y[R];
+    constexpr int NM = S::N0 > S::N1 ? S::N0 : S::N1;
+    float acc[NM];
 #pragma unroll
-    for (int k = 0; k < R; ++k) y[k] = 0.f;
+    for (int k = 0; k < NM; ++k) acc[k] = 0.f;
     bool ok = true;
     for (int kb = 0; kb < nkb; ++kb) {
       const int pb = kb & 1;
@@ -181,74 +206,119 @@ __global__ void __launch_bounds__(256, 1)
       tc_fence_after();
       uint32_t g[32];
 #pragma unroll
-      for (int k0 = 0; k0 < R; k0 += 32) {
-        tmem_ld32(tmem_lane_addr(tbase, warp, A.C + pb * R + k0), g);
+      for (int k0 = 0; k0 < NM; k0 += 32) {
+        if (k0 < ncols) {
+          tmem_ld32(tmem_lane_addr(tbase, warp, pb * 128 + k0), g);
 #pragma unroll
-        for (int i = 0; i < 32; ++i) y[k0 + i] += __uint_as_float(g[i]);
+          for (int i = 0; i < 32; ++i) acc[k0 + i] += __uint_as_float(g[i]);
+        }
       }
       tc_fence_before();
       __syncwarp();
       if (lane == 0) mbar_arrive(&B.part_empty[pb]);
       if (row == 0) ENC_TRACE(2, kb);
     }
-    if (ok && mbar_wait(&B.acc_full, 0, abort, err)) {
-      if (row == 0) ENC_TRACE(3, 0);
-      tc_fence_after();
-      uint32_t g[32];
-      // nearest center: argmin |c_j|^2 - 2 x.c_j, strict < keeps the lowest index
-      float best = INFINITY;
-      int a = 0;
-      for (int c0 = 0; c0 < A.C; c0 += 32) {
-        tmem_ld32(tmem_lane_addr(tbase, warp, c0), g);
+    if (row == 0) ENC_TRACE(3, 0);
+    cluster_wait();
+    if (ok) ok = mbar_wait(&B.ec_full, 0, abort, err);
+    // nearest center on CTA 0 (strict < keeps the lowest index), handed to CTA 1
+    int a = 0;
+    if (rank == 0) {
+      if (ok) {
+        float best = INFINITY;
 #pragma unroll
-        for (int i = 0; i < 32; ++i) {
-          if (c0 + i < A.C) {
-            const float sc = fmaf(-2.f, __uint_as_float(g[i]), sCN[c0 + i]);
-            if (sc < best) { best = sc; a = c0 + i; }
+        for (int j = 0; j < 64; ++j) {
+          if (j < C) {
+            const float sc = fmaf(-2.f, acc[j], sCN[j]);
+            if (sc < best) { best = sc; a = j; }
           }
         }
       }
-      // y = E x - E c_a
-      const float *ec = sEC + a * (R + 1);
-      float m = 0.f;
+      st_cluster_u32(mapa(smem_u32(&B.ids[row]), peer), (uint32_t)a);
+      mbar_arrive_cluster(mapa(smem_u32(&B.ids_full), peer));
+    } else {
+      if (ok) ok = mbar_wait_cluster(&B.ids_full, 0, abort, err);
+      if (ok) a = (int)B.ids[row];
+    }
+    if (row == 0) ENC_TRACE(3, 1);
+    // y = E x - E c_a over this CTA's projection columns
+    constexpr int Y0 = 64;  // first projection column on CTA 0
+    const int ecol0 = rank ? S::P0 : 0;  // in E rows
+    float m = 0.f;
+    if (ok) {
+      const float4 *e4 = reinterpret_cast<const float4 *>(sEC + a * S::ECS);
+      if (rank == 0) {
 #pragma unroll
-      for (int k = 0; k < R; ++k) {
-        y[k] -= ec[k];
-        m = fmaxf(m, fabsf(y[k]));
+        for (int k4 = 0; k4 < S::P0 / 4; ++k4) {
+          const float4 e = e4[k4];
+          acc[Y0 + 4 * k4 + 0] -= e.x;
+          acc[Y0 + 4 * k4 + 1] -= e.y;
+          acc[Y0 + 4 * k4 + 2] -= e.z;
+          acc[Y0 + 4 * k4 + 3] -= e.w;
+        }
+#pragma unroll
+        for (int k = 0; k < S::P0; ++k) m = fmaxf(m, fabsf(acc[Y0 + k]));
+      } else {
+#pragma unroll
+        for (int k4 = 0; k4 < S::N1 / 4; ++k4) {
+          const float4 e = e4[k4];
+          acc[4 * k4 + 0] -= e.x;
+          acc[4 * k4 + 1] -= e.y;
+          acc[4 * k4 + 2] -= e.z;
+          acc[4 * k4 + 3] -= e.w;
+        }
+#pragma unroll
+        for (int k = 0; k < S::N1; ++k) m = fmaxf(m, fabsf(acc[k]));
       }
-      if (row == 0) ENC_TRACE(3, 1);
+    }
+    // row maximum over both CTAs
+    st_cluster_u32(mapa(smem_u32(&B.peer_max[row]), peer), __float_as_uint(m));
+    mbar_arrive_cluster(mapa(smem_u32(&B.max_full), peer));
+    if (ok) ok = mbar_wait_cluster(&B.max_full, 0, abort, err);
+    if (row == 0) ENC_TRACE(3, 2);
+    if (ok) {
+      m = fmaxf(m, B.peer_max[row]);
       const __half sh = __float2half_rn(m / 7.0f);
       const float sf = __half2float(sh);
-      // y * (1/s) with a correctly rounded reciprocal: within an ulp or two of
-      // y / s, so a code can differ only for values within ~1e-7 relative of a
-      // rounding boundary (far inside the tie band)
+      // y * (1/s) with a correctly rounded reciprocal, as in the other encode kernels
       const float inv = sf > 0.f ? __frcp_rn(sf) : 0.f;
-      // INT4 codes, two per byte (code 2i in the low nibble)
-      uint8_t *crow = A.codes[br] + t * (R / 2);
+      uint8_t *crow = A.codes[br] + t * (R / 2) + ecol0 / 2;
+      auto pack8 = [&](int k) {
+        uint32_t w = 0;
 #pragma unroll
-      for (int k0 = 0; k0 < R; k0 += 32) {
-        uint32_t w[4];
-#pragma unroll
-        for (int q = 0; q < 4; ++q) {
-          uint32_t acc = 0;
-#pragma unroll
-          for (int i = 0; i < 8; ++i) {
-            const int code = (int)fminf(7.f, fmaxf(-7.f, rintf(y[k0 + 8 * q + i] * inv)));
-            acc |= (uint32_t)(code & 0xF) << (4 * i);
-          }
-          w[q] = acc;
+        for (int i = 0; i < 8; ++i) {
+          const int code = (int)fminf(7.f, fmaxf(-7.f, rintf(acc[k + i] * inv)));
+          w |= (uint32_t)(code & 0xF) << (4 * i);
         }
-        if (t < A.T) *reinterpret_cast<uint4 *>(crow + k0 / 2) = make_uint4(w[0], w[1], w[2], w[3]);
-      }
+        return w;
+      };
       if (t < A.T) {
-        A.ids[br][t] = (uint8_t)a;
-        A.scales[br][t] = sh;
+        // register indices stay compile-time: one loop per side
+        if (rank == 0) {
+#pragma unroll
+          for (int k0 = 0; k0 < S::P0; k0 += 32)
+            *reinterpret_cast<uint4 *>(crow + k0 / 2) =
+                make_uint4(pack8(Y0 + k0), pack8(Y0 + k0 + 8), pack8(Y0 + k0 + 16), pack8(Y0 + k0 + 24));
+        } else {
+#pragma unroll
+          for (int k0 = 0; k0 < S::N1; k0 += 32)
+            *reinterpret_cast<uint4 *>(crow + k0 / 2) =
+                make_uint4(pack8(k0), pack8(k0 + 8), pack8(k0 + 16), pack8(k0 + 24));
+        }
+        if (rank == 0) {
+          A.ids[br][t] = (uint8_t)a;
+          A.scales[br][t] = sh;
+        }
       }
-      if (row == 0) ENC_TRACE(3, 2);
     }
+    if (row == 0) ENC_TRACE(3, 3);
   }
+  if (warp < 4) cluster_wait();
   tc_fence_before();
   __syncthreads();
+  // the peer's stores and arrives into this CTA's shared memory are done
+  // before either CTA exits
+  cluster_sync();
   if (warp == 0) {
     tc_fence_after();
     tmem_dealloc(tbase, tmem_cols);
@@ -570,7 +640,8 @@ cudaError_t codec_prepare(const Codec &c, void *aux, cudaStream_t st) {
   return cudaGetLastError();
 }
 
-// the single-pass kernel holds E x in registers and [C | E] in one TMEM tile
+// the 2-CTA kernel's column split needs C <= 64 (one padded 64-row center
+// box) and r in {64, 128, 192}
 static bool enc_small(const Codec &c) { return (c.r == 64 || c.r == 128 || c.r == 192) && c.C <= 64; }
 
 bool tc_encode_supported(const Codec &c) {
@@ -578,60 +649,89 @@ bool tc_encode_supported(const Codec &c) {
   return enc_small(c) || (c.r % 64 == 0 && c.r >= 64 && c.r <= 384 && c.C <= 256);
 }
 
-static size_t enc_smem(const Codec &c) {
-  if (!enc_small(c)) {
-    const size_t kb = (size_t)(c.C > kRS ? c.C : kRS) * 128;
-    return LSTG * (kA + kb) + ((size_t)c.C + 256) * sizeof(float) + 1024;
-  }
-  const size_t N = c.C + c.r;
-  return NSTG * (kA + N * 128) + ((size_t)c.C * (c.r + 1) + c.C) * sizeof(float) + 1024;
+static size_t enc_large_smem(const Codec &c) {
+  const size_t kb = (size_t)(c.C > kRS ? c.C : kRS) * 128;
+  return LSTG * (kA + kb) + ((size_t)c.C + 256) * sizeof(float) + 1024;
 }
 
-cudaError_t tc_encode_pair(const Codec *c, const void *const *x, int64_t T, uint8_t *const *ids,
-                           uint8_t *const *codes, void *const *scales, int nbranch, cudaStream_t st) {
-  if (T == 0) return cudaSuccess;
-  CUtensorMap m[2][3];
-  EncArgs a{};
-  const int J = c[0].H * c[0].d;
-  const bool small = enc_small(c[0]);
+static size_t enc_split_smem(const Codec &c) {
+  const int P0 = ((c.r - 64) / 2) / 32 * 32, ecs = c.r - P0 + 4;
+  return SSTG * (kA + 128 * 128) + (size_t)c.C * (ecs + 1) * sizeof(float) + 1024;
+}
+
+template <int R>
+static cudaError_t launch_split(CUtensorMap (&m)[2][4], const EncArgs &a, int64_t T, int nbranch, size_t smem,
+                                cudaStream_t st) {
+  static_assert(SplitCols<R>::ECS == R - SplitCols<R>::P0 + 4, "staged E c stride");
+  ensure_smem((const void *)tc_encode_split_kernel<R>, (int)smem);
+  dim3 grid((unsigned)(2 * ((T + 127) / 128)), (unsigned)nbranch);
+  tc_encode_split_kernel<R><<<grid, 256, smem, st>>>(m[0][0], m[0][1], m[0][2], m[0][3], m[1][0], m[1][1],
+                                                      m[1][2], m[1][3], a);
+  return cudaGetLastError();
+}
+
+static void fill_args(EncArgs &a, const Codec *c, uint8_t *const *ids, uint8_t *const *codes,
+                      void *const *scales, int nbranch, int64_t T) {
   for (int b = 0; b < nbranch; ++b) {
-    if (!make_tmap_bf16_2d(&m[b][0], x[b], T, J, J, 128) ||
-        !make_tmap_bf16_2d(&m[b][1], c[b].centers, c[b].C, J, J, c[b].C) ||
-        !make_tmap_bf16_2d(&m[b][2], c[b].E, c[b].r, J, J, small ? c[b].r : kRS))
-      return cudaErrorInvalidValue;
     a.aux[b] = (const float *)c[b].aux;
     a.ids[b] = ids[b];
     a.codes[b] = codes[b];
     a.scales[b] = (__half *)scales[b];
   }
-  if (nbranch == 1) {
-    for (int i = 0; i < 3; ++i) m[1][i] = m[0][i];
-  }
   a.T = T;
-  a.J = J;
+  a.J = c[0].H * c[0].d;
   a.r = c[0].r;
   a.C = c[0].C;
   a.err = error_word_ptr();
-  const size_t smem = enc_smem(c[0]);
-  dim3 grid((unsigned)((T + 127) / 128), (unsigned)nbranch);
-  if (!small) {
-    ensure_smem((const void *)tc_encode_large_kernel, (int)smem);
-    tc_encode_large_kernel<<<grid, 384, smem, st>>>(m[0][0], m[0][1], m[0][2], m[1][0], m[1][1], m[1][2], a);
-    return cudaGetLastError();
-  }
-#define NANOKV_ENC_CASE(RR)                                                                         \
-  case RR:                                                                                          \
-    ensure_smem((const void *)tc_encode_kernel<RR>, (int)smem); \
-    tc_encode_kernel<RR><<<grid, 256, smem, st>>>(m[0][0], m[0][1], m[0][2], m[1][0], m[1][1], m[1][2], a); \
-    break;
-  switch (c[0].r) {
-    NANOKV_ENC_CASE(64)
-    NANOKV_ENC_CASE(128)
-    NANOKV_ENC_CASE(192)
-    default:
+}
+
+static cudaError_t tc_encode_split(const Codec *c, const void *const *x, int64_t T, uint8_t *const *ids,
+                                   uint8_t *const *codes, void *const *scales, int nbranch, cudaStream_t st) {
+  CUtensorMap m[2][4];
+  const int J = c[0].H * c[0].d, r = c[0].r;
+  const int P0 = ((r - 64) / 2) / 32 * 32, N1 = r - P0;
+  for (int b = 0; b < nbranch; ++b) {
+    // x tile; centers (64-row box, rows >= C read as zero); E rows [0, P0) for
+    // CTA 0 (the centers map stands in when P0 = 0); E rows [P0, r) for CTA 1
+    if (!make_tmap_bf16_2d(&m[b][0], x[b], T, J, J, 128) ||
+        !make_tmap_bf16_2d(&m[b][1], c[b].centers, c[b].C, J, J, 64) ||
+        !(P0 == 0 ? (m[b][2] = m[b][1], true) : make_tmap_bf16_2d(&m[b][2], c[b].E, r, J, J, P0)) ||
+        !make_tmap_bf16_2d(&m[b][3], c[b].E, r, J, J, N1))
       return cudaErrorInvalidValue;
   }
-#undef NANOKV_ENC_CASE
+  if (nbranch == 1)
+    for (int i = 0; i < 4; ++i) m[1][i] = m[0][i];
+  EncArgs a{};
+  fill_args(a, c, ids, codes, scales, nbranch, T);
+  const size_t smem = enc_split_smem(c[0]);
+  switch (r) {
+    case 64: return launch_split<64>(m, a, T, nbranch, smem, st);
+    case 128: return launch_split<128>(m, a, T, nbranch, smem, st);
+    case 192: return launch_split<192>(m, a, T, nbranch, smem, st);
+    default: return cudaErrorInvalidValue;
+  }
+}
+
+cudaError_t tc_encode_pair(const Codec *c, const void *const *x, int64_t T, uint8_t *const *ids,
+                           uint8_t *const *codes, void *const *scales, int nbranch, cudaStream_t st) {
+  if (T == 0) return cudaSuccess;
+  if (enc_small(c[0])) return tc_encode_split(c, x, T, ids, codes, scales, nbranch, st);
+  CUtensorMap m[2][3];
+  const int J = c[0].H * c[0].d;
+  for (int b = 0; b < nbranch; ++b) {
+    if (!make_tmap_bf16_2d(&m[b][0], x[b], T, J, J, 128) ||
+        !make_tmap_bf16_2d(&m[b][1], c[b].centers, c[b].C, J, J, c[b].C) ||
+        !make_tmap_bf16_2d(&m[b][2], c[b].E, c[b].r, J, J, kRS))
+      return cudaErrorInvalidValue;
+  }
+  if (nbranch == 1)
+    for (int i = 0; i < 3; ++i) m[1][i] = m[0][i];
+  EncArgs a{};
+  fill_args(a, c, ids, codes, scales, nbranch, T);
+  const size_t smem = enc_large_smem(c[0]);
+  dim3 grid((unsigned)((T + 127) / 128), (unsigned)nbranch);
+  ensure_smem((const void *)tc_encode_large_kernel, (int)smem);
+  tc_encode_large_kernel<<<grid, 384, smem, st>>>(m[0][0], m[0][1], m[0][2], m[1][0], m[1][1], m[1][2], a);
   return cudaGetLastError();
 }
 

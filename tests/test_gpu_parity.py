@@ -60,12 +60,14 @@ def test_encode_full_size_chunk(name, path):
         P.check_encode(x, c, h, _sd(w), sample=sample)
 
 
-@pytest.mark.parametrize("H,C,r", [(2, 128, 64), (3, 96, 192), (4, 80, 320), (8, 256, 256), (24, 256, 384)])
+@pytest.mark.parametrize("H,C,r", [(2, 16, 64), (4, 48, 128), (8, 32, 192), (2, 128, 64), (3, 96, 192),
+                                   (4, 80, 320), (8, 256, 256), (24, 256, 384)])
 def test_encode_codec_shapes(H, C, r, path):
-    """Codecs past the single-pass tensor-core encode (more than 64 centers or
-    r > 192): E shorter than one 128-row projection slice (r = 64), a 64-wide
-    last slice (r = 320), the long workload's codec, and a ragged token count
-    (300 = 2 tiles + 44)."""
+    """Every column split of the 2-CTA encode (r = 64, 128, 192 with fewer than
+    64 centers, whose padded center rows read as zero), and codecs past it
+    (more than 64 centers or r > 192): E shorter than one 128-row projection
+    slice (r = 64), a 64-wide last slice (r = 320), the long workload's codec.
+    A ragged token count (300 = 2 tiles + 44)."""
     w = scaled(WORKLOADS["long"], H=H, C=C, r=r, rank=min(r, 48), T=300, T_full=300, Tq=64)
     prob = P.problem(w)
     ck, cv, hk, hv = P.encode_history(w, prob)
