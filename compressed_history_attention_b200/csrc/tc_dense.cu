@@ -1,11 +1,16 @@
 // Tensor-core attention of the query chunk over the current, uncompressed
 // chunk (the third branch merged by LSE; NanoKV Fig. 4(d)).  One CTA per
 // (128-row query tile, head):
-//   warp 0      TMA producer: Q once, then K/V tiles (2 stages)
+//   warp 0      TMA producer: Q once, then K tiles (3 stages)
 //   warp 1      MMA issuer:   S = Q K^T (SS), O += P V (P read from TMEM)
+//   warp 2      TMA producer: V tiles (2 stages)
 //   warps 4..11 softmax:      two threads per query row (TMEM lane), each
 //                             owning 64 of the tile's 128 keys
-// S and O accumulate in TMEM; P overwrites S as bf16.  Every wait is bounded.
+// S and O accumulate in TMEM; P overwrites S as bf16.  A K stage is released
+// by the score MMAs that read it and a V stage by the value MMAs, and the two
+// streams have their own producers, so the next tiles' keys load while the
+// softmax runs instead of after the previous value MMA.  Every wait is
+// bounded.
 #include "tc_common.cuh"
 
 namespace nanokv {
@@ -63,9 +68,10 @@ constexpr uint32_t kTileBytes = 128 * 128 * 2;  // one [128 x 128] bf16 operand 
 constexpr uint32_t IDESC_S = idesc_bf16(128, 128, false, false);
 constexpr uint32_t IDESC_PV = idesc_bf16(128, 128, false, true);
 constexpr uint32_t TM_O = 0, TM_S = 128, TM_COLS = 512;  // S: two 128-column buffers
+constexpr int KST = 3;                                     // K stages (V has 2)
 
 struct DenseBars {
-  uint64_t q_full, k_full[2], v_full[2], kv_empty[2], s_full[2], p_full[2], pv_done;
+  uint64_t q_full, k_full[KST], k_empty[KST], v_full[2], v_empty[2], s_full[2], p_full[2], pv_done;
   uint32_t tmem_base;
   int abort;
   uint64_t xbar[2], lbar;  // row-max exchange per tile parity; final row-sum exchange
@@ -81,8 +87,8 @@ __global__ void __launch_bounds__(384, 1)
   extern __shared__ uint8_t smraw[];
   uint8_t *sm = (uint8_t *)(((uintptr_t)smraw + 1023) & ~(uintptr_t)1023);
   uint8_t *sQ = sm;
-  uint8_t *sK[2] = {sm + kTileBytes, sm + 2 * kTileBytes};
-  uint8_t *sV[2] = {sm + 3 * kTileBytes, sm + 4 * kTileBytes};
+  uint8_t *sK[KST] = {sm + kTileBytes, sm + 2 * kTileBytes, sm + 3 * kTileBytes};
+  uint8_t *sV[2] = {sm + 4 * kTileBytes, sm + 5 * kTileBytes};
   __shared__ DenseBars B;
 
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
@@ -93,10 +99,13 @@ __global__ void __launch_bounds__(384, 1)
 
   if (threadIdx.x == 0) {
     mbar_init(&B.q_full, 1);
-    for (int s = 0; s < 2; ++s) {
+    for (int s = 0; s < KST; ++s) {
       mbar_init(&B.k_full[s], 1);
+      mbar_init(&B.k_empty[s], 1);
+    }
+    for (int s = 0; s < 2; ++s) {
       mbar_init(&B.v_full[s], 1);
-      mbar_init(&B.kv_empty[s], 1);
+      mbar_init(&B.v_empty[s], 1);
     }
     for (int s = 0; s < 2; ++s) {
       mbar_init(&B.s_full[s], 1);
@@ -129,23 +138,34 @@ __global__ void __launch_bounds__(384, 1)
       tma_load_2d(sQ + kTileBytes / 2, &tmQ, h * DH + 64, (int)q0, &B.q_full);
       int issued = 0;
       for (int j = 0; j < ntiles; ++j) {
-        const int s = j & 1;
-        if (j >= 2 && !mbar_wait(&B.kv_empty[s], ((j >> 1) - 1) & 1, abort, err)) break;
+        const int s = j % KST;
+        if (j >= KST && !mbar_wait(&B.k_empty[s], ((j / KST) - 1) & 1, abort, err)) break;
         const int k0 = j * BN;
         mbar_arrive_expect_tx(&B.k_full[s], kTileBytes);
         tma_load_2d(sK[s], &tmK, h * DH, k0, &B.k_full[s]);
         tma_load_2d(sK[s] + kTileBytes / 2, &tmK, h * DH + 64, k0, &B.k_full[s]);
+        issued = j + 1;
+      }
+      // drain: every issued copy completes before the CTA may exit
+      mbar_wait(&B.q_full, 0, nullptr, nullptr);
+      for (int j = (issued > KST ? issued - KST : 0); j < issued; ++j)
+        mbar_wait(&B.k_full[j % KST], (j / KST) & 1, nullptr, nullptr);
+    }
+  } else if (warp == 2) {
+    // ---------------- TMA producer: values ----------------
+    if (lane == 0) {
+      int issued = 0;
+      for (int j = 0; j < ntiles; ++j) {
+        const int s = j & 1;
+        if (j >= 2 && !mbar_wait(&B.v_empty[s], ((j >> 1) - 1) & 1, abort, err)) break;
+        const int k0 = j * BN;
         mbar_arrive_expect_tx(&B.v_full[s], kTileBytes);
         tma_load_2d(sV[s], &tmV, h * DH, k0, &B.v_full[s]);
         tma_load_2d(sV[s] + kTileBytes / 2, &tmV, h * DH + 64, k0, &B.v_full[s]);
         issued = j + 1;
       }
-      // drain: every issued copy completes before the CTA may exit
-      mbar_wait(&B.q_full, 0, nullptr, nullptr);
-      for (int j = (issued > 2 ? issued - 2 : 0); j < issued; ++j) {
-        mbar_wait(&B.k_full[j & 1], (j >> 1) & 1, nullptr, nullptr);
+      for (int j = (issued > 2 ? issued - 2 : 0); j < issued; ++j)
         mbar_wait(&B.v_full[j & 1], (j >> 1) & 1, nullptr, nullptr);
-      }
     }
   } else if (warp == 1) {
     // ---------------- MMA issuer ----------------
@@ -153,12 +173,12 @@ __global__ void __launch_bounds__(384, 1)
       bool ok = mbar_wait(&B.q_full, 0, abort, err);
       const uint32_t aQ = smem_u32(sQ);
       auto scores = [&](int j) -> bool {
-        const int s = j & 1;
-        if (!mbar_wait(&B.k_full[s], (j >> 1) & 1, abort, err)) return false;
+        const int s = j & 1, ks3 = j % KST;
+        if (!mbar_wait(&B.k_full[ks3], (j / KST) & 1, abort, err)) return false;
         // the S buffer of tile j last held P of tile j - 2
         if (j >= 2 && !mbar_wait(&B.pv_done, (j - 2) & 1, abort, err)) return false;
         tc_fence_after();
-        const uint32_t aK = smem_u32(sK[s]);
+        const uint32_t aK = smem_u32(sK[ks3]);
 #pragma unroll
         for (int ks = 0; ks < DH / 16; ++ks) {
           const uint32_t off = (ks >> 2) * (kTileBytes / 2) + (ks & 3) * 32;
@@ -166,6 +186,7 @@ __global__ void __launch_bounds__(384, 1)
                  IDESC_S, ks > 0);
         }
         mma_commit(&B.s_full[s]);
+        mma_commit(&B.k_empty[ks3]);
         return true;
       };
       auto values = [&](int j) -> bool {
@@ -179,7 +200,7 @@ __global__ void __launch_bounds__(384, 1)
           mma_ts(tbase + TM_O, tbase + TM_S + s * 128 + ks * 8,
                  sdesc_sw128(aV + ks * 2048, kTileBytes / 2, 1024), IDESC_PV, (j > 0 || ks > 0));
         mma_commit(&B.pv_done);
-        mma_commit(&B.kv_empty[s]);
+        mma_commit(&B.v_empty[s]);
         return true;
       };
       if (ok) ok = scores(0);
@@ -252,7 +273,7 @@ cudaError_t tc_attend_dense(const void *q, int64_t Tq, int H, int d, const void 
   if (!make_tmap_bf16_2d(&mq, q, Tq, J, J, 128) || !make_tmap_bf16_2d(&mk, k, T, J, J, 128) ||
       !make_tmap_bf16_2d(&mv, v, T, J, J, 128))
     return cudaErrorInvalidValue;
-  const size_t smem = 5 * kTileBytes + 1024;
+  const size_t smem = (1 + KST + 2) * kTileBytes + 1024;
   ensure_smem((const void *)tc_dense_kernel, (int)smem);
   dim3 grid((unsigned)((Tq + BM - 1) / BM), (unsigned)H);
   return launch_k(tc_dense_kernel, grid, dim3(384), smem, st, pdl, mq, mk, mv, Tq, T, H, tau * kLog2e,
