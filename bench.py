@@ -41,7 +41,7 @@ BAD_REASONS = ("hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown")
 NCU_TRAFFIC = {
     ("attend_full", "full"): ("tc_full", "4deaa1093a4d50d4", 18819072 + 5870336),
     ("attend_low", "mixed"): ("tc_low", "4fcc55f69a077271", 17918464 + 15104),
-    ("attend_dense", "full"): ("tc_dense", "0b2aa648c02231cb", 43223040 + 1623296),
+    ("attend_dense", "full"): ("tc_dense", "6f930d6c7b63c100", 43229696 + 1877760),
     ("encode", "full"): ("tc_encode", "c8fa4e3280375134", 30489600 + 19712),
 }
 
