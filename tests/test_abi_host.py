@@ -145,3 +145,26 @@ def test_codec_prepare_validation():
     assert L.nanokv_codec_prepare(ctypes.byref(c), None, None) == _lib.ERR_INVALID
     assert L.nanokv_codec_prepare(ctypes.byref(c), ctypes.c_void_p((1 << 20) + 4), None) == _lib.ERR_INVALID
     assert L.nanokv_codec_prepare(ctypes.byref(_codec(E=0)), ctypes.c_void_p(1 << 20), None) == _lib.ERR_INVALID
+
+
+def test_attend_full_tokens_routing():
+    """History tokens attended on the full-dim path: the caller's T_full, or
+    all T tokens when the codec has a full-dim but no low-dim tensor-core
+    kernel (the two forms give the same result); the CUDA-core path keeps
+    the caller's split."""
+    L = nk.lib()
+    bf = dict(d=128, param_dtype=_lib.BF16, scale_dtype=_lib.F16)
+    small = _codec(H=12, r=192, C=64, **bf)
+    large = _codec(H=24, r=384, C=256, **bf)
+    g = lambda c, T, Tf: L.nanokv_attend_full_tokens(ctypes.byref(c), ctypes.byref(c), T, Tf)  # noqa: E731
+    assert g(small, 14040, 4680) == 4680       # low-dim tensor-core kernel covers r = 192, C = 64
+    assert g(large, 93600, 9360) == 93600      # r = 384, C = 256: low-dim tokens run full-dim
+    assert g(large, 93600, 93600) == 93600
+    assert g(_codec(), 256, 100) == 100        # fp32: CUDA-core kernels, split kept
+    assert g(small, 100, 200) == -1            # T_full > T
+    assert g(small, -1, 0) == -1
+    prev = nk.nanokv_set_kernel_path(1)        # CUDA-core path forced: split kept
+    try:
+        assert g(large, 93600, 9360) == 9360
+    finally:
+        nk.nanokv_set_kernel_path(prev)
