@@ -110,6 +110,11 @@ typedef struct {
  * Inputs k, v [T, J]; outputs ids_* [T], codes_* [T, r/2], scales_* [T].
  * Either branch may be skipped by passing its codec as NULL (then its input
  * and outputs are ignored).  T = 0 is a no-op.
+ * Kernels: bf16 codecs with aux, J a multiple of 64, C a multiple of 16
+ * (16..256) and r a multiple of 64 up to 384 run on the tensor cores (a
+ * 2-CTA kernel per 128 tokens for C <= 64 and r in {64, 128, 192}, a
+ * multi-pass kernel otherwise); every other codec runs on the fp32 CUDA-core
+ * kernel.  Both branches share one launch when their shapes agree.
  */
 int nanokv_encode(const nanokv_codec *ck, const nanokv_codec *cv,
                   const void *k, const void *v, int32_t x_dtype, int64_t T,
