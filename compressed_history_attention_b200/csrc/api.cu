@@ -2,6 +2,8 @@
 #include "../../include/nanokv.h"
 #include "common.cuh"
 #include "sm100.cuh"
+
+#include <nvtx3/nvToolsExt.h>
 #include "tc.cuh"
 
 #include <stdarg.h>
@@ -162,6 +164,15 @@ static cudaError_t branch_streams(BranchStreams **out) {
 
 static bool aligned16(const void *p) { return ((uintptr_t)p & 15u) == 0; }
 
+// One NVTX range per API call, so that a profiler timeline shows which
+// library call launched which kernels (no effect without a profiler attached).
+struct ApiRange {
+  explicit ApiRange(const char *name) { nvtxRangePushA(name); }
+  ~ApiRange() { nvtxRangePop(); }
+  ApiRange(const ApiRange &) = delete;
+  ApiRange &operator=(const ApiRange &) = delete;
+};
+
 unsigned *error_word_ptr() {
   // the device address of g_error_word on the current device
   static thread_local int cached_dev = -1;
@@ -305,6 +316,7 @@ int nanokv_selftest_wait(uint64_t limit_ns, void *stream) {
 int nanokv_encode(const nanokv_codec *ck, const nanokv_codec *cv, const void *k, const void *v,
                   int32_t x_dtype, int64_t T, uint8_t *ids_k, uint8_t *codes_k, void *scales_k,
                   uint8_t *ids_v, uint8_t *codes_v, void *scales_v, void *stream) {
+  ApiRange range("nanokv_encode");
   if (T < 0) return fail(NANOKV_ERR_INVALID, "encode: T=%lld < 0", (long long)T);
   if (!ck && !cv) return fail(NANOKV_ERR_INVALID, "encode: both codecs are NULL");
   Codec c[2];
@@ -359,6 +371,7 @@ size_t nanokv_codec_aux_bytes(const nanokv_codec *c_) {
 }
 
 int nanokv_codec_prepare(const nanokv_codec *c_, void *aux, void *stream) {
+  ApiRange range("nanokv_codec_prepare");
   Codec c;
   int s = check_codec(c_, "prepare", true, &c);
   if (s) return s;
@@ -384,6 +397,7 @@ int nanokv_attend(const void *q, int32_t io_dtype, int64_t Tq, const nanokv_code
                   int64_t T, int64_t T_full, const void *k_cur, const void *v_cur, int64_t T_cur,
                   float softmax_scale, void *out, float *lse_out, void *workspace,
                   size_t workspace_bytes, void *stream) {
+  ApiRange range("nanokv_attend");
   Codec ck, cv;
   int s;
   if ((s = check_codec(ck_, "attend ck", false, &ck))) return s;
@@ -521,6 +535,7 @@ int nanokv_attend(const void *q, int32_t io_dtype, int64_t Tq, const nanokv_code
 int nanokv_lse_merge(int32_t n, const float *const *o_parts, const float *const *lse_parts,
                      int64_t Tq, int32_t H, int32_t d, void *out, int32_t out_dtype,
                      float *lse_out, void *stream) {
+  ApiRange range("nanokv_lse_merge");
   if (n < 1 || n > kMaxParts) return fail(NANOKV_ERR_INVALID, "merge: n=%d out of range [1,%d]", n, kMaxParts);
   if (Tq < 0 || H < 1 || d < 4 || (d & 3)) return fail(NANOKV_ERR_INVALID, "merge: bad sizes (d must be a multiple of 4)");
   const int op = io_prec(out_dtype);
