@@ -168,3 +168,22 @@ def test_attend_full_tokens_routing():
         assert g(large, 93600, 9360) == 9360
     finally:
         nk.nanokv_set_kernel_path(prev)
+
+
+def test_workspace_follows_the_routing():
+    """A codec with no low-dim tensor-core kernel attends every history token
+    full-dim, so its workspace does not depend on the caller's split; with
+    the CUDA-core path forced, the split is kept and the low-dim buffers
+    appear."""
+    L = nk.lib()
+    bf = dict(d=128, param_dtype=_lib.BF16, scale_dtype=_lib.F16)
+    large = _codec(H=24, r=384, C=256, **bf)
+    small = _codec(H=12, r=192, C=64, **bf)
+    ws = lambda c, T, Tf: L.nanokv_attend_workspace(4680, ctypes.byref(c), ctypes.byref(c), T, Tf, 4680)  # noqa: E731
+    assert ws(large, 93600, 9360) == ws(large, 93600, 93600) > 0
+    assert ws(small, 14040, 4680) != ws(small, 14040, 14040)
+    prev = nk.nanokv_set_kernel_path(1)
+    try:
+        assert ws(large, 93600, 9360) != ws(large, 93600, 93600)
+    finally:
+        nk.nanokv_set_kernel_path(prev)
