@@ -60,6 +60,23 @@ __device__ __forceinline__ uint32_t pack_bf16x2(float lo, float hi) {
   return *reinterpret_cast<uint32_t *>(&v);
 }
 
+// 8 packed INT4 codes (one 32-bit word, code i in bits [4i, 4i+4)) -> 8 bf16
+// in the order (n0,n4), (n1,n5), (n2,n6), (n3,n7): position p of the group
+// holds code (0,4,1,5,2,6,3,7)[p].  (n XOR 8) | 0x4300 is the bf16 bit
+// pattern of 128 + (n + 8) for a two's-complement nibble n; subtracting 136
+// leaves n exactly.
+__device__ __forceinline__ uint4 unpack8(uint32_t w) {
+  const __nv_bfloat162 bias = __floats2bfloat162_rn(136.f, 136.f);
+  uint32_t o[4];
+#pragma unroll
+  for (int i = 0; i < 4; ++i) {
+    const uint32_t b = ((w >> (4 * i)) & 0x000F000Fu) ^ 0x43084308u;
+    __nv_bfloat162 v = __hsub2(*reinterpret_cast<const __nv_bfloat162 *>(&b), bias);
+    o[i] = *reinterpret_cast<uint32_t *>(&v);
+  }
+  return make_uint4(o[0], o[1], o[2], o[3]);
+}
+
 // TMEM address of (lane base of this warp's quarter, column)
 __device__ __forceinline__ uint32_t tmem_lane_addr(uint32_t base, int warp, uint32_t col) {
   return base + ((uint32_t)((warp & 3) * 32) << 16) + col;
@@ -89,26 +106,63 @@ __device__ unsigned long long g_softmax_trace[8][128];
 // 64 of those columns, updates the row state.  `nk` valid keys; `zscale`
 // multiplies raw scores into log2 units.  Returns the factor by which the
 // caller must rescale O (1 if none); *rescale tells whether any row of the
-// warp needs it.
+// warp needs it.  Full tiles take a compact loop over 32-column chunks (the
+// kernels that call this run many warp roles at once, and their unrolled
+// code competes for the instruction cache); a partial last tile takes a
+// rolled, masked path.
+static __device__ __noinline__ float softmax_tile_partial(uint32_t tbase, int warp, uint32_t s_col, int nk, float zscale,
+                                                   RowState &st, bool &warp_rescale) {
+  float mx = -INFINITY;
+  uint32_t r32[32];
+#pragma unroll 1
+  for (int c = 0; c < 4; ++c) {
+    sm100::tmem_ld32(tmem_lane_addr(tbase, warp, s_col + 32 * c), r32);
+#pragma unroll
+    for (int i = 0; i < 32; ++i) mx = (32 * c + i < nk) ? fmaxf(mx, __uint_as_float(r32[i])) : mx;
+  }
+  mx *= zscale;
+  float corr = 1.f;
+  const bool need = mx > st.m + kRescaleLog2;
+  if (need) {
+    corr = (st.m == -INFINITY) ? 0.f : ex2(st.m - mx);
+    st.l *= corr;
+    st.m = mx;
+  }
+  warp_rescale = __any_sync(0xffffffffu, need) != 0;
+  const float m = st.m;
+  float ls = 0.f;
+#pragma unroll 1
+  for (int c = 0; c < 4; ++c) {
+    sm100::tmem_ld32(tmem_lane_addr(tbase, warp, s_col + 32 * c), r32);
+    uint32_t pk[16];
+#pragma unroll
+    for (int i = 0; i < 16; ++i) {
+      const int k0 = 32 * c + 2 * i;
+      const float p0 = (k0 < nk) ? ex2(fmaf(__uint_as_float(r32[2 * i]), zscale, -m)) : 0.f;
+      const float p1 = (k0 + 1 < nk) ? ex2(fmaf(__uint_as_float(r32[2 * i + 1]), zscale, -m)) : 0.f;
+      ls += p0 + p1;
+      pk[i] = pack_bf16x2(p0, p1);
+    }
+    sm100::tmem_st16(tmem_lane_addr(tbase, warp, s_col + 16 * c), pk);
+  }
+  sm100::tmem_st_wait();
+  st.l += ls;
+  return corr;
+}
+
 __device__ __forceinline__ float softmax_tile(uint32_t tbase, int warp, uint32_t s_col, int nk,
                                               float zscale, RowState &st, bool &warp_rescale,
                                               int trace_j = -1) {
-  uint32_t r[64];
-  const bool full = nk >= 128;
+  if (nk < 128) return softmax_tile_partial(tbase, warp, s_col, nk, zscale, st, warp_rescale);
   // pass 1: row max over the tile, four independent chains
   float mx4[4] = {-INFINITY, -INFINITY, -INFINITY, -INFINITY};
   SOFTMAX_TRACE(0, trace_j);
+  uint32_t r32[32];
+#pragma unroll 1
+  for (int c = 0; c < 4; ++c) {
+    sm100::tmem_ld32(tmem_lane_addr(tbase, warp, s_col + 32 * c), r32);
 #pragma unroll
-  for (int c = 0; c < 2; ++c) {
-    sm100::tmem_ld64(tmem_lane_addr(tbase, warp, s_col + 64 * c), r);
-    if (full) {
-#pragma unroll
-      for (int i = 0; i < 64; ++i) mx4[i & 3] = fmaxf(mx4[i & 3], __uint_as_float(r[i]));
-    } else {
-#pragma unroll
-      for (int i = 0; i < 64; ++i)
-        mx4[i & 3] = (64 * c + i < nk) ? fmaxf(mx4[i & 3], __uint_as_float(r[i])) : mx4[i & 3];
-    }
+    for (int i = 0; i < 32; ++i) mx4[i & 3] = fmaxf(mx4[i & 3], __uint_as_float(r32[i]));
   }
   // scores are scaled after the max (zscale > 0 keeps the order)
   const float mx = fmaxf(fmaxf(mx4[0], mx4[1]), fmaxf(mx4[2], mx4[3])) * zscale;
@@ -123,29 +177,21 @@ __device__ __forceinline__ float softmax_tile(uint32_t tbase, int warp, uint32_t
   SOFTMAX_TRACE(1, trace_j);
   const float m = st.m;
   float ls[4] = {0.f, 0.f, 0.f, 0.f};
-  // pass 2 in 32-column chunks (fewer live registers than 64)
-#pragma unroll
+  // pass 2 in 32-column chunks
+#pragma unroll 1
   for (int c = 0; c < 4; ++c) {
-    uint32_t r32[32];
     sm100::tmem_ld32(tmem_lane_addr(tbase, warp, s_col + 32 * c), r32);
-    if (c == 0) SOFTMAX_TRACE(2, trace_j);
     uint32_t pk[16];
 #pragma unroll
     for (int i = 0; i < 16; ++i) {
-      const int k0 = 32 * c + 2 * i;
-      float p0 = ex2(fmaf(__uint_as_float(r32[2 * i]), zscale, -m));
-      float p1 = ex2(fmaf(__uint_as_float(r32[2 * i + 1]), zscale, -m));
-      if (!full) {
-        p0 = (k0 < nk) ? p0 : 0.f;
-        p1 = (k0 + 1 < nk) ? p1 : 0.f;
-      }
+      const float p0 = ex2(fmaf(__uint_as_float(r32[2 * i]), zscale, -m));
+      const float p1 = ex2(fmaf(__uint_as_float(r32[2 * i + 1]), zscale, -m));
       ls[i & 3] += p0 + p1;
       pk[i] = pack_bf16x2(p0, p1);
     }
     // P of S columns [32c, 32c + 32) goes to columns [16c, 16c + 16), all of
     // which were read by this chunk or an earlier one
     sm100::tmem_st16(tmem_lane_addr(tbase, warp, s_col + 16 * c), pk);
-    SOFTMAX_TRACE(4 + c, trace_j);
   }
   sm100::tmem_st_wait();
   SOFTMAX_TRACE(3, trace_j);
@@ -246,7 +292,7 @@ __device__ __forceinline__ void write_row_half(uint32_t tbase, int warp, uint32_
 // Multiplies this thread's O row (128 fp32 columns at o_col) by f.
 __device__ __forceinline__ void rescale_o(uint32_t tbase, int warp, uint32_t o_col, float f) {
   uint32_t r[16];
-#pragma unroll
+#pragma unroll 1
   for (int c = 0; c < 8; ++c) {
     const uint32_t a = tmem_lane_addr(tbase, warp, o_col + 16 * c);
     sm100::tmem_ld16(a, r);
@@ -265,7 +311,7 @@ __device__ __forceinline__ void write_row(uint32_t tbase, int warp, uint32_t o_c
   const float inv = st.l > 0.f ? 1.f / st.l : 0.f;
   uint32_t r[32];
   float *dst = O + (row * H + h) * 128;
-#pragma unroll
+#pragma unroll 1
   for (int c = 0; c < 4; ++c) {
     sm100::tmem_ld32(tmem_lane_addr(tbase, warp, o_col + 32 * c), r);
     sm100::tmem_ld_wait();

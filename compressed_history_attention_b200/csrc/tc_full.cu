@@ -82,19 +82,6 @@ struct FullBars {
 // 8 packed INT4 codes (one 32-bit word, code i in bits [4i, 4i+4)) -> 8 bf16
 // in the order (n0,n4), (n1,n5), (n2,n6), (n3,n7): position p of the group
 // holds code (0,4,1,5,2,6,3,7)[p]
-__device__ __forceinline__ uint4 unpack8(uint32_t w) {
-  const __nv_bfloat162 bias = __floats2bfloat162_rn(136.f, 136.f);
-  uint32_t o[4];
-#pragma unroll
-  for (int i = 0; i < 4; ++i) {
-    // (nibble XOR 8) | 0x4300 encodes 128 + (n + 8) in bf16; subtract 136
-    const uint32_t b = ((w >> (4 * i)) & 0x000F000Fu) ^ 0x43084308u;
-    __nv_bfloat162 v = __hsub2(*reinterpret_cast<const __nv_bfloat162 *>(&b), bias);
-    o[i] = *reinterpret_cast<uint32_t *>(&v);
-  }
-  return make_uint4(o[0], o[1], o[2], o[3]);
-}
-
 // kLarge (codecs with r > 192 or C > 64): the branch's centers are read from
 // global memory (L2) by the epilogue instead of being staged in shared
 // memory, and the code ring has 2 slots, so that a resident decoder slice of

@@ -65,18 +65,6 @@ struct LowBars {
   int abort;
 };
 
-__device__ __forceinline__ uint4 unpack8(uint32_t w) {
-  const __nv_bfloat162 bias = __floats2bfloat162_rn(136.f, 136.f);
-  uint32_t o[4];
-#pragma unroll
-  for (int i = 0; i < 4; ++i) {
-    const uint32_t b = ((w >> (4 * i)) & 0x000F000Fu) ^ 0x43084308u;
-    __nv_bfloat162 v = __hsub2(*reinterpret_cast<const __nv_bfloat162 *>(&b), bias);
-    o[i] = *reinterpret_cast<uint32_t *>(&v);
-  }
-  return make_uint4(o[0], o[1], o[2], o[3]);
-}
-
 __global__ void __launch_bounds__(384, 1)
     tc_low_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUtensorMap tmDk,
                   const __grid_constant__ CUtensorMap tmCk, const __grid_constant__ CUtensorMap tmDv,
