@@ -128,3 +128,79 @@ def compare_attn(O_gpu, L_gpu, O_ref, L_ref, fp32: bool, rows=None, tol=None):
 
 def tau_of(w):
     return 1.0 / math.sqrt(w.d)
+
+
+U_BF16 = 2.0 ** -8  # unit roundoff of bf16 (8 significant bits, round to nearest)
+
+
+def rounding_bound(q, ck, cv, ohk, ohv, kc, vc, T_full, tau):
+    """Per-element bound on |O_gpu - O_exact| for the tensor-core path, for
+    queries q [R, H, d] over the compressed history (oracle dicts) plus the
+    current chunk kc, vc [Tc, H, d], all in fp64.
+
+    Rounding points of that path (everything else is fp32 with errors ~2^-24):
+      * full-dim history: K_hat = bf16(c + bf16(s) bf16(x)) with x = D code,
+        so each element errs by at most u (2 |s x| + |k_hat|); V_hat alike;
+      * low-dim history: the reduced query D_K^T q (scaled) is rounded to bf16,
+        so a score errs by at most u s sum_r |q~_r| |code_r|; the value side
+        rounds P s_V, P and the restore operands O~ / l, P_C / l to bf16;
+      * every branch rounds P to bf16 for the value MMA; the output is bf16.
+    With score errors dz_t, the weights become w_t e^{dz_t} / A with
+    A = sum_s w_s e^{dz_s}, so O moves by (1/A) sum_t w_t (e^{dz_t} - 1)(v_t - O)
+    exactly, and 1/A <= exp(sum_s w_s |dz_s|) (Jensen); the LSE moves by
+    log A, at most log(1 + sum_t w_t (e^{|dz_t|} - 1)) in magnitude.  Returns
+    (bound on O [R, H, d], bound on LSE [H, R])."""
+    u = U_BF16
+    R, H, d = q.shape
+    T = len(ohk["ids"])
+    T_low = T - T_full
+
+    def decode(h, c, lo, hi):
+        sx = h["scales"][lo:hi, None] * (np.asarray(h["codes"][lo:hi], np.float64) @ c["D"].T)  # s D code
+        return sx, c["centers"][h["ids"][lo:hi]] + sx
+
+    sxk, kf = decode(ohk, ck, T_low, T)
+    sxv, vf = decode(ohv, cv, T_low, T)
+    _, kl = decode(ohk, ck, 0, T_low)
+    _, vl = decode(ohv, cv, 0, T_low)
+    ek = u * (2 * np.abs(sxk) + np.abs(kf))
+    ev = u * (2 * np.abs(sxv) + np.abs(vf))
+    ck_low, sk_low = np.abs(np.asarray(ohk["codes"][:T_low], np.float64)), ohk["scales"][:T_low]
+    cv_low, sv_low = np.abs(np.asarray(ohv["codes"][:T_low], np.float64)), ohv["scales"][:T_low]
+    bound = np.zeros((R, H, d))
+    lse_bound = np.zeros((H, R))
+    for h in range(H):
+        cols = slice(h * d, (h + 1) * d)
+        qh = q[:, h, :]
+        keys = np.concatenate([kl[:, cols], kf[:, cols], kc[:, h, :]])          # [T + Tc, d]
+        vals = np.concatenate([vl[:, cols], vf[:, cols], vc[:, h, :]])
+        z = tau * qh @ keys.T
+        z -= z.max(axis=1, keepdims=True)
+        wgt = np.exp(z)
+        wgt /= wgt.sum(axis=1, keepdims=True)                                    # [R, T + Tc]
+        O = wgt @ vals
+        qred = qh @ ck["D"][cols, :]                                             # [R, r]
+        dz = np.zeros_like(wgt)
+        dz[:, :T_low] = tau * u * (np.abs(qred) @ ck_low.T) * sk_low[None, :]
+        dz[:, T_low:T] = tau * (np.abs(qh) @ ek[:, cols].T)
+        lse_bound[h] = np.log1p((wgt * np.expm1(dz)).sum(axis=1))
+        a = wgt * np.expm1(dz) * np.exp((wgt * dz).sum(axis=1, keepdims=True))
+        b = np.empty((R, d))
+        for r0 in range(0, R, 16):                                               # softmax weights
+            rs = slice(r0, r0 + 16)
+            b[rs] = np.einsum("rt,rtk->rk", a[rs], np.abs(vals[None, :, :] - O[rs, None, :]))
+        b += wgt[:, T_low:T] @ ev[:, cols]                                       # V_hat rounding
+        b += u * (wgt @ np.abs(vals))                                            # P rounding
+        low_coef = (cv_low * sv_low[:, None]) @ np.abs(cv["D"][cols, :]).T       # [T_low, d]
+        b += 2 * u * (wgt[:, :T_low] @ low_coef)                                 # P s_V and O~ / l
+        b += u * (wgt[:, :T_low] @ np.abs(cv["centers"][ohv["ids"][:T_low], cols]))  # P_C / l
+        b += u * np.abs(O)                                                       # bf16 output
+        bound[:, h, :] = b
+    return bound, lse_bound
+
+
+def gpu_rounding_bound(w, prob, hk, hv, T_full, rows, tau):
+    """rounding_bound for rows of a GPU problem and its GPU-encoded history."""
+    return rounding_bound(orc.f64(prob["q"])[rows], oracle_codec(prob["codec_k"]), oracle_codec(prob["codec_v"]),
+                          oracle_hist(hk), oracle_hist(hv), orc.f64(prob["k_cur"]), orc.f64(prob["v_cur"]),
+                          T_full, tau)

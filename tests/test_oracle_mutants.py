@@ -81,7 +81,38 @@ def _softmax_no_tau(q, k, v, tau):
     return _orig_sm(q, k, v, 1.0 if tau != 1.0 else 0.5)
 
 
+_orig_encode = orc.encode
+
+
+def _encode_projects_from_first_center(x, centers, E, scale_dtype):
+    r = _orig_encode(x, centers, E, scale_dtype)
+    y = orc.project(x, centers, np.zeros_like(r["ids"]), E)
+    s = orc.scale_of(y, scale_dtype)
+    return dict(r, y=y, scales=s, codes=orc.quantise(y, s))
+
+
+def _encode_codes_from_unrounded_scale(x, centers, E, scale_dtype):
+    r = _orig_encode(x, centers, E, scale_dtype)
+    m = np.max(np.abs(r["y"]), axis=1) / 7
+    return dict(r, codes=orc.quantise(r["y"], m))
+
+
+def _encode_returns_unquantised(x, centers, E, scale_dtype):
+    r = _orig_encode(x, centers, E, scale_dtype)
+    return dict(r, codes=r["y"])
+
+
+def _encode_scale_from_residual(x, centers, E, scale_dtype):
+    r = _orig_encode(x, centers, E, scale_dtype)
+    s = orc.scale_of(x - centers[r["ids"]], scale_dtype)
+    return dict(r, scales=s, codes=orc.quantise(r["y"], s))
+
+
 MUTANTS = {
+    "encode_projects_from_first_center": ("encode", _encode_projects_from_first_center),
+    "encode_codes_from_unrounded_scale": ("encode", _encode_codes_from_unrounded_scale),
+    "encode_returns_unquantised": ("encode", _encode_returns_unquantised),
+    "encode_scale_from_residual": ("encode", _encode_scale_from_residual),
     "decode_no_center": ("decode", _decode_no_center),
     "decode_no_scale": ("decode", _decode_no_scale),
     "quantise_half_up": ("quantise", _quantise_floor),

@@ -81,6 +81,24 @@ def test_int4_hand_picked_cases():
     assert np.array_equal(orc.unpack_codes(packed), codes)
 
 
+def test_encode_worked_example():
+    """The whole encode (assign, project, scale, quantise, pack) on five tokens
+    worked by hand: an argmin tie, half-steps on both sides of zero, a zero
+    residual, and a token whose fp16-rounded scale moves a code."""
+    g = _load("encode_worked.json")
+    x, cen, E = (np.array(g[k], dtype=np.float64) for k in ("x", "centers", "E"))
+    r = orc.encode(x, cen, E, g["scale_dtype"])
+    assert r["ids"].tolist() == g["ids"]
+    assert np.array_equal(r["y"], np.array(g["y"], dtype=np.float64))
+    assert r["scales"].tolist() == g["scales"]
+    assert r["codes"].tolist() == g["codes"]
+    assert orc.pack_codes(r["codes"]).tolist() == g["packed"]
+    assert orc.argmin_ties(x, cen).tolist() == g["argmin_tie"]
+    s = r["scales"]
+    assert orc.rounding_ties(x, cen, r["ids"], E, r["y"], s).tolist() == g["rounding_tie"]
+    assert orc.scale_ties(r["y"], g["scale_dtype"]).tolist() == g["scale_tie"]
+
+
 def test_int4_clamp_and_zero_scale():
     y = np.array([[10.0, -10.0, 0.2]])
     assert list(orc.quantise(y, np.array([1.0]))[0]) == [7, -7, 0]
