@@ -8,6 +8,11 @@ or low-dim) plus the current chunk, LSE-merged.  Default workload: one layer,
 H=12, d=128 (J=1536), history 3 chunks = 14040 tokens, all full-dim, Tq=4680,
 64 centers, r=192, bf16 I/O, fp16 scales.
 
+The headline `value` is the metric the task names: the attention call's
+algorithmic TFLOP/s (full-dim workload); the Fast (mixed) and long-rollout
+attends are side measurements, and encode is reported in GB/s.  `ms_per_step`
+is the whole step (encode + attend), the `step` object its throughput.
+
     python bench.py [--gpus N] [--steps K] [--warmup W] [--impl ours|reference]
 
 Under torchrun (N > 1) every rank runs its own replica of the workload (no
@@ -30,6 +35,7 @@ ROOT = os.path.dirname(os.path.abspath(__file__))
 sys.path.insert(0, ROOT)
 
 PEAKS_FALLBACK = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0}
+METRIC = "compressed-history attention TFLOP/s (full vs Fast), % bf16 peak; encode GB/s"
 BAD_REASONS = ("hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown")
 
 
@@ -98,6 +104,7 @@ def args_():
     ap.add_argument("--no-fast", action="store_true", help="skip the mixed-dim (Fast) side measurement")
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--no-step30", action="store_true", help="skip the 30-layer step (side measurement)")
+    ap.add_argument("--no-long", action="store_true", help="skip the long-rollout attend (side measurement)")
     ap.add_argument("--path", type=int, default=0, help="kernel family: 0 auto, 1 CUDA-core, 2 tensor-core")
     return ap.parse_args()
 
@@ -361,7 +368,7 @@ def run_ours(a, rank, world, device):
     step_ms, enc_ms, att_ms = max_over_ranks([step_ms, enc_ms, att_ms], world, device)
 
     flops = ak["total"] + ef
-    value = whole_job_tflops(flops, step_ms, world)
+    value = whole_job_tflops(ak["total"], att_ms, world)
     # dominant kernel: the one with the largest share of the timed region
     dom = max(kt.items(), key=lambda kv: kv[1][0])
     dom_name, (dom_ms, dom_n) = dom
@@ -391,15 +398,16 @@ def run_ours(a, rank, world, device):
     hist_tf = (ak["full"] + ak["low"]) / (att_ms * 1e-3) / 1e12
     enc_gbs = eb / (enc_ms * 1e-3) / 1e9
 
-    e2e = run_e2e(s, w, a, device, flops, world)
-    fast = None if a.no_fast else run_fast(a, device, peaks)
-    step30 = None if a.no_step30 else run_step30(a, device, peaks)
-    cpu = None
+    e2e = run_e2e(s, w, a, device, ak["total"], world)
+    cpu, parity = None, None
     if rank == 0 and world == 1 and not a.no_cpu_baseline:
-        cpu = cpu_baseline(w, s, budget_s=12.0)
+        cpu, parity = cpu_baseline(w, s, budget_s=12.0)
+    fast = None if a.no_fast else run_side(a, device, peaks, "mixed")
+    long_ = None if a.no_long else run_side(a, device, peaks, "long")
+    step30 = None if a.no_step30 else run_step30(a, device, peaks)
 
     line = {
-        "metric": "compressed-history attention + encode step throughput (algorithmic TFLOP/s)",
+        "metric": METRIC,
         "value": round(value, 3), "unit": "TFLOP/s", "n_gpus": world, "steps": a.steps,
         "warmup": a.warmup, "ms_per_step": round(step_ms, 4), "higher_is_better": True,
         "scaling": "weak", "vs_baseline": None, "dtype": "bf16" if not w.fp32 else "f32",
@@ -412,13 +420,18 @@ def run_ours(a, rank, world, device):
                    "encode_tokens": s["n_enc"], "l2": "flushed between steps (256 MiB write outside the step events)",
                    "launch": "CUDA graph replay of the encode and attend calls",
                    "parallelism": f"replicas x{world}"},
+        "value_is": "the attention call (history + current chunk + LSE merge) of the step; "
+                    "ms_per_step is the whole step (encode + attend)",
+        "frac_bf16_peak": round(attend_tf / peak_tf, 4),
         "attend": {"ms": round(att_ms, 4), "tflops": round(attend_tf, 3),
                    "history_tflops": round(hist_tf, 3), "frac_bf16_peak": round(attend_tf / peak_tf, 4)},
+        "step": {"ms": round(step_ms, 4), "tflops": round(whole_job_tflops(flops, step_ms, world), 3),
+                 "what": "encode of one chunk (K and V) + attend + merge"},
         "encode": {"ms": round(enc_ms, 4), "gbs": round(enc_gbs, 2),
                    "frac_hbm": round(enc_gbs / peaks["hbm_gbs"], 4)},
         "kernels": kernels,
         "clocks": clocks, "e2e": e2e, "gpu_launches": launches, "roofline": roof,
-        "cpu_baseline": cpu, "fast": fast, "step30": step30,
+        "cpu_baseline": cpu, "parity": parity, "fast": fast, "long": long_, "step30": step30,
     }
     return line
 
@@ -511,17 +524,21 @@ def run_e2e(s, w, a, device, flops, world):
     torch.cuda.synchronize()
     ms_serial = max_over_ranks([f0.elapsed_time(f1) / a.steps], world, device)[0]
     return {"value": round(whole_job_tflops(flops, ms, world), 3), "unit": "TFLOP/s",
+            "work": "the attention call's algorithmic flops over the whole end-to-end step "
+                    "(uploads, encode, attend, readback)",
             "ms_per_step": round(ms, 4), "h2d_bytes_per_step": bi, "d2h_bytes_per_step": bo,
             "pipelined": "H2D of step i+1 and D2H of step i-1 overlap step i (double-buffered)",
             "serial_ms_per_step": round(ms_serial, 4),
             "serial_value": round(whole_job_tflops(flops, ms_serial, world), 3)}
 
 
-def run_fast(a, device, peaks):
-    """Side measurement of the mixed-dimensional (Fast) attend on the mixed
-    workload (same shapes, most recent chunk full-dim, 9360 tokens low-dim)."""
+def run_side(a, device, peaks, name):
+    """Side measurement of one more workload's attend call: `mixed` (the
+    mixed-dimensional Fast attend: same shapes as the headline workload, most
+    recent chunk full-dim, 9360 tokens low-dim) or `long` (the long rollout:
+    H=24, 93600 history tokens, the last two chunks full-dim, C=256, r=384)."""
     from synth.gen import WORKLOADS
-    w = WORKLOADS["mixed"]
+    w = WORKLOADS[name]
     s = setup(w, device)
     for _ in range(2):
         step_attend(s, w)
@@ -546,10 +563,13 @@ def run_fast(a, device, peaks):
             avg = ms_k / cnt
             per[name] = {"ms": round(avg, 4), "tflops": round(work / (avg * 1e-3) / 1e12, 2),
                          "frac_bf16_peak": round(work / (avg * 1e-3) / 1e12 / peaks["bf16_tflops"], 4)}
+    tfa = full_tokens(w, s)
     del s, g
     torch.cuda.empty_cache()
     return {"workload": w.describe(), "attend_ms": round(ms, 4), "tflops": round(tf, 3),
-            "frac_bf16_peak": round(tf / peaks["bf16_tflops"], 4), "iters": n, "kernels": per}
+            "frac_bf16_peak": round(tf / peaks["bf16_tflops"], 4), "iters": n, "kernels": per,
+            "T_full_attended": tfa, "step_gflop": round(ak["total"] / 1e9, 3),
+            "step_gflop_as_named": round(af["total"] / 1e9, 3)}
 
 
 def run_step30(a, device, peaks):
@@ -599,7 +619,9 @@ def run_step30(a, device, peaks):
     del g, layers, ws
     torch.cuda.empty_cache()
     return {"workload": w.describe(), "layers": w.layers, "ms": round(ms, 3), "ms_per_layer": round(ms / w.layers, 4),
-            "tflops": round(tf, 3), "frac_bf16_peak": round(tf / peaks["bf16_tflops"], 4), "iters": n,
+            "tflops": round(tf, 3), "frac_bf16_peak": round(tf / peaks["bf16_tflops"], 4),
+            "frac_bf16_sustained": round(tf / peaks.get("bf16_tflops_sustained", peaks["bf16_tflops"]), 4),
+            "peak_note": "a ~0.15 s graph loop: the sustained bf16 figure is the matching denominator", "iters": n,
             "launch": "one CUDA graph of the 30 layers' encode and attend calls"}
 
 
@@ -635,8 +657,9 @@ def oracle_hist(h):
 
 def oracle_sample(w, D, n_rows, n_enc, seed=0):
     """Runs the oracle on a bounded sample of one step: encode n_enc tokens of
-    K and V and attend n_rows query rows over the whole history plus the
-    current chunk.  Returns (seconds, algorithmic flops of the sample)."""
+    K and V, and attend n_rows query rows over the whole history plus the
+    current chunk.  Returns the timings and algorithmic work of both parts and
+    the oracle's results (for the parity block)."""
     import numpy as np
     from oracle import nanokv_oracle as orc
     from compressed_history_attention_b200.accounting import attend_flops, encode_flops
@@ -645,32 +668,82 @@ def oracle_sample(w, D, n_rows, n_enc, seed=0):
     rows = np.sort(rng.choice(w.Tq, min(n_rows, w.Tq), replace=False))
     n_enc = min(n_enc, D["xk"].shape[0])
     t0 = time.perf_counter()
-    orc.encode(D["xk"][:n_enc], D["ck"]["centers"], D["ck"]["E"], sd)
-    orc.encode(D["xv"][:n_enc], D["cv"]["centers"], D["cv"]["E"], sd)
-    orc.attend(D["q"][rows], D["ck"], D["cv"], D["hk"], D["hv"], w.T_full, D["kc"], D["vc"])
-    dt = time.perf_counter() - t0
-    fl = (2 * encode_flops(n_enc, w.J, w.r, w.C)
-          + attend_flops(len(rows), w.H, w.d, w.r, w.C, w.T_full, w.T_low, w.Tq)["total"])
-    return dt, fl, len(rows), n_enc
+    ek = orc.encode(D["xk"][:n_enc], D["ck"]["centers"], D["ck"]["E"], sd)
+    ev = orc.encode(D["xv"][:n_enc], D["cv"]["centers"], D["cv"]["E"], sd)
+    t1 = time.perf_counter()
+    O, L = orc.attend(D["q"][rows], D["ck"], D["cv"], D["hk"], D["hv"], w.T_full, D["kc"], D["vc"])
+    t2 = time.perf_counter()
+    return {"t_enc": t1 - t0, "t_att": t2 - t1, "enc_flops": 2 * encode_flops(n_enc, w.J, w.r, w.C),
+            "att_flops": attend_flops(len(rows), w.H, w.d, w.r, w.C, w.T_full, w.T_low, w.Tq)["total"],
+            "rows": rows, "n_enc": n_enc, "O": O, "L": L, "enc": (ek, ev)}
 
 
 def _calibrated(w, D, budget_s, rows0, enc0):
-    dt, _, _, _ = oracle_sample(w, D, rows0, enc0)
-    scale = max(1.0, min(64.0, budget_s / max(dt, 1e-3)))
+    r = oracle_sample(w, D, rows0, enc0)
+    scale = max(1.0, min(64.0, budget_s / max(r["t_enc"] + r["t_att"], 1e-3)))
     return int(rows0 * scale), int(enc0 * scale)
+
+
+def encode_parity(x, codec, ids, codes, scales, ref, sd):
+    """GPU encode outputs against the oracle's on the same tokens: ids, scales
+    and codes must agree except at ties (values within rounding error of a
+    decision boundary), which are counted."""
+    import numpy as np
+    from oracle import nanokv_oracle as orc
+    tie_a = orc.argmin_ties(x, codec["centers"])
+    same = ids == ref["ids"]
+    tie_s = orc.scale_ties(ref["y"], sd)
+    if sd == "f16":
+        scale_ok = (scales == ref["scales"]) | tie_s
+    else:
+        scale_ok = np.abs(scales - ref["scales"]) <= 1e-6 * np.abs(ref["scales"])
+    want = orc.codes_given_scale(ref["y"], scales)
+    tie_r = orc.rounding_ties(x, codec["centers"], ref["ids"], codec["E"], ref["y"], scales)
+    flips = (codes != want) & same[:, None]
+    return {"tokens": int(len(ids)), "argmin_ties": int(tie_a.sum()),
+            "ids_differ_outside_ties": int((~same & ~tie_a).sum()),
+            "scale_ties": int(tie_s.sum()) if sd == "f16" else 0,
+            "scales_differ_outside_ties": int((~scale_ok & same).sum()),
+            "rounding_ties": int(tie_r.sum()), "code_flips_at_ties": int((flips & tie_r).sum()),
+            "codes_differ_outside_ties": int((flips & ~tie_r).sum())}
 
 
 def cpu_baseline(w, s, budget_s=12.0):
     """The oracle as it stands, timed on this host's cores on a bounded sample
-    of the same workload (the GPU's inputs and compressed history)."""
+    of the same workload (the GPU's inputs and compressed history); the same
+    sample gives the parity of the GPU's results against the oracle."""
+    import numpy as np
+    from oracle import nanokv_oracle as orc
     p = s["prob"]
     D = oracle_data(w, p["codec_k"], p["codec_v"], s["xk"], s["xv"], oracle_hist(s["hk"]),
                     oracle_hist(s["hv"]), p["q"], p["k_cur"], p["v_cur"])
     n_rows, n_enc = _calibrated(w, D, budget_s, 16, 64)
-    dt, fl, n_rows, n_enc = oracle_sample(w, D, n_rows, n_enc, seed=1)
-    return {"value": round(fl / dt / 1e12, 6), "unit": "TFLOP/s", "cores": _threads_used(), "kind": "oracle",
-            "sample": f"encode {n_enc} K + {n_enc} V tokens and attend {n_rows} of {w.Tq} query rows "
-                      f"over the full history + current chunk; {dt:.1f} s fp64 numpy"}
+    r = oracle_sample(w, D, n_rows, n_enc, seed=1)
+    n_rows, n_enc, rows = len(r["rows"]), r["n_enc"], r["rows"]
+    cpu = {"value": round(r["att_flops"] / r["t_att"] / 1e12, 6), "unit": "TFLOP/s", "cores": _threads_used(),
+           "kind": "oracle",
+           "sample": f"attend {n_rows} of {w.Tq} query rows over the full history + current chunk "
+                     f"({r['t_att']:.1f} s fp64 numpy; value = its attention TFLOP/s); encode {n_enc} K + "
+                     f"{n_enc} V tokens ({r['t_enc']:.1f} s)",
+           "encode_gbs": round(2 * n_enc * w.J * (4 if w.fp32 else 2) / r["t_enc"] / 1e9, 6)}
+    # parity of the GPU's last step on the same rows and tokens
+    O = orc.f64(s["out"])[rows]
+    L = orc.f64(s["lse"])[:, rows]
+    err = np.abs(O - r["O"])
+    fin = np.isfinite(r["L"])
+    sd = "f32" if w.fp32 else "f16"
+    enc = {}
+    for name, x, c, h, ref in (("k", D["xk"], D["ck"], s["tail_k"], r["enc"][0]),
+                               ("v", D["xv"], D["cv"], s["tail_v"], r["enc"][1])):
+        hh = oracle_hist(h)
+        enc[name] = encode_parity(x[:n_enc], c, hh["ids"][:n_enc], hh["codes"][:n_enc], hh["scales"][:n_enc],
+                                  ref, sd)
+    parity = {"attend_rows": n_rows, "max_abs": float(err.max()),
+              "rel_l2": float(np.linalg.norm(O - r["O"]) / np.linalg.norm(r["O"])),
+              "lse_max_abs": float(np.abs(L[fin] - r["L"][fin]).max()),
+              "tolerance": "bf16 I/O: max-abs 2e-2 and rel-L2 5e-3" if not w.fp32 else "fp32: max-abs 1e-5",
+              "encode": enc}
+    return cpu, parity
 
 
 def run_reference(a, rank, world):
@@ -695,17 +768,19 @@ def run_reference(a, rank, world):
     n_rows, n_enc = _calibrated(w, D, budget, 8, 32)
     for _ in range(a.warmup):
         oracle_sample(w, D, n_rows, n_enc)
-    tot_t, tot_f = 0.0, 0
+    tot_t, tot_att, tot_f = 0.0, 0.0, 0
     for i in range(a.steps):
-        dt, fl, n_rows, n_enc = oracle_sample(w, D, n_rows, n_enc, seed=i)
-        tot_t += dt
-        tot_f += fl
-    v = tot_f / tot_t / 1e12
+        r = oracle_sample(w, D, n_rows, n_enc, seed=i)
+        n_rows, n_enc = len(r["rows"]), r["n_enc"]
+        tot_t += r["t_enc"] + r["t_att"]
+        tot_att += r["t_att"]
+        tot_f += r["att_flops"]
+    v = tot_f / tot_att / 1e12
     sample = (f"per step: encode {n_enc} K + {n_enc} V tokens and attend {n_rows} of {w.Tq} query rows "
-              "over the full history + current chunk (fp64 numpy oracle)")
+              "over the full history + current chunk (fp64 numpy oracle); value = the attend's TFLOP/s")
     return {
         "impl": "reference",
-        "metric": "compressed-history attention + encode step throughput (algorithmic TFLOP/s)",
+        "metric": METRIC,
         "value": round(v, 6), "unit": "TFLOP/s", "n_gpus": world, "steps": a.steps, "warmup": a.warmup,
         "ms_per_step": round(1e3 * tot_t / a.steps, 2), "higher_is_better": True, "scaling": "weak",
         "vs_baseline": None, "dtype": "f64", "data": "synthetic",

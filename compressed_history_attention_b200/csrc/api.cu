@@ -230,6 +230,12 @@ static int64_t effective_T_full(int path, bool tc_low_ok, bool tc_full_ok, int64
   return T_full;
 }
 
+// a low-dim tensor-core kernel exists for these codecs: the single-CTA one
+// (r <= 192, C <= 64) or the 2-CTA one for larger codecs
+static bool tc_low_any(const Codec &ck, const Codec &cv) {
+  return tc_low_supported(ck, cv) || tc_low_pair_supported(ck, cv);
+}
+
 // workspace carve-up (every region 256-byte aligned)
 struct WsLayout {
   // branch b (0 low-dim, 1 full-dim, 2 current chunk) has nparts[b]
@@ -302,7 +308,7 @@ int64_t nanokv_attend_full_tokens(const nanokv_codec *ck, const nanokv_codec *cv
   Codec a, b;
   if (T < 0 || T_full < 0 || T_full > T) return -1;
   if (check_codec(ck, "ck", false, &a) || check_codec(cv, "cv", false, &b)) return -1;
-  return effective_T_full(g_kernel_path.load(), tc_low_supported(a, b), tc_full_supported(a, b), T, T_full);
+  return effective_T_full(g_kernel_path.load(), tc_low_any(a, b), tc_full_supported(a, b), T, T_full);
 }
 
 int nanokv_selftest_wait(uint64_t limit_ns, void *stream) {
@@ -385,9 +391,9 @@ size_t nanokv_attend_workspace(int64_t Tq, const nanokv_codec *ck, const nanokv_
   if (Tq < 0 || T < 0 || T_full < 0 || T_full > T || T_cur < 0) return 0;
   if (check_codec(ck, "ck", false, &a) || check_codec(cv, "cv", false, &b)) return 0;
   const int path = g_kernel_path.load();
-  const bool tc_low = path != 1 && tc_low_supported(a, b);
+  const bool tc_low = path != 1 && tc_low_any(a, b);
   const bool tc_full = path != 1 && tc_full_supported(a, b);
-  T_full = effective_T_full(path, tc_low_supported(a, b), tc_full_supported(a, b), T, T_full);
+  T_full = effective_T_full(path, tc_low_any(a, b), tc_full_supported(a, b), T, T_full);
   const int splits = (tc_full && T_full > 0 && Tq > 0) ? tc_full_splits(Tq, a.H, a.d, T_full) : 1;
   return ws_layout(Tq, a, T - T_full, T_full, T_cur, tc_low, splits).total;
 }
@@ -427,7 +433,7 @@ int nanokv_attend(const void *q, int32_t io_dtype, int64_t Tq, const nanokv_code
 
   const int path = g_kernel_path.load();
   const bool tc_full_ok = tc_full_supported(ck, cv);
-  const bool tc_low_ok = tc_low_supported(ck, cv);
+  const bool tc_low_ok = tc_low_any(ck, cv);
   T_full = effective_T_full(path, tc_low_ok, tc_full_ok, T, T_full);
   const int64_t T_low = T - T_full;
   const bool tc_dense_ok = tc_dense_supported(ck.prec, ck.d);
@@ -479,7 +485,8 @@ int nanokv_attend(const void *q, int32_t io_dtype, int64_t Tq, const nanokv_code
     if (e != cudaSuccess) return cuda_status(e, "attend fork");
     if (use_tc_low) {
       e = timed(NANOKV_K_LOW, 1, bst, [&] {
-        return tc_attend_low(q, Tq, ck, cv, hk, hv, 0, T_low, softmax_scale, p, bst);
+        return tc_low_supported(ck, cv) ? tc_attend_low(q, Tq, ck, cv, hk, hv, 0, T_low, softmax_scale, p, bst)
+                                        : tc_attend_low_pair(q, Tq, ck, cv, hk, hv, 0, T_low, softmax_scale, p, bst);
       });
     } else {
       float *qred = (float *)(ws + w.off_qred), *qc = (float *)(ws + w.off_qc);

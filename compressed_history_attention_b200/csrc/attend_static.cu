@@ -4,6 +4,7 @@
 // array compiled into this library instead of a caller-provided workspace.
 #include "../../include/nanokv.h"
 
+#include <cuda.h>
 #include <cuda_runtime.h>
 
 #include <mutex>
@@ -23,21 +24,44 @@ __device__ __align__(256) unsigned char g_attend_scratch[kStaticScratchBytes];
 constexpr int kMaxDevices = 64;
 std::mutex g_mu;
 void *g_scratch_ptr[kMaxDevices] = {};
+CUcontext g_scratch_ctx[kMaxDevices] = {};
+
+// the current driver context, through the runtime's entry-point query (the
+// library takes no link-time dependency on the driver library)
+CUcontext current_context() {
+  using Fn = CUresult (*)(CUcontext *);
+  static Fn fn = [] {
+    void *p = nullptr;
+    cudaDriverEntryPointQueryResult q;
+    return (cudaGetDriverEntryPoint("cuCtxGetCurrent", &p, cudaEnableDefault, &q) == cudaSuccess &&
+            q == cudaDriverEntryPointSuccess)
+               ? (Fn)p
+               : (Fn) nullptr;
+  }();
+  CUcontext c = nullptr;
+  if (fn) fn(&c);
+  return c;
+}
 
 // Device address of the scratch array on the current device.  Host code can
-// only name the array's host-side stand-in, so the address is looked up once
-// per device (with that device current) and cached.
+// only name the array's host-side stand-in, so the address is looked up (with
+// that device current) and cached per device together with the context it
+// belongs to: after a device reset, or under another context of the same
+// device, the array lives at a new address and is looked up again.
 int scratch_for_current_device(void **out) {
   int dev = 0;
   if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= kMaxDevices)
     return nanokv::set_error(NANOKV_ERR_CUDA, "attend_static: no usable current device");
+  CUcontext ctx = current_context();  // NULL before the runtime has made the primary context current
   std::lock_guard<std::mutex> lk(g_mu);
-  if (!g_scratch_ptr[dev]) {
+  if (!g_scratch_ptr[dev] || !ctx || ctx != g_scratch_ctx[dev]) {
     void *p = nullptr;
     const cudaError_t e = cudaGetSymbolAddress(&p, g_attend_scratch);
     if (e != cudaSuccess || !p)
       return nanokv::set_error(NANOKV_ERR_CUDA, "attend_static: cudaGetSymbolAddress of the scratch array failed");
+    if (!ctx) ctx = current_context();  // the lookup made the primary context current
     g_scratch_ptr[dev] = p;
+    g_scratch_ctx[dev] = ctx;
   }
   *out = g_scratch_ptr[dev];
   return NANOKV_OK;

@@ -331,6 +331,55 @@ __device__ __forceinline__ void mma_commit_mc(uint64_t *bar, uint16_t cta_mask) 
       : "memory");
 }
 
+// ---------------------------------------------------------------------------
+// tcgen05 across a CTA pair (cta_group::2).  One thread of the even CTA of a
+// 2-CTA cluster issues each MMA for both; every operand descriptor names the
+// same shared-memory offset in both CTAs, each CTA holding its half of A
+// (rows) and of B (N), and each CTA's TMEM receives its rows of D.  For M =
+// 256 a CTA's 128 rows occupy all lanes, N columns; for M = 128 its 64 rows
+// occupy lanes [0, 64) for D columns [0, N/2) and lanes [64, 128) for
+// columns [N/2, N), both in N/2 TMEM columns.
+// ---------------------------------------------------------------------------
+// (warp-wide, the same warp index in both CTAs) allocate `ncols` TMEM columns
+// in both CTAs of the pair; the base is written to *slot in each CTA
+__device__ __forceinline__ void tmem_alloc2(uint32_t *slot, uint32_t ncols) {
+  asm volatile("tcgen05.alloc.cta_group::2.sync.aligned.shared::cta.b32 [%0], %1;" ::"r"(smem_u32(slot)),
+               "r"(ncols)
+               : "memory");
+}
+__device__ __forceinline__ void tmem_relinquish2() {
+  asm volatile("tcgen05.relinquish_alloc_permit.cta_group::2.sync.aligned;" ::: "memory");
+}
+__device__ __forceinline__ void tmem_dealloc2(uint32_t taddr, uint32_t ncols) {
+  asm volatile("tcgen05.dealloc.cta_group::2.sync.aligned.b32 %0, %1;" ::"r"(taddr), "r"(ncols)
+               : "memory");
+}
+__device__ __forceinline__ void mma2_ss(uint32_t d_tmem, uint64_t a_desc, uint64_t b_desc, uint32_t idesc,
+                                        uint32_t accumulate) {
+  asm volatile(
+      "{ .reg .pred p; setp.ne.b32 p, %4, 0; "
+      "tcgen05.mma.cta_group::2.kind::f16 [%0], %1, %2, %3, p; }" ::"r"(d_tmem),
+      "l"(a_desc), "l"(b_desc), "r"(idesc), "r"(accumulate)
+      : "memory");
+}
+__device__ __forceinline__ void mma2_ts(uint32_t d_tmem, uint32_t a_tmem, uint64_t b_desc, uint32_t idesc,
+                                        uint32_t accumulate) {
+  asm volatile(
+      "{ .reg .pred p; setp.ne.b32 p, %4, 0; "
+      "tcgen05.mma.cta_group::2.kind::f16 [%0], [%1], %2, %3, p; }" ::"r"(d_tmem),
+      "r"(a_tmem), "l"(b_desc), "r"(idesc), "r"(accumulate)
+      : "memory");
+}
+// arrive on the mbarrier at the same offset in every CTA of `cta_mask` once
+// all previously issued pair MMAs of this thread complete
+__device__ __forceinline__ void mma2_commit_mc(uint64_t *bar, uint16_t cta_mask) {
+  asm volatile(
+      "tcgen05.commit.cta_group::2.mbarrier::arrive::one.shared::cluster.multicast::cluster.b64 [%0], "
+      "%1;" ::"r"(smem_u32(bar)),
+      "h"(cta_mask)
+      : "memory");
+}
+
 // programmatic dependent launch: let the next kernel in the stream start on
 // SMs this grid leaves idle (used only where the next kernel does not read
 // this one's output)

@@ -8,6 +8,8 @@ namespace nanokv {
 bool tc_encode_supported(const Codec &c);
 bool tc_full_supported(const Codec &ck, const Codec &cv);
 bool tc_low_supported(const Codec &ck, const Codec &cv);
+// larger codecs (r in {128, 256, 384}, up to 256 centers): a 2-CTA kernel
+bool tc_low_pair_supported(const Codec &ck, const Codec &cv);
 bool tc_dense_supported(int prec, int d);
 
 // encodes nbranch (1 or 2) branches with equal C and r in one launch
@@ -27,6 +29,9 @@ cudaError_t tc_attend_full(const void *q, int64_t Tq, const Codec &ck, const Cod
 cudaError_t tc_attend_low(const void *q, int64_t Tq, const Codec &ck, const Codec &cv,
                           const Hist &hk, const Hist &hv, int64_t t0, int64_t T, float tau,
                           Part out, cudaStream_t st);
+cudaError_t tc_attend_low_pair(const void *q, int64_t Tq, const Codec &ck, const Codec &cv,
+                               const Hist &hk, const Hist &hv, int64_t t0, int64_t T, float tau,
+                               Part out, cudaStream_t st);
 cudaError_t tc_attend_dense(const void *q, int64_t Tq, int H, int d, const void *k, const void *v,
                             int64_t T, float tau, Part out, cudaStream_t st, bool pdl);
 

@@ -166,8 +166,9 @@ int nanokv_attend(const void *q, int32_t io_dtype, int64_t Tq,
  * the library keeps until the process exits; calls whose
  * nanokv_attend_workspace(...) exceeds it return NANOKV_ERR_INVALID with a
  * message.  No allocation or free happens in this call.  The first call on a
- * device looks up the array's device address (cudaGetSymbolAddress) and caches
- * it, so make that first call before any stream capture.  All calls share the
+ * device (and the first after a device reset, or under another CUDA context)
+ * looks up the array's device address (cudaGetSymbolAddress) and caches it
+ * with the context, so make that first call before any stream capture.  All calls share the
  * array: calls that may overlap on the GPU (other streams, other threads) race
  * on it and must be serialised by the caller.  Nothing in the array needs to be
  * zero on entry; it keeps the last call's partial results.

@@ -156,28 +156,30 @@ def test_attend_full_tokens_routing():
     bf = dict(d=128, param_dtype=_lib.BF16, scale_dtype=_lib.F16)
     small = _codec(H=12, r=192, C=64, **bf)
     large = _codec(H=24, r=384, C=256, **bf)
+    odd = _codec(H=24, r=320, C=256, **bf)
     g = lambda c, T, Tf: L.nanokv_attend_full_tokens(ctypes.byref(c), ctypes.byref(c), T, Tf)  # noqa: E731
-    assert g(small, 14040, 4680) == 4680       # low-dim tensor-core kernel covers r = 192, C = 64
-    assert g(large, 93600, 9360) == 93600      # r = 384, C = 256: low-dim tokens run full-dim
-    assert g(large, 93600, 93600) == 93600
+    assert g(small, 14040, 4680) == 4680       # single-CTA low-dim kernel: r = 192, C = 64
+    assert g(large, 93600, 9360) == 9360       # 2-CTA low-dim kernel: r = 384, C = 256
+    assert g(odd, 93600, 9360) == 93600        # r = 320: no low-dim kernel, low-dim tokens run full-dim
+    assert g(odd, 93600, 93600) == 93600
     assert g(_codec(), 256, 100) == 100        # fp32: CUDA-core kernels, split kept
     assert g(small, 100, 200) == -1            # T_full > T
     assert g(small, -1, 0) == -1
     prev = nk.nanokv_set_kernel_path(1)        # CUDA-core path forced: split kept
     try:
-        assert g(large, 93600, 9360) == 9360
+        assert g(odd, 93600, 9360) == 9360
     finally:
         nk.nanokv_set_kernel_path(prev)
 
 
 def test_workspace_follows_the_routing():
-    """A codec with no low-dim tensor-core kernel attends every history token
-    full-dim, so its workspace does not depend on the caller's split; with
-    the CUDA-core path forced, the split is kept and the low-dim buffers
-    appear."""
+    """A codec with no low-dim tensor-core kernel (r = 320) attends every
+    history token full-dim, so its workspace does not depend on the caller's
+    split; with the CUDA-core path forced, the split is kept and the low-dim
+    buffers appear."""
     L = nk.lib()
     bf = dict(d=128, param_dtype=_lib.BF16, scale_dtype=_lib.F16)
-    large = _codec(H=24, r=384, C=256, **bf)
+    large = _codec(H=24, r=320, C=256, **bf)
     small = _codec(H=12, r=192, C=64, **bf)
     ws = lambda c, T, Tf: L.nanokv_attend_workspace(4680, ctypes.byref(c), ctypes.byref(c), T, Tf, 4680)  # noqa: E731
     assert ws(large, 93600, 9360) == ws(large, 93600, 93600) > 0

@@ -48,18 +48,31 @@ def test_long_low_dim_main_term():
     assert af["low"] > main  # plus the query prep and the output restore
 
 
-@pytest.mark.parametrize("name", ["full", "mixed", "step30"])
-def test_work_as_run_equals_named_where_low_dim_kernel_exists(name):
+@pytest.mark.parametrize("name", ["full", "mixed", "long", "step30"])
+def test_work_as_run_equals_named(name):
+    """Every workload's codecs have a low-dim tensor-core kernel (the long
+    rollout's C = 256, r = 384 included), so the history runs split as named."""
     _, (af, ak, _, _) = _work(name)
     assert ak == af
 
 
-def test_long_work_as_run_is_full_dim():
-    """r = 384 > d = 128 and 256 centers: no low-dim tensor-core kernel, so
-    every history token is attended full-dim; that is less arithmetic than
-    the named low-dim split, and the throughput numerator counts it."""
-    w, (af, ak, _, _) = _work("long")
-    assert ak["low"] == 0
-    assert ak["full"] == 4 * w.Tq * w.T * w.J + 4 * w.T * w.J * w.r
-    assert ak["total"] / 1e12 == pytest.approx(6.093, rel=1e-3)
-    assert ak["total"] < af["total"]
+def test_encode_parity_counts_mismatches_outside_ties():
+    """The bench's parity block: identical outputs give zero mismatches; a
+    changed id and a changed code outside any tie are counted."""
+    import numpy as np
+    from oracle import nanokv_oracle as orc
+    rng = np.random.default_rng(0)
+    cen = rng.standard_normal((8, 32))
+    E = np.linalg.qr(rng.standard_normal((32, 8)))[0].T
+    x = cen[rng.integers(0, 8, 40)] + 0.3 * rng.standard_normal((40, 32))
+    ref = orc.encode(x, cen, E, "f16")
+    codec = {"centers": cen, "E": E}
+    same = bench.encode_parity(x, codec, ref["ids"].copy(), ref["codes"].copy(), ref["scales"].copy(), ref, "f16")
+    assert same["ids_differ_outside_ties"] == 0 and same["codes_differ_outside_ties"] == 0
+    assert same["scales_differ_outside_ties"] == 0 and same["tokens"] == 40
+    ids, codes = ref["ids"].copy(), ref["codes"].copy()
+    ids[3] = (ids[3] + 1) % 8
+    codes[5, 2] += 1 if codes[5, 2] < 7 else -1
+    bad = bench.encode_parity(x, codec, ids, codes, ref["scales"].copy(), ref, "f16")
+    assert bad["ids_differ_outside_ties"] == 1
+    assert bad["codes_differ_outside_ties"] == 1
