@@ -44,10 +44,11 @@ BAD_REASONS = ("hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown")
 # of the sources they were taken on: a kernel whose source has changed since
 # reports null traffic.
 NCU_TRAFFIC = {
-    ("attend_full", "full"): ("tc_full", "4deaa1093a4d50d4", 18819072 + 5870336),
+    ("attend_full", "full"): ("tc_full", "ad7a7c99a295bffa", 18877440 + 5851904),
+    ("attend_low", "long"): ("tc_low_pair", "cf31160a163436dd", 71376384 + 31356928),
     ("attend_low", "mixed"): ("tc_low", "4fcc55f69a077271", 17918464 + 15104),
     ("attend_dense", "full"): ("tc_dense", "6f930d6c7b63c100", 43229696 + 1877760),
-    ("encode", "full"): ("tc_encode", "c8fa4e3280375134", 30489600 + 19712),
+    ("encode", "full"): ("tc_encode", "4b9f263521ef0a34", 30489600 + 18688),
 }
 
 
