@@ -24,7 +24,7 @@ SYMBOLS = ("nanokv_encode", "nanokv_attend", "nanokv_attend_workspace", "nanokv_
            "nanokv_set_kernel_path", "nanokv_check", "nanokv_last_error", "nanokv_version",
            "nanokv_timing_enable", "nanokv_timing_read", "nanokv_codec_aux_bytes",
            "nanokv_codec_prepare", "nanokv_attend_static", "nanokv_selftest_wait",
-           "nanokv_attend_full_tokens")
+           "nanokv_attend_full_tokens", "nanokv_attend_routed", "nanokv_attend_routed_workspace")
 
 # kernel identities of the diagnostics (nanokv_kernel_id)
 KERNELS = {0: "encode", 1: "attend_full", 2: "attend_low", 3: "attend_dense", 4: "lse_merge"}
@@ -46,6 +46,13 @@ class _Codec(ctypes.Structure):
 
 class _Hist(ctypes.Structure):
     _fields_ = [("ids", ctypes.c_void_p), ("codes", ctypes.c_void_p), ("scales", ctypes.c_void_p)]
+
+
+class _Range(ctypes.Structure):
+    _fields_ = [("start", ctypes.c_int64), ("count", ctypes.c_int64)]
+
+
+MAX_RANGES = 64
 
 
 _lib = None
@@ -93,6 +100,11 @@ def lib() -> ctypes.CDLL:
     L.nanokv_selftest_wait.restype = ctypes.c_int
     L.nanokv_attend_full_tokens.argtypes = [P(_Codec), P(_Codec), i64, i64]
     L.nanokv_attend_full_tokens.restype = i64
+    L.nanokv_attend_routed.argtypes = [vp, i32, i64, P(_Codec), P(_Codec), P(_Hist), P(_Hist), i64,
+                                       P(_Range), i32, vp, vp, vp, i64, f32, vp, vp, vp, sz, vp]
+    L.nanokv_attend_routed.restype = ctypes.c_int
+    L.nanokv_attend_routed_workspace.argtypes = [i64, P(_Codec), P(_Codec), i64, P(_Range), i32, vp, i64]
+    L.nanokv_attend_routed_workspace.restype = sz
     _lib = L
     return L
 
@@ -248,6 +260,63 @@ def nanokv_attend(q: torch.Tensor, ck: Codec, cv: Codec, hk: Hist | None, hv: Hi
     st = lib().nanokv_attend(
         _ptr(q), _dt(q), Tq, ctypes.byref(sk), ctypes.byref(sv),
         ctypes.byref(shk) if shk else None, ctypes.byref(shv) if shv else None, T, T_full,
+        _ptr(k_cur), _ptr(v_cur), T_cur, ctypes.c_float(softmax_scale), _ptr(out), _ptr(lse),
+        _ptr(workspace), workspace.numel() * workspace.element_size(), _stream(dev))
+    _raise(st)
+    return out, lse
+
+
+def _ranges(full):
+    arr = (_Range * max(1, len(full)))(*[_Range(int(a), int(c)) for a, c in full])
+    return arr, len(full)
+
+
+def _heads(full_heads, H):
+    if full_heads is None:
+        return None, None
+    buf = (ctypes.c_uint8 * H)(*[1 if h else 0 for h in full_heads])
+    return buf, ctypes.cast(buf, ctypes.c_void_p)
+
+
+def nanokv_attend_routed_workspace(Tq: int, ck: Codec, cv: Codec, T: int, full, full_heads, T_cur: int) -> int:
+    sk, sv = ck.struct(), cv.struct()
+    arr, n = _ranges(full)
+    _keep, hp = _heads(full_heads, ck.H)
+    return int(lib().nanokv_attend_routed_workspace(Tq, ctypes.byref(sk), ctypes.byref(sv), T, arr, n, hp, T_cur))
+
+
+def nanokv_attend_routed(q: torch.Tensor, ck: Codec, cv: Codec, hk: Hist | None, hv: Hist | None, full,
+                         full_heads=None, k_cur: torch.Tensor | None = None, v_cur: torch.Tensor | None = None,
+                         softmax_scale: float | None = None, out: torch.Tensor | None = None,
+                         lse: torch.Tensor | bool | None = True, workspace: torch.Tensor | None = None):
+    """nanokv_attend under a routing policy: `full` is a list of (start,
+    count) history token ranges read full-dim (sorted, disjoint), the rest
+    low-dim; `full_heads` (H truth values, or None) marks heads that read all
+    their history full-dim.  Returns (out, lse) as nanokv_attend."""
+    Tq, H, d = q.shape
+    T = len(hk) if hk is not None else 0
+    T_cur = k_cur.shape[0] if k_cur is not None else 0
+    if softmax_scale is None:
+        softmax_scale = 1.0 / math.sqrt(d)
+    dev = q.device
+    if out is None:
+        out = torch.empty_like(q)
+    if lse is True:
+        lse = torch.empty(H, Tq, dtype=torch.float32, device=dev)
+    elif lse is False:
+        lse = None
+    # (0 for arguments the call itself then refuses with its own status)
+    need = nanokv_attend_routed_workspace(Tq, ck, cv, T, full, full_heads, T_cur)
+    if workspace is None or workspace.numel() * workspace.element_size() < need:
+        workspace = torch.empty(max(need, 16), dtype=torch.uint8, device=dev)
+    sk, sv = ck.struct(), cv.struct()
+    shk = hk.struct() if hk is not None and T else None
+    shv = hv.struct() if hv is not None and T else None
+    arr, n = _ranges(full)
+    _keep, hp = _heads(full_heads, H)
+    st = lib().nanokv_attend_routed(
+        _ptr(q), _dt(q), Tq, ctypes.byref(sk), ctypes.byref(sv),
+        ctypes.byref(shk) if shk else None, ctypes.byref(shv) if shv else None, T, arr, n, hp,
         _ptr(k_cur), _ptr(v_cur), T_cur, ctypes.c_float(softmax_scale), _ptr(out), _ptr(lse),
         _ptr(workspace), workspace.numel() * workspace.element_size(), _stream(dev))
     _raise(st)

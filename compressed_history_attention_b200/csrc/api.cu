@@ -271,6 +271,77 @@ static WsLayout ws_layout(int64_t Tq, const Codec &ck, int64_t T_low, int64_t T_
   return w;
 }
 
+// ---------------------------------------------------------------------------
+// routed attend: a full-dim routing policy given as token ranges and heads
+// ---------------------------------------------------------------------------
+struct RoutedPlan {
+  int64_t T_f = 0, T_l = 0;  // history tokens read full-dim / low-dim (ordinary heads)
+  GatherSegs full{}, low{};  // segments of the two sets
+  int nfh = 0;               // heads kept full-dim
+  uint32_t mask[8] = {};
+  // workspace: gathered histories [set][branch] (ids, codes, scales), head lists
+  size_t off_ids[2][2], off_codes[2][2], off_scales[2][2], off_heads, total;
+};
+
+static int routed_plan(const Codec &ck, const Codec &cv, int64_t T, const nanokv_range *full, int32_t n_full,
+                       const uint8_t *full_heads, size_t base, RoutedPlan *p) {
+  if (n_full < 0 || n_full > NANOKV_MAX_RANGES)
+    return fail(NANOKV_ERR_INVALID, "routed: n_full=%d out of range [0,%d]", n_full, NANOKV_MAX_RANGES);
+  if (n_full > 0 && !full) return fail(NANOKV_ERR_INVALID, "routed: NULL range array with n_full > 0");
+  RoutedPlan r;
+  int64_t prev_end = 0;
+  for (int i = 0; i < n_full; ++i) {
+    const int64_t s0 = full[i].start, c = full[i].count;
+    if (s0 < prev_end || c < 0 || s0 + c > T)
+      return fail(NANOKV_ERR_INVALID, "routed: range %d [%lld, +%lld) not sorted, disjoint and inside [0, %lld)", i,
+                  (long long)s0, (long long)c, (long long)T);
+    if (c > 0) {
+      if (s0 > prev_end) {  // the gap before this range is low-dim
+        r.low.src[r.low.n] = prev_end;
+        r.low.dst[r.low.n] = r.T_l;
+        r.low.cnt[r.low.n++] = s0 - prev_end;
+        r.T_l += s0 - prev_end;
+      }
+      r.full.src[r.full.n] = s0;
+      r.full.dst[r.full.n] = r.T_f;
+      r.full.cnt[r.full.n++] = c;
+      r.T_f += c;
+      prev_end = s0 + c;
+    }
+  }
+  if (T > prev_end) {
+    r.low.src[r.low.n] = prev_end;
+    r.low.dst[r.low.n] = r.T_l;
+    r.low.cnt[r.low.n++] = T - prev_end;
+    r.T_l += T - prev_end;
+  }
+  if (full_heads)
+    for (int h = 0; h < ck.H; ++h)
+      if (full_heads[h]) {
+        r.mask[h >> 5] |= 1u << (h & 31);
+        ++r.nfh;
+      }
+  // gathered histories, then the head lists
+  size_t off = base;
+  const int64_t n[2] = {r.T_f, r.T_l};
+  const Codec *c[2] = {&ck, &cv};
+  const size_t sb = ck.prec == PREC_F32 ? 4 : 2;
+  for (int set = 0; set < 2; ++set)
+    for (int br = 0; br < 2; ++br) {
+      r.off_ids[set][br] = off;
+      off += al256((size_t)n[set]);
+      r.off_codes[set][br] = off;
+      off += al256((size_t)n[set] * (c[br]->r / 2));
+      r.off_scales[set][br] = off;
+      off += al256((size_t)n[set] * sb);
+    }
+  r.off_heads = off;
+  off += al256((size_t)2 * ck.H * sizeof(int32_t));
+  r.total = off;
+  *p = r;
+  return NANOKV_OK;
+}
+
 }  // namespace nanokv
 
 using namespace nanokv;
@@ -537,6 +608,217 @@ int nanokv_attend(const void *q, int32_t io_dtype, int64_t Tq, const nanokv_code
   e = timed(NANOKV_K_MERGE, 1, st,
             [&] { return lse_merge_launch(pl, Tq, ck.H, ck.d, out, ck.prec, lse_out, st); });
   return cuda_status(e, "attend merge launch");
+}
+
+// How a routed call runs its two history sets.  `full_set`: the routed
+// tokens, all heads, full-dim.  `low_set` for the ordinary heads: the
+// low-dim kernel (tensor-core or CUDA-core), or the tensor-core full-dim
+// kernel where no low-dim one exists (as in nanokv_attend); for the heads
+// kept full-dim: the full-dim kernel.
+struct RoutedKernels {
+  bool tc_full, tc_low, tc_dense, low_via_full, low_simt;
+};
+
+static int routed_kernels(int path, const Codec &ck, const Codec &cv, const RoutedPlan &r, int64_t T_cur,
+                          RoutedKernels *k) {
+  const bool full_ok = tc_full_supported(ck, cv), low_ok = tc_low_any(ck, cv);
+  k->tc_full = path != 1 && full_ok;
+  k->tc_low = path != 1 && low_ok;
+  k->tc_dense = path != 1 && tc_dense_supported(ck.prec, ck.d);
+  k->low_via_full = !k->tc_low && k->tc_full;
+  k->low_simt = r.T_l > 0 && r.nfh < ck.H && !k->tc_low && !k->low_via_full;
+  if (path == 2 && ((r.T_f > 0 && !k->tc_full) || (r.T_l > 0 && !k->tc_low && !k->low_via_full) ||
+                    (T_cur > 0 && !k->tc_dense)))
+    return fail(NANOKV_ERR_UNSUPPORTED, "routed: no tensor-core kernel for this shape");
+  const bool split_heads = r.T_l > 0 && r.nfh > 0 && r.nfh < ck.H && !k->low_via_full;
+  if (split_heads && !(k->tc_full && k->tc_low))
+    return fail(NANOKV_ERR_UNSUPPORTED,
+                "routed: heads of both kinds in one call need the tensor-core kernels for this codec");
+  return NANOKV_OK;
+}
+
+size_t nanokv_attend_routed_workspace(int64_t Tq, const nanokv_codec *ck_, const nanokv_codec *cv_, int64_t T,
+                                      const nanokv_range *full, int32_t n_full, const uint8_t *full_heads,
+                                      int64_t T_cur) {
+  Codec ck, cv;
+  if (Tq < 0 || T < 0 || T_cur < 0) return 0;
+  if (check_codec(ck_, "ck", false, &ck) || check_codec(cv_, "cv", false, &cv)) return 0;
+  RoutedPlan r;
+  if (routed_plan(ck, cv, T, full, n_full, full_heads, 0, &r)) return 0;
+  RoutedKernels k;
+  if (routed_kernels(g_kernel_path.load(), ck, cv, r, T_cur, &k)) return 0;
+  const int splits = (k.tc_full && r.T_f > 0 && Tq > 0) ? tc_full_splits(Tq, ck.H, ck.d, r.T_f) : 1;
+  const WsLayout w = ws_layout(Tq, ck, r.T_l, r.T_f, T_cur, !k.low_simt, splits);
+  RoutedPlan r2;
+  routed_plan(ck, cv, T, full, n_full, full_heads, w.total, &r2);
+  return r2.total;
+}
+
+int nanokv_attend_routed(const void *q, int32_t io_dtype, int64_t Tq, const nanokv_codec *ck_,
+                         const nanokv_codec *cv_, const nanokv_hist *hk_, const nanokv_hist *hv_, int64_t T,
+                         const nanokv_range *full, int32_t n_full, const uint8_t *full_heads, const void *k_cur,
+                         const void *v_cur, int64_t T_cur, float softmax_scale, void *out, float *lse_out,
+                         void *workspace, size_t workspace_bytes, void *stream) {
+  ApiRange range("nanokv_attend_routed");
+  Codec ck, cv;
+  int s;
+  if ((s = check_codec(ck_, "routed ck", false, &ck))) return s;
+  if ((s = check_codec(cv_, "routed cv", false, &cv))) return s;
+  if (ck.H != cv.H || ck.d != cv.d || ck.prec != cv.prec)
+    return fail(NANOKV_ERR_INVALID, "routed: ck and cv must share H, d and dtypes");
+  if (io_prec(io_dtype) != ck.prec) return fail(NANOKV_ERR_UNSUPPORTED, "routed: io_dtype must equal param_dtype");
+  if (Tq < 0 || T < 0 || T_cur < 0)
+    return fail(NANOKV_ERR_INVALID, "routed: bad sizes Tq=%lld T=%lld T_cur=%lld", (long long)Tq, (long long)T,
+                (long long)T_cur);
+  if (!(softmax_scale == softmax_scale) || softmax_scale <= 0.f || softmax_scale > 1e4f)
+    return fail(NANOKV_ERR_INVALID, "routed: softmax_scale must be finite and positive");
+  RoutedPlan r;
+  if ((s = routed_plan(ck, cv, T, full, n_full, full_heads, 0, &r))) return s;
+  if (Tq == 0) return NANOKV_OK;
+  if (!q || !out) return fail(NANOKV_ERR_INVALID, "routed: NULL q or out");
+  if (!aligned16(q) || !aligned16(out) || (lse_out && !aligned16(lse_out)))
+    return fail(NANOKV_ERR_INVALID, "routed: q/out/lse_out must be 16-byte aligned");
+  if (T > 0 && (!hk_ || !hv_ || !hk_->ids || !hk_->codes || !hk_->scales || !hv_->ids || !hv_->codes || !hv_->scales))
+    return fail(NANOKV_ERR_INVALID, "routed: NULL history pointer with T > 0");
+  if (T_cur > 0 && (!k_cur || !v_cur || !aligned16(k_cur) || !aligned16(v_cur)))
+    return fail(NANOKV_ERR_INVALID, "routed: k_cur/v_cur NULL or misaligned with T_cur > 0");
+  const int path = g_kernel_path.load();
+  RoutedKernels k;
+  if ((s = routed_kernels(path, ck, cv, r, T_cur, &k))) return s;
+  const int splits = (k.tc_full && r.T_f > 0) ? tc_full_splits(Tq, ck.H, ck.d, r.T_f) : 1;
+  const WsLayout w = ws_layout(Tq, ck, r.T_l, r.T_f, T_cur, !k.low_simt, splits);
+  routed_plan(ck, cv, T, full, n_full, full_heads, w.total, &r);
+  if (r.total > 0 && (!workspace || workspace_bytes < r.total))
+    return fail(NANOKV_ERR_INVALID, "routed: workspace needs %zu bytes, got %zu", r.total, workspace_bytes);
+  if (workspace && !aligned16(workspace)) return fail(NANOKV_ERR_INVALID, "routed: workspace must be 16-byte aligned");
+
+  cudaStream_t st = (cudaStream_t)stream;
+  char *ws = (char *)workspace;
+  cudaError_t e = cudaSuccess;
+  // 1. gather the two sets (and the head lists) into the workspace
+  Hist hs[2][2];  // [set][branch]
+  const int sb = ck.prec == PREC_F32 ? 4 : 2;
+  if (T > 0) {
+    GatherArgs g{};
+    const nanokv_hist *src[2] = {hk_, hv_};
+    const Codec *c[2] = {&ck, &cv};
+    for (int br = 0; br < 2; ++br) {
+      g.ids[br] = src[br]->ids;
+      g.codes[br] = src[br]->codes;
+      g.scales[br] = (const uint8_t *)src[br]->scales;
+      g.row_bytes[br] = c[br]->r / 2;
+      for (int set = 0; set < 2; ++set) {
+        g.d_ids[set][br] = (uint8_t *)(ws + r.off_ids[set][br]);
+        g.d_codes[set][br] = (uint8_t *)(ws + r.off_codes[set][br]);
+        g.d_scales[set][br] = (uint8_t *)(ws + r.off_scales[set][br]);
+        hs[set][br] = Hist{g.d_ids[set][br], g.d_codes[set][br], g.d_scales[set][br]};
+      }
+    }
+    g.n_out[0] = r.T_f;
+    g.n_out[1] = r.T_l;
+    g.scale_bytes = sb;
+    for (int i = 0; i < 8; ++i) g.head_mask[i] = r.mask[i];
+    g.H = ck.H;
+    g.head_lists = (int32_t *)(ws + r.off_heads);
+    if ((e = gather_launch(r.full, r.low, g, st)) != cudaSuccess) return cuda_status(e, "routed gather launch");
+  }
+  const int32_t *heads_full = (const int32_t *)(ws + r.off_heads), *heads_low = heads_full + ck.H;
+  const int nlh = ck.H - r.nfh;
+
+  // 2. branches: routed tokens full-dim (all heads); the other tokens low-dim
+  // for the ordinary heads and full-dim for the heads kept full; the current
+  // chunk.  Independent: on the helper streams, as in nanokv_attend.
+  PartList pl{};
+  const bool on[3] = {r.T_l > 0, r.T_f > 0, T_cur > 0};
+  const int nbranch = (int)on[0] + (int)on[1] + (int)on[2];
+  std::unique_lock<std::mutex> lk(g_bs_mu, std::defer_lock);
+  BranchStreams *bs = nullptr;
+  if (nbranch > 1 && !g_timing.load()) {
+    lk.lock();
+    if ((e = branch_streams(&bs)) != cudaSuccess) return cuda_status(e, "routed helper streams");
+    if ((e = cudaEventRecord(bs->fork, st)) != cudaSuccess) return cuda_status(e, "routed fork");
+  }
+  auto bstream = [&](int b) -> cudaStream_t {
+    if (!bs) return st;
+    e = cudaStreamWaitEvent(bs->s[b], bs->fork, 0);
+    return bs->s[b];
+  };
+  auto join = [&](int b) -> cudaError_t {
+    if (!bs) return cudaSuccess;
+    cudaError_t e2 = cudaEventRecord(bs->join[b], bs->s[b]);
+    return e2 == cudaSuccess ? cudaStreamWaitEvent(st, bs->join[b], 0) : e2;
+  };
+  if (on[0]) {
+    Part p{(float *)(ws + w.off_O[0]), (float *)(ws + w.off_L[0])};
+    cudaStream_t bst = bstream(0);
+    if (e != cudaSuccess) return cuda_status(e, "routed fork");
+    const Hist &lk_ = hs[1][0], &lv_ = hs[1][1];
+    if (r.nfh == ck.H || k.low_via_full) {
+      // every head reads these tokens full-dim
+      e = timed(NANOKV_K_FULL, 1, bst, [&] {
+        return k.tc_full ? tc_attend_full(q, Tq, ck, cv, lk_, lv_, 0, r.T_l, softmax_scale, p, 1, 0, 0, bst, false)
+                         : simt_attend_full(q, Tq, ck, cv, lk_, lv_, 0, r.T_l, softmax_scale, p, bst);
+      });
+    } else {
+      const HeadSel lows = r.nfh ? HeadSel{heads_low, nlh} : HeadSel{nullptr, 0};
+      if (r.nfh)  // the heads kept full-dim, into the same partial (disjoint heads)
+        e = timed(NANOKV_K_FULL, 1, bst, [&] {
+          return tc_attend_full(q, Tq, ck, cv, lk_, lv_, 0, r.T_l, softmax_scale, p, 1, 0, 0, bst, false,
+                                HeadSel{heads_full, r.nfh});
+        });
+      if (e == cudaSuccess && k.tc_low) {
+        e = timed(NANOKV_K_LOW, 1, bst, [&] {
+          return tc_low_supported(ck, cv)
+                     ? tc_attend_low(q, Tq, ck, cv, lk_, lv_, 0, r.T_l, softmax_scale, p, bst, lows)
+                     : tc_attend_low_pair(q, Tq, ck, cv, lk_, lv_, 0, r.T_l, softmax_scale, p, bst, lows);
+        });
+      } else if (e == cudaSuccess) {
+        float *qred = (float *)(ws + w.off_qred), *qc = (float *)(ws + w.off_qc);
+        e = timed(NANOKV_K_LOW, 2, bst, [&] {
+          cudaError_t e2 = simt_low_prep(q, Tq, ck, qred, qc, bst);
+          if (e2 == cudaSuccess) e2 = simt_attend_low(qred, qc, Tq, ck, cv, lk_, lv_, 0, r.T_l, softmax_scale, p, bst);
+          return e2;
+        });
+      }
+    }
+    if (e == cudaSuccess) e = join(0);
+    if (e != cudaSuccess) return cuda_status(e, "routed low-set launch");
+    pl.O[pl.n] = p.O;
+    pl.LSE[pl.n++] = p.LSE;
+  }
+  if (on[1]) {
+    Part p{(float *)(ws + w.off_O[1]), (float *)(ws + w.off_L[1])};
+    cudaStream_t bst = bstream(1);
+    if (e != cudaSuccess) return cuda_status(e, "routed fork");
+    e = timed(NANOKV_K_FULL, 1, bst, [&] {
+      return k.tc_full ? tc_attend_full(q, Tq, ck, cv, hs[0][0], hs[0][1], 0, r.T_f, softmax_scale, p, splits,
+                                        w.osz / sizeof(float), w.lsz / sizeof(float), bst, false)
+                       : simt_attend_full(q, Tq, ck, cv, hs[0][0], hs[0][1], 0, r.T_f, softmax_scale, p, bst);
+    });
+    if (e == cudaSuccess) e = join(1);
+    if (e != cudaSuccess) return cuda_status(e, "routed full-set launch");
+    for (int z = 0; z < w.nparts[1]; ++z) {
+      pl.O[pl.n] = (const float *)(ws + w.off_O[1] + z * w.osz);
+      pl.LSE[pl.n++] = (const float *)(ws + w.off_L[1] + z * w.lsz);
+    }
+  }
+  if (on[2]) {
+    Part p{(float *)(ws + w.off_O[2]), (float *)(ws + w.off_L[2])};
+    cudaStream_t bst = bstream(2);
+    if (e != cudaSuccess) return cuda_status(e, "routed fork");
+    e = timed(NANOKV_K_DENSE, 1, bst, [&] {
+      return k.tc_dense ? tc_attend_dense(q, Tq, ck.H, ck.d, k_cur, v_cur, T_cur, softmax_scale, p, bst, false)
+                        : simt_attend_dense(ck.prec, q, Tq, ck.H, ck.d, k_cur, v_cur, T_cur, softmax_scale, p, bst);
+    });
+    if (e == cudaSuccess) e = join(2);
+    if (e != cudaSuccess) return cuda_status(e, "routed current-chunk launch");
+    pl.O[pl.n] = p.O;
+    pl.LSE[pl.n++] = p.LSE;
+  }
+  if (lk.owns_lock()) lk.unlock();
+  e = timed(NANOKV_K_MERGE, 1, st,
+            [&] { return lse_merge_launch(pl, Tq, ck.H, ck.d, out, ck.prec, lse_out, st); });
+  return cuda_status(e, "routed merge launch");
 }
 
 int nanokv_lse_merge(int32_t n, const float *const *o_parts, const float *const *lse_parts,

@@ -56,6 +56,13 @@ struct Hist {
 
 enum Prec { PREC_F32 = 0, PREC_BF16 = 1 };
 
+// The heads one history-kernel launch covers: all H (map == nullptr), or the
+// n heads listed in the device array map (grid y indexes the list).
+struct HeadSel {
+  const int32_t *map;
+  int n;
+};
+
 // fp32 partial output of one attention branch: O [Tq, H, d], LSE [H, Tq]
 struct Part {
   float *O, *LSE;
@@ -67,6 +74,27 @@ struct PartList {
   const float *LSE[kMaxParts];
   int n;
 };
+
+// Gather of routed history tokens into contiguous compressed histories.
+// A set is a list of segments: output tokens [dst, dst + cnt) are source
+// tokens [src, src + cnt).  Up to 64 routed ranges give up to 65 segments of
+// the complement.
+constexpr int kMaxSegs = 65;
+struct GatherSegs {
+  int64_t src[kMaxSegs], dst[kMaxSegs], cnt[kMaxSegs];
+  int n;
+};
+struct GatherArgs {
+  const uint8_t *ids[2], *codes[2], *scales[2];            // source history, [K / V]
+  uint8_t *d_ids[2][2], *d_codes[2][2], *d_scales[2][2];   // destinations, [set][K / V]
+  int64_t n_out[2];                                       // tokens per set (full-dim, low-dim)
+  int row_bytes[2];                                       // packed code bytes per token, [K / V]
+  int scale_bytes;                                        // 2 (fp16) or 4 (fp32)
+  uint32_t head_mask[8];                                  // heads kept full-dim (bit h)
+  int H;
+  int32_t *head_lists;                                    // [2][H]: those heads, then the others
+};
+cudaError_t gather_launch(const GatherSegs &full, const GatherSegs &low, const GatherArgs &a, cudaStream_t st);
 
 // Raises a kernel's dynamic shared-memory limit to `bytes` on the current
 // device the first time a launch needs it (the attribute call is not repeated

@@ -25,13 +25,13 @@ int tc_full_splits(int64_t Tq, int H, int d, int64_t T);
 cudaError_t tc_attend_full(const void *q, int64_t Tq, const Codec &ck, const Codec &cv,
                            const Hist &hk, const Hist &hv, int64_t t0, int64_t T, float tau,
                            Part out, int nsplit, size_t ostride, size_t lstride, cudaStream_t st,
-                           bool pdl);
+                           bool pdl, HeadSel hs = HeadSel{nullptr, 0});
 cudaError_t tc_attend_low(const void *q, int64_t Tq, const Codec &ck, const Codec &cv,
                           const Hist &hk, const Hist &hv, int64_t t0, int64_t T, float tau,
-                          Part out, cudaStream_t st);
+                          Part out, cudaStream_t st, HeadSel hs = HeadSel{nullptr, 0});
 cudaError_t tc_attend_low_pair(const void *q, int64_t Tq, const Codec &ck, const Codec &cv,
                                const Hist &hk, const Hist &hv, int64_t t0, int64_t T, float tau,
-                               Part out, cudaStream_t st);
+                               Part out, cudaStream_t st, HeadSel hs = HeadSel{nullptr, 0});
 cudaError_t tc_attend_dense(const void *q, int64_t Tq, int H, int d, const void *k, const void *v,
                             int64_t T, float tau, Part out, cudaStream_t st, bool pdl);
 

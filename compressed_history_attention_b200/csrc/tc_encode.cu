@@ -597,28 +597,64 @@ __global__ void __launch_bounds__(384, 1)
   }
 }
 
-// EC[j][k] = E[k] . c_j and |c_j|^2 in fp32: one warp per output
+// EC[j][k] = E[k] . c_j and |c_j|^2 in fp32, a small GEMM of the codec's
+// centers against its encoder.  A block stages 8 center rows and 16 encoder
+// rows (in 384-wide chunks of J, converted to fp32) in shared memory and
+// computes their 128 products, two threads per product (one per half of the
+// chunk, combined by a shuffle); the blocks of the first encoder tile also
+// form the squared norms of their centers.  Each center and encoder row is
+// read from global memory once per block that uses it.
+constexpr int kPrepC = 8, kPrepR = 16, kPrepJ = 384, kPrepLD = kPrepJ + 4;
+
 template <typename TP>
-__global__ void codec_prepare_kernel(const TP *__restrict__ cen, const TP *__restrict__ E, int C, int r,
-                                     int J, float *__restrict__ aux) {
-  const int lane = threadIdx.x & 31;
-  const int64_t wid = ((int64_t)blockIdx.x * blockDim.x + threadIdx.x) >> 5;
-  const int64_t n = (int64_t)C * r + C;
-  if (wid >= n) return;
-  float acc = 0.f;
-  if (wid < (int64_t)C * r) {
-    const int j = (int)(wid / r), k = (int)(wid % r);
-    const TP *cr = cen + (size_t)j * J, *er = E + (size_t)k * J;
-    for (int i = lane; i < J; i += 32) acc = fmaf(to_f(er[i]), to_f(cr[i]), acc);
-  } else {
-    const TP *cr = cen + (size_t)(wid - (int64_t)C * r) * J;
-    for (int i = lane; i < J; i += 32) {
-      const float v = to_f(cr[i]);
-      acc = fmaf(v, v, acc);
+__global__ void __launch_bounds__(256) codec_prepare_kernel(const TP *__restrict__ cen, const TP *__restrict__ E,
+                                                            int C, int r, int J, float *__restrict__ aux) {
+  __shared__ __align__(16) float cs[kPrepC][kPrepLD];
+  __shared__ __align__(16) float es[kPrepR][kPrepLD];
+  const int j0 = blockIdx.x * kPrepC, k0 = blockIdx.y * kPrepR;
+  const int t = threadIdx.x, o = t & 127, half = t >> 7;
+  const int jj = o / kPrepR, kk = o % kPrepR;
+  const int warp = t >> 5, lane = t & 31;
+  float acc = 0.f, nrm = 0.f;
+  for (int c0 = 0; c0 < J; c0 += kPrepJ) {
+    const int n = J - c0 < kPrepJ ? J - c0 : kPrepJ;
+    for (int idx = t; idx < (kPrepC + kPrepR) * kPrepJ; idx += 256) {
+      const int row = idx / kPrepJ, i = idx % kPrepJ;
+      float v = 0.f;
+      if (i < n) {
+        if (row < kPrepC) {
+          if (j0 + row < C) v = to_f(cen[(size_t)(j0 + row) * J + c0 + i]);
+        } else if (k0 + row - kPrepC < r) {
+          v = to_f(E[(size_t)(k0 + row - kPrepC) * J + c0 + i]);
+        }
+      }
+      if (row < kPrepC) cs[row][i] = v;
+      else es[row - kPrepC][i] = v;
     }
+    __syncthreads();
+    const float *a = cs[jj] + half * (kPrepJ / 2), *b = es[kk] + half * (kPrepJ / 2);
+#pragma unroll 4
+    for (int i = 0; i < kPrepJ / 2; i += 4) {
+      const float4 x = *reinterpret_cast<const float4 *>(a + i), y = *reinterpret_cast<const float4 *>(b + i);
+      acc = fmaf(x.x, y.x, acc);
+      acc = fmaf(x.y, y.y, acc);
+      acc = fmaf(x.z, y.z, acc);
+      acc = fmaf(x.w, y.w, acc);
+    }
+    if (blockIdx.y == 0)  // warp w: center j0 + w
+      for (int i = lane; i < kPrepJ; i += 32) nrm = fmaf(cs[warp][i], cs[warp][i], nrm);
+    __syncthreads();
   }
-  acc = warp_sum(acc);
-  if (lane == 0) aux[wid] = acc;
+  // the two halves of each product are threads t and t + 128: combine
+  // through shared memory (reusing the staging buffer)
+  float *part = &cs[0][0];
+  if (half) part[o] = acc;
+  __syncthreads();
+  if (!half && j0 + jj < C && k0 + kk < r) aux[(size_t)(j0 + jj) * r + k0 + kk] = acc + part[o];
+  if (blockIdx.y == 0) {
+    nrm = warp_sum(nrm);
+    if (lane == 0 && j0 + warp < C) aux[(size_t)C * r + j0 + warp] = nrm;
+  }
 }
 
 }  // namespace
@@ -628,14 +664,12 @@ size_t codec_aux_bytes(const Codec &c) {
 }
 
 cudaError_t codec_prepare(const Codec &c, void *aux, cudaStream_t st) {
-  const int64_t n = (int64_t)c.C * c.r + c.C;
-  const int threads = 256;
-  const int64_t blocks = (n * 32 + threads - 1) / threads;
+  const dim3 grid((unsigned)((c.C + kPrepC - 1) / kPrepC), (unsigned)((c.r + kPrepR - 1) / kPrepR));
   if (c.prec == PREC_F32)
-    codec_prepare_kernel<float><<<(unsigned)blocks, threads, 0, st>>>(
-        (const float *)c.centers, (const float *)c.E, c.C, c.r, c.H * c.d, (float *)aux);
+    codec_prepare_kernel<float><<<grid, 256, 0, st>>>((const float *)c.centers, (const float *)c.E, c.C, c.r,
+                                                      c.H * c.d, (float *)aux);
   else
-    codec_prepare_kernel<__nv_bfloat16><<<(unsigned)blocks, threads, 0, st>>>(
+    codec_prepare_kernel<__nv_bfloat16><<<grid, 256, 0, st>>>(
         (const __nv_bfloat16 *)c.centers, (const __nv_bfloat16 *)c.E, c.C, c.r, c.H * c.d, (float *)aux);
   return cudaGetLastError();
 }

@@ -67,6 +67,7 @@ struct FullArgs {
   float zscale;
   float *O, *L;
   unsigned *err;
+  const int32_t *head_map;      // heads of grid y (nullptr: y is the head)
 };
 
 struct FullBars {
@@ -105,7 +106,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(384, 1)
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const uint32_t rank = cluster_ctarank();  // 0: decodes K, 1: decodes V
   const uint32_t peer = rank ^ 1u;
-  const int h = blockIdx.y;
+  const int h = A.head_map ? A.head_map[blockIdx.y] : (int)blockIdx.y;
   const int64_t q0 = (int64_t)blockIdx.x * BM;
   // this CTA's share of the history: split blockIdx.z, tokens [t0, t0 + T)
   const int64_t tb = (int64_t)blockIdx.z * A.Tsplit;
@@ -581,7 +582,7 @@ int tc_full_splits(int64_t Tq, int H, int d, int64_t T) {
 cudaError_t tc_attend_full(const void *q, int64_t Tq, const Codec &ck, const Codec &cv,
                            const Hist &hk, const Hist &hv, int64_t t0, int64_t T, float tau,
                            Part out, int nsplit, size_t ostride, size_t lstride, cudaStream_t st,
-                           bool pdl) {
+                           bool pdl, HeadSel hs) {
   if (Tq == 0 || T == 0) return cudaSuccess;
   const int64_t ntiles = (T + BN - 1) / BN;
   if (nsplit < 1 || nsplit > ntiles) return cudaErrorInvalidValue;
@@ -613,6 +614,7 @@ cudaError_t tc_attend_full(const void *q, int64_t Tq, const Codec &ck, const Cod
   a.O = out.O;
   a.L = out.LSE;
   a.err = error_word_ptr();
+  a.head_map = hs.map;
   const int Cmax = ck.C > cv.C ? ck.C : cv.C;
   const bool large = full_large(ck.r, Cmax);
   const size_t smem = tc_full_smem(ck.r, Cmax);
@@ -620,7 +622,7 @@ cudaError_t tc_attend_full(const void *q, int64_t Tq, const Codec &ck, const Cod
   const unsigned qt = (unsigned)((Tq + BM - 1) / BM);
   // every split must get at least one key tile (the caller merges nsplit partials)
   if ((T + a.Tsplit - 1) / a.Tsplit != nsplit) return cudaErrorInvalidValue;
-  dim3 grid((qt + 1) & ~1u, (unsigned)ck.H, (unsigned)nsplit);
+  dim3 grid((qt + 1) & ~1u, (unsigned)(hs.map ? hs.n : ck.H), (unsigned)nsplit);
   return large ? launch_k(tc_full_kernel<true>, grid, dim3(384), smem, st, pdl, mq, a)
                : launch_k(tc_full_kernel<false>, grid, dim3(384), smem, st, pdl, mq, a);
 }

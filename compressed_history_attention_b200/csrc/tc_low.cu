@@ -53,6 +53,7 @@ struct LowArgs {
   float zscale;
   float *O, *L;
   unsigned *err;
+  const int32_t *head_map;  // heads of grid y (nullptr: y is the head)
 };
 
 
@@ -95,7 +96,7 @@ __global__ void __launch_bounds__(384, 1)
   __shared__ LowBars B;
 
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-  const int h = blockIdx.y;
+  const int h = A.head_map ? A.head_map[blockIdx.y] : (int)blockIdx.y;
   const int64_t q0 = (int64_t)blockIdx.x * BM;
   const int ntiles = (int)((A.T + BN - 1) / BN);
   volatile int *abort = &B.abort;
@@ -537,7 +538,8 @@ static size_t low_smem(int r, int C) {
 }
 
 cudaError_t tc_attend_low(const void *q, int64_t Tq, const Codec &ck, const Codec &cv, const Hist &hk,
-                          const Hist &hv, int64_t t0, int64_t T, float tau, Part out, cudaStream_t st) {
+                          const Hist &hv, int64_t t0, int64_t T, float tau, Part out, cudaStream_t st,
+                          HeadSel hs) {
   if (Tq == 0 || T == 0) return cudaSuccess;
   const int J = ck.H * DH;
   CUtensorMap mq, mdk, mck, mdv, mcv;
@@ -567,9 +569,10 @@ cudaError_t tc_attend_low(const void *q, int64_t Tq, const Codec &ck, const Code
   a.O = out.O;
   a.L = out.LSE;
   a.err = error_word_ptr();
+  a.head_map = hs.map;
   const size_t smem = low_smem(ck.r, ck.C);
   ensure_smem((const void *)tc_low_kernel, (int)smem);
-  dim3 grid((unsigned)((Tq + BM - 1) / BM), (unsigned)ck.H);
+  dim3 grid((unsigned)((Tq + BM - 1) / BM), (unsigned)(hs.map ? hs.n : ck.H));
   tc_low_kernel<<<grid, 384, smem, st>>>(mq, mdk, mck, mdv, mcv, a);
   return cudaGetLastError();
 }

@@ -57,6 +57,7 @@ struct PairArgs {
   float zscale;
   float *O, *L;
   unsigned *err;
+  const int32_t *head_map;  // heads of grid y (nullptr: y is the head)
 };
 
 // barriers and small arrays, at the end of the dynamic shared memory
@@ -103,7 +104,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(384, 1)
 
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const uint32_t rank = cluster_ctarank();
-  const int h = blockIdx.y;
+  const int h = A.head_map ? A.head_map[blockIdx.y] : (int)blockIdx.y;
   const int64_t q0 = (int64_t)(blockIdx.x >> 1) * 128 + 64 * rank;  // this CTA's first query row
   const int ntiles = (int)((A.T + BN - 1) / BN);
   const int J = A.H * DH;
@@ -508,7 +509,8 @@ bool tc_low_pair_supported(const Codec &ck, const Codec &cv) {
 }
 
 cudaError_t tc_attend_low_pair(const void *q, int64_t Tq, const Codec &ck, const Codec &cv, const Hist &hk,
-                               const Hist &hv, int64_t t0, int64_t T, float tau, Part out, cudaStream_t st) {
+                               const Hist &hv, int64_t t0, int64_t T, float tau, Part out, cudaStream_t st,
+                               HeadSel hs) {
   if (Tq == 0 || T == 0) return cudaSuccess;
   const int J = ck.H * DH;
   CUtensorMap mq, mdk, mdv;
@@ -535,9 +537,10 @@ cudaError_t tc_attend_low_pair(const void *q, int64_t Tq, const Codec &ck, const
   a.O = out.O;
   a.L = out.LSE;
   a.err = error_word_ptr();
+  a.head_map = hs.map;
   const size_t smem = tc_low_pair_smem(ck.r);
   ensure_smem((const void *)tc_low_pair_kernel, (int)smem);
-  dim3 grid(2 * (unsigned)((Tq + 127) / 128), (unsigned)ck.H);
+  dim3 grid(2 * (unsigned)((Tq + 127) / 128), (unsigned)(hs.map ? hs.n : ck.H));
   tc_low_pair_kernel<<<grid, 384, smem, st>>>(mq, mdk, mdv, a);
   return cudaGetLastError();
 }

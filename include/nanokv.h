@@ -180,6 +180,47 @@ int nanokv_attend_static(const void *q, int32_t io_dtype, int64_t Tq,
                          const void *k_cur, const void *v_cur, int64_t T_cur,
                          float softmax_scale, void *out, float *lse_out, void *stream);
 
+/*
+ * nanokv_attend_routed -- nanokv_attend under a general full-dim routing
+ * policy instead of "the most recent T_full tokens" (NanoKV-Fast, Table 7:
+ * full-dimensional routing by recent frames, periodic anchor frames, sink
+ * frames, per-layer full fallback, and head-layer pairs kept at full
+ * dimension; Fig. 4(d): a fixed policy routes history to full- or
+ * low-dimensional attention, the branches are LSE-merged).
+ *   full, n_full  HOST array of n_full (0 <= n_full <= NANOKV_MAX_RANGES)
+ *                 history token ranges [start, start + count), sorted by start,
+ *                 disjoint, inside [0, T): these tokens use full-dim
+ *                 decode-attention, every other history token low-dim.  A
+ *                 per-layer full fallback is the single range [0, T).
+ *   full_heads    HOST array of H bytes or NULL: a head with a non-zero entry
+ *                 attends ALL its history tokens full-dim (a sensitive head kept
+ *                 at full dimension).  Heads of both kinds in one call need the
+ *                 tensor-core kernels (NANOKV_ERR_UNSUPPORTED on the CUDA-core
+ *                 path).
+ * Everything else (arguments, layouts, the current chunk, outputs, errors) is
+ * as for nanokv_attend.  The routed tokens of each branch are first gathered
+ * into contiguous compressed histories in the workspace (attention does not
+ * depend on the order of its keys), so the result is the attention over the
+ * same key set as nanokv_attend, up to rounding.
+ */
+#define NANOKV_MAX_RANGES 64
+typedef struct {
+  int64_t start, count;
+} nanokv_range;
+
+int nanokv_attend_routed(const void *q, int32_t io_dtype, int64_t Tq,
+                         const nanokv_codec *ck, const nanokv_codec *cv,
+                         const nanokv_hist *hk, const nanokv_hist *hv, int64_t T,
+                         const nanokv_range *full, int32_t n_full, const uint8_t *full_heads,
+                         const void *k_cur, const void *v_cur, int64_t T_cur,
+                         float softmax_scale, void *out, float *lse_out,
+                         void *workspace, size_t workspace_bytes, void *stream);
+
+/* Workspace bytes nanokv_attend_routed needs (0 for invalid arguments). */
+size_t nanokv_attend_routed_workspace(int64_t Tq, const nanokv_codec *ck, const nanokv_codec *cv,
+                                      int64_t T, const nanokv_range *full, int32_t n_full,
+                                      const uint8_t *full_heads, int64_t T_cur);
+
 /* Workspace bytes nanokv_attend needs for these sizes (0 is possible). */
 size_t nanokv_attend_workspace(int64_t Tq, const nanokv_codec *ck, const nanokv_codec *cv,
                                int64_t T, int64_t T_full, int64_t T_cur);

@@ -237,6 +237,36 @@ def attend(q, ck, cv, hk, hv, T_full: int, k_cur=None, v_cur=None, tau=None):
     return lse_merge(parts)
 
 
+def take_history(h: dict, idx) -> dict:
+    return {"ids": h["ids"][idx], "codes": h["codes"][idx], "scales": h["scales"][idx]}
+
+
+def attend_routed(q, ck, cv, hk, hv, full_mask, full_heads=None, k_cur=None, v_cur=None, tau=None):
+    """Compressed-history attention under a general full-dim routing policy
+    (NanoKV-Fast Table 7: recent, anchor and sink frames read at full
+    dimension, per-layer full fallback, sensitive heads kept at full
+    dimension; Fig. 4(d): LSE merging of the branches).  History tokens with
+    full_mask[t] go through full-dim decode-attention and the others through
+    the low-dim branch; a head with full_heads[h] reads every history token
+    full-dim.  The current chunk is the third branch, as in attend()."""
+    Tq, H, d = q.shape
+    if tau is None:
+        tau = 1.0 / np.sqrt(d)
+    full_mask = np.asarray(full_mask, dtype=bool)
+    f_idx, l_idx = np.nonzero(full_mask)[0], np.nonzero(~full_mask)[0]
+    cur = [softmax_attention(q, k_cur, v_cur, tau)] if k_cur is not None and len(k_cur) else []
+    routed = lse_merge([attend_full(q, ck, cv, take_history(hk, f_idx), take_history(hv, f_idx), tau),
+                        attend_low(q, ck, cv, take_history(hk, l_idx), take_history(hv, l_idx), tau)] + cur)
+    if full_heads is None or not np.any(full_heads):
+        return routed
+    all_idx = np.arange(len(full_mask))
+    kept = lse_merge([attend_full(q, ck, cv, take_history(hk, all_idx), take_history(hv, all_idx), tau)] + cur)
+    sel = np.asarray(full_heads, dtype=bool)
+    O = np.where(sel[None, :, None], kept[0], routed[0])
+    lse = np.where(sel[:, None], kept[1], routed[1])
+    return O, lse
+
+
 # ----------------------------------------------------------------------------
 # Tie accounting: an integer decided by floating point (argmin, rounding, the
 # fp16 scale) may legitimately differ between two correct implementations only

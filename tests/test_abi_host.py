@@ -189,3 +189,29 @@ def test_workspace_follows_the_routing():
         assert ws(large, 93600, 9360) != ws(large, 93600, 93600)
     finally:
         nk.nanokv_set_kernel_path(prev)
+
+
+def test_routed_rejects_bad_ranges():
+    """Routing ranges must be sorted, disjoint, inside [0, T), at most
+    NANOKV_MAX_RANGES; bad ones are refused before anything is launched."""
+    L = nk.lib()
+    c = _codec()
+    p = ctypes.c_void_p(1 << 20)
+    h = _lib._Hist(1 << 20, 1 << 20, 1 << 20)
+
+    def call(ranges, T=100, n=None):
+        arr = (_lib._Range * max(1, len(ranges)))(*[_lib._Range(a, b) for a, b in ranges])
+        return L.nanokv_attend_routed(p, _lib.F32, 4, ctypes.byref(c), ctypes.byref(c), ctypes.byref(h),
+                                      ctypes.byref(h), T, arr, len(ranges) if n is None else n, None, None, None,
+                                      0, ctypes.c_float(0.25), p, None, p, 1 << 20, None)
+
+    assert call([(10, 5), (12, 5)]) == _lib.ERR_INVALID   # overlap
+    assert call([(50, 5), (10, 5)]) == _lib.ERR_INVALID   # not sorted
+    assert call([(90, 20)]) == _lib.ERR_INVALID           # past T
+    assert call([(5, -1)]) == _lib.ERR_INVALID            # negative count
+    assert call([(0, 1)], n=_lib.MAX_RANGES + 1) == _lib.ERR_INVALID
+    ws = lambda ranges: L.nanokv_attend_routed_workspace(  # noqa: E731
+        4, ctypes.byref(c), ctypes.byref(c), 100,
+        (_lib._Range * max(1, len(ranges)))(*[_lib._Range(a, b) for a, b in ranges]), len(ranges), None, 0)
+    assert ws([(10, 5), (12, 5)]) == 0
+    assert ws([(10, 5), (40, 5)]) > 0

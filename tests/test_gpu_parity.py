@@ -171,6 +171,25 @@ def test_attend_peaked_softmax(path):
         assert np.all(lerr <= lse_bound + 1e-4), f"max LSE err/bound {np.max(lerr / (lse_bound + 1e-4)):.3f}"
 
 
+@pytest.mark.parametrize("H,C,r", [(12, 64, 192), (24, 256, 384), (2, 8, 8)])
+def test_codec_prepare_tables(H, C, r):
+    """The derived encode tables E c_j and |c_j|^2 against fp64: bf16 (or
+    fp32) products summed in fp32, so within J * 2^-24 of the sum of |terms|."""
+    g = torch.Generator(device="cpu").manual_seed(7)
+    J = H * (16 if C == 8 else 128)
+    dt = torch.float32 if C == 8 else torch.bfloat16
+    cen = torch.randn(C, J, generator=g).to(dt).cuda()
+    E = (torch.randn(r, J, generator=g) / math.sqrt(J)).to(dt).cuda()
+    c = nk.Codec(H, J // H, cen, torch.zeros(J, r, dtype=dt, device="cuda"), E).prepare()
+    torch.cuda.synchronize()
+    aux = c.aux.view(torch.float32)[: C * r + C].double().cpu().numpy()
+    cd, ed = P.orc.f64(cen), P.orc.f64(E)
+    ec, mag = cd @ ed.T, np.abs(cd) @ np.abs(ed).T
+    assert np.all(np.abs(aux[: C * r].reshape(C, r) - ec) <= J * 2.0 ** -24 * mag + 1e-30)
+    nrm = (cd * cd).sum(axis=1)
+    assert np.all(np.abs(aux[C * r:] - nrm) <= J * 2.0 ** -24 * nrm)
+
+
 def test_lse_merge_parity():
     from oracle import nanokv_oracle as orc
     g = torch.Generator(device="cuda").manual_seed(5)

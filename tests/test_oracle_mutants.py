@@ -108,7 +108,28 @@ def _encode_scale_from_residual(x, centers, E, scale_dtype):
     return dict(r, scales=s, codes=orc.quantise(r["y"], s))
 
 
+_orig_routed = orc.attend_routed
+
+
+def _routed_drops_low_tokens(q, ck, cv, hk, hv, full_mask, full_heads=None, k_cur=None, v_cur=None, tau=None):
+    m = np.asarray(full_mask, dtype=bool)
+    keep = np.nonzero(m)[0]
+    return _orig_routed(q, ck, cv, orc.take_history(hk, keep), orc.take_history(hv, keep), m[keep],
+                        full_heads, k_cur, v_cur, tau)
+
+
+def _routed_kept_heads_skip_current(q, ck, cv, hk, hv, full_mask, full_heads=None, k_cur=None, v_cur=None, tau=None):
+    O, L = _orig_routed(q, ck, cv, hk, hv, full_mask, full_heads, k_cur, v_cur, tau)
+    if full_heads is None:
+        return O, L
+    O2, L2 = _orig_routed(q, ck, cv, hk, hv, np.ones_like(np.asarray(full_mask, bool)), None, None, None, tau)
+    sel = np.asarray(full_heads, dtype=bool)
+    return np.where(sel[None, :, None], O2, O), np.where(sel[:, None], L2, L)
+
+
 MUTANTS = {
+    "routed_drops_low_tokens": ("attend_routed", _routed_drops_low_tokens),
+    "routed_kept_heads_skip_current": ("attend_routed", _routed_kept_heads_skip_current),
     "encode_projects_from_first_center": ("encode", _encode_projects_from_first_center),
     "encode_codes_from_unrounded_scale": ("encode", _encode_codes_from_unrounded_scale),
     "encode_returns_unquantised": ("encode", _encode_returns_unquantised),

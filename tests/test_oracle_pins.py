@@ -335,3 +335,61 @@ def test_table6_head_layer_counts():
     g = _load("head_dims.json")
     for row in g["rows"]:
         assert sum(row["counts"]) == row["layers"] * row["heads"], row
+
+
+# --------------------------------------------------------------------------
+# routed attention (Table 7 policies) and the policy builder
+# --------------------------------------------------------------------------
+
+def _decoded_softmax(q, ck, cv, hk, hv, kc, vc, tau):
+    """One textbook softmax over every decoded history key plus the current chunk."""
+    Tq, H, d = q.shape
+    kh = orc.decode(hk["ids"], hk["codes"], hk["scales"], ck["centers"], ck["D"]).reshape(-1, H, d)
+    vh = orc.decode(hv["ids"], hv["codes"], hv["scales"], cv["centers"], cv["D"]).reshape(-1, H, d)
+    return orc.softmax_attention(q, np.concatenate([kh, kc]), np.concatenate([vh, vc]), tau)
+
+
+def test_routed_attention_equals_one_softmax():
+    """Any token routing and any set of heads kept full-dim gives the attention
+    over the concatenation of all keys (the low-dim branch only reorders the
+    contraction; LSE merging recombines the branches)."""
+    for seed in (0, 1, 2):
+        rng = np.random.default_rng(seed)
+        H, d, r, C, T, Tq, Tc = 3, 8, 6, 5, 40, 7, 6
+        ck, cv, hk, hv = _rand_codec(rng, H, d, r, C, T)
+        q = rng.standard_normal((Tq, H, d))
+        kc, vc = rng.standard_normal((Tc, H, d)), rng.standard_normal((Tc, H, d))
+        mask = rng.random(T) < 0.4
+        heads = np.array([False, True, False]) if seed else None
+        O, L = orc.attend_routed(q, ck, cv, hk, hv, mask, heads, kc, vc, tau=0.7)
+        Or, Lr = _decoded_softmax(q, ck, cv, hk, hv, kc, vc, 0.7)
+        assert np.allclose(O, Or, rtol=0, atol=1e-12) and np.allclose(L, Lr, rtol=0, atol=1e-12)
+
+
+def test_routed_attention_recent_range_is_attend():
+    """The fixed policy of the configs (the most recent T_full tokens) as a
+    routing mask gives attend() with that T_full."""
+    rng = np.random.default_rng(5)
+    H, d, r, C, T, Tq = 2, 8, 6, 4, 30, 5
+    ck, cv, hk, hv = _rand_codec(rng, H, d, r, C, T)
+    q = rng.standard_normal((Tq, H, d))
+    mask = np.zeros(T, dtype=bool)
+    mask[T - 12:] = True
+    O, L = orc.attend_routed(q, ck, cv, hk, hv, mask, tau=0.5)
+    Or, Lr = orc.attend(q, ck, cv, hk, hv, 12, tau=0.5)
+    assert np.allclose(O, Or, rtol=0, atol=1e-13) and np.allclose(L, Lr, rtol=0, atol=1e-13)
+
+
+def test_frame_policy_ranges():
+    """Hand-worked policies: 10 frames of 100 tokens, 4 recent, 1 sink, an
+    anchor every 4 older frames -> frames {0, 4, 6, 7, 8, 9}; a partial last
+    frame is clipped; the per-layer fallback reads everything full-dim."""
+    from compressed_history_attention_b200.routing import frame_policy, full_mask
+    assert frame_policy(1000, 100, recent=4, sinks=1, anchor_every=4) == [(0, 100), (400, 100), (600, 400)]
+    assert frame_policy(950, 100, recent=4, sinks=1, anchor_every=4) == [(0, 100), (400, 100), (600, 350)]
+    assert frame_policy(1000, 100, recent=2) == [(800, 200)]
+    assert frame_policy(1000, 100, sinks=3, recent=2) == [(0, 300), (800, 200)]
+    assert frame_policy(1000, 100, full_layer=True) == [(0, 1000)]
+    assert frame_policy(0, 100, recent=2) == []
+    m = full_mask([(0, 100), (400, 100), (600, 350)], 950)
+    assert m.sum() == 550 and m[0] and not m[100] and m[949]
