@@ -21,7 +21,11 @@ plain readings below (each also listed in the design notes):
   * head h owns joint columns [h*d, (h+1)*d) of K/V and rows of D;
   * the current chunk is a third, uncompressed attention branch merged by LSE;
   * routing: the most recent T_full history tokens are full-dim, the older
-    T - T_full tokens low-dim.
+    T - T_full tokens low-dim;
+  * reduced attention dimension (Table 6): head h attends in R^{d_h} through
+    orthonormal maps U_h (queries, keys) and W_h (values, output restore);
+    the analytical maps are the leading left singular vectors of the head's
+    decoder rows (see the section on reduced dimensions below).
 
 Every stored value (bf16 / fp16 / fp32) converts exactly to fp64, and all
 arithmetic here is fp64 numpy.  Parity of every function is pinned by the
@@ -241,22 +245,33 @@ def take_history(h: dict, idx) -> dict:
     return {"ids": h["ids"][idx], "codes": h["codes"][idx], "scales": h["scales"][idx]}
 
 
-def attend_routed(q, ck, cv, hk, hv, full_mask, full_heads=None, k_cur=None, v_cur=None, tau=None):
+def attend_routed(q, ck, cv, hk, hv, full_mask, full_heads=None, k_cur=None, v_cur=None, tau=None,
+                  lowdim=None):
     """Compressed-history attention under a general full-dim routing policy
     (NanoKV-Fast Table 7: recent, anchor and sink frames read at full
     dimension, per-layer full fallback, sensitive heads kept at full
     dimension; Fig. 4(d): LSE merging of the branches).  History tokens with
     full_mask[t] go through full-dim decode-attention and the others through
     the low-dim branch; a head with full_heads[h] reads every history token
-    full-dim.  The current chunk is the third branch, as in attend()."""
+    full-dim.  With lowdim (maps as in attend_reduced, d_h[h] = 0 for heads
+    not reduced), the low-dim tokens of a reduced head go through attention
+    at its reduced dimension (Table 6) instead.  The current chunk is the
+    third branch, as in attend()."""
     Tq, H, d = q.shape
     if tau is None:
         tau = 1.0 / np.sqrt(d)
     full_mask = np.asarray(full_mask, dtype=bool)
     f_idx, l_idx = np.nonzero(full_mask)[0], np.nonzero(~full_mask)[0]
     cur = [softmax_attention(q, k_cur, v_cur, tau)] if k_cur is not None and len(k_cur) else []
-    routed = lse_merge([attend_full(q, ck, cv, take_history(hk, f_idx), take_history(hv, f_idx), tau),
-                        attend_low(q, ck, cv, take_history(hk, l_idx), take_history(hv, l_idx), tau)] + cur)
+    hk_f, hv_f = take_history(hk, f_idx), take_history(hv, f_idx)
+    hk_l, hv_l = take_history(hk, l_idx), take_history(hv, l_idx)
+    full_part = attend_full(q, ck, cv, hk_f, hv_f, tau)
+    routed = lse_merge([full_part, attend_low(q, ck, cv, hk_l, hv_l, tau)] + cur)
+    if lowdim is not None and np.any(np.asarray(lowdim["d_h"]) > 0):
+        red = np.asarray(lowdim["d_h"]) > 0
+        dims = {"U": lowdim["U"], "W": lowdim["W"], "d_h": np.where(red, lowdim["d_h"], d)}
+        reduced = lse_merge([full_part, attend_reduced(q, ck, cv, hk_l, hv_l, dims, tau)] + cur)
+        routed = (np.where(red[None, :, None], reduced[0], routed[0]), np.where(red[:, None], reduced[1], routed[1]))
     if full_heads is None or not np.any(full_heads):
         return routed
     all_idx = np.arange(len(full_mask))
@@ -264,6 +279,68 @@ def attend_routed(q, ck, cv, hk, hv, full_mask, full_heads=None, k_cur=None, v_c
     sel = np.asarray(full_heads, dtype=bool)
     O = np.where(sel[None, :, None], kept[0], routed[0])
     lse = np.where(sel[:, None], kept[1], routed[1])
+    return O, lse
+
+
+# ----------------------------------------------------------------------------
+# Reduced attention dimension per head (NanoKV-Fast: Table 6, head-layer
+# pairs deployed at d_h in {32, 64, 96, 128}; Fig. 4(d), the low-dimensional
+# branch reduces the queries and restores the output dimension; Table 8,
+# low-dimensional maps with an analytical initialization).
+#
+# Readings (the pages print no formulas for the maps):
+#   * head h has a key/query map U_h and a value map W_h, each [d, d_h] with
+#     orthonormal columns; the attention of that head runs in R^{d_h}:
+#         q~ = U_h^T q,  k~_t = U_h^T K_hat_t,  v~_t = W_h^T V_hat_t,
+#         o~ = softmax(tau q~ k~^T) v~,        O_h = W_h o~;
+#     tau stays the model's softmax scale;
+#   * the stored coefficients are reused: k~_t = U_h^T c_K[a_t] +
+#     s_t (U_h^T D_K,h) code_t, i.e. the decoder and centers are mapped once
+#     and the coefficients decode straight into d_h dimensions;
+#   * the analytical initialization takes U_h (W_h) as the leading d_h left
+#     singular vectors of the head's decoder rows D_K,h (D_V,h), [d, r];
+#   * maps are stored padded as [H, d, d]: head h uses columns [0, d_h).
+# ----------------------------------------------------------------------------
+
+def lowdim_maps(D: np.ndarray, H: int, d: int) -> np.ndarray:
+    """Analytical low-dimensional maps [H, d, d]: head h's left singular
+    vectors of its decoder rows D[h*d:(h+1)*d, :], by decreasing singular
+    value (a complete orthonormal basis of R^d, so any leading d_h columns
+    form the rank-d_h truncation's column space)."""
+    out = np.zeros((H, d, d))
+    for h in range(H):
+        u, _, _ = np.linalg.svd(D[h * d:(h + 1) * d, :], full_matrices=True)
+        out[h] = u
+    return out
+
+
+def attend_reduced(q, ck: dict, cv: dict, hk: dict, hv: dict, maps: dict, tau: float):
+    """History attention of every head at its reduced dimension.  maps:
+    {"U": [H, d, d], "W": [H, d, d], "d_h": [H]} with 0 < d_h[h] <= d."""
+    Tq, H, d = q.shape
+    T = len(hk["ids"])
+    O = np.zeros((Tq, H, d))
+    lse = np.full((H, Tq), -np.inf)
+    if T == 0:
+        return O, lse
+    codes_k = np.asarray(hk["codes"], np.float64)
+    codes_v = np.asarray(hv["codes"], np.float64)
+    for h in range(H):
+        n = int(maps["d_h"][h])
+        U = np.asarray(maps["U"][h], np.float64)[:, :n]          # [d, d_h]
+        W = np.asarray(maps["W"][h], np.float64)[:, :n]
+        cols = slice(h * d, (h + 1) * d)
+        q_red = q[:, h, :] @ U                                    # reduce the queries
+        Dk, Dv = U.T @ ck["D"][cols, :], W.T @ cv["D"][cols, :]   # decoders into d_h
+        ck_red, cv_red = ck["centers"][:, cols] @ U, cv["centers"][:, cols] @ W
+        k_red = ck_red[hk["ids"]] + hk["scales"][:, None] * (codes_k @ Dk.T)
+        v_red = cv_red[hv["ids"]] + hv["scales"][:, None] * (codes_v @ Dv.T)
+        z = tau * (q_red @ k_red.T)
+        m = z.max(axis=1, keepdims=True)
+        p = np.exp(z - m)
+        l = p.sum(axis=1, keepdims=True)
+        O[:, h, :] = ((p @ v_red) / l) @ W.T                      # restore to d
+        lse[h] = (m + np.log(l))[:, 0]
     return O, lse
 
 

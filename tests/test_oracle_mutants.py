@@ -111,15 +111,17 @@ def _encode_scale_from_residual(x, centers, E, scale_dtype):
 _orig_routed = orc.attend_routed
 
 
-def _routed_drops_low_tokens(q, ck, cv, hk, hv, full_mask, full_heads=None, k_cur=None, v_cur=None, tau=None):
+def _routed_drops_low_tokens(q, ck, cv, hk, hv, full_mask, full_heads=None, k_cur=None, v_cur=None, tau=None,
+                             lowdim=None):
     m = np.asarray(full_mask, dtype=bool)
     keep = np.nonzero(m)[0]
     return _orig_routed(q, ck, cv, orc.take_history(hk, keep), orc.take_history(hv, keep), m[keep],
-                        full_heads, k_cur, v_cur, tau)
+                        full_heads, k_cur, v_cur, tau, lowdim)
 
 
-def _routed_kept_heads_skip_current(q, ck, cv, hk, hv, full_mask, full_heads=None, k_cur=None, v_cur=None, tau=None):
-    O, L = _orig_routed(q, ck, cv, hk, hv, full_mask, full_heads, k_cur, v_cur, tau)
+def _routed_kept_heads_skip_current(q, ck, cv, hk, hv, full_mask, full_heads=None, k_cur=None, v_cur=None, tau=None,
+                                    lowdim=None):
+    O, L = _orig_routed(q, ck, cv, hk, hv, full_mask, full_heads, k_cur, v_cur, tau, lowdim)
     if full_heads is None:
         return O, L
     O2, L2 = _orig_routed(q, ck, cv, hk, hv, np.ones_like(np.asarray(full_mask, bool)), None, None, None, tau)
@@ -127,7 +129,61 @@ def _routed_kept_heads_skip_current(q, ck, cv, hk, hv, full_mask, full_heads=Non
     return np.where(sel[None, :, None], O2, O), np.where(sel[:, None], L2, L)
 
 
+_orig_reduced = orc.attend_reduced
+
+
+def _reduced_swaps_maps(q, ck, cv, hk, hv, maps, tau):
+    return _orig_reduced(q, ck, cv, hk, hv, dict(maps, U=maps["W"], W=maps["U"]), tau)
+
+
+def _reduced_trailing_columns(q, ck, cv, hk, hv, maps, tau):
+    U, W = np.asarray(maps["U"]), np.asarray(maps["W"])
+    return _orig_reduced(q, ck, cv, hk, hv, dict(maps, U=U[:, :, ::-1], W=W[:, :, ::-1]), tau)
+
+
+def _reduced_rescales_tau(q, ck, cv, hk, hv, maps, tau):
+    d = q.shape[2]
+    O = np.zeros(q.shape)
+    L = np.zeros((q.shape[1], q.shape[0]))
+    for h in range(q.shape[1]):
+        n = int(maps["d_h"][h])
+        o, lse = _orig_reduced(q, ck, cv, hk, hv, maps, tau * np.sqrt(d / n))
+        O[:, h], L[h] = o[:, h], lse[h]
+    return O, L
+
+
+def _reduced_restores_with_key_map(q, ck, cv, hk, hv, maps, tau):
+    Tq, H, d = q.shape
+    O, L = _orig_reduced(q, ck, cv, hk, hv, maps, tau)
+    for h in range(H):
+        n = int(maps["d_h"][h])
+        U, W = np.asarray(maps["U"][h])[:, :n], np.asarray(maps["W"][h])[:, :n]
+        O[:, h] = O[:, h] @ W @ U.T
+    return O, L
+
+
+_orig_maps = orc.lowdim_maps
+
+
+def _maps_ascending(D, H, d):
+    return _orig_maps(D, H, d)[:, :, ::-1]
+
+
+def _routed_reduces_full_set(q, ck, cv, hk, hv, full_mask, full_heads=None, k_cur=None, v_cur=None, tau=None,
+                             lowdim=None):
+    if lowdim is None:
+        return _orig_routed(q, ck, cv, hk, hv, full_mask, full_heads, k_cur, v_cur, tau)
+    return _orig_routed(q, ck, cv, hk, hv, np.zeros_like(np.asarray(full_mask, bool)), full_heads, k_cur, v_cur,
+                        tau, lowdim)
+
+
 MUTANTS = {
+    "reduced_swaps_maps": ("attend_reduced", _reduced_swaps_maps),
+    "reduced_trailing_columns": ("attend_reduced", _reduced_trailing_columns),
+    "reduced_rescales_tau": ("attend_reduced", _reduced_rescales_tau),
+    "reduced_restores_with_key_map": ("attend_reduced", _reduced_restores_with_key_map),
+    "maps_ascending": ("lowdim_maps", _maps_ascending),
+    "routed_reduces_full_set": ("attend_routed", _routed_reduces_full_set),
     "routed_drops_low_tokens": ("attend_routed", _routed_drops_low_tokens),
     "routed_kept_heads_skip_current": ("attend_routed", _routed_kept_heads_skip_current),
     "encode_projects_from_first_center": ("encode", _encode_projects_from_first_center),

@@ -393,3 +393,124 @@ def test_frame_policy_ranges():
     assert frame_policy(0, 100, recent=2) == []
     m = full_mask([(0, 100), (400, 100), (600, 350)], 950)
     assert m.sum() == 550 and m[0] and not m[100] and m[949]
+
+
+# --------------------------------------------------------------------------
+# reduced attention dimension per head (Table 6; Fig. 4(d) reduce / restore;
+# Table 8 analytical maps)
+# --------------------------------------------------------------------------
+
+def _orthonormal(rng, H, d):
+    return np.stack([np.linalg.qr(rng.standard_normal((d, d)))[0] for _ in range(H)])
+
+
+def _subspace_codec(rng, maps, n, d, r, C, T, key):
+    """A codec whose decoder columns and centers lie, per head, in the span
+    of the first n columns of that head's map (U for keys, W for values)."""
+    H = maps.shape[0]
+    D = np.concatenate([maps[h][:, :n] @ rng.standard_normal((n, r)) for h in range(H)])
+    cen = np.concatenate([(maps[h][:, :n] @ rng.standard_normal((n, C))).T for h in range(H)], axis=1)
+    hist = {"ids": rng.integers(0, C, T), "codes": rng.integers(-7, 8, (T, r)), "scales": rng.uniform(0.05, 0.6, T)}
+    return {"centers": cen, "D": D}, hist
+
+
+def test_reduced_at_full_dimension_is_full_attention():
+    """d_h = d with any orthonormal maps: U^T q . U^T k = q . k and W W^T = I,
+    so the reduced branch is the full-dim branch."""
+    rng = np.random.default_rng(21)
+    H, d, r, C, T, Tq = 3, 8, 6, 5, 30, 7
+    ck, cv, hk, hv = _rand_codec(rng, H, d, r, C, T)
+    q = rng.standard_normal((Tq, H, d))
+    maps = {"U": _orthonormal(rng, H, d), "W": _orthonormal(rng, H, d), "d_h": [d] * H}
+    O, L = orc.attend_reduced(q, ck, cv, hk, hv, maps, 0.6)
+    Of, Lf = orc.attend_full(q, ck, cv, hk, hv, 0.6)
+    assert np.allclose(O, Of, rtol=0, atol=1e-12) and np.allclose(L, Lf, rtol=0, atol=1e-12)
+
+
+def test_reduced_is_exact_when_keys_and_values_live_in_the_maps():
+    """Keys confined to span(U_h[:, :d_h]) and values to span(W_h[:, :d_h])
+    (different subspaces, d_h < d, queries arbitrary): the reduction loses
+    nothing, so attention at d_h equals full-dim attention."""
+    rng = np.random.default_rng(22)
+    H, d, r, C, T, Tq = 2, 12, 7, 4, 25, 6
+    for n in (3, 5):
+        U, W = _orthonormal(rng, H, d), _orthonormal(rng, H, d)
+        ck, hk = _subspace_codec(rng, U, n, d, r, C, T, "k")
+        cv, hv = _subspace_codec(rng, W, n, d, r, C, T, "v")
+        q = rng.standard_normal((Tq, H, d))
+        O, L = orc.attend_reduced(q, ck, cv, hk, hv, {"U": U, "W": W, "d_h": [n] * H}, 0.8)
+        Of, Lf = orc.attend_full(q, ck, cv, hk, hv, 0.8)
+        assert np.allclose(O, Of, rtol=0, atol=1e-11) and np.allclose(L, Lf, rtol=0, atol=1e-11)
+        # and it is a real reduction: the same maps on an unconfined codec differ
+        ck2, cv2, hk2, hv2 = _rand_codec(rng, H, d, r, C, T)
+        O2, _ = orc.attend_reduced(q, ck2, cv2, hk2, hv2, {"U": U, "W": W, "d_h": [n] * H}, 0.8)
+        Of2, _ = orc.attend_full(q, ck2, cv2, hk2, hv2, 0.8)
+        assert np.abs(O2 - Of2).max() > 1e-3
+
+
+def test_analytic_maps_are_the_decoder_principal_subspace():
+    """The leading n columns of lowdim_maps span the top-n eigenvectors of
+    D_h D_h^T (the symmetric eigensolver, another routine) for every n up to
+    the rank, and each head's map is orthonormal."""
+    rng = np.random.default_rng(23)
+    H, d, r = 2, 10, 7
+    D = rng.standard_normal((H * d, r)) * np.linspace(2.0, 0.3, r)[None, :]
+    maps = orc.lowdim_maps(D, H, d)
+    for h in range(H):
+        Dh = D[h * d:(h + 1) * d]
+        w, v = np.linalg.eigh(Dh @ Dh.T)
+        v = v[:, np.argsort(w)[::-1]]
+        assert np.allclose(maps[h].T @ maps[h], np.eye(d), atol=1e-12)
+        for n in range(1, r + 1):
+            P1 = maps[h][:, :n] @ maps[h][:, :n].T
+            P2 = v[:, :n] @ v[:, :n].T
+            assert np.allclose(P1, P2, atol=1e-9), (h, n)
+
+
+def test_analytic_maps_are_exact_for_low_rank_decoders():
+    """Decoders of rank n with centers in their column space: the analytical
+    maps at d_h = n reproduce full-dim attention (Eckart-Young: the rank-n
+    truncation of a rank-n decoder is the decoder)."""
+    rng = np.random.default_rng(24)
+    H, d, r, C, T, Tq, n = 2, 12, 8, 4, 20, 5, 4
+    ck, hk = _subspace_codec(rng, _orthonormal(rng, H, d), n, d, r, C, T, "k")
+    cv, hv = _subspace_codec(rng, _orthonormal(rng, H, d), n, d, r, C, T, "v")
+    maps = {"U": orc.lowdim_maps(ck["D"], H, d), "W": orc.lowdim_maps(cv["D"], H, d), "d_h": [n] * H}
+    q = rng.standard_normal((Tq, H, d))
+    O, L = orc.attend_reduced(q, ck, cv, hk, hv, maps, 0.5)
+    Of, Lf = orc.attend_full(q, ck, cv, hk, hv, 0.5)
+    assert np.allclose(O, Of, rtol=0, atol=1e-11) and np.allclose(L, Lf, rtol=0, atol=1e-11)
+
+
+def test_routed_with_reduced_heads():
+    """Reduced heads read their low-dim tokens at d_h and their full-dim
+    tokens full-dim: with keys/values confined to the maps' subspaces the
+    whole call equals one softmax over every key; on an unconfined codec the
+    reduced heads equal the LSE merge of full-dim attention over the routed
+    tokens, reduced attention over the others and the current chunk, and the
+    other heads are untouched."""
+    rng = np.random.default_rng(25)
+    H, d, r, C, T, Tq, Tc, n = 3, 12, 7, 4, 30, 5, 4, 5
+    U, W = _orthonormal(rng, H, d), _orthonormal(rng, H, d)
+    ck, hk = _subspace_codec(rng, U, n, d, r, C, T, "k")
+    cv, hv = _subspace_codec(rng, W, n, d, r, C, T, "v")
+    q = rng.standard_normal((Tq, H, d))
+    kc, vc = rng.standard_normal((Tc, H, d)), rng.standard_normal((Tc, H, d))
+    mask = rng.random(T) < 0.3
+    lowdim = {"U": U, "W": W, "d_h": np.array([n, 0, n])}
+    O, L = orc.attend_routed(q, ck, cv, hk, hv, mask, None, kc, vc, tau=0.7, lowdim=lowdim)
+    Or, Lr = _decoded_softmax(q, ck, cv, hk, hv, kc, vc, 0.7)
+    assert np.allclose(O, Or, rtol=0, atol=1e-11) and np.allclose(L, Lr, rtol=0, atol=1e-11)
+
+    ck, cv, hk, hv = _rand_codec(rng, H, d, r, C, T)
+    O, L = orc.attend_routed(q, ck, cv, hk, hv, mask, None, kc, vc, tau=0.7, lowdim=lowdim)
+    O0, L0 = orc.attend_routed(q, ck, cv, hk, hv, mask, None, kc, vc, tau=0.7)
+    f, l = np.nonzero(mask)[0], np.nonzero(~mask)[0]
+    maps = {"U": U, "W": W, "d_h": [n] * H}
+    Oe, Le = orc.lse_merge([orc.attend_full(q, ck, cv, orc.take_history(hk, f), orc.take_history(hv, f), 0.7),
+                            orc.attend_reduced(q, ck, cv, orc.take_history(hk, l), orc.take_history(hv, l), maps, 0.7),
+                            orc.softmax_attention(q, kc, vc, 0.7)])
+    for h in (0, 2):
+        assert np.allclose(O[:, h], Oe[:, h], rtol=0, atol=1e-12) and np.allclose(L[h], Le[h], rtol=0, atol=1e-12)
+    assert np.array_equal(O[:, 1], O0[:, 1]) and np.array_equal(L[1], L0[1])
+    assert np.abs(O[:, 0] - O0[:, 0]).max() > 1e-3
