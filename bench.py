@@ -106,6 +106,8 @@ def args_():
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--no-step30", action="store_true", help="skip the 30-layer step (side measurement)")
     ap.add_argument("--no-long", action="store_true", help="skip the long-rollout attend (side measurement)")
+    ap.add_argument("--no-reduced", action="store_true",
+                    help="skip the Fast attend with heads at reduced attention dimensions (side measurement)")
     ap.add_argument("--path", type=int, default=0, help="kernel family: 0 auto, 1 CUDA-core, 2 tensor-core")
     return ap.parse_args()
 
@@ -405,6 +407,7 @@ def run_ours(a, rank, world, device):
         cpu, parity = cpu_baseline(w, s, budget_s=12.0)
     fast = None if a.no_fast else run_side(a, device, peaks, "mixed")
     long_ = None if a.no_long else run_side(a, device, peaks, "long")
+    reduced = None if a.no_reduced else run_reduced(a, device, peaks)
     step30 = None if a.no_step30 else run_step30(a, device, peaks)
 
     line = {
@@ -432,7 +435,8 @@ def run_ours(a, rank, world, device):
                    "frac_hbm": round(enc_gbs / peaks["hbm_gbs"], 4)},
         "kernels": kernels,
         "clocks": clocks, "e2e": e2e, "gpu_launches": launches, "roofline": roof,
-        "cpu_baseline": cpu, "parity": parity, "fast": fast, "long": long_, "step30": step30,
+        "cpu_baseline": cpu, "parity": parity, "fast": fast, "long": long_, "fast_reduced": reduced,
+        "step30": step30,
     }
     return line
 
@@ -571,6 +575,78 @@ def run_side(a, device, peaks, name):
             "frac_bf16_peak": round(tf / peaks["bf16_tflops"], 4), "iters": n, "kernels": per,
             "T_full_attended": tfa, "step_gflop": round(ak["total"] / 1e9, 3),
             "step_gflop_as_named": round(af["total"] / 1e9, 3)}
+
+
+# Attention dimension of each head in the reduced-dimension measurement: the
+# shares of the HY-WorldPlay 32x row of Table 6 (440 / 192 / 24 / 208 of 864
+# head-layer pairs at 32 / 64 / 96 / 128) rounded to 12 heads; 128 = kept at
+# full dimension.
+TABLE6_MIX = (32, 64, 32, 128, 32, 64, 32, 128, 32, 64, 32, 128)
+
+
+def run_reduced(a, device, peaks):
+    """Side measurement of the Fast attend on the `mixed` workload with heads
+    at reduced attention dimensions (TABLE6_MIX): the most recent chunk
+    full-dim for every head, the 9360 older tokens at d_h = 32 / 64 for the
+    reduced heads and full-dim for the heads kept at 128, through
+    nanokv_attend_routed with random orthonormal maps."""
+    import compressed_history_attention_b200 as nk
+    from compressed_history_attention_b200.accounting import routed_flops
+    from synth.gen import WORKLOADS, make_lowdim_maps
+    w = WORKLOADS["mixed"]
+    s = setup(w, device)
+    mix = [TABLE6_MIX[h % len(TABLE6_MIX)] for h in range(w.H)]
+    d_h = [x if x < w.d else 0 for x in mix]
+    kept = [x == w.d for x in mix]
+    m = make_lowdim_maps(w, 11, device=device)
+    ld = nk.nanokv_lowdim_prepare(s["ck"], s["cv"], m["U"], m["W"])
+    full = [(w.T - w.T_full, w.T_full)]
+    p = s["prob"]
+    need = nk.nanokv_attend_routed_workspace(w.Tq, s["ck"], s["cv"], w.T, full, kept, w.Tq, ld, d_h)
+    ws = torch.empty(max(need, 16), dtype=torch.uint8, device=device)
+
+    def call():
+        nk.nanokv_attend_routed(p["q"], s["ck"], s["cv"], s["hk"], s["hv"], full, kept, p["k_cur"], p["v_cur"],
+                                out=s["out"], lse=s["lse"], workspace=ws, lowdim=ld, d_h=d_h)
+    for _ in range(2):
+        call()
+    flush = torch.empty(256 * 1024 * 1024, dtype=torch.uint8, device=device)
+    n = max(3, a.steps // 2)
+    g = capture(call)
+    ev = [[torch.cuda.Event(enable_timing=True) for _ in range(2)] for _ in range(n)]
+    for i in range(n):
+        flush.zero_()
+        ev[i][0].record()
+        g.replay()
+        ev[i][1].record()
+    torch.cuda.synchronize()
+    ms = sum(e[0].elapsed_time(e[1]) for e in ev) / n
+    dims = [x for x in d_h if x]
+    work = routed_flops(w.Tq, w.H, w.d, w.r, w.C, w.T_full, w.T_low, w.Tq, kept=sum(kept), dims=dims)
+    nk.nanokv_timing_read()
+    nk.nanokv_timing_enable(True)
+    for _ in range(n):
+        flush.zero_()
+        call()
+    torch.cuda.synchronize()
+    nk.nanokv_timing_enable(False)
+    kt = nk.nanokv_timing_read()
+    per = {}
+    for name, wk in (("attend_low", work["reduced"]), ("attend_full", work["full"]), ("attend_dense", work["current"])):
+        ms_k, cnt = kt[name]
+        if cnt:
+            per[name] = {"ms": round(ms_k / n, 4), "launches_per_call": cnt // n,
+                         "tflops": round(wk / (ms_k / n * 1e-3) / 1e12, 2)}
+    tf = work["total"] / (ms * 1e-3) / 1e12
+    del s, g, ws, ld
+    torch.cuda.empty_cache()
+    return {"workload": w.describe() + "; heads at d_h " + "/".join(map(str, mix)) + " (128 = kept full-dim)",
+            "attend_ms": round(ms, 4), "tflops": round(tf, 3), "frac_bf16_peak": round(tf / peaks["bf16_tflops"], 4),
+            "iters": n, "step_gflop": round(work["total"] / 1e9, 3),
+            "gflop_reduced_heads": round(work["reduced"] / 1e9, 3),
+            "kernels": per,
+            "note": "attend_low holds the query reduction and the reduced-width launches; attend_full the routed "
+                    "tokens of every head and the kept heads' other tokens"}
 
 
 def run_step30(a, device, peaks):

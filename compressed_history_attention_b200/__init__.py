@@ -9,5 +9,6 @@ from ._lib import (  # noqa: F401
     nanokv_attend_static, nanokv_check, nanokv_encode, nanokv_lse_merge, nanokv_set_kernel_path,
     nanokv_timing_enable,
     nanokv_timing_read, nanokv_version, nanokv_selftest_wait, nanokv_attend_full_tokens,
-    nanokv_attend_routed, nanokv_attend_routed_workspace,
+    nanokv_attend_routed, nanokv_attend_routed_workspace, Lowdim, nanokv_lowdim_prepare,
+    nanokv_lowdim_analytic,
 )

@@ -24,7 +24,8 @@ SYMBOLS = ("nanokv_encode", "nanokv_attend", "nanokv_attend_workspace", "nanokv_
            "nanokv_set_kernel_path", "nanokv_check", "nanokv_last_error", "nanokv_version",
            "nanokv_timing_enable", "nanokv_timing_read", "nanokv_codec_aux_bytes",
            "nanokv_codec_prepare", "nanokv_attend_static", "nanokv_selftest_wait",
-           "nanokv_attend_full_tokens", "nanokv_attend_routed", "nanokv_attend_routed_workspace")
+           "nanokv_attend_full_tokens", "nanokv_attend_routed", "nanokv_attend_routed_workspace",
+           "nanokv_lowdim_aux_bytes", "nanokv_lowdim_prepare", "nanokv_lowdim_analytic")
 
 # kernel identities of the diagnostics (nanokv_kernel_id)
 KERNELS = {0: "encode", 1: "attend_full", 2: "attend_low", 3: "attend_dense", 4: "lse_merge"}
@@ -53,6 +54,11 @@ class _Range(ctypes.Structure):
 
 
 MAX_RANGES = 64
+
+
+class _Lowdim(ctypes.Structure):
+    _fields_ = [("d_h", ctypes.POINTER(ctypes.c_int32)), ("U", ctypes.c_void_p), ("W", ctypes.c_void_p),
+                ("aux", ctypes.c_void_p)]
 
 
 _lib = None
@@ -101,10 +107,17 @@ def lib() -> ctypes.CDLL:
     L.nanokv_attend_full_tokens.argtypes = [P(_Codec), P(_Codec), i64, i64]
     L.nanokv_attend_full_tokens.restype = i64
     L.nanokv_attend_routed.argtypes = [vp, i32, i64, P(_Codec), P(_Codec), P(_Hist), P(_Hist), i64,
-                                       P(_Range), i32, vp, vp, vp, i64, f32, vp, vp, vp, sz, vp]
+                                       P(_Range), i32, vp, P(_Lowdim), vp, vp, i64, f32, vp, vp, vp, sz, vp]
     L.nanokv_attend_routed.restype = ctypes.c_int
-    L.nanokv_attend_routed_workspace.argtypes = [i64, P(_Codec), P(_Codec), i64, P(_Range), i32, vp, i64]
+    L.nanokv_attend_routed_workspace.argtypes = [i64, P(_Codec), P(_Codec), i64, P(_Range), i32, vp,
+                                                 P(_Lowdim), i64]
     L.nanokv_attend_routed_workspace.restype = sz
+    L.nanokv_lowdim_aux_bytes.argtypes = [P(_Codec), P(_Codec)]
+    L.nanokv_lowdim_aux_bytes.restype = sz
+    L.nanokv_lowdim_prepare.argtypes = [P(_Codec), P(_Codec), P(_Lowdim), vp]
+    L.nanokv_lowdim_prepare.restype = ctypes.c_int
+    L.nanokv_lowdim_analytic.argtypes = [P(_Codec), vp, vp]
+    L.nanokv_lowdim_analytic.restype = ctypes.c_int
     _lib = L
     return L
 
@@ -278,21 +291,73 @@ def _heads(full_heads, H):
     return buf, ctypes.cast(buf, ctypes.c_void_p)
 
 
-def nanokv_attend_routed_workspace(Tq: int, ck: Codec, cv: Codec, T: int, full, full_heads, T_cur: int) -> int:
+@dataclasses.dataclass
+class Lowdim:
+    """Maps of the heads deployed at a reduced attention dimension: U, W
+    [H, d, d] (head h's map in the leading columns of U[h] / W[h]) and the
+    mapped decoder / center tables (aux) that nanokv_lowdim_prepare wrote."""
+    U: torch.Tensor
+    W: torch.Tensor
+    aux: torch.Tensor
+
+    def struct(self, d_h) -> tuple:
+        arr = (ctypes.c_int32 * len(d_h))(*[int(v) for v in d_h])
+        return arr, _Lowdim(arr, self.U.data_ptr(), self.W.data_ptr(), self.aux.data_ptr())
+
+
+def nanokv_lowdim_prepare(ck: Codec, cv: Codec, U: torch.Tensor, W: torch.Tensor) -> Lowdim:
+    """Maps the codecs' decoder rows and centers through U (keys) and W
+    (values) once (nanokv_lowdim_prepare), into a buffer kept on the result."""
+    sk, sv = ck.struct(), cv.struct()
+    n = int(lib().nanokv_lowdim_aux_bytes(ctypes.byref(sk), ctypes.byref(sv)))
+    if n == 0:
+        _raise(ERR_UNSUPPORTED)
+    ld = Lowdim(U.contiguous(), W.contiguous(), torch.empty(n, dtype=torch.uint8, device=ck.D.device))
+    _keep, s = ld.struct([0] * ck.H)
+    _raise(lib().nanokv_lowdim_prepare(ctypes.byref(sk), ctypes.byref(sv), ctypes.byref(s), _stream(ck.D.device)))
+    return ld
+
+
+def nanokv_lowdim_analytic(c: Codec) -> torch.Tensor:
+    """Analytical maps [H, d, d] of a codec (nanokv_lowdim_analytic): the
+    left singular vectors of each head's decoder rows, by decreasing
+    singular value."""
+    maps = torch.empty(c.H, c.d, c.d, dtype=c.D.dtype, device=c.D.device)
+    sc = c.struct()
+    _raise(lib().nanokv_lowdim_analytic(ctypes.byref(sc), _ptr(maps), _stream(c.D.device)))
+    return maps
+
+
+def _lowdim(lowdim: Lowdim | None, d_h):
+    if lowdim is None:
+        return None, None
+    if d_h is None:
+        raise ValueError("a Lowdim needs the per-head d_h")
+    keep, s = lowdim.struct(d_h)
+    return (keep, s), ctypes.byref(s)
+
+
+def nanokv_attend_routed_workspace(Tq: int, ck: Codec, cv: Codec, T: int, full, full_heads, T_cur: int,
+                                   lowdim: Lowdim | None = None, d_h=None) -> int:
     sk, sv = ck.struct(), cv.struct()
     arr, n = _ranges(full)
     _keep, hp = _heads(full_heads, ck.H)
-    return int(lib().nanokv_attend_routed_workspace(Tq, ctypes.byref(sk), ctypes.byref(sv), T, arr, n, hp, T_cur))
+    _keep2, lp = _lowdim(lowdim, d_h)
+    return int(lib().nanokv_attend_routed_workspace(Tq, ctypes.byref(sk), ctypes.byref(sv), T, arr, n, hp, lp,
+                                                    T_cur))
 
 
 def nanokv_attend_routed(q: torch.Tensor, ck: Codec, cv: Codec, hk: Hist | None, hv: Hist | None, full,
                          full_heads=None, k_cur: torch.Tensor | None = None, v_cur: torch.Tensor | None = None,
                          softmax_scale: float | None = None, out: torch.Tensor | None = None,
-                         lse: torch.Tensor | bool | None = True, workspace: torch.Tensor | None = None):
+                         lse: torch.Tensor | bool | None = True, workspace: torch.Tensor | None = None,
+                         lowdim: Lowdim | None = None, d_h=None):
     """nanokv_attend under a routing policy: `full` is a list of (start,
     count) history token ranges read full-dim (sorted, disjoint), the rest
     low-dim; `full_heads` (H truth values, or None) marks heads that read all
-    their history full-dim.  Returns (out, lse) as nanokv_attend."""
+    their history full-dim; `lowdim` with `d_h` (H ints: 0, 32, 64 or 96)
+    puts heads at a reduced attention dimension for their low-dim tokens.
+    Returns (out, lse) as nanokv_attend."""
     Tq, H, d = q.shape
     T = len(hk) if hk is not None else 0
     T_cur = k_cur.shape[0] if k_cur is not None else 0
@@ -306,7 +371,7 @@ def nanokv_attend_routed(q: torch.Tensor, ck: Codec, cv: Codec, hk: Hist | None,
     elif lse is False:
         lse = None
     # (0 for arguments the call itself then refuses with its own status)
-    need = nanokv_attend_routed_workspace(Tq, ck, cv, T, full, full_heads, T_cur)
+    need = nanokv_attend_routed_workspace(Tq, ck, cv, T, full, full_heads, T_cur, lowdim, d_h)
     if workspace is None or workspace.numel() * workspace.element_size() < need:
         workspace = torch.empty(max(need, 16), dtype=torch.uint8, device=dev)
     sk, sv = ck.struct(), cv.struct()
@@ -314,9 +379,10 @@ def nanokv_attend_routed(q: torch.Tensor, ck: Codec, cv: Codec, hk: Hist | None,
     shv = hv.struct() if hv is not None and T else None
     arr, n = _ranges(full)
     _keep, hp = _heads(full_heads, H)
+    _keep2, lp = _lowdim(lowdim, d_h)
     st = lib().nanokv_attend_routed(
         _ptr(q), _dt(q), Tq, ctypes.byref(sk), ctypes.byref(sv),
-        ctypes.byref(shk) if shk else None, ctypes.byref(shv) if shv else None, T, arr, n, hp,
+        ctypes.byref(shk) if shk else None, ctypes.byref(shv) if shv else None, T, arr, n, hp, lp,
         _ptr(k_cur), _ptr(v_cur), T_cur, ctypes.c_float(softmax_scale), _ptr(out), _ptr(lse),
         _ptr(workspace), workspace.numel() * workspace.element_size(), _stream(dev))
     _raise(st)

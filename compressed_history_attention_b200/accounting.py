@@ -31,3 +31,33 @@ def encode_bytes(T: int, J: int, r: int, x_bytes: int = 2, scale_bytes: int = 2)
 def token_bytes(r: int, scale_bytes: int = 2) -> int:
     """Compressed bytes of one token in one branch: id + codes + scale."""
     return 1 + r // 2 + scale_bytes
+
+
+def reduced_flops(Tq: int, T_low: int, d: int, r: int, dims) -> int:
+    """Low-dim tokens of heads at reduced attention dimensions `dims` (one
+    d_h per reduced head): scores and value products of width d_h, the decode
+    of each token's key and value into d_h (once per token), the query
+    reduction and the output restore (once per query row)."""
+    if not (Tq and T_low):
+        return 0
+    return sum(4 * Tq * T_low * n + 4 * T_low * n * r + 2 * Tq * d * n + 2 * Tq * n * d for n in dims)
+
+
+def routed_flops(Tq: int, H: int, d: int, r: int, C: int, T_full: int, T_low: int, T_cur: int,
+                 kept: int = 0, dims=(), low_full: bool = False) -> dict:
+    """A routed call: T_full tokens full-dim for every head; the T_low others
+    full-dim for the `kept` heads (and for the ordinary heads too when
+    `low_full`: codecs whose low-dim tokens run on the full-dim kernel), at
+    reduced widths `dims` for the reduced heads, in the coefficient space for
+    the rest; the current chunk and merge as in attend_flops."""
+    nred = len(dims)
+    nlow = H - kept - nred
+    base = attend_flops(Tq, H, d, r, C, T_full, 0, T_cur)
+    per_head = attend_flops(Tq, 1, d, r, C, T_low, 0, 0)["full"]     # one head, full-dim over T_low
+    low_one = attend_flops(Tq, 1, d, r, C, 0, T_low, 0)["low"]       # one head, coefficient space
+    full_low = (kept + (nlow if low_full else 0)) * per_head
+    low = (0 if low_full else nlow) * low_one
+    red = reduced_flops(Tq, T_low, d, r, dims)
+    out = {"full": base["full"] + full_low, "low": low, "reduced": red, "current": base["current"]}
+    out["total"] = out["full"] + out["low"] + out["reduced"] + out["current"]
+    return out

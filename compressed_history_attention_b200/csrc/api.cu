@@ -277,14 +277,23 @@ static WsLayout ws_layout(int64_t Tq, const Codec &ck, int64_t T_low, int64_t T_
 struct RoutedPlan {
   int64_t T_f = 0, T_l = 0;  // history tokens read full-dim / low-dim (ordinary heads)
   GatherSegs full{}, low{};  // segments of the two sets
-  int nfh = 0;               // heads kept full-dim
-  uint32_t mask[8] = {};
-  // workspace: gathered histories [set][branch] (ids, codes, scales), head lists
-  size_t off_ids[2][2], off_codes[2][2], off_scales[2][2], off_heads, total;
+  uint8_t cls[256] = {};     // HeadClass of each head's low-dim tokens
+  int ncls[HC_COUNT] = {};   // heads per class
+  int nred = 0;              // heads at a reduced attention dimension
+  HeadDims dims{};
+  // workspace: gathered histories [set][branch] (ids, codes, scales), head
+  // lists, reduced queries
+  size_t off_ids[2][2], off_codes[2][2], off_scales[2][2], off_heads, off_qred, total;
 };
 
-static int routed_plan(const Codec &ck, const Codec &cv, int64_t T, const nanokv_range *full, int32_t n_full,
-                       const uint8_t *full_heads, size_t base, RoutedPlan *p) {
+static bool lowdim_codecs_ok(const Codec &ck, const Codec &cv) {
+  return ck.prec == PREC_BF16 && cv.prec == PREC_BF16 && ck.d == 128 && cv.d == 128 && ck.H == cv.H &&
+         ck.r == cv.r;
+}
+
+static int routed_plan(const Codec &ck, const Codec &cv, int64_t Tq, int64_t T, const nanokv_range *full,
+                       int32_t n_full, const uint8_t *full_heads, const nanokv_lowdim *lowdim, size_t base,
+                       RoutedPlan *p) {
   if (n_full < 0 || n_full > NANOKV_MAX_RANGES)
     return fail(NANOKV_ERR_INVALID, "routed: n_full=%d out of range [0,%d]", n_full, NANOKV_MAX_RANGES);
   if (n_full > 0 && !full) return fail(NANOKV_ERR_INVALID, "routed: NULL range array with n_full > 0");
@@ -315,13 +324,29 @@ static int routed_plan(const Codec &ck, const Codec &cv, int64_t T, const nanokv
     r.low.cnt[r.low.n++] = T - prev_end;
     r.T_l += T - prev_end;
   }
-  if (full_heads)
-    for (int h = 0; h < ck.H; ++h)
-      if (full_heads[h]) {
-        r.mask[h >> 5] |= 1u << (h & 31);
-        ++r.nfh;
-      }
-  // gathered histories, then the head lists
+  if (lowdim && !lowdim->d_h) return fail(NANOKV_ERR_INVALID, "routed: lowdim given with a NULL d_h array");
+  for (int h = 0; h < ck.H; ++h) {
+    const int dh = lowdim ? lowdim->d_h[h] : 0;
+    if (!(dh == 0 || tc_reduced_dim_ok(dh)))
+      return fail(NANOKV_ERR_INVALID, "routed: d_h[%d]=%d (0, 32, 64 or 96; full 128 goes in full_heads)", h, dh);
+    uint8_t c = HC_LOW;
+    if (full_heads && full_heads[h]) c = HC_FULL;
+    else if (dh) {
+      c = dh == 32 ? HC_R32 : dh == 64 ? HC_R64 : HC_R96;
+      r.dims.d[h] = (uint8_t)dh;
+      ++r.nred;
+    }
+    r.cls[h] = c;
+    ++r.ncls[c];
+  }
+  if (r.nred > 0) {
+    if (!lowdim_codecs_ok(ck, cv))
+      return fail(NANOKV_ERR_UNSUPPORTED, "routed: reduced attention dimensions need bf16 codecs with d = 128");
+    if (!lowdim->U || !lowdim->W || !lowdim->aux || !aligned16(lowdim->U) || !aligned16(lowdim->W) ||
+        !aligned16(lowdim->aux))
+      return fail(NANOKV_ERR_INVALID, "routed: lowdim U, W and aux must be non-NULL and 16-byte aligned");
+  }
+  // gathered histories, then the head lists, then the reduced queries
   size_t off = base;
   const int64_t n[2] = {r.T_f, r.T_l};
   const Codec *c[2] = {&ck, &cv};
@@ -336,7 +361,9 @@ static int routed_plan(const Codec &ck, const Codec &cv, int64_t T, const nanokv
       off += al256((size_t)n[set] * sb);
     }
   r.off_heads = off;
-  off += al256((size_t)2 * ck.H * sizeof(int32_t));
+  off += al256((size_t)(HC_COUNT + 1) * ck.H * sizeof(int32_t));
+  r.off_qred = off;
+  if (r.nred > 0 && r.T_l > 0) off += al256((size_t)Tq * ck.H * 128 * 2);
   r.total = off;
   *p = r;
   return NANOKV_OK;
@@ -611,12 +638,15 @@ int nanokv_attend(const void *q, int32_t io_dtype, int64_t Tq, const nanokv_code
 }
 
 // How a routed call runs its two history sets.  `full_set`: the routed
-// tokens, all heads, full-dim.  `low_set` for the ordinary heads: the
-// low-dim kernel (tensor-core or CUDA-core), or the tensor-core full-dim
-// kernel where no low-dim one exists (as in nanokv_attend); for the heads
-// kept full-dim: the full-dim kernel.
+// tokens, all heads, full-dim.  `low_set`, per head class: the heads kept
+// full-dim on the full-dim kernel; the ordinary heads on the low-dim kernel
+// (tensor-core or CUDA-core), or on the tensor-core full-dim kernel where no
+// low-dim one exists (as in nanokv_attend); the reduced heads on the full-dim
+// kernel at their width.  `cls` / `ncls`: the classes after that choice.
 struct RoutedKernels {
   bool tc_full, tc_low, tc_dense, low_via_full, low_simt;
+  uint8_t cls[256];
+  int ncls[HC_COUNT];
 };
 
 static int routed_kernels(int path, const Codec &ck, const Codec &cv, const RoutedPlan &r, int64_t T_cur,
@@ -626,39 +656,51 @@ static int routed_kernels(int path, const Codec &ck, const Codec &cv, const Rout
   k->tc_low = path != 1 && low_ok;
   k->tc_dense = path != 1 && tc_dense_supported(ck.prec, ck.d);
   k->low_via_full = !k->tc_low && k->tc_full;
-  k->low_simt = r.T_l > 0 && r.nfh < ck.H && !k->tc_low && !k->low_via_full;
-  if (path == 2 && ((r.T_f > 0 && !k->tc_full) || (r.T_l > 0 && !k->tc_low && !k->low_via_full) ||
+  const int nlow = r.ncls[HC_LOW];
+  k->low_simt = r.T_l > 0 && nlow > 0 && !k->tc_low && !k->low_via_full;
+  if (path == 2 && ((r.T_f > 0 && !k->tc_full) || (r.T_l > 0 && nlow > 0 && !k->tc_low && !k->low_via_full) ||
                     (T_cur > 0 && !k->tc_dense)))
     return fail(NANOKV_ERR_UNSUPPORTED, "routed: no tensor-core kernel for this shape");
-  const bool split_heads = r.T_l > 0 && r.nfh > 0 && r.nfh < ck.H && !k->low_via_full;
-  if (split_heads && !(k->tc_full && k->tc_low))
+  if (r.T_l > 0 && r.nred > 0 && !k->tc_full)
+    return fail(NANOKV_ERR_UNSUPPORTED, "routed: reduced attention dimensions need the tensor-core kernels");
+  for (int c = 0; c < HC_COUNT; ++c) k->ncls[c] = 0;
+  for (int h = 0; h < ck.H; ++h) {
+    k->cls[h] = (r.cls[h] == HC_LOW && k->low_via_full) ? (uint8_t)HC_FULL : r.cls[h];
+    ++k->ncls[k->cls[h]];
+  }
+  int present = 0;
+  for (int c = 0; c < HC_COUNT; ++c) present += k->ncls[c] > 0;
+  // a launch over part of the heads needs a kernel that takes a head list
+  if (r.T_l > 0 && present > 1 &&
+      ((k->ncls[HC_FULL] > 0 && !k->tc_full) || (k->ncls[HC_LOW] > 0 && !k->tc_low)))
     return fail(NANOKV_ERR_UNSUPPORTED,
-                "routed: heads of both kinds in one call need the tensor-core kernels for this codec");
+                "routed: heads of several kinds in one call need the tensor-core kernels for this codec");
   return NANOKV_OK;
 }
 
 size_t nanokv_attend_routed_workspace(int64_t Tq, const nanokv_codec *ck_, const nanokv_codec *cv_, int64_t T,
                                       const nanokv_range *full, int32_t n_full, const uint8_t *full_heads,
-                                      int64_t T_cur) {
+                                      const nanokv_lowdim *lowdim, int64_t T_cur) {
   Codec ck, cv;
   if (Tq < 0 || T < 0 || T_cur < 0) return 0;
   if (check_codec(ck_, "ck", false, &ck) || check_codec(cv_, "cv", false, &cv)) return 0;
   RoutedPlan r;
-  if (routed_plan(ck, cv, T, full, n_full, full_heads, 0, &r)) return 0;
+  if (routed_plan(ck, cv, Tq, T, full, n_full, full_heads, lowdim, 0, &r)) return 0;
   RoutedKernels k;
   if (routed_kernels(g_kernel_path.load(), ck, cv, r, T_cur, &k)) return 0;
   const int splits = (k.tc_full && r.T_f > 0 && Tq > 0) ? tc_full_splits(Tq, ck.H, ck.d, r.T_f) : 1;
   const WsLayout w = ws_layout(Tq, ck, r.T_l, r.T_f, T_cur, !k.low_simt, splits);
   RoutedPlan r2;
-  routed_plan(ck, cv, T, full, n_full, full_heads, w.total, &r2);
+  routed_plan(ck, cv, Tq, T, full, n_full, full_heads, lowdim, w.total, &r2);
   return r2.total;
 }
 
 int nanokv_attend_routed(const void *q, int32_t io_dtype, int64_t Tq, const nanokv_codec *ck_,
                          const nanokv_codec *cv_, const nanokv_hist *hk_, const nanokv_hist *hv_, int64_t T,
-                         const nanokv_range *full, int32_t n_full, const uint8_t *full_heads, const void *k_cur,
-                         const void *v_cur, int64_t T_cur, float softmax_scale, void *out, float *lse_out,
-                         void *workspace, size_t workspace_bytes, void *stream) {
+                         const nanokv_range *full, int32_t n_full, const uint8_t *full_heads,
+                         const nanokv_lowdim *lowdim, const void *k_cur, const void *v_cur, int64_t T_cur,
+                         float softmax_scale, void *out, float *lse_out, void *workspace, size_t workspace_bytes,
+                         void *stream) {
   ApiRange range("nanokv_attend_routed");
   Codec ck, cv;
   int s;
@@ -673,7 +715,7 @@ int nanokv_attend_routed(const void *q, int32_t io_dtype, int64_t Tq, const nano
   if (!(softmax_scale == softmax_scale) || softmax_scale <= 0.f || softmax_scale > 1e4f)
     return fail(NANOKV_ERR_INVALID, "routed: softmax_scale must be finite and positive");
   RoutedPlan r;
-  if ((s = routed_plan(ck, cv, T, full, n_full, full_heads, 0, &r))) return s;
+  if ((s = routed_plan(ck, cv, Tq, T, full, n_full, full_heads, lowdim, 0, &r))) return s;
   if (Tq == 0) return NANOKV_OK;
   if (!q || !out) return fail(NANOKV_ERR_INVALID, "routed: NULL q or out");
   if (!aligned16(q) || !aligned16(out) || (lse_out && !aligned16(lse_out)))
@@ -687,7 +729,7 @@ int nanokv_attend_routed(const void *q, int32_t io_dtype, int64_t Tq, const nano
   if ((s = routed_kernels(path, ck, cv, r, T_cur, &k))) return s;
   const int splits = (k.tc_full && r.T_f > 0) ? tc_full_splits(Tq, ck.H, ck.d, r.T_f) : 1;
   const WsLayout w = ws_layout(Tq, ck, r.T_l, r.T_f, T_cur, !k.low_simt, splits);
-  routed_plan(ck, cv, T, full, n_full, full_heads, w.total, &r);
+  routed_plan(ck, cv, Tq, T, full, n_full, full_heads, lowdim, w.total, &r);
   if (r.total > 0 && (!workspace || workspace_bytes < r.total))
     return fail(NANOKV_ERR_INVALID, "routed: workspace needs %zu bytes, got %zu", r.total, workspace_bytes);
   if (workspace && !aligned16(workspace)) return fail(NANOKV_ERR_INVALID, "routed: workspace must be 16-byte aligned");
@@ -717,13 +759,16 @@ int nanokv_attend_routed(const void *q, int32_t io_dtype, int64_t Tq, const nano
     g.n_out[0] = r.T_f;
     g.n_out[1] = r.T_l;
     g.scale_bytes = sb;
-    for (int i = 0; i < 8; ++i) g.head_mask[i] = r.mask[i];
+    for (int h = 0; h < ck.H; ++h) g.head_class[h] = k.cls[h];
     g.H = ck.H;
     g.head_lists = (int32_t *)(ws + r.off_heads);
     if ((e = gather_launch(r.full, r.low, g, st)) != cudaSuccess) return cuda_status(e, "routed gather launch");
   }
-  const int32_t *heads_full = (const int32_t *)(ws + r.off_heads), *heads_low = heads_full + ck.H;
-  const int nlh = ck.H - r.nfh;
+  const int32_t *lists = (const int32_t *)(ws + r.off_heads);
+  // the heads of class c: all heads (no list) when the class holds every head
+  auto sel = [&](int c) {
+    return k.ncls[c] == ck.H ? HeadSel{nullptr, 0} : HeadSel{lists + (size_t)c * ck.H, k.ncls[c]};
+  };
 
   // 2. branches: routed tokens full-dim (all heads); the other tokens low-dim
   // for the ordinary heads and full-dim for the heads kept full; the current
@@ -753,31 +798,51 @@ int nanokv_attend_routed(const void *q, int32_t io_dtype, int64_t Tq, const nano
     cudaStream_t bst = bstream(0);
     if (e != cudaSuccess) return cuda_status(e, "routed fork");
     const Hist &lk_ = hs[1][0], &lv_ = hs[1][1];
-    if (r.nfh == ck.H || k.low_via_full) {
-      // every head reads these tokens full-dim
+    // each head class into the same partial (disjoint heads)
+    if (k.ncls[HC_FULL]) {
       e = timed(NANOKV_K_FULL, 1, bst, [&] {
-        return k.tc_full ? tc_attend_full(q, Tq, ck, cv, lk_, lv_, 0, r.T_l, softmax_scale, p, 1, 0, 0, bst, false)
+        return k.tc_full ? tc_attend_full(q, Tq, ck, cv, lk_, lv_, 0, r.T_l, softmax_scale, p, 1, 0, 0, bst, false,
+                                          sel(HC_FULL))
                          : simt_attend_full(q, Tq, ck, cv, lk_, lv_, 0, r.T_l, softmax_scale, p, bst);
       });
-    } else {
-      const HeadSel lows = r.nfh ? HeadSel{heads_low, nlh} : HeadSel{nullptr, 0};
-      if (r.nfh)  // the heads kept full-dim, into the same partial (disjoint heads)
-        e = timed(NANOKV_K_FULL, 1, bst, [&] {
-          return tc_attend_full(q, Tq, ck, cv, lk_, lv_, 0, r.T_l, softmax_scale, p, 1, 0, 0, bst, false,
-                                HeadSel{heads_full, r.nfh});
-        });
-      if (e == cudaSuccess && k.tc_low) {
+    }
+    if (e == cudaSuccess && k.ncls[HC_LOW]) {
+      if (k.tc_low) {
         e = timed(NANOKV_K_LOW, 1, bst, [&] {
           return tc_low_supported(ck, cv)
-                     ? tc_attend_low(q, Tq, ck, cv, lk_, lv_, 0, r.T_l, softmax_scale, p, bst, lows)
-                     : tc_attend_low_pair(q, Tq, ck, cv, lk_, lv_, 0, r.T_l, softmax_scale, p, bst, lows);
+                     ? tc_attend_low(q, Tq, ck, cv, lk_, lv_, 0, r.T_l, softmax_scale, p, bst, sel(HC_LOW))
+                     : tc_attend_low_pair(q, Tq, ck, cv, lk_, lv_, 0, r.T_l, softmax_scale, p, bst, sel(HC_LOW));
         });
-      } else if (e == cudaSuccess) {
+      } else {
         float *qred = (float *)(ws + w.off_qred), *qc = (float *)(ws + w.off_qc);
         e = timed(NANOKV_K_LOW, 2, bst, [&] {
           cudaError_t e2 = simt_low_prep(q, Tq, ck, qred, qc, bst);
           if (e2 == cudaSuccess) e2 = simt_attend_low(qred, qc, Tq, ck, cv, lk_, lv_, 0, r.T_l, softmax_scale, p, bst);
           return e2;
+        });
+      }
+    }
+    if (e == cudaSuccess && r.nred) {
+      // reduced heads: reduce their queries once, then one launch per width
+      void *qr = ws + r.off_qred;
+      e = timed(NANOKV_K_LOW, 1, bst, [&] {
+        return reduce_queries(q, Tq, ck.H, lowdim->U, HeadSel{lists + (size_t)HC_COUNT * ck.H, r.nred}, r.dims, qr,
+                              bst);
+      });
+      const LowdimTables tb = lowdim_tables(ck, cv, lowdim->aux);
+      Codec ckr = ck, cvr = cv;
+      ckr.D = tb.D[0];
+      ckr.centers = tb.cen[0];
+      cvr.D = tb.D[1];
+      cvr.centers = tb.cen[1];
+      ckr.aux = cvr.aux = nullptr;
+      const int width[3] = {32, 64, 96};
+      for (int i = 0; i < 3 && e == cudaSuccess; ++i) {
+        const int c = HC_R32 + i;
+        if (!k.ncls[c]) continue;
+        e = timed(NANOKV_K_LOW, 1, bst, [&] {
+          return tc_attend_reduced(width[i], qr, Tq, ckr, cvr, lowdim->W, lk_, lv_, 0, r.T_l, softmax_scale, p, bst,
+                                   sel(c));
         });
       }
     }
@@ -819,6 +884,36 @@ int nanokv_attend_routed(const void *q, int32_t io_dtype, int64_t Tq, const nano
   e = timed(NANOKV_K_MERGE, 1, st,
             [&] { return lse_merge_launch(pl, Tq, ck.H, ck.d, out, ck.prec, lse_out, st); });
   return cuda_status(e, "routed merge launch");
+}
+
+size_t nanokv_lowdim_aux_bytes(const nanokv_codec *ck_, const nanokv_codec *cv_) {
+  Codec ck, cv;
+  if (check_codec(ck_, "lowdim ck", false, &ck) || check_codec(cv_, "lowdim cv", false, &cv)) return 0;
+  return lowdim_codecs_ok(ck, cv) ? lowdim_aux_bytes(ck, cv) : 0;
+}
+
+int nanokv_lowdim_prepare(const nanokv_codec *ck_, const nanokv_codec *cv_, const nanokv_lowdim *ld, void *stream) {
+  ApiRange range("nanokv_lowdim_prepare");
+  Codec ck, cv;
+  int s;
+  if ((s = check_codec(ck_, "lowdim ck", false, &ck))) return s;
+  if ((s = check_codec(cv_, "lowdim cv", false, &cv))) return s;
+  if (!lowdim_codecs_ok(ck, cv))
+    return fail(NANOKV_ERR_UNSUPPORTED, "lowdim: needs bf16 codecs with d = 128 and equal H and r for K and V");
+  if (!ld || !ld->U || !ld->W || !ld->aux || !aligned16(ld->U) || !aligned16(ld->W) || !aligned16(ld->aux))
+    return fail(NANOKV_ERR_INVALID, "lowdim: U, W and aux must be non-NULL and 16-byte aligned");
+  return cuda_status(lowdim_prepare(ck, cv, ld->U, ld->W, ld->aux, (cudaStream_t)stream), "lowdim prepare launch");
+}
+
+int nanokv_lowdim_analytic(const nanokv_codec *c_, void *maps, void *stream) {
+  ApiRange range("nanokv_lowdim_analytic");
+  Codec c;
+  int s;
+  if ((s = check_codec(c_, "lowdim analytic", false, &c))) return s;
+  if (c.prec != PREC_BF16 || c.d != 128)
+    return fail(NANOKV_ERR_UNSUPPORTED, "lowdim analytic: needs a bf16 codec with d = 128");
+  if (!maps || !aligned16(maps)) return fail(NANOKV_ERR_INVALID, "lowdim analytic: maps NULL or misaligned");
+  return cuda_status(lowdim_analytic(c, maps, (cudaStream_t)stream), "lowdim analytic launch");
 }
 
 int nanokv_lse_merge(int32_t n, const float *const *o_parts, const float *const *lse_parts,

@@ -84,17 +84,38 @@ struct GatherSegs {
   int64_t src[kMaxSegs], dst[kMaxSegs], cnt[kMaxSegs];
   int n;
 };
+// How a routed call reads a head's low-dim tokens: full-dim (heads kept at
+// full dimension), in the coefficient space (the low-dim kernels), or at a
+// reduced attention dimension of 32, 64 or 96.
+enum HeadClass : uint8_t { HC_FULL = 0, HC_LOW = 1, HC_R32 = 2, HC_R64 = 3, HC_R96 = 4, HC_COUNT = 5 };
 struct GatherArgs {
   const uint8_t *ids[2], *codes[2], *scales[2];            // source history, [K / V]
   uint8_t *d_ids[2][2], *d_codes[2][2], *d_scales[2][2];   // destinations, [set][K / V]
   int64_t n_out[2];                                       // tokens per set (full-dim, low-dim)
   int row_bytes[2];                                       // packed code bytes per token, [K / V]
   int scale_bytes;                                        // 2 (fp16) or 4 (fp32)
-  uint32_t head_mask[8];                                  // heads kept full-dim (bit h)
+  uint8_t head_class[256];                                // HeadClass of each head
   int H;
-  int32_t *head_lists;                                    // [2][H]: those heads, then the others
+  int32_t *head_lists;  // [HC_COUNT + 1][H]: the heads of each class, in order; then all reduced heads
 };
 cudaError_t gather_launch(const GatherSegs &full, const GatherSegs &low, const GatherArgs &a, cudaStream_t st);
+
+// Reduced attention dimension (lowdim.cu): mapped decoder rows [H*128, r]
+// and centers [C, H*128] (bf16) of each branch, in a caller buffer.
+struct LowdimTables {
+  void *D[2], *cen[2];
+};
+struct HeadDims {
+  uint8_t d[256];  // reduced attention dimension of each head (0: not reduced)
+};
+size_t lowdim_aux_bytes(const Codec &ck, const Codec &cv);
+LowdimTables lowdim_tables(const Codec &ck, const Codec &cv, void *aux);
+cudaError_t lowdim_prepare(const Codec &ck, const Codec &cv, const void *U, const void *W, void *aux,
+                           cudaStream_t st);
+cudaError_t reduce_queries(const void *q, int64_t Tq, int H, const void *U, HeadSel heads, const HeadDims &dims,
+                           void *qred, cudaStream_t st);
+// analytical maps [H, 128, 128] bf16 from a codec's decoder (bf16, d = 128)
+cudaError_t lowdim_analytic(const Codec &c, void *maps, cudaStream_t st);
 
 // Raises a kernel's dynamic shared-memory limit to `bytes` on the current
 // device the first time a launch needs it (the attribute call is not repeated

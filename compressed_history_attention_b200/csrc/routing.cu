@@ -12,13 +12,13 @@ namespace nanokv {
 namespace {
 
 __global__ void __launch_bounds__(256) gather_kernel(GatherSegs full, GatherSegs low, GatherArgs A) {
-  // head lists: heads kept full-dim in order, then the others
+  // head lists: the heads of each class, in order
   if (A.head_lists && blockIdx.x == 0 && blockIdx.y == 0 && threadIdx.x == 0) {
-    int nf = 0, nl = 0;
+    int n[HC_COUNT] = {}, nr = 0;
     for (int h = 0; h < A.H; ++h) {
-      const bool f = (A.head_mask[h >> 5] >> (h & 31)) & 1u;
-      if (f) A.head_lists[nf++] = h;
-      else A.head_lists[A.H + nl++] = h;
+      const int c = A.head_class[h] < HC_COUNT ? A.head_class[h] : HC_LOW;
+      A.head_lists[c * A.H + n[c]++] = h;
+      if (c >= HC_R32) A.head_lists[HC_COUNT * A.H + nr++] = h;  // and every reduced head
     }
   }
   const int set = blockIdx.y;

@@ -26,6 +26,14 @@ cudaError_t tc_attend_full(const void *q, int64_t Tq, const Codec &ck, const Cod
                            const Hist &hk, const Hist &hv, int64_t t0, int64_t T, float tau,
                            Part out, int nsplit, size_t ostride, size_t lstride, cudaStream_t st,
                            bool pdl, HeadSel hs = HeadSel{nullptr, 0});
+// Heads at a reduced attention dimension d_h (32, 64 or 96): the full-dim
+// kernel at width d_h on the reduced queries [Tq, H*128] and the mapped
+// decoder / centers (ck_red, cv_red), restoring its rows with the value maps
+// W [H, 128, 128].  One history split.
+bool tc_reduced_dim_ok(int d_h);
+cudaError_t tc_attend_reduced(int d_h, const void *q_red, int64_t Tq, const Codec &ck_red, const Codec &cv_red,
+                              const void *W, const Hist &hk, const Hist &hv, int64_t t0, int64_t T, float tau,
+                              Part out, cudaStream_t st, HeadSel hs);
 cudaError_t tc_attend_low(const void *q, int64_t Tq, const Codec &ck, const Codec &cv,
                           const Hist &hk, const Hist &hv, int64_t t0, int64_t T, float tau,
                           Part out, cudaStream_t st, HeadSel hs = HeadSel{nullptr, 0});

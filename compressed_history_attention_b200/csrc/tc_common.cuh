@@ -289,11 +289,11 @@ __device__ __forceinline__ void write_row_half(uint32_t tbase, int warp, uint32_
   }
 }
 
-// Multiplies this thread's O row (128 fp32 columns at o_col) by f.
-__device__ __forceinline__ void rescale_o(uint32_t tbase, int warp, uint32_t o_col, float f) {
+// Multiplies this thread's O row (16 * n16 fp32 columns at o_col) by f.
+__device__ __forceinline__ void rescale_o(uint32_t tbase, int warp, uint32_t o_col, float f, int n16 = 8) {
   uint32_t r[16];
 #pragma unroll 1
-  for (int c = 0; c < 8; ++c) {
+  for (int c = 0; c < n16; ++c) {
     const uint32_t a = tmem_lane_addr(tbase, warp, o_col + 16 * c);
     sm100::tmem_ld16(a, r);
     sm100::tmem_ld_wait();
@@ -323,6 +323,50 @@ __device__ __forceinline__ void write_row(uint32_t tbase, int warp, uint32_t o_c
         *reinterpret_cast<float4 *>(dst + 32 * c + i) = v;
       }
     }
+  }
+  if (row < Tq) L[(int64_t)h * Tq + row] = st.l > 0.f ? (st.m + log2f(st.l)) * kLn2 : -INFINITY;
+}
+
+// Reduced attention dimension: normalises this thread's o~ row (DHR fp32
+// columns at o_col) and writes the restored row O = W_h o~ (128 columns,
+// fp32 accumulation) and the LSE.  Wh: the head's value map [128, 128] bf16,
+// row-major, columns [0, DHR) used; every lane reads the same map element at
+// the same time.
+template <int DHR>
+__device__ __forceinline__ void write_row_restored(uint32_t tbase, int warp, uint32_t o_col, const RowState &st,
+                                                   int64_t row, int64_t Tq, int h, int H,
+                                                   const __nv_bfloat16 *__restrict__ Wh, float *__restrict__ O,
+                                                   float *__restrict__ L) {
+  const float inv = st.l > 0.f ? 1.f / st.l : 0.f;
+  float ot[DHR];
+#pragma unroll
+  for (int c = 0; c < DHR / 32; ++c) {
+    uint32_t r[32];
+    sm100::tmem_ld32(tmem_lane_addr(tbase, warp, o_col + 32 * c), r);
+    sm100::tmem_ld_wait();
+#pragma unroll
+    for (int i = 0; i < 32; ++i) ot[32 * c + i] = __uint_as_float(r[i]) * inv;
+  }
+  float *dst = O + (row * H + h) * 128;
+#pragma unroll 1
+  for (int i = 0; i < 128; i += 4) {
+    float acc[4] = {0.f, 0.f, 0.f, 0.f};
+#pragma unroll
+    for (int u = 0; u < 4; ++u) {
+      const uint4 *wrow = reinterpret_cast<const uint4 *>(Wh + (size_t)(i + u) * 128);
+#pragma unroll
+      for (int g = 0; g < DHR / 8; ++g) {
+        const uint4 wv = __ldg(wrow + g);
+        const uint32_t w4[4] = {wv.x, wv.y, wv.z, wv.w};
+#pragma unroll
+        for (int k = 0; k < 4; ++k) {
+          const float2 f = __bfloat1622float2(*reinterpret_cast<const __nv_bfloat162 *>(&w4[k]));
+          acc[u] = fmaf(f.x, ot[8 * g + 2 * k], acc[u]);
+          acc[u] = fmaf(f.y, ot[8 * g + 2 * k + 1], acc[u]);
+        }
+      }
+    }
+    if (row < Tq) *reinterpret_cast<float4 *>(dst + i) = make_float4(acc[0], acc[1], acc[2], acc[3]);
   }
   if (row < Tq) L[(int64_t)h * Tq + row] = st.l > 0.f ? (st.m + log2f(st.l)) * kLn2 : -INFINITY;
 }

@@ -22,6 +22,14 @@
 // Codes are unpacked in an order permuted within each group of 8; the
 // decoder slice is stored with the same permutation, so the contraction over
 // the rank index is unchanged.  Every wait is bounded.
+//
+// The same kernel serves heads deployed at a reduced attention dimension
+// d_h in {32, 64, 96} (NanoKV-Fast, Table 6; Fig. 4(d): reduced queries,
+// restored outputs).  Its inputs are then the reduced queries U_h^T q and the
+// mapped decoder rows U_h^T D_h and centers (W_h for values), so the
+// coefficients decode straight into d_h dimensions and every tile, MMA and
+// TMEM column range shrinks to d_h; at the end each softmax thread restores
+// its normalised row to d dimensions, O = W_h o~, in fp32.
 #include "tc_common.cuh"
 
 namespace nanokv {
@@ -49,9 +57,7 @@ constexpr int DH = 128;
 constexpr uint32_t kTile = 128 * 128 * 2;   // [128 x 128] bf16
 constexpr uint32_t kChunk = 128 * 64 * 2;   // [128 keys x 64 codes] bf16
 constexpr int NRING = 4;  // unpacked code chunks in flight (2 for r > 192: shared memory)
-constexpr uint32_t IDESC_DEC = idesc_bf16(128, 128, false, false);
 constexpr uint32_t IDESC_S = idesc_bf16(128, 128, false, false);
-constexpr uint32_t IDESC_PV = idesc_bf16(128, 128, false, true);
 constexpr uint32_t TM_O = 0, TM_S = 128, TM_X = 384, TM_COLS = 512;  // S: two 128-column buffers
 
 struct FullArgs {
@@ -68,6 +74,7 @@ struct FullArgs {
   float *O, *L;
   unsigned *err;
   const int32_t *head_map;      // heads of grid y (nullptr: y is the head)
+  const __nv_bfloat16 *W;       // reduced dimension: value maps [H, 128, 128] (restore)
 };
 
 struct FullBars {
@@ -87,20 +94,36 @@ struct FullBars {
 // global memory (L2) by the epilogue instead of being staged in shared
 // memory, and the code ring has 2 slots, so that a resident decoder slice of
 // up to r = 384 fits.
-template <bool kLarge>
+//
+// DHR: attention dimension of the launch (128, or a reduced d_h of 32, 64 or
+// 96).  Q and decoded tiles are [128 x DHR] in 64-column blocks (NAT of
+// them); the decoder slice holds DHR rows.
+template <int DHR>
+struct FullDims {
+  static constexpr int NAT = (DHR + 63) / 64;
+  static constexpr uint32_t kTileR = NAT * (kTile / 2);  // bytes of a Q / decoded tile
+  static constexpr uint32_t kDChunk = DHR * 128;          // decoder bytes per 64-wide rank block
+  static constexpr uint32_t IDEC = idesc_bf16(128, DHR, false, false);
+  static constexpr uint32_t IPV = idesc_bf16(128, DHR, false, true);
+};
+
+template <bool kLarge, int DHR>
 __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(384, 1)
     tc_full_kernel(const __grid_constant__ CUtensorMap tmQ, const FullArgs A) {
+  using F = FullDims<DHR>;
+  constexpr int NAT = F::NAT;
+  constexpr uint32_t kTileR = F::kTileR;
   extern __shared__ uint8_t smraw[];
   uint8_t *sm = (uint8_t *)(((uintptr_t)smraw + 1023) & ~(uintptr_t)1023);
   const int nrb = A.r / 64;  // 64-wide rank blocks
   uint8_t *sQ = sm;
-  uint8_t *sD = sQ + kTile;
-  uint8_t *sRing = sD + nrb * kChunk;
+  uint8_t *sD = sQ + kTileR;
+  uint8_t *sRing = sD + nrb * F::kDChunk;
   constexpr bool kCenGlobal = kLarge;
   constexpr int nring = kLarge ? 2 : NRING;
   uint8_t *sKh = sRing + nring * kChunk;
-  uint8_t *sVh = sKh + kTile;
-  uint8_t *sCen = sVh + kTile;  // this CTA's branch centers, head slice [C][128] bf16
+  uint8_t *sVh = sKh + kTileR;
+  uint8_t *sCen = sVh + kTileR;  // this CTA's branch centers, head slice [C][DHR] bf16, 256-byte rows
   __shared__ FullBars B;
 
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
@@ -139,7 +162,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(384, 1)
     }
     B.abort = 0;
     // phase 0 of the barrier of the tile this CTA receives
-    mbar_arrive_expect_tx(rank == 1 ? &B.kh_full : &B.vh_full, kTile);
+    mbar_arrive_expect_tx(rank == 1 ? &B.kh_full : &B.vh_full, kTileR);
     fence_mbar_init();
   }
   if (warp == 0) {
@@ -154,7 +177,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(384, 1)
   {
     const __nv_bfloat16 *Dsrc = A.D[rank] + (size_t)h * DH * A.r;
     const int gpr = A.r / 8;  // 8-element groups per row
-    const int groups = DH * gpr;
+    const int groups = DHR * gpr;
     constexpr int U = 8;
     for (int g0 = threadIdx.x; g0 < groups; g0 += U * 384) {
       uint4 v[U];
@@ -170,24 +193,25 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(384, 1)
           // element order (0,4,1,5,2,6,3,7): 16-bit halves of the source words
           const uint4 o = make_uint4(__byte_perm(v[u].x, v[u].z, 0x5410), __byte_perm(v[u].x, v[u].z, 0x7632),
                                      __byte_perm(v[u].y, v[u].w, 0x5410), __byte_perm(v[u].y, v[u].w, 0x7632));
-          *reinterpret_cast<uint4 *>(sD + sw128_offset(gidx / gpr, 8 * (gidx % gpr), DH)) = o;
+          *reinterpret_cast<uint4 *>(sD + sw128_offset(gidx / gpr, 8 * (gidx % gpr), DHR)) = o;
         }
       }
     }
     const int C = kCenGlobal ? 0 : A.C[rank];  // nothing to stage when centers are read from L2
     const __nv_bfloat16 *cen = A.cen[rank] + (size_t)h * DH;
-    for (int i0 = threadIdx.x; i0 < C * 16; i0 += 4 * 384) {
+    constexpr int CPR = DHR / 8;  // 16-byte chunks per center row
+    for (int i0 = threadIdx.x; i0 < C * CPR; i0 += 4 * 384) {
       uint4 v[4];
 #pragma unroll
       for (int u = 0; u < 4; ++u) {
         const int i = i0 + u * 384;
-        if (i < C * 16) v[u] = *reinterpret_cast<const uint4 *>(cen + (size_t)(i >> 4) * J + 8 * (i & 15));
+        if (i < C * CPR) v[u] = *reinterpret_cast<const uint4 *>(cen + (size_t)(i / CPR) * J + 8 * (i % CPR));
       }
 #pragma unroll
       for (int u = 0; u < 4; ++u) {
         const int i = i0 + u * 384;
-        if (i < C * 16) {
-          const int a = i >> 4, k = i & 15;
+        if (i < C * CPR) {
+          const int a = i / CPR, k = i % CPR;
           *reinterpret_cast<uint4 *>(sCen + a * 256 + ((k ^ (a & 15)) << 4)) = v[u];
         }
       }
@@ -205,9 +229,9 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(384, 1)
     // ---------------- Q load and MMA issuer ----------------
     if (lane == 0) {
       prefetch_tmap(&tmQ);
-      mbar_arrive_expect_tx(&B.q_full, kTile);
-      tma_load_2d(sQ, &tmQ, h * DH, (int)q0, &B.q_full);
-      tma_load_2d(sQ + kTile / 2, &tmQ, h * DH + 64, (int)q0, &B.q_full);
+      mbar_arrive_expect_tx(&B.q_full, kTileR);
+#pragma unroll
+      for (int c = 0; c < NAT; ++c) tma_load_2d(sQ + c * (kTile / 2), &tmQ, h * DH + 64 * c, (int)q0, &B.q_full);
       const uint32_t aQ = smem_u32(sQ), aD = smem_u32(sD), aR = smem_u32(sRing);
       const uint32_t aK = smem_u32(sKh), aV = smem_u32(sVh);
       bool ok = mbar_wait(&B.q_full, 0, abort, err);
@@ -226,10 +250,10 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(384, 1)
           if (mbar_test(&B.ring_full[slot], (cc / nring) & 1)) {
             if (cb == 0) FULL_TRACE(0, jd);
             tc_fence_after();
-            const uint32_t a = aR + slot * kChunk, b = aD + cb * kChunk;
+            const uint32_t a = aR + slot * kChunk, b = aD + cb * F::kDChunk;
 #pragma unroll
             for (int k = 0; k < 4; ++k)
-              mma_ss(tbase + TM_X, sdesc_sw128(a + 32 * k, 16, 1024), sdesc_sw128(b + 32 * k, 16, 1024), IDESC_DEC,
+              mma_ss(tbase + TM_X, sdesc_sw128(a + 32 * k, 16, 1024), sdesc_sw128(b + 32 * k, 16, 1024), F::IDEC,
                      (cb > 0 || k > 0));
             mma_commit(&B.ring_empty[slot]);
             ++cc;
@@ -248,11 +272,11 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(384, 1)
           FULL_TRACE(2, js);
           // the K_hat receiver arms the next phase (its bytes can only come
           // after this tile's scores are done in both CTAs)
-          if (rank == 1 && js + 1 < ntiles) mbar_arrive_expect_tx(&B.kh_full, kTile);
+          if (rank == 1 && js + 1 < ntiles) mbar_arrive_expect_tx(&B.kh_full, kTileR);
           tc_fence_after();
           const uint32_t dS = tbase + TM_S + (js & 1) * 128;
 #pragma unroll
-          for (int ks = 0; ks < DH / 16; ++ks) {
+          for (int ks = 0; ks < DHR / 16; ++ks) {
             const uint32_t off = (ks >> 2) * (kTile / 2) + (ks & 3) * 32;
             mma_ss(dS, sdesc_sw128(aQ + off, 16, 1024), sdesc_sw128(aK + off, 16, 1024), IDESC_S, ks > 0);
           }
@@ -264,12 +288,12 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(384, 1)
         // ---- values stream
         if (jv < js && mbar_test(&B.p_full[jv & 1], (jv >> 1) & 1) && mbar_test_cluster(&B.vh_full, jv & 1)) {
           FULL_TRACE(3, jv);
-          if (rank == 0 && jv + 1 < ntiles) mbar_arrive_expect_tx(&B.vh_full, kTile);
+          if (rank == 0 && jv + 1 < ntiles) mbar_arrive_expect_tx(&B.vh_full, kTileR);
           tc_fence_after();
           const uint32_t sP = tbase + TM_S + (jv & 1) * 128;
 #pragma unroll
           for (int ks = 0; ks < BN / 16; ++ks)
-            mma_ts(tbase + TM_O, sP + ks * 8, sdesc_sw128(aV + ks * 2048, kTile / 2, 1024), IDESC_PV,
+            mma_ts(tbase + TM_O, sP + ks * 8, sdesc_sw128(aV + ks * 2048, kTile / 2, 1024), F::IPV,
                    (jv > 0 || ks > 0));
           mma_commit(&B.pv_done[jv & 1]);
           mma_commit_mc(&B.vh_empty, 0x2);  // V_hat consumed: tell the V decoder (CTA 1)
@@ -366,13 +390,13 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(384, 1)
       if (j + 1 < ntiles) key_meta(j + 1, a_next, s_next);
       const uint8_t *crow = sCen + a * 256;
       const int sw = a & 15;
-      uint32_t o[64];
+      uint32_t o[DHR / 2];
       if constexpr (kCenGlobal) {
         // the key's center row (known a tile ahead) from L2, into the output
         // registers, before X is ready: o = c + s x is then formed in place
         const uint4 *src = reinterpret_cast<const uint4 *>(A.cen[rank] + (size_t)a * J + (size_t)h * DH);
 #pragma unroll
-        for (int g = 0; g < 16; ++g) {
+        for (int g = 0; g < DHR / 8; ++g) {
           const uint4 cv = __ldg(src + g);
           o[4 * g] = cv.x;
           o[4 * g + 1] = cv.y;
@@ -389,10 +413,10 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(384, 1)
       // buffer is waited for, so the next decode overlaps the hand-off.
       const __nv_bfloat162 s2 = __floats2bfloat162_rn(s, s);
 #pragma unroll
-      for (int c = 0; c < 4; ++c) {
+      for (int c = 0; c < DHR / 32; ++c) {
         uint32_t x[32];
         tmem_ld32(tmem_lane_addr(tbase, warp, TM_X + 32 * c), x);
-        if (c == 3) {
+        if (c == DHR / 32 - 1) {
           // X is no longer read by this warp: let the next decode start now
           tc_fence_before();
           __syncwarp();
@@ -427,11 +451,14 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(384, 1)
       if (t == 0) FULL_TRACE(5, j);
       bool ok = true;
 #pragma unroll
-      for (int c = 0; c < 2; ++c) {
+      for (int c = 0; c < NAT; ++c) {
+        constexpr int G = DHR >= 64 ? 8 : DHR / 8;  // 8-column groups of a block (the last one may hold fewer)
 #pragma unroll
-        for (int g = 0; g < 8; ++g)
-          st_shared_v4(dst_local + sw128_offset(t, 64 * c + 8 * g, 128),
-                       make_uint4(o[32 * c + 4 * g], o[32 * c + 4 * g + 1], o[32 * c + 4 * g + 2], o[32 * c + 4 * g + 3]));
+        for (int g = 0; g < G; ++g)
+          if (64 * c + 8 * g < DHR)
+            st_shared_v4(dst_local + sw128_offset(t, 64 * c + 8 * g, 128),
+                         make_uint4(o[32 * c + 4 * g], o[32 * c + 4 * g + 1], o[32 * c + 4 * g + 2],
+                                    o[32 * c + 4 * g + 3]));
         // columns [64c, 64c + 64) of every key form one 16 KB block of the
         // tile: hand it to the local MMA / the peer as soon as it is complete
         if (t == 0 && c == 0) FULL_TRACE(12, j);
@@ -444,7 +471,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(384, 1)
           if (!mbar_wait(&B.half_done[c], j & 1, abort, err)) { ok = false; break; }
           FULL_TRACE(15 + c, j);
           bulk_s2cluster(dst_remote + c * (kTile / 2), dstL + c * (kTile / 2), kTile / 2, full_remote);
-          if (c == 1) {
+          if (c == NAT - 1) {
             mbar_arrive(full_bar);
             FULL_TRACE(6, j);
           }
@@ -473,7 +500,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(384, 1)
       if (j > 0 && wr) {
         if (!mbar_wait(&B.pv_done[(j - 1) & 1], ((j - 1) >> 1) & 1, abort, err)) { ok = false; break; }
         tc_fence_after();
-        rescale_o(tbase, warp, TM_O, corr);
+        rescale_o(tbase, warp, TM_O, corr, DHR / 16);
       }
       tc_fence_before();
       __syncwarp();
@@ -485,8 +512,12 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(384, 1)
     if (ok && ntiles >= 2) ok = mbar_wait(&B.pv_done[(ntiles - 2) & 1], ((ntiles - 2) >> 1) & 1, abort, err);
     if (ok && mbar_wait(&B.pv_done[(ntiles - 1) & 1], ((ntiles - 1) >> 1) & 1, abort, err)) {
       tc_fence_after();
-      write_row(tbase, warp, TM_O, st, q0 + row, A.Tq, h, A.H, A.O + blockIdx.z * A.ostride,
-                A.L + blockIdx.z * A.lstride);
+      if constexpr (DHR == DH)
+        write_row(tbase, warp, TM_O, st, q0 + row, A.Tq, h, A.H, A.O + blockIdx.z * A.ostride,
+                  A.L + blockIdx.z * A.lstride);
+      else
+        write_row_restored<DHR>(tbase, warp, TM_O, st, q0 + row, A.Tq, h, A.H, A.W + (size_t)h * DH * DH,
+                                A.O + blockIdx.z * A.ostride, A.L + blockIdx.z * A.lstride);
     }
   }
   tc_fence_before();
@@ -511,9 +542,10 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(384, 1)
 
 static bool full_large(int r, int C) { return r > 192 || C > 64; }
 
-size_t tc_full_smem(int r, int C) {
+static size_t tc_full_smem(int r, int C, int dhr = DH) {
   const bool large = full_large(r, C);
-  return (size_t)3 * kTile + (size_t)(r / 64) * kChunk + (size_t)(large ? 2 : NRING) * kChunk +
+  const size_t tile = (size_t)((dhr + 63) / 64) * (kTile / 2);
+  return 3 * tile + (size_t)(r / 64) * dhr * 128 + (size_t)(large ? 2 : NRING) * kChunk +
          (large ? 0 : (size_t)C * 256) + 1024;
 }
 
@@ -524,6 +556,8 @@ bool tc_full_supported(const Codec &ck, const Codec &cv) {
   return ck.prec == PREC_BF16 && ck.d == DH && ck.r == cv.r && ck.r % 64 == 0 && ck.r <= 384 &&
          C <= 256 && tc_full_smem(ck.r, C) <= 232448;
 }
+
+bool tc_reduced_dim_ok(int d_h) { return d_h == 32 || d_h == 64 || d_h == 96; }
 
 // Largest number of two-CTA clusters of the full-dim kernel that can be
 // resident at once on the current device (cached per device).
@@ -536,13 +570,13 @@ static int full_cluster_capacity() {
   cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
   int cap = sms / 2;
   const size_t smem = tc_full_smem(192, 64);
-  if (ensure_smem((const void *)tc_full_kernel<false>, (int)smem) == cudaSuccess) {
+  if (ensure_smem((const void *)tc_full_kernel<false, DH>, (int)smem) == cudaSuccess) {
     cudaLaunchConfig_t cfg{};
     cfg.gridDim = dim3(2, 1, 1);
     cfg.blockDim = dim3(384);
     cfg.dynamicSmemBytes = smem;
     int n = 0;
-    if (cudaOccupancyMaxActiveClusters(&n, (const void *)tc_full_kernel<false>, &cfg) == cudaSuccess && n > 0)
+    if (cudaOccupancyMaxActiveClusters(&n, (const void *)tc_full_kernel<false, DH>, &cfg) == cudaSuccess && n > 0)
       cap = n;
   }
   cudaGetLastError();
@@ -579,10 +613,20 @@ int tc_full_splits(int64_t Tq, int H, int d, int64_t T) {
   return best;
 }
 
-cudaError_t tc_attend_full(const void *q, int64_t Tq, const Codec &ck, const Codec &cv,
-                           const Hist &hk, const Hist &hv, int64_t t0, int64_t T, float tau,
-                           Part out, int nsplit, size_t ostride, size_t lstride, cudaStream_t st,
-                           bool pdl, HeadSel hs) {
+template <int DHR>
+static cudaError_t launch_full(const CUtensorMap &mq, const FullArgs &a, dim3 grid, bool large, size_t smem,
+                               cudaStream_t st, bool pdl) {
+  const void *fn = large ? (const void *)tc_full_kernel<true, DHR> : (const void *)tc_full_kernel<false, DHR>;
+  cudaError_t e = ensure_smem(fn, (int)smem);
+  if (e != cudaSuccess) return e;
+  return large ? launch_k(tc_full_kernel<true, DHR>, grid, dim3(384), smem, st, pdl, mq, a)
+               : launch_k(tc_full_kernel<false, DHR>, grid, dim3(384), smem, st, pdl, mq, a);
+}
+
+static cudaError_t attend_full_dim(int dhr, const void *q, int64_t Tq, const Codec &ck, const Codec &cv,
+                                   const Hist &hk, const Hist &hv, int64_t t0, int64_t T, float tau, Part out,
+                                   int nsplit, size_t ostride, size_t lstride, cudaStream_t st, bool pdl, HeadSel hs,
+                                   const void *W) {
   if (Tq == 0 || T == 0) return cudaSuccess;
   const int64_t ntiles = (T + BN - 1) / BN;
   if (nsplit < 1 || nsplit > ntiles) return cudaErrorInvalidValue;
@@ -615,16 +659,35 @@ cudaError_t tc_attend_full(const void *q, int64_t Tq, const Codec &ck, const Cod
   a.L = out.LSE;
   a.err = error_word_ptr();
   a.head_map = hs.map;
+  a.W = (const __nv_bfloat16 *)W;
   const int Cmax = ck.C > cv.C ? ck.C : cv.C;
   const bool large = full_large(ck.r, Cmax);
-  const size_t smem = tc_full_smem(ck.r, Cmax);
-  ensure_smem(large ? (const void *)tc_full_kernel<true> : (const void *)tc_full_kernel<false>, (int)smem);
+  const size_t smem = tc_full_smem(ck.r, Cmax, dhr);
+  if (smem > 232448) return cudaErrorInvalidConfiguration;
   const unsigned qt = (unsigned)((Tq + BM - 1) / BM);
   // every split must get at least one key tile (the caller merges nsplit partials)
   if ((T + a.Tsplit - 1) / a.Tsplit != nsplit) return cudaErrorInvalidValue;
   dim3 grid((qt + 1) & ~1u, (unsigned)(hs.map ? hs.n : ck.H), (unsigned)nsplit);
-  return large ? launch_k(tc_full_kernel<true>, grid, dim3(384), smem, st, pdl, mq, a)
-               : launch_k(tc_full_kernel<false>, grid, dim3(384), smem, st, pdl, mq, a);
+  switch (dhr) {
+    case 32: return launch_full<32>(mq, a, grid, large, smem, st, pdl);
+    case 64: return launch_full<64>(mq, a, grid, large, smem, st, pdl);
+    case 96: return launch_full<96>(mq, a, grid, large, smem, st, pdl);
+    case DH: return launch_full<DH>(mq, a, grid, large, smem, st, pdl);
+    default: return cudaErrorInvalidValue;
+  }
+}
+
+cudaError_t tc_attend_full(const void *q, int64_t Tq, const Codec &ck, const Codec &cv, const Hist &hk,
+                           const Hist &hv, int64_t t0, int64_t T, float tau, Part out, int nsplit, size_t ostride,
+                           size_t lstride, cudaStream_t st, bool pdl, HeadSel hs) {
+  return attend_full_dim(DH, q, Tq, ck, cv, hk, hv, t0, T, tau, out, nsplit, ostride, lstride, st, pdl, hs, nullptr);
+}
+
+cudaError_t tc_attend_reduced(int d_h, const void *q_red, int64_t Tq, const Codec &ck_red, const Codec &cv_red,
+                              const void *W, const Hist &hk, const Hist &hv, int64_t t0, int64_t T, float tau,
+                              Part out, cudaStream_t st, HeadSel hs) {
+  if (!tc_reduced_dim_ok(d_h) || !W) return cudaErrorInvalidValue;
+  return attend_full_dim(d_h, q_red, Tq, ck_red, cv_red, hk, hv, t0, T, tau, out, 1, 0, 0, st, false, hs, W);
 }
 
 #ifdef NANOKV_TRACE

@@ -197,21 +197,77 @@ int nanokv_attend_static(const void *q, int32_t io_dtype, int64_t Tq,
  *                 at full dimension).  Heads of both kinds in one call need the
  *                 tensor-core kernels (NANOKV_ERR_UNSUPPORTED on the CUDA-core
  *                 path).
+ *   lowdim        NULL, or the heads deployed at a reduced attention dimension
+ *                 (nanokv_lowdim, prepared by nanokv_lowdim_prepare): a head
+ *                 with d_h[h] > 0 that is not in full_heads reads its low-dim
+ *                 tokens at dimension d_h[h] instead of in the coefficient
+ *                 space.  Needs the tensor-core kernels (bf16 codecs, d = 128;
+ *                 NANOKV_ERR_UNSUPPORTED otherwise).
  * Everything else (arguments, layouts, the current chunk, outputs, errors) is
  * as for nanokv_attend.  The routed tokens of each branch are first gathered
  * into contiguous compressed histories in the workspace (attention does not
  * depend on the order of its keys), so the result is the attention over the
- * same key set as nanokv_attend, up to rounding.
+ * same key set as nanokv_attend, up to rounding (and, for reduced heads, with
+ * their low-dim tokens seen through the maps).
  */
 #define NANOKV_MAX_RANGES 64
 typedef struct {
   int64_t start, count;
 } nanokv_range;
 
+/*
+ * Reduced attention dimension per head (NanoKV-Fast, Table 6: head-layer
+ * pairs deployed at d_h in {32, 64, 96, 128}; Fig. 4(d): the low-dimensional
+ * branch reduces the queries and restores the output dimension; Table 8:
+ * low-dimensional maps).  Head h attends its low-dim tokens through
+ * orthonormal maps U_h (queries and keys) and W_h (values and the output
+ * restore), each [d, d_h]:
+ *     q~ = U_h^T q,   k~_t = U_h^T c_K[a_t] + s_t (U_h^T D_K,h) code_t,
+ *     v~_t likewise with W_h,   o~ = softmax(tau q~ k~^T) v~,   O = W_h o~.
+ * The stored coefficients decode straight into d_h dimensions through the
+ * mapped decoder rows and centers.  Fields (d = 128, bf16 codecs only):
+ *   d_h   HOST array [H]: 0 (not reduced), 32, 64 or 96.  A head kept at the
+ *         full 128 dimensions goes in full_heads instead.
+ *   U, W  device [H, d, d] row-major bf16, 16-byte aligned, caller-owned:
+ *         head h's map in columns [0, d_h[h]) of U[h] / W[h] (the leading
+ *         columns, so maps ordered by importance serve every d_h).
+ *   aux   device buffer of nanokv_lowdim_aux_bytes() bytes, 256-byte aligned,
+ *         caller-owned: the mapped decoder rows and centers of both branches,
+ *         written by nanokv_lowdim_prepare; valid while U, W and the codecs'
+ *         D / centers are unchanged.
+ */
+typedef struct {
+  const int32_t *d_h;
+  const void *U, *W;
+  void *aux;
+} nanokv_lowdim;
+
+/* Bytes of nanokv_lowdim.aux for these codecs (0 if they have no reduced
+ * path: not bf16, d != 128, or K and V disagree on H or r). */
+size_t nanokv_lowdim_aux_bytes(const nanokv_codec *ck, const nanokv_codec *cv);
+
+/* Analytical maps (Table 8, "analytical initialization" of the
+ * low-dimensional maps): maps[h] [d, d] row-major bf16 holds, as its columns,
+ * the left singular vectors of the head's decoder rows D_h = rows
+ * [h*d, (h+1)*d) of c->D, by decreasing singular value, so that its leading
+ * d_h columns span the best rank-d_h approximation of D_h's column space
+ * (Eckart-Young).  Pass ck for U and cv for W.  Computed on the GPU as the
+ * eigenvectors of D_h D_h^T (cyclic Jacobi, fp32); the sign of each column
+ * is arbitrary (attention does not depend on it).  maps: device, H*d*d bf16,
+ * 16-byte aligned, caller-owned.  bf16 codecs with d = 128 only. */
+int nanokv_lowdim_analytic(const nanokv_codec *c, void *maps, void *stream);
+
+/* Writes ld->aux from the maps and the codecs (all d mapped rows of every
+ * head, so any d_h can use them): asynchronous on `stream`; NANOKV_OK, or
+ * NANOKV_ERR_INVALID / NANOKV_ERR_UNSUPPORTED before anything is launched. */
+int nanokv_lowdim_prepare(const nanokv_codec *ck, const nanokv_codec *cv, const nanokv_lowdim *ld,
+                          void *stream);
+
 int nanokv_attend_routed(const void *q, int32_t io_dtype, int64_t Tq,
                          const nanokv_codec *ck, const nanokv_codec *cv,
                          const nanokv_hist *hk, const nanokv_hist *hv, int64_t T,
                          const nanokv_range *full, int32_t n_full, const uint8_t *full_heads,
+                         const nanokv_lowdim *lowdim,
                          const void *k_cur, const void *v_cur, int64_t T_cur,
                          float softmax_scale, void *out, float *lse_out,
                          void *workspace, size_t workspace_bytes, void *stream);
@@ -219,7 +275,8 @@ int nanokv_attend_routed(const void *q, int32_t io_dtype, int64_t Tq,
 /* Workspace bytes nanokv_attend_routed needs (0 for invalid arguments). */
 size_t nanokv_attend_routed_workspace(int64_t Tq, const nanokv_codec *ck, const nanokv_codec *cv,
                                       int64_t T, const nanokv_range *full, int32_t n_full,
-                                      const uint8_t *full_heads, int64_t T_cur);
+                                      const uint8_t *full_heads, const nanokv_lowdim *lowdim,
+                                      int64_t T_cur);
 
 /* Workspace bytes nanokv_attend needs for these sizes (0 is possible). */
 size_t nanokv_attend_workspace(int64_t Tq, const nanokv_codec *ck, const nanokv_codec *cv,

@@ -162,3 +162,16 @@ def scaled(w: Workload, **kw) -> Workload:
     """A smaller copy of a workload (for parity cases that the oracle finishes
     in seconds): same codec structure, other sizes."""
     return dataclasses.replace(w, **kw)
+
+
+def make_lowdim_maps(w: Workload, seed: int, device="cpu") -> dict:
+    """Maps for heads at a reduced attention dimension: U and W [H, d, d],
+    each head a random orthonormal basis (QR of a Gaussian draw) rounded to
+    the storage dtype.  Any orthonormal map is a valid input (the deployed
+    maps are learned); which columns a head uses is the caller's d_h."""
+    g = _gen(seed, device)
+
+    def one():
+        m = torch.randn(w.H, w.d, w.d, generator=g, device=device, dtype=torch.float64)
+        return _round(torch.linalg.qr(m)[0], w.dtype).contiguous()
+    return {"U": one(), "W": one()}

@@ -203,7 +203,7 @@ def test_routed_rejects_bad_ranges():
         arr = (_lib._Range * max(1, len(ranges)))(*[_lib._Range(a, b) for a, b in ranges])
         return L.nanokv_attend_routed(p, _lib.F32, 4, ctypes.byref(c), ctypes.byref(c), ctypes.byref(h),
                                       ctypes.byref(h), T, arr, len(ranges) if n is None else n, None, None, None,
-                                      0, ctypes.c_float(0.25), p, None, p, 1 << 20, None)
+                                      None, 0, ctypes.c_float(0.25), p, None, p, 1 << 20, None)
 
     assert call([(10, 5), (12, 5)]) == _lib.ERR_INVALID   # overlap
     assert call([(50, 5), (10, 5)]) == _lib.ERR_INVALID   # not sorted
@@ -212,6 +212,48 @@ def test_routed_rejects_bad_ranges():
     assert call([(0, 1)], n=_lib.MAX_RANGES + 1) == _lib.ERR_INVALID
     ws = lambda ranges: L.nanokv_attend_routed_workspace(  # noqa: E731
         4, ctypes.byref(c), ctypes.byref(c), 100,
-        (_lib._Range * max(1, len(ranges)))(*[_lib._Range(a, b) for a, b in ranges]), len(ranges), None, 0)
+        (_lib._Range * max(1, len(ranges)))(*[_lib._Range(a, b) for a, b in ranges]), len(ranges), None, None, 0)
     assert ws([(10, 5), (12, 5)]) == 0
     assert ws([(10, 5), (40, 5)]) > 0
+
+
+def test_lowdim_validation():
+    """Reduced attention dimensions: bf16 codecs with d = 128 only; d_h in
+    {0, 32, 64, 96}; maps and tables non-NULL and aligned; all refused before
+    anything is launched."""
+    L = nk.lib()
+    bf = dict(H=4, d=128, r=192, C=64, param_dtype=_lib.BF16, scale_dtype=_lib.F16)
+    c, c32 = _codec(**bf), _codec()
+    n = L.nanokv_lowdim_aux_bytes(ctypes.byref(c), ctypes.byref(c))
+    assert n >= 2 * (4 * 128 * 192 * 2) + 2 * (64 * 4 * 128 * 2)
+    assert L.nanokv_lowdim_aux_bytes(ctypes.byref(c32), ctypes.byref(c32)) == 0      # fp32, d = 16
+    assert L.nanokv_lowdim_aux_bytes(ctypes.byref(c), ctypes.byref(_codec(**dict(bf, r=128)))) == 0
+    p = ctypes.c_void_p(1 << 20)
+    good = _lib._Lowdim(None, p, p, p)
+    assert L.nanokv_lowdim_prepare(ctypes.byref(c32), ctypes.byref(c32), ctypes.byref(good), None) == _lib.ERR_UNSUPPORTED
+    assert L.nanokv_lowdim_prepare(ctypes.byref(c), ctypes.byref(c), None, None) == _lib.ERR_INVALID
+    assert L.nanokv_lowdim_prepare(ctypes.byref(c), ctypes.byref(c), ctypes.byref(_lib._Lowdim(None, None, p, p)),
+                                   None) == _lib.ERR_INVALID
+    assert L.nanokv_lowdim_prepare(ctypes.byref(c), ctypes.byref(c),
+                                   ctypes.byref(_lib._Lowdim(None, p, p, ctypes.c_void_p((1 << 20) + 8))),
+                                   None) == _lib.ERR_INVALID
+
+    h = _lib._Hist(1 << 20, 1 << 20, 1 << 20)
+    arr = (_lib._Range * 1)(_lib._Range(0, 10))
+
+    def call(codec, dims, U=p, io=_lib.BF16):
+        d = (ctypes.c_int32 * codec.H)(*dims)
+        ld = _lib._Lowdim(d, U, p, p)
+        return L.nanokv_attend_routed(p, io, 4, ctypes.byref(codec), ctypes.byref(codec), ctypes.byref(h),
+                                      ctypes.byref(h), 100, arr, 1, None, ctypes.byref(ld), None, None, 0,
+                                      ctypes.c_float(0.1), p, None, p, 1 << 30, None)
+
+    assert call(c, [48, 0, 0, 0]) == _lib.ERR_INVALID       # not a deployed width
+    assert call(c, [128, 0, 0, 0]) == _lib.ERR_INVALID      # full width: full_heads instead
+    assert call(c, [32, 0, 0, 0], U=None) == _lib.ERR_INVALID
+    assert call(_codec(H=4), [32, 0, 0, 0], io=_lib.F32) == _lib.ERR_UNSUPPORTED
+    ws = lambda dims: L.nanokv_attend_routed_workspace(  # noqa: E731
+        64, ctypes.byref(c), ctypes.byref(c), 100, arr, 1, None,
+        ctypes.byref(_lib._Lowdim((ctypes.c_int32 * 4)(*dims), p, p, p)), 0)
+    # the reduced queries [Tq, H, 128] bf16 join the workspace
+    assert ws([32, 0, 64, 0]) >= ws([0, 0, 0, 0]) + 64 * 4 * 128 * 2

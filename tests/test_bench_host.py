@@ -76,3 +76,21 @@ def test_encode_parity_counts_mismatches_outside_ties():
     bad = bench.encode_parity(x, codec, ids, codes, ref["scales"].copy(), ref, "f16")
     assert bad["ids_differ_outside_ties"] == 1
     assert bad["codes_differ_outside_ties"] == 1
+
+
+def test_routed_work_accounting():
+    """routed_flops reduces to attend_flops for the fixed policy, counts a
+    kept head's low-dim tokens full-dim, and a reduced head's at its width:
+    scores and values of width d_h, a decode into d_h per token, the query
+    reduction and the restore per query row."""
+    from compressed_history_attention_b200.accounting import attend_flops, routed_flops
+    Tq, H, d, r, C, Tf, Tl, Tc = 100, 4, 128, 192, 64, 300, 500, 100
+    base = attend_flops(Tq, H, d, r, C, Tf, Tl, Tc)
+    assert routed_flops(Tq, H, d, r, C, Tf, Tl, Tc)["total"] == base["total"]
+    assert routed_flops(Tq, H, d, r, C, Tf, Tl, Tc, kept=H)["total"] == attend_flops(Tq, H, d, r, C, Tf + Tl, 0, Tc)["total"]
+    assert routed_flops(Tq, H, d, r, C, Tf, Tl, Tc, low_full=True)["total"] == \
+        attend_flops(Tq, H, d, r, C, Tf + Tl, 0, Tc)["total"]
+    one = routed_flops(Tq, H, d, r, C, Tf, Tl, Tc, dims=[32])
+    assert one["reduced"] == 4 * Tq * Tl * 32 + 4 * Tl * 32 * r + 4 * Tq * d * 32
+    assert one["low"] == base["low"] * (H - 1) // H
+    assert one["total"] < base["total"]
