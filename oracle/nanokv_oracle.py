@@ -22,6 +22,9 @@ plain readings below (each also listed in the design notes):
   * the current chunk is a third, uncompressed attention branch merged by LSE;
   * routing: the most recent T_full history tokens are full-dim, the older
     T - T_full tokens low-dim;
+  * calibration (Tables 2, 5; Fig. 3(a)): Lloyd k-means from given initial
+    centers, then the leading eigenvectors of the residual second moment
+    (see the calibration section below);
   * reduced attention dimension (Table 6): head h attends in R^{d_h} through
     orthonormal maps U_h (queries, keys) and W_h (values, output restore);
     the analytical maps are the leading left singular vectors of the head's
@@ -280,6 +283,67 @@ def attend_routed(q, ck, cv, hk, hv, full_mask, full_heads=None, k_cur=None, v_c
     O = np.where(sel[None, :, None], kept[0], routed[0])
     lse = np.where(sel[:, None], kept[1], routed[1])
     return O, lse
+
+
+# ----------------------------------------------------------------------------
+# Calibration of a codec on a chunk of tokens (Table 5: centers fitted
+# separately for K and V; Table 2: joint PCA with INT4 coefficients, then
+# shared centers; Fig. 3(a): joint head-channel PCA retains the most KV
+# variance at matched dimensional compression).
+#
+# Readings (the pages give no algorithm):
+#   * centers: Lloyd's k-means from caller-given initial centers, a fixed
+#     number of rounds; each round assigns every token to its nearest center
+#     (assign(): ties to the lowest index), then moves every center to the
+#     mean of its tokens; a center with no tokens stays where it is;
+#   * decoder: the r leading eigenvectors (decreasing eigenvalue) of the
+#     residual second-moment matrix (1/N) sum_t rho_t rho_t^T over the joint
+#     H*d channels, rho_t = x_t - c_{a_t} with the final centers and their
+#     assignment; E = D^T;
+#   * each eigenvector's sign: its entry of largest magnitude is positive
+#     (the first such entry on a tie).
+# ----------------------------------------------------------------------------
+
+def kmeans(x: np.ndarray, init_centers: np.ndarray, rounds: int):
+    """Lloyd rounds from init_centers [C, J]; returns (centers, ids), ids the
+    assignment to the returned centers."""
+    c = np.array(init_centers, dtype=np.float64, copy=True)
+    for _ in range(rounds):
+        ids = assign(x, c)
+        for j in range(c.shape[0]):
+            members = ids == j
+            if members.any():
+                c[j] = x[members].mean(axis=0)
+    return c, assign(x, c)
+
+
+def sign_fixed(v: np.ndarray) -> np.ndarray:
+    """Columns of v with the sign that makes each column's entry of largest
+    magnitude positive (first such entry on a tie)."""
+    v = np.array(v, dtype=np.float64, copy=True)
+    for i in range(v.shape[1]):
+        k = int(np.argmax(np.abs(v[:, i])))
+        if v[k, i] < 0:
+            v[:, i] = -v[:, i]
+    return v
+
+
+def joint_pca(x: np.ndarray, centers: np.ndarray, ids: np.ndarray, r: int):
+    """Decoder D [J, r] and the eigenvalues [r] of the residual second-moment
+    matrix (leading r, decreasing)."""
+    rho = x - centers[ids]
+    S = rho.T @ rho / x.shape[0]
+    w, v = np.linalg.eigh(S)
+    order = np.argsort(-w, kind="stable")[:r]
+    return sign_fixed(v[:, order]), w[order]
+
+
+def calibrate(x: np.ndarray, init_centers: np.ndarray, rounds: int, r: int) -> dict:
+    """Codec of one branch from a calibration chunk x [N, J]: centers [C, J],
+    D [J, r], E = D^T, plus the final assignment and the eigenvalues."""
+    centers, ids = kmeans(x, init_centers, rounds)
+    D, w = joint_pca(x, centers, ids, r)
+    return {"centers": centers, "D": D, "E": D.T.copy(), "ids": ids, "eigenvalues": w}
 
 
 # ----------------------------------------------------------------------------

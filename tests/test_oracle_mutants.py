@@ -177,7 +177,63 @@ def _routed_reduces_full_set(q, ck, cv, hk, hv, full_mask, full_heads=None, k_cu
                         tau, lowdim)
 
 
+_orig_kmeans = orc.kmeans
+_orig_pca = orc.joint_pca
+
+
+def _kmeans_sums(x, init_centers, rounds):
+    c = np.array(init_centers, dtype=np.float64, copy=True)
+    for _ in range(rounds):
+        ids = orc.assign(x, c)
+        for j in range(c.shape[0]):
+            if (ids == j).any():
+                c[j] = x[ids == j].sum(axis=0)
+    return c, orc.assign(x, c)
+
+
+def _kmeans_assigns_once(x, init_centers, rounds):
+    c = np.array(init_centers, dtype=np.float64, copy=True)
+    ids = orc.assign(x, c)
+    for _ in range(rounds):
+        for j in range(c.shape[0]):
+            if (ids == j).any():
+                c[j] = x[ids == j].mean(axis=0)
+    return c, orc.assign(x, c)
+
+
+def _kmeans_empty_to_zero(x, init_centers, rounds):
+    c = np.array(init_centers, dtype=np.float64, copy=True)
+    for _ in range(rounds):
+        ids = orc.assign(x, c)
+        for j in range(c.shape[0]):
+            c[j] = x[ids == j].mean(axis=0) if (ids == j).any() else 0.0
+    return c, orc.assign(x, c)
+
+
+def _pca_ascending(x, centers, ids, r):
+    rho = x - centers[ids]
+    w, v = np.linalg.eigh(rho.T @ rho / x.shape[0])
+    return orc.sign_fixed(v[:, :r]), w[:r]
+
+
+def _pca_of_raw_tokens(x, centers, ids, r):
+    return _orig_pca(x, np.zeros_like(centers), ids, r)
+
+
+def _pca_no_sign_rule(x, centers, ids, r):
+    rho = x - centers[ids]
+    w, v = np.linalg.eigh(rho.T @ rho / x.shape[0])
+    order = np.argsort(-w)[:r]
+    return -orc.sign_fixed(v[:, order]), w[order]
+
+
 MUTANTS = {
+    "kmeans_sums": ("kmeans", _kmeans_sums),
+    "kmeans_assigns_once": ("kmeans", _kmeans_assigns_once),
+    "kmeans_empty_to_zero": ("kmeans", _kmeans_empty_to_zero),
+    "pca_ascending": ("joint_pca", _pca_ascending),
+    "pca_of_raw_tokens": ("joint_pca", _pca_of_raw_tokens),
+    "pca_no_sign_rule": ("joint_pca", _pca_no_sign_rule),
     "reduced_swaps_maps": ("attend_reduced", _reduced_swaps_maps),
     "reduced_trailing_columns": ("attend_reduced", _reduced_trailing_columns),
     "reduced_rescales_tau": ("attend_reduced", _reduced_rescales_tau),

@@ -514,3 +514,91 @@ def test_routed_with_reduced_heads():
         assert np.allclose(O[:, h], Oe[:, h], rtol=0, atol=1e-12) and np.allclose(L[h], Le[h], rtol=0, atol=1e-12)
     assert np.array_equal(O[:, 1], O0[:, 1]) and np.array_equal(L[1], L0[1])
     assert np.abs(O[:, 0] - O0[:, 0]).max() > 1e-3
+
+
+# --------------------------------------------------------------------------
+# calibration: k-means centers and joint PCA (Tables 2, 5; Fig. 3(a))
+# --------------------------------------------------------------------------
+
+def test_kmeans_worked_example():
+    g = _load("kmeans_worked.json")
+    x, init = np.array(g["x"]), np.array(g["init"])
+    for n in range(1, len(g["rounds"]) + 1):
+        c, ids = orc.kmeans(x, init, n)
+        assert np.allclose(c, np.array(g["rounds"][n - 1]["centers"]), rtol=0, atol=1e-12), n
+        nxt = g["rounds"][min(n, len(g["rounds"]) - 1)]["ids"]
+        assert ids.tolist() == nxt, n
+
+
+def test_kmeans_single_center_is_the_mean():
+    rng = np.random.default_rng(31)
+    x = rng.standard_normal((50, 7))
+    c, ids = orc.kmeans(x, rng.standard_normal((1, 7)), 1)
+    assert np.allclose(c[0], x.mean(axis=0), rtol=0, atol=1e-14) and (ids == 0).all()
+
+
+def test_kmeans_center_without_tokens_stays():
+    rng = np.random.default_rng(32)
+    x = rng.standard_normal((40, 5))
+    init = np.stack([x[0], x[1], np.full(5, 1e3)])
+    c, ids = orc.kmeans(x, init, 3)
+    assert np.array_equal(c[2], init[2]) and not (ids == 2).any()
+
+
+def test_kmeans_objective_never_increases_and_is_permutation_equivariant():
+    rng = np.random.default_rng(33)
+    x = np.concatenate([rng.standard_normal((60, 6)) + 4 * rng.standard_normal(6) for _ in range(4)])
+    init = x[rng.choice(len(x), 5, replace=False)]
+    prev = np.inf
+    for n in range(6):
+        c, ids = orc.kmeans(x, init, n)
+        obj = ((x - c[ids]) ** 2).sum()
+        assert obj <= prev + 1e-9
+        prev = obj
+    perm = np.array([3, 0, 4, 1, 2])
+    c1, ids1 = orc.kmeans(x, init, 4)
+    c2, ids2 = orc.kmeans(x, init[perm], 4)
+    assert np.allclose(c2, c1[perm], rtol=0, atol=1e-12)
+    assert np.array_equal(perm[ids2], ids1)
+
+
+def test_joint_pca_eigenpairs_match_the_svd_of_the_residuals():
+    """D's columns are orthonormal eigenvectors of the residual second moment,
+    eigenvalues decreasing, equal to the squared singular values of
+    rho / sqrt(N) (np.linalg.svd, another routine), and their span is the
+    leading right-singular subspace; each column's largest entry is
+    positive."""
+    rng = np.random.default_rng(34)
+    N, J, C, r = 200, 12, 3, 5
+    x = rng.standard_normal((N, J)) * np.linspace(3.0, 0.2, J)[None, :]
+    centers, ids = orc.kmeans(x, x[:C], 2)
+    D, w = orc.joint_pca(x, centers, ids, r)
+    rho = x - centers[ids]
+    S = rho.T @ rho / N
+    assert np.allclose(D.T @ D, np.eye(r), atol=1e-12)
+    assert np.allclose(S @ D, D * w[None, :], atol=1e-10)
+    assert (np.diff(w) <= 0).all()
+    _, sv, vt = np.linalg.svd(rho / np.sqrt(N), full_matrices=False)
+    assert np.allclose(w, sv[:r] ** 2, rtol=1e-10, atol=1e-12)
+    assert np.allclose(D @ D.T, vt[:r].T @ vt[:r], atol=1e-9)
+    for i in range(r):
+        assert D[np.argmax(np.abs(D[:, i])), i] > 0
+
+
+def test_calibrated_codec_is_exact_on_low_rank_residuals():
+    """Tokens = a center + a residual in a rank-r subspace: k-means from the
+    true centers keeps them, and the calibrated D reconstructs every residual
+    exactly (x = c_a + D D^T (x - c_a))."""
+    rng = np.random.default_rng(35)
+    N, J, C, r = 120, 16, 3, 4
+    true_c = 30 * rng.standard_normal((C, J))
+    B = np.linalg.qr(rng.standard_normal((J, r)))[0]
+    z = rng.integers(0, C, N)
+    g = rng.standard_normal((N, r))
+    g -= np.stack([g[z == j].mean(axis=0) for j in range(C)])[z]   # residuals of zero mean per cluster
+    x = true_c[z] + g @ B.T
+    cal = orc.calibrate(x, true_c, 2, r)
+    assert np.array_equal(cal["ids"], z)
+    rho = x - cal["centers"][cal["ids"]]
+    assert np.allclose(rho @ cal["D"] @ cal["E"], rho, atol=1e-10)
+    assert np.allclose(cal["E"], cal["D"].T)
