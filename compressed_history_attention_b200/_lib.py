@@ -25,7 +25,8 @@ SYMBOLS = ("nanokv_encode", "nanokv_attend", "nanokv_attend_workspace", "nanokv_
            "nanokv_timing_enable", "nanokv_timing_read", "nanokv_codec_aux_bytes",
            "nanokv_codec_prepare", "nanokv_attend_static", "nanokv_selftest_wait",
            "nanokv_attend_full_tokens", "nanokv_attend_routed", "nanokv_attend_routed_workspace",
-           "nanokv_lowdim_aux_bytes", "nanokv_lowdim_prepare", "nanokv_lowdim_analytic")
+           "nanokv_lowdim_aux_bytes", "nanokv_lowdim_prepare", "nanokv_lowdim_analytic",
+           "nanokv_calibrate_workspace", "nanokv_calibrate")
 
 # kernel identities of the diagnostics (nanokv_kernel_id)
 KERNELS = {0: "encode", 1: "attend_full", 2: "attend_low", 3: "attend_dense", 4: "lse_merge"}
@@ -118,6 +119,10 @@ def lib() -> ctypes.CDLL:
     L.nanokv_lowdim_prepare.restype = ctypes.c_int
     L.nanokv_lowdim_analytic.argtypes = [P(_Codec), vp, vp]
     L.nanokv_lowdim_analytic.restype = ctypes.c_int
+    L.nanokv_calibrate_workspace.argtypes = [i64, i32, i32]
+    L.nanokv_calibrate_workspace.restype = sz
+    L.nanokv_calibrate.argtypes = [vp, i32, i64, i32, i32, i32, vp, i32, vp, vp, vp, vp, vp, vp, sz, vp]
+    L.nanokv_calibrate.restype = ctypes.c_int
     _lib = L
     return L
 
@@ -326,6 +331,28 @@ def nanokv_lowdim_analytic(c: Codec) -> torch.Tensor:
     sc = c.struct()
     _raise(lib().nanokv_lowdim_analytic(ctypes.byref(sc), _ptr(maps), _stream(c.D.device)))
     return maps
+
+
+def nanokv_calibrate(x: torch.Tensor, init_centers: torch.Tensor, rounds: int, r: int) -> dict:
+    """Codec of one branch fitted on tokens x [N, J] (nanokv_calibrate):
+    k-means centers from init_centers [C, J], then the r leading eigenvectors
+    of the residual second moment as D [J, r] and E = D^T, in x's dtype; also
+    the final assignment and the eigenvalues."""
+    x = x.contiguous()
+    N, J = x.shape
+    C = init_centers.shape[0]
+    dev = x.device
+    out = {"centers": torch.empty(C, J, dtype=x.dtype, device=dev),
+           "D": torch.empty(J, r, dtype=x.dtype, device=dev), "E": torch.empty(r, J, dtype=x.dtype, device=dev),
+           "ids": torch.empty(N, dtype=torch.uint8, device=dev),
+           "eigenvalues": torch.empty(r, dtype=torch.float32, device=dev)}
+    n = int(lib().nanokv_calibrate_workspace(N, J, C))
+    ws = torch.empty(max(n, 16), dtype=torch.uint8, device=dev)
+    init = init_centers.to(torch.float32).contiguous()
+    _raise(lib().nanokv_calibrate(_ptr(x), _dt(x), N, J, C, r, _ptr(init), rounds, _ptr(out["centers"]),
+                                  _ptr(out["D"]), _ptr(out["E"]), _ptr(out["ids"]), _ptr(out["eigenvalues"]),
+                                  _ptr(ws), n, _stream(dev)))
+    return out
 
 
 def _lowdim(lowdim: Lowdim | None, d_h):

@@ -125,9 +125,12 @@ __global__ void selftest_wait_kernel(uint64_t limit_ns, unsigned *err) {
 // the others leave idle (a partial last wave).  Created once per device and
 // kept for the life of the process; callers on several host threads
 // serialise on the mutex while they enqueue.
+// Helper streams: 0 low-dim set, 1 full-dim set, 2 current chunk; 3 and 4
+// the reduced-dimension heads of a routed call.
+constexpr int kBranchStreams = 5;
 struct BranchStreams {
-  cudaStream_t s[3] = {};
-  cudaEvent_t fork = nullptr, join[3] = {};
+  cudaStream_t s[kBranchStreams] = {};
+  cudaEvent_t fork = nullptr, join[kBranchStreams] = {}, aux = nullptr;
   bool ready = false;
 };
 constexpr int kMaxDevices = 64;
@@ -149,11 +152,14 @@ static cudaError_t branch_streams(BranchStreams **out) {
     int least = 0, greatest = 0;
     e = cudaDeviceGetStreamPriorityRange(&least, &greatest);
     // numerically smaller is higher priority
-    const int prio[3] = {greatest < least ? greatest + 1 : least, greatest, least};
-    for (int i = 0; i < 3 && e == cudaSuccess; ++i)
+    const int mid = greatest < least ? greatest + 1 : least;
+    const int prio[kBranchStreams] = {mid, greatest, least, mid, mid};
+    for (int i = 0; i < kBranchStreams && e == cudaSuccess; ++i)
       e = cudaStreamCreateWithPriority(&b.s[i], cudaStreamNonBlocking, prio[i]);
     if (e == cudaSuccess) e = cudaEventCreateWithFlags(&b.fork, cudaEventDisableTiming);
-    for (int i = 0; i < 3 && e == cudaSuccess; ++i) e = cudaEventCreateWithFlags(&b.join[i], cudaEventDisableTiming);
+    if (e == cudaSuccess) e = cudaEventCreateWithFlags(&b.aux, cudaEventDisableTiming);
+    for (int i = 0; i < kBranchStreams && e == cudaSuccess; ++i)
+      e = cudaEventCreateWithFlags(&b.join[i], cudaEventDisableTiming);
     cudaThreadExchangeStreamCaptureMode(&mode);
     if (e != cudaSuccess) return e;
     b.ready = true;
@@ -775,7 +781,7 @@ int nanokv_attend_routed(const void *q, int32_t io_dtype, int64_t Tq, const nano
   // chunk.  Independent: on the helper streams, as in nanokv_attend.
   PartList pl{};
   const bool on[3] = {r.T_l > 0, r.T_f > 0, T_cur > 0};
-  const int nbranch = (int)on[0] + (int)on[1] + (int)on[2];
+  const int nbranch = (int)on[0] + (int)on[1] + (int)on[2] + (int)(on[0] && r.nred > 0);
   std::unique_lock<std::mutex> lk(g_bs_mu, std::defer_lock);
   BranchStreams *bs = nullptr;
   if (nbranch > 1 && !g_timing.load()) {
@@ -823,12 +829,25 @@ int nanokv_attend_routed(const void *q, int32_t io_dtype, int64_t Tq, const nano
       }
     }
     if (e == cudaSuccess && r.nred) {
-      // reduced heads: reduce their queries once, then one launch per width
+      // reduced heads: reduce their queries once, then one launch per width;
+      // beside the other classes, on helper streams 3 (the reduction, the
+      // 32- and 96-wide launches) and 4 (the 64-wide launch, after the
+      // reduction)
       void *qr = ws + r.off_qred;
-      e = timed(NANOKV_K_LOW, 1, bst, [&] {
+      cudaStream_t rs[2] = {bst, bst};
+      if (bs) {
+        rs[0] = bstream(3);
+        if (e == cudaSuccess) rs[1] = bstream(4);
+        if (e != cudaSuccess) return cuda_status(e, "routed fork");
+      }
+      e = timed(NANOKV_K_LOW, 1, rs[0], [&] {
         return reduce_queries(q, Tq, ck.H, lowdim->U, HeadSel{lists + (size_t)HC_COUNT * ck.H, r.nred}, r.dims, qr,
-                              bst);
+                              rs[0]);
       });
+      if (bs && e == cudaSuccess) {
+        e = cudaEventRecord(bs->aux, rs[0]);
+        if (e == cudaSuccess) e = cudaStreamWaitEvent(rs[1], bs->aux, 0);
+      }
       const LowdimTables tb = lowdim_tables(ck, cv, lowdim->aux);
       Codec ckr = ck, cvr = cv;
       ckr.D = tb.D[0];
@@ -840,11 +859,14 @@ int nanokv_attend_routed(const void *q, int32_t io_dtype, int64_t Tq, const nano
       for (int i = 0; i < 3 && e == cudaSuccess; ++i) {
         const int c = HC_R32 + i;
         if (!k.ncls[c]) continue;
-        e = timed(NANOKV_K_LOW, 1, bst, [&] {
-          return tc_attend_reduced(width[i], qr, Tq, ckr, cvr, lowdim->W, lk_, lv_, 0, r.T_l, softmax_scale, p, bst,
+        cudaStream_t cs_ = rs[i == 1 ? 1 : 0];
+        e = timed(NANOKV_K_LOW, 1, cs_, [&] {
+          return tc_attend_reduced(width[i], qr, Tq, ckr, cvr, lowdim->W, lk_, lv_, 0, r.T_l, softmax_scale, p, cs_,
                                    sel(c));
         });
       }
+      if (bs && e == cudaSuccess) e = join(3);
+      if (bs && e == cudaSuccess) e = join(4);
     }
     if (e == cudaSuccess) e = join(0);
     if (e != cudaSuccess) return cuda_status(e, "routed low-set launch");
@@ -914,6 +936,48 @@ int nanokv_lowdim_analytic(const nanokv_codec *c_, void *maps, void *stream) {
     return fail(NANOKV_ERR_UNSUPPORTED, "lowdim analytic: needs a bf16 codec with d = 128");
   if (!maps || !aligned16(maps)) return fail(NANOKV_ERR_INVALID, "lowdim analytic: maps NULL or misaligned");
   return cuda_status(lowdim_analytic(c, maps, (cudaStream_t)stream), "lowdim analytic launch");
+}
+
+size_t nanokv_calibrate_workspace(int64_t N, int32_t J, int32_t C) {
+  if (N < 1 || J < 32 || J > 3072 || (J & 31) || C < 1 || C > 256) return 0;
+  return calibrate_workspace(N, J, C);
+}
+
+int nanokv_calibrate(const void *x, int32_t dtype, int64_t N, int32_t J, int32_t C, int32_t r,
+                     const float *init_centers, int32_t rounds, void *centers_out, void *D_out, void *E_out,
+                     uint8_t *ids_out, float *eigenvalues_out, void *workspace, size_t workspace_bytes,
+                     void *stream) {
+  ApiRange range("nanokv_calibrate");
+  const int prec = io_prec(dtype);
+  if (prec < 0) return fail(NANOKV_ERR_UNSUPPORTED, "calibrate: dtype must be F32 or BF16");
+  if (N < 1 || J < 32 || J > 3072 || (J & 31))
+    return fail(NANOKV_ERR_INVALID, "calibrate: N=%lld must be >= 1 and J=%d a multiple of 32 in [32, 3072]",
+                (long long)N, J);
+  if (C < 1 || C > 256 || r < 1 || r > J || rounds < 0 || rounds > 1000)
+    return fail(NANOKV_ERR_INVALID, "calibrate: C=%d (1..256), r=%d (1..J), rounds=%d (0..1000)", C, r, rounds);
+  if (!x || !init_centers || !centers_out || !D_out || !E_out || !workspace)
+    return fail(NANOKV_ERR_INVALID, "calibrate: NULL pointer");
+  if (!aligned16(x) || !aligned16(init_centers) || !aligned16(workspace))
+    return fail(NANOKV_ERR_INVALID, "calibrate: x, init_centers and workspace must be 16-byte aligned");
+  const size_t need = calibrate_workspace(N, J, C);
+  if (workspace_bytes < need)
+    return fail(NANOKV_ERR_INVALID, "calibrate: workspace needs %zu bytes, got %zu", need, workspace_bytes);
+  CalibArgs a{};
+  a.x = x;
+  a.N = N;
+  a.J = J;
+  a.C = C;
+  a.r = r;
+  a.rounds = rounds;
+  a.prec = prec;
+  a.init = init_centers;
+  a.centers = centers_out;
+  a.D = D_out;
+  a.E = E_out;
+  a.ids = ids_out;
+  a.evals = eigenvalues_out;
+  calibrate_carve(a, workspace);
+  return cuda_status(calibrate_launch(a, (cudaStream_t)stream), "calibrate");
 }
 
 int nanokv_lse_merge(int32_t n, const float *const *o_parts, const float *const *lse_parts,

@@ -117,6 +117,27 @@ cudaError_t reduce_queries(const void *q, int64_t Tq, int H, const void *U, Head
 // analytical maps [H, 128, 128] bf16 from a codec's decoder (bf16, d = 128)
 cudaError_t lowdim_analytic(const Codec &c, void *maps, cudaStream_t st);
 
+// Codec calibration (calibrate.cu): k-means centers, then the leading
+// eigenvectors of the residual second moment.  Outputs in the tokens' dtype.
+constexpr int kCalibSweeps = 30;  // Jacobi sweeps at most (stops once converged)
+struct CalibArgs {
+  const void *x;        // [N, J] tokens (fp32 or bf16, prec)
+  int64_t N;
+  int J, C, r, rounds, prec;
+  const float *init;    // [C, J] initial centers
+  void *centers, *D, *E;  // outputs [C, J], [J, r], [r, J]
+  uint8_t *ids;         // [N] final assignment (workspace when the caller passes none)
+  float *evals;         // [r] or nullptr
+  float *cen32;          // workspace: fp32 centers
+  double *S, *V;         // workspace: the second moment / its eigenvectors (fp64)
+  void *rot;
+  int *done;
+};
+size_t calibrate_workspace(int64_t N, int J, int C);
+void calibrate_carve(CalibArgs &a, void *ws);
+// synchronises the stream once per Jacobi sweep (the convergence test)
+cudaError_t calibrate_launch(const CalibArgs &a, cudaStream_t st);
+
 // Raises a kernel's dynamic shared-memory limit to `bytes` on the current
 // device the first time a launch needs it (the attribute call is not repeated
 // on every launch).

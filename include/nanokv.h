@@ -257,6 +257,38 @@ size_t nanokv_lowdim_aux_bytes(const nanokv_codec *ck, const nanokv_codec *cv);
  * 16-byte aligned, caller-owned.  bf16 codecs with d = 128 only. */
 int nanokv_lowdim_analytic(const nanokv_codec *c, void *maps, void *stream);
 
+/*
+ * nanokv_calibrate -- fit one branch's codec on a calibration chunk, the step
+ * before encode (Table 5: centers fitted separately for K and V; Table 2:
+ * joint PCA with INT4 coefficients, then shared centers; Fig. 3(a): joint
+ * head-channel PCA retains the most KV variance at matched compression).
+ *   1. `rounds` Lloyd k-means rounds from init_centers: every token to its
+ *      nearest center (squared Euclidean over the joint J = H*d channels,
+ *      ties to the lowest index), every center to the mean of its tokens (a
+ *      center without tokens stays); then the final assignment (ids_out).
+ *   2. D = the r leading eigenvectors, by decreasing eigenvalue, of the
+ *      residual second moment (1/N) sum_t rho_t rho_t^T, rho_t = x_t -
+ *      c_{a_t}; each column's largest-magnitude entry positive; E = D^T.
+ *   x             device [N, J] in dtype (F32 or BF16), 16-byte aligned
+ *   init_centers  device [C, J] fp32 (the caller's choice, e.g. C tokens)
+ *   centers_out   device [C, J], D_out [J, r], E_out [r, J], in dtype
+ *   ids_out       device [N] u8 or NULL; eigenvalues_out device [r] fp32 or NULL
+ *   workspace     device, nanokv_calibrate_workspace(N, J, C) bytes
+ * J a multiple of 32 up to 3072, C <= 256, 1 <= r <= J.  All work is fp32
+ * on the GPU: k-means kernels, a tiled second-moment kernel and cyclic
+ * Jacobi rotations (three launches per round of J/2 disjoint pairs).  The
+ * call synchronises `stream` once per Jacobi sweep to test convergence (so
+ * it cannot be captured in a CUDA graph) and returns when the work is done.
+ * Eigenvectors of (nearly) equal eigenvalues are determined only as a
+ * subspace.  Errors: NANOKV_ERR_INVALID / _UNSUPPORTED before any launch,
+ * NANOKV_ERR_CUDA on a CUDA error.
+ */
+size_t nanokv_calibrate_workspace(int64_t N, int32_t J, int32_t C);
+int nanokv_calibrate(const void *x, int32_t dtype, int64_t N, int32_t J, int32_t C, int32_t r,
+                     const float *init_centers, int32_t rounds, void *centers_out, void *D_out,
+                     void *E_out, uint8_t *ids_out, float *eigenvalues_out, void *workspace,
+                     size_t workspace_bytes, void *stream);
+
 /* Writes ld->aux from the maps and the codecs (all d mapped rows of every
  * head, so any d_h can use them): asynchronous on `stream`; NANOKV_OK, or
  * NANOKV_ERR_INVALID / NANOKV_ERR_UNSUPPORTED before anything is launched. */

@@ -257,3 +257,26 @@ def test_lowdim_validation():
         ctypes.byref(_lib._Lowdim((ctypes.c_int32 * 4)(*dims), p, p, p)), 0)
     # the reduced queries [Tq, H, 128] bf16 join the workspace
     assert ws([32, 0, 64, 0]) >= ws([0, 0, 0, 0]) + 64 * 4 * 128 * 2
+
+
+def test_calibrate_validation():
+    """Calibration: J a multiple of 32 up to 3072, 1 <= C <= 256, 1 <= r <= J,
+    aligned pointers and a large enough workspace; refused before any launch."""
+    L = nk.lib()
+    assert L.nanokv_calibrate_workspace(100, 48, 4) == 0
+    assert L.nanokv_calibrate_workspace(100, 4096, 4) == 0
+    n = L.nanokv_calibrate_workspace(100, 64, 4)
+    assert n >= 2 * 64 * 64 * 4 + 4 * 64 * 4
+    p = ctypes.c_void_p(1 << 20)
+
+    def call(dt=_lib.BF16, N=100, J=64, C=4, r=8, rounds=2, ws=1 << 30, x=p):
+        return L.nanokv_calibrate(x, dt, N, J, C, r, p, rounds, p, p, p, None, None, p, ws, None)
+
+    assert call(dt=_lib.F16) == _lib.ERR_UNSUPPORTED
+    assert call(J=48) == _lib.ERR_INVALID
+    assert call(C=0) == _lib.ERR_INVALID
+    assert call(r=65) == _lib.ERR_INVALID
+    assert call(rounds=-1) == _lib.ERR_INVALID
+    assert call(ws=16) == _lib.ERR_INVALID
+    assert call(x=ctypes.c_void_p((1 << 20) + 4)) == _lib.ERR_INVALID
+    assert call(x=None) == _lib.ERR_INVALID
