@@ -44,11 +44,11 @@ BAD_REASONS = ("hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown")
 # of the sources they were taken on: a kernel whose source has changed since
 # reports null traffic.
 NCU_TRAFFIC = {
-    ("attend_full", "full"): ("tc_full", "ad7a7c99a295bffa", 18877440 + 5851904),
-    ("attend_low", "long"): ("tc_low_pair", "cf31160a163436dd", 71376384 + 31356928),
-    ("attend_low", "mixed"): ("tc_low", "4fcc55f69a077271", 17918464 + 15104),
-    ("attend_dense", "full"): ("tc_dense", "6f930d6c7b63c100", 43229696 + 1877760),
-    ("encode", "full"): ("tc_encode", "4b9f263521ef0a34", 30489600 + 18688),
+    ("attend_full", "full"): ("tc_full", "cbc8940b3c4cfc1f", 18916480 + 2877355),
+    ("attend_low", "long"): ("tc_low_pair", "1af5729c0430d001", 71728100 + 27869668),
+    ("attend_low", "mixed"): ("tc_low", "d15b7a8cf47b4f75", 17933966 + 19342),
+    ("attend_dense", "full"): ("tc_dense", "bc840a866ba6a1e1", 43226496 + 128366),
+    ("encode", "full"): ("tc_encode", "2dd3bbffe1bdaec5", 30490261 + 181),
 }
 
 

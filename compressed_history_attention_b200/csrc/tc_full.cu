@@ -80,7 +80,7 @@ struct FullArgs {
 struct FullBars {
   uint64_t q_full;
   uint64_t ring_full[NRING], ring_empty[NRING];
-  uint64_t x_full, x_empty, half_done[2];
+  uint64_t x_full, x_empty;
   uint64_t kh_full, vh_full, kh_empty, vh_empty;
   uint64_t s_full[2], p_full[2], pv_done[2];  // pv_done[b]: P*V of the tiles using S buffer b
   uint32_t tmem_base;
@@ -146,13 +146,11 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(384, 1)
     for (int i = 0; i < nring; ++i) { mbar_init(&B.ring_full[i], 2); mbar_init(&B.ring_empty[i], 1); }
     mbar_init(&B.x_full, 1);
     mbar_init(&B.x_empty, 4);  // one arrive per epilogue warp once its last X load is done
-    mbar_init(&B.half_done[0], 4);
-    mbar_init(&B.half_done[1], 4);
-    // decoded-tile barriers: in the decoding CTA one arrive by its epilogue;
-    // in the receiving CTA one expect_tx arrive, by its own MMA thread, that
-    // arms each phase for the bytes of the two bulk copies from the decoder
-    mbar_init(&B.kh_full, 1);
-    mbar_init(&B.vh_full, 1);
+    // decoded-tile barriers: in the decoding CTA one arrive per epilogue
+    // warp; in the receiving CTA one expect_tx arrive, by its own MMA
+    // thread, that arms each phase for the bytes of the decoder's bulk copies
+    mbar_init(&B.kh_full, rank == 0 ? 4 : 1);
+    mbar_init(&B.vh_full, rank == 1 ? 4 : 1);
     mbar_init(&B.kh_empty, 2);
     mbar_init(&B.vh_empty, 2);
     for (int i = 0; i < 2; ++i) {
@@ -449,7 +447,6 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(384, 1)
       // bulk copy that carried it to the peer had completed before that)
       if (j > 0 && !mbar_wait_cluster(empty_bar, (j - 1) & 1, abort, err)) break;
       if (t == 0) FULL_TRACE(5, j);
-      bool ok = true;
 #pragma unroll
       for (int c = 0; c < NAT; ++c) {
         constexpr int G = DHR >= 64 ? 8 : DHR / 8;  // 8-column groups of a block (the last one may hold fewer)
@@ -460,24 +457,18 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(384, 1)
                          make_uint4(o[32 * c + 4 * g], o[32 * c + 4 * g + 1], o[32 * c + 4 * g + 2],
                                     o[32 * c + 4 * g + 3]));
         // columns [64c, 64c + 64) of every key form one 16 KB block of the
-        // tile: hand it to the local MMA / the peer as soon as it is complete
+        // tile, and this warp's 32 key rows of it are contiguous: each warp
+        // hands its rows to the peer as soon as it has stored them
         if (t == 0 && c == 0) FULL_TRACE(12, j);
         fence_proxy_async_smem();  // read by this CTA's MMA and by the bulk copy
-        if (t == 0 && c == 0) FULL_TRACE(13, j);
-        if (t == 96 && c == 0) FULL_TRACE(14, j);
         __syncwarp();
-        if (lane == 0) mbar_arrive(&B.half_done[c]);
-        if (t == 0) {
-          if (!mbar_wait(&B.half_done[c], j & 1, abort, err)) { ok = false; break; }
-          FULL_TRACE(15 + c, j);
-          bulk_s2cluster(dst_remote + c * (kTile / 2), dstL + c * (kTile / 2), kTile / 2, full_remote);
-          if (c == NAT - 1) {
-            mbar_arrive(full_bar);
-            FULL_TRACE(6, j);
-          }
+        if (lane == 0) {
+          const uint32_t off = c * (kTile / 2) + (uint32_t)(warp - 4) * 32 * 128;
+          bulk_s2cluster(dst_remote + off, dstL + off, 32 * 128, full_remote);
         }
       }
-      if (!ok) break;
+      if (lane == 0) mbar_arrive(full_bar);  // the local MMA may read this warp's rows
+      if (t == 0) FULL_TRACE(6, j);
     }
   } else if (warp >= 8) {
     // ---------------- softmax (thread = query row) ----------------
