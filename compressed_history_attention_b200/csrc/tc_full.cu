@@ -332,10 +332,12 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(384, 1)
         v[2 * i + 1] = __ldg(src + 1);
       }
     };
-    uint4 cur[4], nxt[4];
+    uint4 cur[4], nxt[4], nx2[4], nx3[4];
     load(0, cur);
+    if (1 < nchunk) load(1, nxt);
+    if (2 < nchunk) load(2, nx2);
     for (int c = 0; c < nchunk; ++c) {
-      if (c + 1 < nchunk) load(c + 1, nxt);
+      if (c + 3 < nchunk) load(c + 3, nx3);
       const int rs = c % nring, cb = c % nrb;
       if (warp == 2 && lane == 0 && cb == 0) FULL_TRACE(9, c / nrb);
       if (warp == 2 && lane == 0 && cb == 1) FULL_TRACE(17, c / nrb);
@@ -360,7 +362,11 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(384, 1)
       if (warp == 2 && lane == 0 && cb == nrb - 1) FULL_TRACE(11, c / nrb);
       if (warp == 2 && lane == 0 && cb == 1) FULL_TRACE(20, c / nrb);
 #pragma unroll
-      for (int k = 0; k < 4; ++k) cur[k] = nxt[k];
+      for (int k = 0; k < 4; ++k) {
+        cur[k] = nxt[k];
+        nxt[k] = nx2[k];
+        nx2[k] = nx3[k];
+      }
     }
   } else if (warp >= 4 && warp < 8) {
     // ---------------- decode epilogue (thread = key) ----------------
