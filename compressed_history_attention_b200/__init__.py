@@ -10,5 +10,5 @@ from ._lib import (  # noqa: F401
     nanokv_timing_enable,
     nanokv_timing_read, nanokv_version, nanokv_selftest_wait, nanokv_attend_full_tokens,
     nanokv_attend_routed, nanokv_attend_routed_workspace, Lowdim, nanokv_lowdim_prepare,
-    nanokv_lowdim_analytic, nanokv_calibrate,
+    nanokv_lowdim_analytic, nanokv_calibrate, nanokv_attend_partial,
 )

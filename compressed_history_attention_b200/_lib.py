@@ -26,7 +26,7 @@ SYMBOLS = ("nanokv_encode", "nanokv_attend", "nanokv_attend_workspace", "nanokv_
            "nanokv_codec_prepare", "nanokv_attend_static", "nanokv_selftest_wait",
            "nanokv_attend_full_tokens", "nanokv_attend_routed", "nanokv_attend_routed_workspace",
            "nanokv_lowdim_aux_bytes", "nanokv_lowdim_prepare", "nanokv_lowdim_analytic",
-           "nanokv_calibrate_workspace", "nanokv_calibrate")
+           "nanokv_calibrate_workspace", "nanokv_calibrate", "nanokv_attend_partial")
 
 # kernel identities of the diagnostics (nanokv_kernel_id)
 KERNELS = {0: "encode", 1: "attend_full", 2: "attend_low", 3: "attend_dense", 4: "lse_merge"}
@@ -123,6 +123,8 @@ def lib() -> ctypes.CDLL:
     L.nanokv_calibrate_workspace.restype = sz
     L.nanokv_calibrate.argtypes = [vp, i32, i64, i32, i32, i32, vp, i32, vp, vp, vp, vp, vp, vp, sz, vp]
     L.nanokv_calibrate.restype = ctypes.c_int
+    L.nanokv_attend_partial.argtypes = L.nanokv_attend.argtypes
+    L.nanokv_attend_partial.restype = ctypes.c_int
     _lib = L
     return L
 
@@ -438,6 +440,35 @@ def nanokv_attend_static(q: torch.Tensor, ck: Codec, cv: Codec, hk: Hist | None,
         ctypes.byref(shk) if shk else None, ctypes.byref(shv) if shv else None, T, T_full,
         _ptr(k_cur), _ptr(v_cur), T_cur, ctypes.c_float(softmax_scale), _ptr(out), _ptr(lse),
         _stream(q.device))
+    _raise(st)
+    return out, lse
+
+
+def nanokv_attend_partial(q: torch.Tensor, ck: Codec, cv: Codec, hk: Hist | None, hv: Hist | None,
+                          T_full: int, k_cur: torch.Tensor | None = None, v_cur: torch.Tensor | None = None,
+                          softmax_scale: float | None = None, workspace: torch.Tensor | None = None):
+    """nanokv_attend with an fp32 output: the partial (O [Tq, H, d] fp32,
+    LSE [H, Tq]) over this call's keys, for an LSE merge with partials over
+    other keys (nanokv_attend_partial)."""
+    Tq, H, d = q.shape
+    T = len(hk) if hk is not None else 0
+    T_cur = k_cur.shape[0] if k_cur is not None else 0
+    if softmax_scale is None:
+        softmax_scale = 1.0 / math.sqrt(d)
+    dev = q.device
+    out = torch.empty(Tq, H, d, dtype=torch.float32, device=dev)
+    lse = torch.empty(H, Tq, dtype=torch.float32, device=dev)
+    need = nanokv_attend_workspace(Tq, ck, cv, T, T_full, T_cur)
+    if workspace is None or workspace.numel() * workspace.element_size() < need:
+        workspace = torch.empty(max(need, 16), dtype=torch.uint8, device=dev)
+    sk, sv = ck.struct(), cv.struct()
+    shk = hk.struct() if hk is not None and T else None
+    shv = hv.struct() if hv is not None and T else None
+    st = lib().nanokv_attend_partial(
+        _ptr(q), _dt(q), Tq, ctypes.byref(sk), ctypes.byref(sv),
+        ctypes.byref(shk) if shk else None, ctypes.byref(shv) if shv else None, T, T_full,
+        _ptr(k_cur), _ptr(v_cur), T_cur, ctypes.c_float(softmax_scale), _ptr(out), _ptr(lse),
+        _ptr(workspace), workspace.numel() * workspace.element_size(), _stream(dev))
     _raise(st)
     return out, lse
 

@@ -502,12 +502,13 @@ size_t nanokv_attend_workspace(int64_t Tq, const nanokv_codec *ck, const nanokv_
   return ws_layout(Tq, a, T - T_full, T_full, T_cur, tc_low, splits).total;
 }
 
-int nanokv_attend(const void *q, int32_t io_dtype, int64_t Tq, const nanokv_codec *ck_,
-                  const nanokv_codec *cv_, const nanokv_hist *hk_, const nanokv_hist *hv_,
-                  int64_t T, int64_t T_full, const void *k_cur, const void *v_cur, int64_t T_cur,
-                  float softmax_scale, void *out, float *lse_out, void *workspace,
-                  size_t workspace_bytes, void *stream) {
-  ApiRange range("nanokv_attend");
+// nanokv_attend, with its output in the codecs' precision (out_f32 false) or
+// in fp32 (nanokv_attend_partial)
+static int attend_impl(const void *q, int32_t io_dtype, int64_t Tq, const nanokv_codec *ck_,
+                       const nanokv_codec *cv_, const nanokv_hist *hk_, const nanokv_hist *hv_, int64_t T,
+                       int64_t T_full, const void *k_cur, const void *v_cur, int64_t T_cur, float softmax_scale,
+                       void *out, float *lse_out, void *workspace, size_t workspace_bytes, void *stream,
+                       bool out_f32) {
   Codec ck, cv;
   int s;
   if ((s = check_codec(ck_, "attend ck", false, &ck))) return s;
@@ -639,8 +640,29 @@ int nanokv_attend(const void *q, int32_t io_dtype, int64_t Tq, const nanokv_code
   }
   if (lk.owns_lock()) lk.unlock();
   e = timed(NANOKV_K_MERGE, 1, st,
-            [&] { return lse_merge_launch(pl, Tq, ck.H, ck.d, out, ck.prec, lse_out, st); });
+            [&] { return lse_merge_launch(pl, Tq, ck.H, ck.d, out, out_f32 ? (int)PREC_F32 : ck.prec, lse_out, st); });
   return cuda_status(e, "attend merge launch");
+}
+
+int nanokv_attend(const void *q, int32_t io_dtype, int64_t Tq, const nanokv_codec *ck_,
+                  const nanokv_codec *cv_, const nanokv_hist *hk_, const nanokv_hist *hv_,
+                  int64_t T, int64_t T_full, const void *k_cur, const void *v_cur, int64_t T_cur,
+                  float softmax_scale, void *out, float *lse_out, void *workspace,
+                  size_t workspace_bytes, void *stream) {
+  ApiRange range("nanokv_attend");
+  return attend_impl(q, io_dtype, Tq, ck_, cv_, hk_, hv_, T, T_full, k_cur, v_cur, T_cur, softmax_scale, out,
+                     lse_out, workspace, workspace_bytes, stream, false);
+}
+
+int nanokv_attend_partial(const void *q, int32_t io_dtype, int64_t Tq, const nanokv_codec *ck_,
+                          const nanokv_codec *cv_, const nanokv_hist *hk_, const nanokv_hist *hv_, int64_t T,
+                          int64_t T_full, const void *k_cur, const void *v_cur, int64_t T_cur,
+                          float softmax_scale, float *out, float *lse_out, void *workspace,
+                          size_t workspace_bytes, void *stream) {
+  ApiRange range("nanokv_attend_partial");
+  if (Tq > 0 && !lse_out) return fail(NANOKV_ERR_INVALID, "attend_partial: lse_out is required");
+  return attend_impl(q, io_dtype, Tq, ck_, cv_, hk_, hv_, T, T_full, k_cur, v_cur, T_cur, softmax_scale, out,
+                     lse_out, workspace, workspace_bytes, stream, true);
 }
 
 // How a routed call runs its two history sets.  `full_set`: the routed

@@ -181,6 +181,27 @@ int nanokv_attend_static(const void *q, int32_t io_dtype, int64_t Tq,
                          float softmax_scale, void *out, float *lse_out, void *stream);
 
 /*
+ * nanokv_attend_partial -- nanokv_attend with its output in fp32: the
+ * attention of the queries over THIS call's keys (its history, routed by
+ * T_full, and the current chunk if given) as a partial result (O, LSE) for
+ * an LSE merge with partials over other keys (nanokv_lse_merge; Fig. 4(d)).
+ * A history held in several pieces -- e.g. sharded across GPUs, one (O, LSE)
+ * exchange before the merge -- attends each piece with this call and merges
+ * the partials; pass the current chunk to exactly one piece.
+ *   out      device [Tq, H, d] fp32, 16-byte aligned
+ *   lse_out  device [H, Tq] fp32, required
+ * Everything else (arguments, workspace = nanokv_attend_workspace, errors)
+ * is as for nanokv_attend.
+ */
+int nanokv_attend_partial(const void *q, int32_t io_dtype, int64_t Tq,
+                          const nanokv_codec *ck, const nanokv_codec *cv,
+                          const nanokv_hist *hk, const nanokv_hist *hv,
+                          int64_t T, int64_t T_full,
+                          const void *k_cur, const void *v_cur, int64_t T_cur,
+                          float softmax_scale, float *out, float *lse_out,
+                          void *workspace, size_t workspace_bytes, void *stream);
+
+/*
  * nanokv_attend_routed -- nanokv_attend under a general full-dim routing
  * policy instead of "the most recent T_full tokens" (NanoKV-Fast, Table 7:
  * full-dimensional routing by recent frames, periodic anchor frames, sink

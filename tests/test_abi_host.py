@@ -280,3 +280,18 @@ def test_calibrate_validation():
     assert call(ws=16) == _lib.ERR_INVALID
     assert call(x=ctypes.c_void_p((1 << 20) + 4)) == _lib.ERR_INVALID
     assert call(x=None) == _lib.ERR_INVALID
+
+
+def test_attend_partial_validation():
+    """The fp32-partial attend checks its arguments like nanokv_attend and
+    requires the LSE output (a partial without it cannot be merged)."""
+    L = nk.lib()
+    c = _codec()
+    p = ctypes.c_void_p(1 << 20)
+    h = _lib._Hist(1 << 20, 1 << 20, 1 << 20)
+    call = lambda lse, T_full=8, Tq=4: L.nanokv_attend_partial(  # noqa: E731
+        p, _lib.F32, Tq, ctypes.byref(c), ctypes.byref(c), ctypes.byref(h), ctypes.byref(h), 8, T_full, None, None,
+        0, ctypes.c_float(0.25), p, lse, p, 1 << 20, None)
+    assert call(None) == _lib.ERR_INVALID
+    assert call(p, T_full=9) == _lib.ERR_INVALID
+    assert call(None, Tq=0) == _lib.OK
