@@ -75,3 +75,20 @@ def test_calibrate_matches_oracle(name):
             # within rounding of each other either sign is correct
             err = np.abs(v - u).max() if top[1] < 0.98 * top[0] else min(np.abs(v - u).max(), np.abs(v + u).max())
             assert err <= 2 * eps * top[0] + 1e-6 / gap + 1e-5, (i, gap, err)
+
+
+def test_calibrate_center_without_tokens_stays():
+    """An initial center far from every token keeps its place (and no token
+    is assigned to it), as in the oracle."""
+    w, rounds, r = CASES["small"]
+    x, init = _tokens(w)
+    init[3] = 1e3
+    got = nk.nanokv_calibrate(x, init, rounds, r)
+    torch.cuda.synchronize()
+    ids = got["ids"].cpu().numpy()
+    assert not (ids == 3).any()
+    assert torch.equal(got["centers"][3].float().cpu(), init[3].to(got["centers"].dtype).float().cpu())
+    orc = P.orc
+    ref = orc.calibrate(orc.f64(x), orc.f64(init), rounds, r)
+    ties = orc.argmin_ties(orc.f64(x), ref["centers"])
+    assert ((ids.astype(np.int64) == ref["ids"]) | ties).all()

@@ -209,3 +209,30 @@ def test_analytic_maps(name):
                 P2 = ref[h][:, :n] @ ref[h][:, :n].T
                 tol = 5e-3 + 1e-5 / max(gap, 1e-12)
                 assert np.abs(P1 - P2).max() < tol, (h, n, gap, np.abs(P1 - P2).max())
+
+
+def test_routed_many_ranges_and_empty_ones():
+    """The largest policy the ABI takes: 64 ranges (single tokens spread over
+    the history, some of count 0), against the oracle."""
+    w, prob, ck, cv, hk, hv, _, _ = _case("mixed_small", 0)
+    starts = np.linspace(0, w.T - 1, _lib.MAX_RANGES).astype(int)
+    full = [(int(s), 0 if i % 7 == 3 else 1) for i, s in enumerate(starts)]
+    O, L = nk.nanokv_attend_routed(prob["q"], ck, cv, hk, hv, full, None, prob["k_cur"], prob["v_cur"])
+    torch.cuda.synchronize()
+    Or, Lr = _oracle(w, prob, hk, hv, full, None)
+    P.compare_attn(O, L, Or, Lr, False)
+
+
+def test_routed_reduced_heads_without_low_tokens():
+    """With every history token routed full-dim, heads at reduced dimensions
+    have nothing to reduce: the call equals nanokv_attend with T_full = T
+    bit for bit."""
+    w, prob, ck, cv, hk, hv, _, _ = _case("mixed_small", 0)
+    U, W = _maps(w, 12)
+    ld = nk.nanokv_lowdim_prepare(ck, cv, U, W)
+    d_h = [32, 64, 96, 0] * (w.H // 4)
+    got = nk.nanokv_attend_routed(prob["q"], ck, cv, hk, hv, [(0, w.T)], None, prob["k_cur"], prob["v_cur"],
+                                  lowdim=ld, d_h=d_h)
+    ref = nk.nanokv_attend(prob["q"], ck, cv, hk, hv, w.T, prob["k_cur"], prob["v_cur"])
+    torch.cuda.synchronize()
+    assert torch.equal(got[0], ref[0]) and torch.equal(got[1], ref[1])
