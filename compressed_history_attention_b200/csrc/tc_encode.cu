@@ -598,62 +598,101 @@ __global__ void __launch_bounds__(384, 1)
 }
 
 // EC[j][k] = E[k] . c_j and |c_j|^2 in fp32, a small GEMM of the codec's
-// centers against its encoder.  A block stages 8 center rows and 16 encoder
-// rows (in 384-wide chunks of J, converted to fp32) in shared memory and
-// computes their 128 products, two threads per product (one per half of the
-// chunk, combined by a shuffle); the blocks of the first encoder tile also
-// form the squared norms of their centers.  Each center and encoder row is
-// read from global memory once per block that uses it.
-constexpr int kPrepC = 8, kPrepR = 16, kPrepJ = 384, kPrepLD = kPrepJ + 4;
+// centers against its encoder (2 C r J flops; reads dominate).  One block
+// per 4 centers x 8 encoder rows, its 8 warps over eighths of J: each lane
+// takes 8-element (16-byte) groups, keeps the 4 center and 8 encoder values
+// of a group in registers and accumulates the 32 products and the 4
+// squared norms; the sums meet by warp shuffles and then across the warps
+// in shared memory.  Each row is read once per block that uses it.
+template <typename TP>
+__device__ __forceinline__ void load8f(const TP *p, float (&v)[8]);
+template <>
+__device__ __forceinline__ void load8f<__nv_bfloat16>(const __nv_bfloat16 *p, float (&v)[8]) {
+  const uint4 w = __ldg(reinterpret_cast<const uint4 *>(p));
+  const uint32_t u[4] = {w.x, w.y, w.z, w.w};
+#pragma unroll
+  for (int i = 0; i < 4; ++i) {
+    const float2 f = __bfloat1622float2(*reinterpret_cast<const __nv_bfloat162 *>(&u[i]));
+    v[2 * i] = f.x;
+    v[2 * i + 1] = f.y;
+  }
+}
+template <>
+__device__ __forceinline__ void load8f<float>(const float *p, float (&v)[8]) {
+  const float4 a = __ldg(reinterpret_cast<const float4 *>(p)), b = __ldg(reinterpret_cast<const float4 *>(p) + 1);
+  v[0] = a.x; v[1] = a.y; v[2] = a.z; v[3] = a.w;
+  v[4] = b.x; v[5] = b.y; v[6] = b.z; v[7] = b.w;
+}
+
+constexpr int kPrepC = 4, kPrepR = 8;  // centers x encoder rows per block
+constexpr int kPrepW = 8;              // warps per block, each over 1/8 of J
 
 template <typename TP>
 __global__ void __launch_bounds__(256) codec_prepare_kernel(const TP *__restrict__ cen, const TP *__restrict__ E,
                                                             int C, int r, int J, float *__restrict__ aux) {
-  __shared__ __align__(16) float cs[kPrepC][kPrepLD];
-  __shared__ __align__(16) float es[kPrepR][kPrepLD];
-  const int j0 = blockIdx.x * kPrepC, k0 = blockIdx.y * kPrepR;
-  const int t = threadIdx.x, o = t & 127, half = t >> 7;
-  const int jj = o / kPrepR, kk = o % kPrepR;
-  const int warp = t >> 5, lane = t & 31;
-  float acc = 0.f, nrm = 0.f;
-  for (int c0 = 0; c0 < J; c0 += kPrepJ) {
-    const int n = J - c0 < kPrepJ ? J - c0 : kPrepJ;
-    for (int idx = t; idx < (kPrepC + kPrepR) * kPrepJ; idx += 256) {
-      const int row = idx / kPrepJ, i = idx % kPrepJ;
-      float v = 0.f;
-      if (i < n) {
-        if (row < kPrepC) {
-          if (j0 + row < C) v = to_f(cen[(size_t)(j0 + row) * J + c0 + i]);
-        } else if (k0 + row - kPrepC < r) {
-          v = to_f(E[(size_t)(k0 + row - kPrepC) * J + c0 + i]);
-        }
-      }
-      if (row < kPrepC) cs[row][i] = v;
-      else es[row - kPrepC][i] = v;
-    }
-    __syncthreads();
-    const float *a = cs[jj] + half * (kPrepJ / 2), *b = es[kk] + half * (kPrepJ / 2);
-#pragma unroll 4
-    for (int i = 0; i < kPrepJ / 2; i += 4) {
-      const float4 x = *reinterpret_cast<const float4 *>(a + i), y = *reinterpret_cast<const float4 *>(b + i);
-      acc = fmaf(x.x, y.x, acc);
-      acc = fmaf(x.y, y.y, acc);
-      acc = fmaf(x.z, y.z, acc);
-      acc = fmaf(x.w, y.w, acc);
-    }
-    if (blockIdx.y == 0)  // warp w: center j0 + w
-      for (int i = lane; i < kPrepJ; i += 32) nrm = fmaf(cs[warp][i], cs[warp][i], nrm);
-    __syncthreads();
+  __shared__ float part[kPrepW][kPrepC * kPrepR + kPrepC];
+  const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
+  const int nkg = (r + kPrepR - 1) / kPrepR;
+  const int j0 = (blockIdx.x / nkg) * kPrepC, k0 = (blockIdx.x % nkg) * kPrepR;
+  // this warp's slice of J, in 8-element groups
+  const int ng = J / 8, g0 = (ng * warp) / kPrepW, g1 = (ng * (warp + 1)) / kPrepW;
+  float acc[kPrepC][kPrepR], nrm[kPrepC];
+#pragma unroll
+  for (int a = 0; a < kPrepC; ++a) {
+    nrm[a] = 0.f;
+#pragma unroll
+    for (int b = 0; b < kPrepR; ++b) acc[a][b] = 0.f;
   }
-  // the two halves of each product are threads t and t + 128: combine
-  // through shared memory (reusing the staging buffer)
-  float *part = &cs[0][0];
-  if (half) part[o] = acc;
+  for (int g = g0 + lane; g < g1; g += 32) {
+    const int i = 8 * g;
+    float c[kPrepC][8], e[kPrepR][8];
+#pragma unroll
+    for (int a = 0; a < kPrepC; ++a) {
+      if (j0 + a < C) load8f(cen + (size_t)(j0 + a) * J + i, c[a]);
+      else
+#pragma unroll
+        for (int q = 0; q < 8; ++q) c[a][q] = 0.f;
+    }
+#pragma unroll
+    for (int b = 0; b < kPrepR; ++b) {
+      if (k0 + b < r) load8f(E + (size_t)(k0 + b) * J + i, e[b]);
+      else
+#pragma unroll
+        for (int q = 0; q < 8; ++q) e[b][q] = 0.f;
+    }
+#pragma unroll
+    for (int a = 0; a < kPrepC; ++a)
+#pragma unroll
+      for (int q = 0; q < 8; ++q) {
+        nrm[a] = fmaf(c[a][q], c[a][q], nrm[a]);
+#pragma unroll
+        for (int b = 0; b < kPrepR; ++b) acc[a][b] = fmaf(c[a][q], e[b][q], acc[a][b]);
+      }
+  }
+  // lanes, then warps
+#pragma unroll
+  for (int a = 0; a < kPrepC; ++a) {
+#pragma unroll
+    for (int b = 0; b < kPrepR; ++b) {
+      const float v = warp_sum(acc[a][b]);
+      if (lane == 0) part[warp][a * kPrepR + b] = v;
+    }
+    const float v = warp_sum(nrm[a]);
+    if (lane == 0) part[warp][kPrepC * kPrepR + a] = v;
+  }
   __syncthreads();
-  if (!half && j0 + jj < C && k0 + kk < r) aux[(size_t)(j0 + jj) * r + k0 + kk] = acc + part[o];
-  if (blockIdx.y == 0) {
-    nrm = warp_sum(nrm);
-    if (lane == 0 && j0 + warp < C) aux[(size_t)C * r + j0 + warp] = nrm;
+  const int o = threadIdx.x;
+  if (o < kPrepC * kPrepR + kPrepC) {
+    float v = 0.f;
+#pragma unroll
+    for (int w = 0; w < kPrepW; ++w) v += part[w][o];
+    if (o < kPrepC * kPrepR) {
+      const int a = o / kPrepR, b = o % kPrepR;
+      if (j0 + a < C && k0 + b < r) aux[(size_t)(j0 + a) * r + k0 + b] = v;
+    } else {
+      const int a = o - kPrepC * kPrepR;
+      if (k0 == 0 && j0 + a < C) aux[(size_t)C * r + j0 + a] = v;
+    }
   }
 }
 
@@ -664,7 +703,7 @@ size_t codec_aux_bytes(const Codec &c) {
 }
 
 cudaError_t codec_prepare(const Codec &c, void *aux, cudaStream_t st) {
-  const dim3 grid((unsigned)((c.C + kPrepC - 1) / kPrepC), (unsigned)((c.r + kPrepR - 1) / kPrepR));
+  const dim3 grid((unsigned)(((c.C + kPrepC - 1) / kPrepC) * ((c.r + kPrepR - 1) / kPrepR)));
   if (c.prec == PREC_F32)
     codec_prepare_kernel<float><<<grid, 256, 0, st>>>((const float *)c.centers, (const float *)c.E, c.C, c.r,
                                                       c.H * c.d, (float *)aux);
