@@ -252,7 +252,7 @@ typedef struct {
  *   U, W  device [H, d, d] row-major bf16, 16-byte aligned, caller-owned:
  *         head h's map in columns [0, d_h[h]) of U[h] / W[h] (the leading
  *         columns, so maps ordered by importance serve every d_h).
- *   aux   device buffer of nanokv_lowdim_aux_bytes() bytes, 256-byte aligned,
+ *   aux   device buffer of nanokv_lowdim_aux_bytes() bytes, 16-byte aligned,
  *         caller-owned: the mapped decoder rows and centers of both branches,
  *         written by nanokv_lowdim_prepare; valid while U, W and the codecs'
  *         D / centers are unchanged.
