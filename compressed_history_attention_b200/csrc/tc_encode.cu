@@ -597,87 +597,121 @@ __global__ void __launch_bounds__(384, 1)
   }
 }
 
-// EC[j][k] = E[k] . c_j and |c_j|^2 in fp32, a small GEMM of the codec's
-// centers against its encoder (2 C r J flops; reads dominate).  One warp
-// per 4 centers x 8 encoder rows: each lane takes 8-element (16-byte)
-// groups of J, keeps the 4 center and 8 encoder values of a group in
-// registers and accumulates the 32 products (and, in the warps of the first
-// encoder rows, the 4 squared norms); the sums meet by warp shuffles.  Each
-// row is read once per warp that uses it.  (Splitting J over a block's
-// warps, combined in shared memory, measured slower: 12.9 against 10.7 us
-// at the full codec, 108 against 41 us at the long one.)
-template <typename TP>
-__device__ __forceinline__ void load8f(const TP *p, float (&v)[8]);
-template <>
-__device__ __forceinline__ void load8f<__nv_bfloat16>(const __nv_bfloat16 *p, float (&v)[8]) {
-  const uint4 w = __ldg(reinterpret_cast<const uint4 *>(p));
-  const uint32_t u[4] = {w.x, w.y, w.z, w.w};
-#pragma unroll
-  for (int i = 0; i < 4; ++i) {
-    const float2 f = __bfloat1622float2(*reinterpret_cast<const __nv_bfloat162 *>(&u[i]));
-    v[2 * i] = f.x;
-    v[2 * i + 1] = f.y;
-  }
-}
-template <>
-__device__ __forceinline__ void load8f<float>(const float *p, float (&v)[8]) {
-  const float4 a = __ldg(reinterpret_cast<const float4 *>(p)), b = __ldg(reinterpret_cast<const float4 *>(p) + 1);
-  v[0] = a.x; v[1] = a.y; v[2] = a.z; v[3] = a.w;
-  v[4] = b.x; v[5] = b.y; v[6] = b.z; v[7] = b.w;
-}
+// EC[j][k] = E[k] . c_j and |c_j|^2 in fp32: a small GEMM of the codec's
+// centers against its encoder (2 C r J flops; reads dominate), once per codec.
 
-constexpr int kPrepC = 4, kPrepR = 8;  // centers x encoder rows per warp
+// 8 consecutive parameters as they are stored: 16 bytes of bf16 or 32 of fp32
+template <typename TP>
+struct Raw8;
+template <>
+struct Raw8<__nv_bfloat16> {
+  uint4 w;
+  __device__ __forceinline__ void load(const __nv_bfloat16 *p) { w = __ldg(reinterpret_cast<const uint4 *>(p)); }
+  __device__ __forceinline__ void zero() { w = make_uint4(0, 0, 0, 0); }
+  __device__ __forceinline__ float get(int q) const {
+    const uint32_t u = q < 2 ? w.x : q < 4 ? w.y : q < 6 ? w.z : w.w;
+    return __uint_as_float((q & 1) ? (u & 0xffff0000u) : (u << 16));
+  }
+};
+template <>
+struct Raw8<float> {
+  float4 a, b;
+  __device__ __forceinline__ void load(const float *p) {
+    a = __ldg(reinterpret_cast<const float4 *>(p));
+    b = __ldg(reinterpret_cast<const float4 *>(p) + 1);
+  }
+  __device__ __forceinline__ void zero() { a = b = make_float4(0.f, 0.f, 0.f, 0.f); }
+  __device__ __forceinline__ float get(int q) const {
+    const float4 &v = q < 4 ? a : b;
+    const int k = q & 3;
+    return k == 0 ? v.x : k == 1 ? v.y : k == 2 ? v.z : v.w;
+  }
+};
+
+// E c_j and |c_j|^2, one 8 x 8 tile of (center, encoder row) pairs per block.
+// Each thread loads its 8-element slices of the tile's 8 center rows and 8
+// encoder rows (every load of a pass in flight at once: one pass covers
+// J = 1536), kept as stored, and forms the 64 partial dot products in fp32
+// element by element; the block then sums them in a fixed order: a shuffle
+// reduce-scatter inside each warp (after which lane L holds the warp's sums
+// of products 2L and 2L + 1), then the warps in order.  The norms come from
+// the blocks of the first column.  Two blocks fit an SM.
+constexpr int kPrepT = 8;    // centers (and encoder rows) per tile
+constexpr int kPrepNT = 192;  // threads per block
 
 template <typename TP>
-__global__ void __launch_bounds__(128) codec_prepare_kernel(const TP *__restrict__ cen, const TP *__restrict__ E,
-                                                            int C, int r, int J, float *__restrict__ aux) {
-  const int lane = threadIdx.x & 31;
-  const int nkg = (r + kPrepR - 1) / kPrepR;
-  const int wid = blockIdx.x * 4 + (threadIdx.x >> 5);
-  if (wid >= ((C + kPrepC - 1) / kPrepC) * nkg) return;
-  const int j0 = (wid / nkg) * kPrepC, k0 = (wid % nkg) * kPrepR;
-  float acc[kPrepC][kPrepR], nrm[kPrepC];
+__global__ void __launch_bounds__(kPrepNT, sizeof(TP) == 2 ? 2 : 1)
+    codec_prepare_kernel(const TP *__restrict__ cen, const TP *__restrict__ E, int C, int r, int J,
+                         float *__restrict__ aux) {
+  constexpr int NW = kPrepNT / 32;
+  __shared__ float red[NW][kPrepT * kPrepT + kPrepT];
+  const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
+  const int k0 = blockIdx.x * kPrepT, j0 = blockIdx.y * kPrepT;
+  const bool norms = blockIdx.x == 0;
+  float acc[kPrepT * kPrepT], nrm[kPrepT];
 #pragma unroll
-  for (int a = 0; a < kPrepC; ++a) {
-    nrm[a] = 0.f;
+  for (int i = 0; i < kPrepT * kPrepT; ++i) acc[i] = 0.f;
 #pragma unroll
-    for (int b = 0; b < kPrepR; ++b) acc[a][b] = 0.f;
-  }
-  for (int i = lane * 8; i < J; i += 256) {
-    float c[kPrepC][8], e[kPrepR][8];
+  for (int a = 0; a < kPrepT; ++a) nrm[a] = 0.f;
+  for (int i = threadIdx.x * 8; i < J; i += kPrepNT * 8) {
+    Raw8<TP> c[kPrepT], e[kPrepT];
 #pragma unroll
-    for (int a = 0; a < kPrepC; ++a) {
-      if (j0 + a < C) load8f(cen + (size_t)(j0 + a) * J + i, c[a]);
-      else
-#pragma unroll
-        for (int q = 0; q < 8; ++q) c[a][q] = 0.f;
+    for (int a = 0; a < kPrepT; ++a) {
+      if (j0 + a < C) c[a].load(cen + (size_t)(j0 + a) * J + i);
+      else c[a].zero();
     }
 #pragma unroll
-    for (int b = 0; b < kPrepR; ++b) {
-      if (k0 + b < r) load8f(E + (size_t)(k0 + b) * J + i, e[b]);
-      else
-#pragma unroll
-        for (int q = 0; q < 8; ++q) e[b][q] = 0.f;
+    for (int b = 0; b < kPrepT; ++b) {
+      if (k0 + b < r) e[b].load(E + (size_t)(k0 + b) * J + i);
+      else e[b].zero();
     }
 #pragma unroll
-    for (int a = 0; a < kPrepC; ++a)
+    for (int q = 0; q < 8; ++q) {
+      float cq[kPrepT], eq[kPrepT];
 #pragma unroll
-      for (int q = 0; q < 8; ++q) {
-        nrm[a] = fmaf(c[a][q], c[a][q], nrm[a]);
+      for (int a = 0; a < kPrepT; ++a) cq[a] = c[a].get(q);
 #pragma unroll
-        for (int b = 0; b < kPrepR; ++b) acc[a][b] = fmaf(c[a][q], e[b][q], acc[a][b]);
+      for (int b = 0; b < kPrepT; ++b) eq[b] = e[b].get(q);
+#pragma unroll
+      for (int a = 0; a < kPrepT; ++a) {
+        nrm[a] = fmaf(cq[a], cq[a], nrm[a]);
+#pragma unroll
+        for (int b = 0; b < kPrepT; ++b) acc[a * kPrepT + b] = fmaf(cq[a], eq[b], acc[a * kPrepT + b]);
       }
-  }
-#pragma unroll
-  for (int a = 0; a < kPrepC; ++a) {
-#pragma unroll
-    for (int b = 0; b < kPrepR; ++b) {
-      const float v = warp_sum(acc[a][b]);
-      if (lane == 0 && j0 + a < C && k0 + b < r) aux[(size_t)(j0 + a) * r + k0 + b] = v;
     }
-    if (k0 == 0) {
+  }
+  // reduce-scatter over the warp: at offset o each lane keeps the half of its
+  // values selected by its lane bit o and adds the partner's copy of that half
+#pragma unroll
+  for (int o = 16, n = 32; o >= 1; o >>= 1, n >>= 1) {
+    const bool hi = (lane & o) != 0;
+#pragma unroll
+    for (int i = 0; i < n; ++i) {
+      const float send = hi ? acc[i] : acc[i + n];
+      const float keep = hi ? acc[i + n] : acc[i];
+      acc[i] = keep + __shfl_xor_sync(0xffffffffu, send, o);
+    }
+  }
+  red[warp][2 * lane] = acc[0];
+  red[warp][2 * lane + 1] = acc[1];
+  if (norms) {
+#pragma unroll
+    for (int a = 0; a < kPrepT; ++a) {
       const float v = warp_sum(nrm[a]);
-      if (lane == 0 && j0 + a < C) aux[(size_t)C * r + j0 + a] = v;
+      if (lane == 0) red[warp][kPrepT * kPrepT + a] = v;
+    }
+  }
+  __syncthreads();
+  const int t = threadIdx.x;
+  if (t < kPrepT * kPrepT + (norms ? kPrepT : 0)) {
+    float v = 0.f;
+#pragma unroll
+    for (int w = 0; w < NW; ++w) v += red[w][t];
+    if (t < kPrepT * kPrepT) {
+      const int a = t / kPrepT, b = t % kPrepT;
+      if (j0 + a < C && k0 + b < r) aux[(size_t)(j0 + a) * r + k0 + b] = v;
+    } else if (j0 + t - kPrepT * kPrepT < C) {
+      aux[(size_t)C * r + j0 + t - kPrepT * kPrepT] = v;
     }
   }
 }
@@ -689,13 +723,12 @@ size_t codec_aux_bytes(const Codec &c) {
 }
 
 cudaError_t codec_prepare(const Codec &c, void *aux, cudaStream_t st) {
-  const int warps = ((c.C + kPrepC - 1) / kPrepC) * ((c.r + kPrepR - 1) / kPrepR);
-  const dim3 grid((unsigned)((warps + 3) / 4));
+  const dim3 grid((unsigned)((c.r + kPrepT - 1) / kPrepT), (unsigned)((c.C + kPrepT - 1) / kPrepT));
   if (c.prec == PREC_F32)
-    codec_prepare_kernel<float><<<grid, 128, 0, st>>>((const float *)c.centers, (const float *)c.E, c.C, c.r,
-                                                      c.H * c.d, (float *)aux);
+    codec_prepare_kernel<float><<<grid, kPrepNT, 0, st>>>((const float *)c.centers, (const float *)c.E, c.C, c.r,
+                                                          c.H * c.d, (float *)aux);
   else
-    codec_prepare_kernel<__nv_bfloat16><<<grid, 128, 0, st>>>(
+    codec_prepare_kernel<__nv_bfloat16><<<grid, kPrepNT, 0, st>>>(
         (const __nv_bfloat16 *)c.centers, (const __nv_bfloat16 *)c.E, c.C, c.r, c.H * c.d, (float *)aux);
   return cudaGetLastError();
 }
