@@ -48,7 +48,7 @@ NCU_TRAFFIC = {
     ("attend_low", "long"): ("tc_low_pair", "1af5729c0430d001", 71728100 + 27869668),
     ("attend_low", "mixed"): ("tc_low", "d15b7a8cf47b4f75", 17933966 + 19342),
     ("attend_dense", "full"): ("tc_dense", "bc840a866ba6a1e1", 43226496 + 128366),
-    ("encode", "full"): ("tc_encode", "c7e3bff988e11590", 30490829 + 0),
+    ("encode", "full"): ("tc_encode", "70d83cae2d835770", 30490368 + 0),
 }
 
 
