@@ -602,3 +602,39 @@ def test_calibrated_codec_is_exact_on_low_rank_residuals():
     rho = x - cal["centers"][cal["ids"]]
     assert np.allclose(rho @ cal["D"] @ cal["E"], rho, atol=1e-10)
     assert np.allclose(cal["E"], cal["D"].T)
+
+
+def test_zero_residual_tie_rule_of_the_encode_comparison():
+    """The encode comparison's rule for residuals within rounding of zero,
+    checked on the CPU with encodes made by the oracle: tokens on a center
+    are counted and may carry any codes under a scale at the rounding floor;
+    a larger scale fails, and ordinary tokens are never counted."""
+    import torch
+    from compressed_history_attention_b200._lib import Hist
+    from tests import _parity as P
+
+    rng = np.random.default_rng(3)
+    C, J, r = 8, 64, 8
+    cen = orc.f64(torch.tensor(rng.standard_normal((C, J)), dtype=torch.bfloat16))
+    E = orc.f64(torch.tensor(rng.standard_normal((r, J)) / np.sqrt(J), dtype=torch.bfloat16))
+    x = np.concatenate([cen, cen[:2] + rng.standard_normal((2, J))])
+    codec = {"centers": torch.tensor(cen), "E": torch.tensor(E)}
+    xt = torch.tensor(x)
+    ref = orc.encode(x, cen, E, "f16")
+
+    def hist(scales, codes):
+        return Hist(torch.tensor(ref["ids"].astype(np.uint8)), torch.tensor(orc.pack_codes(codes)),
+                    torch.tensor(scales.astype(np.float16)))
+
+    ties = P.check_encode(xt, codec, hist(ref["scales"], ref["codes"]), "f16")
+    assert ties["zero_residual_ties"] == C  # the on-center tokens, not the others
+    # on-center tokens with a scale at the fp16 floor and arbitrary codes pass
+    s = ref["scales"].copy()
+    s[:C] = 2.0 ** -24
+    codes = ref["codes"].copy()
+    codes[:C] = rng.integers(-7, 8, (C, r))
+    P.check_encode(xt, codec, hist(s, codes), "f16")
+    # a scale well above the rounding bound fails
+    s[0] = 1e-2
+    with pytest.raises(AssertionError):
+        P.check_encode(xt, codec, hist(s, codes), "f16")
