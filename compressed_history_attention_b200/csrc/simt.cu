@@ -83,8 +83,13 @@ cudaError_t simt_encode(const Codec &c, const void *x, int64_t T, uint8_t *ids, 
                         void *scales, cudaStream_t st) {
   if (T == 0) return cudaSuccess;
   const int J = c.H * c.d;
-  const int wpb = 8;
-  const size_t smem = (size_t)wpb * (J + c.r) * sizeof(float);
+  // warps per block: up to 8, as many as the per-warp token and residual
+  // buffers (J + r floats each) leave room for in 227 KB of shared memory;
+  // the widest codec (J = 32768, r = 512) runs one warp per block
+  const size_t per_warp = (size_t)(J + c.r) * sizeof(float);
+  int wpb = (int)(size_t(232448) / per_warp);
+  wpb = wpb < 1 ? 1 : (wpb > 8 ? 8 : wpb);
+  const size_t smem = (size_t)wpb * per_warp;
   int64_t blocks = (T + wpb - 1) / wpb;
   if (blocks > 148 * 16) blocks = 148 * 16;
   if (c.prec == PREC_F32) {

@@ -106,3 +106,26 @@ def test_attend_zero_queries(name, path):
     assert np.abs(lse - np.log(n)).max() <= (1e-5 if w.fp32 else 2e-3) * max(1.0, np.log(n))
     Or, Lr = P.oracle_attend(w, prob, hk, hv, w.T_full)
     P.compare_attn(O, L, Or, Lr, w.fp32)
+
+
+# The widest codec the ABI takes (H = 256 heads of d = 128: J = 32768) and
+# the largest rank with the most centers (r = 512, C = 256), which no
+# tensor-core kernel covers: both kernel families, encode and attend.
+EXTREMES = {
+    "widest": scaled(WORKLOADS["mixed"], H=256, C=16, r=64, rank=48, T=256, T_full=128, Tq=64),
+    "max_rank": scaled(WORKLOADS["mixed"], H=8, C=256, r=512, rank=160, T=300, T_full=100, Tq=64),
+}
+
+
+@pytest.mark.parametrize("name", sorted(EXTREMES))
+def test_extreme_codec_shapes(name, path):
+    w = EXTREMES[name]
+    prob = P.problem(w)
+    ck, cv, hk, hv = P.encode_history(w, prob)
+    torch.cuda.synchronize()
+    for x, c, h in ((prob["hist_k"], prob["codec_k"], hk), (prob["hist_v"], prob["codec_v"], hv)):
+        P.check_encode(x, c, h, _sd(w))
+    O, L = nk.nanokv_attend(prob["q"], ck, cv, hk, hv, w.T_full, prob["k_cur"], prob["v_cur"])
+    torch.cuda.synchronize()
+    Or, Lr = P.oracle_attend(w, prob, hk, hv, w.T_full)
+    P.compare_attn(O, L, Or, Lr, w.fp32)
