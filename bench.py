@@ -437,8 +437,22 @@ def run_ours(a, rank, world, device):
         "clocks": clocks, "e2e": e2e, "gpu_launches": launches, "roofline": roof,
         "cpu_baseline": cpu, "parity": parity, "fast": fast, "long": long_, "fast_reduced": reduced,
         "step30": step30,
+        "storage": storage_block(w),
     }
     return line
+
+
+def storage_block(w) -> dict:
+    """The compressed history's size against the uncompressed K/V cache of
+    the workload (bf16, or fp32 in the fp32 mode): per token, and for the
+    whole history with the codec parameters counted."""
+    from compressed_history_attention_b200.accounting import storage
+    b = 4 if w.fp32 else 2
+    st = storage(w.T, w.H, w.d, w.r, w.C, x_bytes=b, param_bytes=b, scale_bytes=b)
+    return {"history_tokens": w.T, "raw_mb": round(st["raw_bytes"] / 1e6, 3),
+            "compressed_mb": round(st["compressed_bytes"] / 1e6, 3), "codec_mb": round(st["codec_bytes"] / 1e6, 3),
+            "per_token_ratio": round(st["per_token_ratio"], 2), "effective_ratio": round(st["effective_ratio"], 2),
+            "effective_ratio_with_encoder": round(st["effective_ratio_with_encoder"], 2)}
 
 
 def run_e2e(s, w, a, device, flops, world):

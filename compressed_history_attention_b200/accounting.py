@@ -61,3 +61,27 @@ def routed_flops(Tq: int, H: int, d: int, r: int, C: int, T_full: int, T_low: in
     out = {"full": base["full"] + full_low, "low": low, "reduced": red, "current": base["current"]}
     out["total"] = out["full"] + out["low"] + out["reduced"] + out["current"]
     return out
+
+
+def storage(T: int, H: int, d: int, r: int, C: int, x_bytes: int = 2, param_bytes: int = 2,
+            scale_bytes: int = 2) -> dict:
+    """Storage of a compressed history of T tokens (K and V), against the
+    uncompressed cache (the pages' KV compression ratio, counted here for
+    this layout): per token, J values of x_bytes against an id, r/2 bytes
+    of codes and a scale; for the whole history, the two branches' codec
+    parameters added (centers [C, J] and decoder D [J, r]; the encoder E,
+    which attention never reads, in the second figure)."""
+    J = H * d
+    raw = 2 * T * J * x_bytes
+    coded = 2 * T * token_bytes(r, scale_bytes)
+    centers_d = 2 * (C * J + J * r) * param_bytes
+    enc = 2 * r * J * param_bytes
+    return {
+        "raw_bytes": raw,
+        "compressed_bytes": coded,
+        "codec_bytes": centers_d,
+        "encoder_bytes": enc,
+        "per_token_ratio": (J * x_bytes) / token_bytes(r, scale_bytes),
+        "effective_ratio": raw / (coded + centers_d) if T else 0.0,
+        "effective_ratio_with_encoder": raw / (coded + centers_d + enc) if T else 0.0,
+    }

@@ -94,3 +94,22 @@ def test_routed_work_accounting():
     assert one["reduced"] == 4 * Tq * Tl * 32 + 4 * Tl * 32 * r + 4 * Tq * d * 32
     assert one["low"] == base["low"] * (H - 1) // H
     assert one["total"] < base["total"]
+
+
+@pytest.mark.parametrize("name,per_token,effective,with_encoder", [
+    # bf16 K/V of J values per token against 1 id byte + r/2 code bytes + a
+    # 2-byte scale; the effective figures add the two branches' centers and
+    # decoders (and encoders): e.g. full, T = 14040, J = 1536, C = 64, r = 192:
+    # 2*14040*3072 / (2*14040*99 + 2*(64*1536 + 1536*192)*2) = 19.82
+    ("full", 3072 / 99, 86261760 / (2779920 + 1572864), 86261760 / (2779920 + 1572864 + 1179648)),
+    ("long", 6144 / 195, 2 * 93600 * 6144 / (2 * 93600 * 195 + 2 * (256 * 3072 + 3072 * 384) * 2),
+     2 * 93600 * 6144 / (2 * 93600 * 195 + 2 * (256 * 3072 + 3072 * 384) * 2 + 2 * 384 * 3072 * 2)),
+    ("step30", 3072 / 99, 2 * 46800 * 3072 / (2 * 46800 * 99 + 1572864),
+     2 * 46800 * 3072 / (2 * 46800 * 99 + 1572864 + 1179648)),
+])
+def test_storage_accounting(name, per_token, effective, with_encoder):
+    st = bench.storage_block(WORKLOADS[name])
+    assert st["per_token_ratio"] == pytest.approx(per_token, abs=0.01)
+    assert st["effective_ratio"] == pytest.approx(effective, abs=0.01)
+    assert st["effective_ratio_with_encoder"] == pytest.approx(with_encoder, abs=0.01)
+    assert st["history_tokens"] == WORKLOADS[name].T
