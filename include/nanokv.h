@@ -84,8 +84,11 @@ size_t nanokv_codec_aux_bytes(const nanokv_codec *c);
  * nanokv_codec_prepare -- fill `aux` (device, 16-byte aligned, at least
  * nanokv_codec_aux_bytes bytes) with the tables the tensor-core encode reads:
  * EC[j][k] = sum_i E[k][i] c_j[i] (fp32, [C][r]) and |c_j|^2 (fp32, [C]).
- * They depend on the codec only, so a caller prepares once per codec and
- * stores the pointer in nanokv_codec.aux.  Needs E.  Asynchronous on stream.
+ * The encode of Fig. 4(b) projects y = E (x - c_a); the tensor-core encode
+ * forms it as E x - EC[a] and finds the nearest center through |c_j|^2 -
+ * 2 x.c_j.  The tables depend on the codec only, so a caller prepares once
+ * per codec and stores the pointer in nanokv_codec.aux; they are summed in a
+ * fixed order, the same on every call.  Needs E.  Asynchronous on stream.
  */
 int nanokv_codec_prepare(const nanokv_codec *c, void *aux, void *stream);
 
