@@ -12,7 +12,8 @@
 // Q~ is stored with the same order and O~ is un-permuted before the restore.
 //   warp 0      TMA: Q, D_{K,h}, C_{K,h}; later D_{V,h}, C_{V,h}
 //   warp 1      MMA issuer
-//   warps 4..7  unpack: thread = key; K codes, V codes, one-hot of a_V
+//   warps 2,3   key-side unpack: K codes, center ids and scales (two keys a thread)
+//   warps 4..7  value-side unpack: thread = key; V codes, one-hot of a_V
 //   warps 8..11 softmax, one thread per query row; prologue/epilogue stores
 #include "tc_common.cuh"
 
@@ -107,7 +108,7 @@ __global__ void __launch_bounds__(384, 1)
     mbar_init(&B.pro_full, 1);
     mbar_init(&B.pro_done, 1);
     mbar_init(&B.qt_ready, 4);
-    mbar_init(&B.kc_full, 4);
+    mbar_init(&B.kc_full, 2);  // the two key-side unpack warps
     mbar_init(&B.kc_empty, 1);
     mbar_init(&B.vc_full, 4);
     mbar_init(&B.v_empty, 1);
@@ -115,8 +116,8 @@ __global__ void __launch_bounds__(384, 1)
     mbar_init(&B.s_full[1], 1);
     mbar_init(&B.p_full[0], 4);
     mbar_init(&B.p_full[1], 4);
-    mbar_init(&B.info_full[0], 4);
-    mbar_init(&B.info_full[1], 4);
+    mbar_init(&B.info_full[0], 2);
+    mbar_init(&B.info_full[1], 2);
     mbar_init(&B.pv_done[0], 1);
     mbar_init(&B.pv_done[1], 1);
     mbar_init(&B.last_done, 1);
@@ -246,53 +247,64 @@ __global__ void __launch_bounds__(384, 1)
         mma_commit(&B.fin_done);
       }
     }
-  } else if (warp >= 4 && warp < 8) {
-    // ---------------- unpack (thread = key) ----------------
-    // The key's ids, scales and packed K / V codes of tile j + 1 are loaded
-    // into registers while tile j is unpacked, so no global-memory latency
-    // sits between the tiles.
-    const int t = (warp - 4) * 32 + lane;
+  } else if (warp == 2 || warp == 3) {
+    // ---------------- key-side unpack: two keys per thread ----------------
+    // Keys t and t + 64 of every tile: their K codes into the K buffer (freed
+    // by the previous tile's scores MMA) and their center id and scales into
+    // the per-key arrays of the tile's parity, which the softmax of tile
+    // j - 2 read last.  The value side runs in warps 4..7 on its own chain,
+    // so the next tile's scores never wait behind this tile's value MMAs.
+    // Each key's ids, scales and codes of tile j + 1 are loaded into
+    // registers while tile j is unpacked.
+    const int t = (warp - 2) * 32 + lane;
     const int cw = r / 32;  // uint4 words of packed codes per key
-    struct KeyData {
-      int ak, av;
+    struct KeyK {
+      int ak;
       float sk, sv;
-      uint4 ck[kMaxCodeWords], cv[kMaxCodeWords];
+      uint4 ck[kMaxCodeWords];
     };
-    auto load_key = [&](int j, KeyData &d) {
-      const int64_t tt = A.t0 + (int64_t)j * BN + t;
-      const bool valid = (int64_t)j * BN + t < A.T;
-      int ak = valid ? (int)A.idk[tt] : 0, av = valid ? (int)A.idv[tt] : 0;
+    auto load_key = [&](int j, int key, KeyK &d) {
+      const int64_t tt = A.t0 + (int64_t)j * BN + key;
+      const bool valid = (int64_t)j * BN + key < A.T;
+      const int ak = valid ? (int)A.idk[tt] : 0;
       d.ak = ak < C ? ak : C - 1;
-      d.av = valid ? (av < C ? av : C - 1) : -1;  // -1: no one-hot entry
       d.sk = valid ? __half2float(A.sk[tt]) : 0.f;
       d.sv = valid ? __half2float(A.sv[tt]) : 0.f;
       const uint4 *pk = reinterpret_cast<const uint4 *>(A.codk + tt * (r / 2));
-      const uint4 *pv = reinterpret_cast<const uint4 *>(A.codv + tt * (r / 2));
 #pragma unroll
-      for (int q = 0; q < kMaxCodeWords; ++q) {
-        d.ck[q] = (q < cw && valid) ? __ldg(pk + q) : make_uint4(0, 0, 0, 0);
-        d.cv[q] = (q < cw && valid) ? __ldg(pv + q) : make_uint4(0, 0, 0, 0);
-      }
+      for (int q = 0; q < kMaxCodeWords; ++q) d.ck[q] = (q < cw && valid) ? __ldg(pk + q) : make_uint4(0, 0, 0, 0);
     };
-    // one tile: unpack `cur` (tile j) after starting the loads of tile j + 1 into `nxt`
-    auto tile = [&](int j, const KeyData &cur, KeyData &nxt) -> bool {
-      if (j + 1 < ntiles) load_key(j + 1, nxt);
-      // ---- K codes
-      // (key info [j & 1] was last read by the softmax of tile j - 2, which finished
-      // before PV of tile j - 2, which the V part of tile j - 1 waited for)
-      if (j >= 1 && !mbar_wait(&B.kc_empty, (j - 1) & 1, abort, err)) return false;
-      if (t == 0) LOW_TRACE(4, j);
+    auto store_key = [&](int j, int key, const KeyK &d) {
 #pragma unroll
       for (int q = 0; q < kMaxCodeWords; ++q) {
         if (q >= cw) break;
-        const uint32_t w[4] = {cur.ck[q].x, cur.ck[q].y, cur.ck[q].z, cur.ck[q].w};
+        const uint32_t w[4] = {d.ck[q].x, d.ck[q].y, d.ck[q].z, d.ck[q].w};
 #pragma unroll
         for (int i = 0; i < 4; ++i)
-          *reinterpret_cast<uint4 *>(sKc + sw128_offset(t, 32 * q + 8 * i, 128)) = unpack8(w[i]);
+          *reinterpret_cast<uint4 *>(sKc + sw128_offset(key, 32 * q + 8 * i, 128)) = unpack8(w[i]);
       }
-      kAK[(j & 1) * 128 + t] = cur.ak;
-      kSK[(j & 1) * 128 + t] = cur.sk;
-      kSV[(j & 1) * 128 + t] = cur.sv;
+      kAK[(j & 1) * 128 + key] = d.ak;
+      kSK[(j & 1) * 128 + key] = d.sk;
+      kSV[(j & 1) * 128 + key] = d.sv;
+    };
+    KeyK cur[2], nxt[2];
+    bool ok = mbar_wait(&B.pro_done, 0, abort, err);  // prologue buffers alias the tiles
+    if (ok && ntiles > 0) {
+      load_key(0, t, cur[0]);
+      load_key(0, t + 64, cur[1]);
+    }
+    for (int j = 0; ok && j < ntiles; ++j) {
+      if (j + 1 < ntiles) {
+        load_key(j + 1, t, nxt[0]);
+        load_key(j + 1, t + 64, nxt[1]);
+      }
+      // the K buffer: tile j - 1's scores are done; the key arrays of this
+      // parity: the softmax of tile j - 2 is done with them
+      if (j >= 1 && !mbar_wait(&B.kc_empty, (j - 1) & 1, abort, err)) { ok = false; break; }
+      if (j >= 2 && !mbar_wait(&B.p_full[j & 1], ((j - 2) >> 1) & 1, abort, err)) { ok = false; break; }
+      if (t == 0) LOW_TRACE(4, j);
+      store_key(j, t, cur[0]);
+      store_key(j, t + 64, cur[1]);
       fence_proxy_async_smem();
       __syncwarp();
       if (lane == 0) {
@@ -300,8 +312,35 @@ __global__ void __launch_bounds__(384, 1)
         mbar_arrive(&B.info_full[j & 1]);
       }
       if (t == 0) LOW_TRACE(5, j);
-      // ---- V codes and one-hot of the value center
-      if (j >= 1 && !mbar_wait(&B.v_empty, (j - 1) & 1, abort, err)) return false;
+      cur[0] = nxt[0];
+      cur[1] = nxt[1];
+    }
+  } else if (warp >= 4 && warp < 8) {
+    // ---------------- value-side unpack (thread = key) ----------------
+    // V codes and the one-hot of the value center into their buffers, freed
+    // by the previous tile's value MMAs; tile j + 1's codes and id are loaded
+    // into registers while tile j is unpacked.
+    const int t = (warp - 4) * 32 + lane;
+    const int cw = r / 32;
+    struct KeyV {
+      int av;
+      uint4 cv[kMaxCodeWords];
+    };
+    auto load_key = [&](int j, KeyV &d) {
+      const int64_t tt = A.t0 + (int64_t)j * BN + t;
+      const bool valid = (int64_t)j * BN + t < A.T;
+      const int av = valid ? (int)A.idv[tt] : 0;
+      d.av = valid ? (av < C ? av : C - 1) : -1;  // -1: no one-hot entry
+      const uint4 *pv = reinterpret_cast<const uint4 *>(A.codv + tt * (r / 2));
+#pragma unroll
+      for (int q = 0; q < kMaxCodeWords; ++q) d.cv[q] = (q < cw && valid) ? __ldg(pv + q) : make_uint4(0, 0, 0, 0);
+    };
+    KeyV cur, nxt;
+    bool ok = mbar_wait(&B.pro_done, 0, abort, err);
+    if (ok && ntiles > 0) load_key(0, cur);
+    for (int j = 0; ok && j < ntiles; ++j) {
+      if (j + 1 < ntiles) load_key(j + 1, nxt);
+      if (j >= 1 && !mbar_wait(&B.v_empty, (j - 1) & 1, abort, err)) { ok = false; break; }
       if (t == 0) LOW_TRACE(6, j);
 #pragma unroll
       for (int q = 0; q < kMaxCodeWords; ++q) {
@@ -328,14 +367,7 @@ __global__ void __launch_bounds__(384, 1)
       __syncwarp();
       if (lane == 0) mbar_arrive(&B.vc_full);
       if (t == 0) LOW_TRACE(7, j);
-      return true;
-    };
-    KeyData ka, kb;
-    bool ok = mbar_wait(&B.pro_done, 0, abort, err);  // prologue buffers alias the tiles
-    if (ok && ntiles > 0) load_key(0, ka);
-    for (int j = 0; ok && j < ntiles; j += 2) {
-      ok = tile(j, ka, kb);
-      if (ok && j + 1 < ntiles) ok = tile(j + 1, kb, ka);
+      cur = nxt;
     }
   } else if (warp >= 8) {
     // ---------------- softmax (thread = query row) ----------------
