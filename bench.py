@@ -46,7 +46,7 @@ BAD_REASONS = ("hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown")
 NCU_TRAFFIC = {
     ("attend_full", "full"): ("tc_full", "952ad7385a3d9deb", 18900341 + 2955424),
     ("attend_low", "long"): ("tc_low_pair", "1af5729c0430d001", 71728100 + 27869668),
-    ("attend_low", "mixed"): ("tc_low", "d15b7a8cf47b4f75", 17933966 + 19342),
+    ("attend_low", "mixed"): ("tc_low", "d71444f9108e510c", 17933850 + 2739),
     ("attend_dense", "full"): ("tc_dense", "bc840a866ba6a1e1", 43226496 + 128366),
     ("encode", "full"): ("tc_encode", "70d83cae2d835770", 30490368 + 0),
 }
